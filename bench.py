@@ -1,0 +1,462 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused EntroPack decode on B200: decoded Gparams/s and the HBM-roofline fraction.
+
+Workload: the 276-layer DiT-like set (seeded synthetic stand-in for the Z-Image-Turbo linear layers of
+the EntroPack README, section 性能), in BF16, compressed at target 4.0 bpp by the host encoder. It is
+then decoded layer by layer into one reused output buffer. A step is one decode pass over all 276
+blobs: 6,174,965,760 parameters. The blobs (about 3.1 GB) are resident in HBM when timing starts.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank decodes its own full replica of the set. No collective touches the data
+path, and the ranks only agree on the time. The JSON line reports weak scaling, with `value` =
+N x params / max-over-ranks step time.
+
+--impl reference times the CPU oracle decoder on the host cores instead: a bounded sample of tiles
+from the same layers each step, with the same metric and unit. The other ranks exit without work.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "decode Gparams/s and % of HBM roofline (276-layer DiT set, 4 bpp) on 1 B200"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--target-bpp", type=float, default=4.0)
+    ap.add_argument("--layers", type=int, default=276, help="debug only: fewer layers makes the line invalid")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="wall-time budget of the CPU baseline sample")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quick", action="store_true",
+                    help="profiling runs: skip rel-L2, the e2e pass and the CPU baseline")
+    ap.add_argument("--json-out", default="")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- environment
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("decode.cu", "epk_format.h"):
+        h.update(open(os.path.join(ROOT, "decode_ep_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic():
+    """DRAM traffic per algorithmic byte from the committed ncu summary. None if the kernel source
+    has changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None
+    if d.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    return d
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.f = None
+
+    def __enter__(self):
+        try:
+            self.f = tempfile.TemporaryFile(mode="w+")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.index)], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.f is None:
+            return None
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for k, n in enumerate(names):
+                if r[5 + k].strip().lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------------- workload
+
+def layer_list(n_layers: int):
+    shapes = synth.dit_layer_shapes()[:n_layers]
+    return [(i, name, M, N) for i, (name, M, N) in enumerate(shapes)]
+
+
+def build_blobs(layers, target_bpp, workers, device=None):
+    """Generates and compresses every layer with the product host encoder, one encoder thread per
+    layer and layers in parallel. If `device` is given, each layer is decoded on the GPU as it
+    arrives, and rel-L2 is accumulated: pooled sqrt(ΣΔ²/ΣW²) in fp64, plus the per-layer mean."""
+    import decode_ep_b200 as ep
+
+    def job(item):
+        i, _, M, N = item
+        w = synth.dit_layer(i, shape=(M, N))
+        t0 = time.perf_counter()
+        c = ep.compress(w, ep.EntroPackLossyConfig(target_bpp, threads=1))
+        return i, c, time.perf_counter() - t0, (w if device is not None else None)
+
+    torch_threads = torch.get_num_threads()
+    torch.set_num_threads(1)
+    out = [None] * len(layers)
+    enc_cpu = num = den = 0.0
+    per = []
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+        for i, c, dt, w in ex.map(job, layers):
+            out[i] = c
+            enc_cpu += dt
+            if w is not None:
+                wd = w.to(device).double()
+                y = ep.decompress(c, device=device).double()
+                d2, w2 = float(((y - wd) ** 2).sum()), float((wd ** 2).sum())
+                num, den = num + d2, den + w2
+                per.append((d2 / w2) ** 0.5)
+                del wd, y
+    wall = time.perf_counter() - t0
+    torch.set_num_threads(torch_threads)
+    rel = ((num / den) ** 0.5, float(np.mean(per))) if per else (None, None)
+    return out, wall, enc_cpu, rel
+
+
+# --------------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import decode_ep_b200 as ep
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+
+    layers = layer_list(args.layers)
+    workers = max(1, min(os.cpu_count() or 1, 64) // max(world, 1))
+    blobs, enc_wall, enc_cpu, (rel_l2, rel_l2_mean) = build_blobs(layers, args.target_bpp, workers,
+                                                                  device if rank == 0 and not args.quick else None)
+    n_params = sum(M * N for _, _, M, N in layers)
+    blob_bytes = sum(len(c.blob) for c in blobs)
+    max_numel = max(M * N for _, _, M, N in layers)
+
+    L = ep.lib()
+    dblobs = [c.device_blob(device) for c in blobs]
+    hdrs = [c.header for c in blobs]
+    ptrs = [d.data_ptr() for d in dblobs]
+    sizes = [len(c.blob) for c in blobs]
+    out = torch.empty(max_numel, dtype=torch.bfloat16, device=device)
+    out_ptr, out_bytes = out.data_ptr(), out.numel() * out.element_size()
+    stream = torch.cuda.current_stream(device)
+    sptr = stream.cuda_stream
+
+    def step():
+        st = 0
+        for h, p, n in zip(hdrs, ptrs, sizes):
+            st |= L.ep_decompress_into(h, p, n, out_ptr, out_bytes, sptr)
+        if st:
+            raise RuntimeError(L.ep_last_error().decode())
+
+    assert ep.device_status(stream) == 0
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize(device)
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        stop.record(stream)
+        torch.cuda.synchronize(device)
+    ms_total = start.elapsed_time(stop)
+    status = ep.device_status(stream)
+    if status:
+        raise RuntimeError(f"device status {status} after the timed region")
+    t = torch.tensor([ms_total], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.barrier()
+    ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    value = world * n_params / (ms_per_step * 1e-3) / 1e9
+
+    # Roofline of the decode kernel: algorithmic bytes (blob read once + container written once)
+    # over the summed per-launch event durations of one pass.
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in layers]
+    for (a, b), h, p, n in zip(evs, hdrs, ptrs, sizes):
+        a.record(stream)
+        L.ep_decompress_into(h, p, n, out_ptr, out_bytes, sptr)
+        b.record(stream)
+    torch.cuda.synchronize(device)
+    kernel_ms = sum(a.elapsed_time(b) for a, b in evs)
+    alg_bytes = blob_bytes + 2 * n_params
+    achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    tr = committed_traffic()
+    traffic = None
+    if tr is not None:
+        traffic = tr["dram_bytes_per_algorithmic_byte"] * alg_bytes / len(layers)
+
+    e2e = run_e2e(args, L, blobs, layers, device, stream) if rank == 0 and not args.quick else None
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
+        cpu = cpu_baseline(blobs, layers, args.cpu_seconds)
+
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "Gparams/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u32+f32", "data": "synthetic",
+        "config": {"workload": "dit276_bf16_4bpp", "layers": len(layers), "params": n_params,
+                   "target_bpp": args.target_bpp, "actual_bpp": round(8 * blob_bytes / n_params, 4),
+                   "container": "bf16", "rounds_per_tile": 16, "blob_bytes": blob_bytes,
+                   "output": f"one reused {2 * max_numel / 1e6:.1f} MB buffer",
+                   "l2": "inputs larger than L2 (blobs %.2f GB read per step)" % (blob_bytes / 1e9),
+                   "parallelism": f"replicas x{world}",
+                   "rel_l2_pooled": None if rel_l2 is None else round(rel_l2, 5),
+                   "rel_l2_layer_mean": None if rel_l2_mean is None else round(rel_l2_mean, 5),
+                   "encode_wall_s": round(enc_wall, 2), "encode_cpu_s": round(enc_cpu, 2),
+                   "encode_threads": workers},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_kind} copy bandwidth",
+                     "per_launch_algorithmic_bytes": alg_bytes / len(layers),
+                     "per_launch_us": round(1e3 * kernel_ms / len(layers), 3),
+                     "kernel_ms_per_pass": round(kernel_ms, 4),
+                     "frac_of_nominal_8TBs": round(achieved / 8000.0, 4)},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clk.summary(),
+        "gpu_launches": len(layers) * args.steps,
+    }
+    return line
+
+
+def run_e2e(args, L, blobs, layers, device, stream):
+    """Same metric through the C ABI with host buffers. Every step copies each blob from pinned host
+    memory to the device, decodes it, and reads the decoded layer back into pinned host memory."""
+    max_blob = max(len(c.blob) for c in blobs)
+    max_numel = max(M * N for _, _, M, N in layers)
+    pinned = [torch.frombuffer(bytearray(c.blob), dtype=torch.uint8).pin_memory() for c in blobs]
+    stage = torch.empty(max_blob + 256, dtype=torch.uint8, device=device)
+    out = torch.empty(max_numel, dtype=torch.bfloat16, device=device)
+    host_out = torch.empty(max_numel, dtype=torch.bfloat16).pin_memory()
+    sptr = stream.cuda_stream
+    numels = [M * N for _, _, M, N in layers]
+
+    def step():
+        st = 0
+        for c, hb, n in zip(blobs, pinned, numels):
+            stage[: hb.numel()].copy_(hb, non_blocking=True)
+            st |= L.ep_decompress_into(c.header, stage.data_ptr(), len(c.blob), out.data_ptr(), out.numel() * 2, sptr)
+            host_out[:n].copy_(out[:n], non_blocking=True)
+        if st:
+            raise RuntimeError(L.ep_last_error().decode())
+
+    step()
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / args.e2e_steps
+    n_params = sum(numels)
+    return {"value": round(n_params / (ms * 1e-3) / 1e9, 2), "unit": "Gparams/s",
+            "h2d_bytes_per_step": int(sum(len(c.blob) for c in blobs)),
+            "d2h_bytes_per_step": int(2 * n_params), "ms_per_step": round(ms, 3), "steps": args.e2e_steps}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def cpu_sample_plan(blobs, layers, run=16):
+    """Runs of `run` consecutive tiles, taken round-robin across the layers: (layer, t0, t1)."""
+    import oracle
+    per = [oracle.blob_info(c.blob)["num_tiles"] for c in blobs]
+    plan = []
+    k = 0
+    while len(plan) < 20000 and k < max(per):
+        for li, T in enumerate(per):
+            if k < T:
+                plan.append((li, k, min(T, k + run)))
+        k += run
+    return plan
+
+
+def oracle_decode_for(seconds, blobs, layers, plan, workers):
+    """Decodes the planned tile runs on `workers` threads until `seconds` of wall time have passed.
+    Returns (params decoded, elapsed seconds)."""
+    import oracle
+    outs = {li: np.zeros(blobs[li].shape, np.uint16) for li in {p[0] for p in plan}}
+
+    def job(item):
+        li, t0, t1 = item
+        oracle.decode_tiles(blobs[li].blob, t0, t1, outs[li])
+        _, _, M, N = layers[li]
+        return min(t1 * 4096, M * N) - t0 * 4096
+
+    done = 0
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+        it = iter(plan)
+        futs = set()
+        for _ in range(2 * workers):
+            item = next(it, None)
+            if item is None:
+                break
+            futs.add(ex.submit(job, item))
+        while futs:
+            fin, futs = cf.wait(futs, return_when=cf.FIRST_COMPLETED)
+            for f in fin:
+                done += f.result()
+            if time.perf_counter() - t0 < seconds:
+                for _ in range(len(fin)):
+                    item = next(it, None)
+                    if item is not None:
+                        futs.add(ex.submit(job, item))
+    return done, time.perf_counter() - t0
+
+
+def cpu_baseline(blobs, layers, seconds):
+    import oracle
+    oracle.build()
+    workers = os.cpu_count() or 1
+    plan = cpu_sample_plan(blobs, layers)
+    n, dt = oracle_decode_for(seconds, blobs, layers, plan, workers)
+    return {"value": round(n / dt / 1e9, 5), "unit": "Gparams/s", "cores": workers, "kind": "oracle",
+            "sample": f"{n} parameters: runs of 16 tiles taken round-robin across all {len(layers)} layers, "
+                      f"decoded by the C oracle on {workers} threads for {dt:.1f} s"}
+
+
+# ------------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    # The bounded sample: four layers, one of each large shape class, encoded by the oracle encoder
+    # (untimed setup). Each step decodes the same fixed set of their tiles.
+    sel = [0, 4, 6, 7]
+    layers = [layer_list(276)[i] for i in sel]
+
+    class B:
+        pass
+    blobs = []
+    for i, _, M, N in layers:
+        w = synth.dit_layer(i, shape=(M, N))
+        b = B()
+        b.blob, _ = oracle.compress(synth.container_bits(w), 1, args.target_bpp)
+        b.shape = (M, N)
+        blobs.append(b)
+    layers = [(k, name, M, N) for k, (_, name, M, N) in enumerate(layers)]
+    workers = os.cpu_count() or 1
+    plan = cpu_sample_plan(blobs, layers)[: 6 * workers]
+    for _ in range(args.warmup):
+        oracle_decode_for(1e9, blobs, layers, plan[:workers], workers)
+    tot_n = tot_t = 0.0
+    for _ in range(args.steps):
+        n, dt = oracle_decode_for(1e9, blobs, layers, plan, workers)
+        tot_n += n
+        tot_t += dt
+    value = tot_n / tot_t / 1e9
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "Gparams/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot_t / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32+f32", "data": "synthetic",
+        "config": {"workload": "dit276_bf16_4bpp", "target_bpp": args.target_bpp, "container": "bf16",
+                   "sample_layers": sel, "sample_tile_runs_per_step": len(plan)},
+        "cpu_baseline": {"value": round(value, 5), "unit": "Gparams/s", "cores": workers, "kind": "oracle",
+                         "sample": f"{len(plan)} runs of 16 tiles (4096 parameters each) per step from layers {sel}, "
+                                   f"C oracle on {workers} threads"},
+        "e2e": {"value": round(value, 5), "unit": "Gparams/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if line is not None:
+        s = json.dumps(line)
+        print(s, flush=True)
+        if args.json_out:
+            with open(args.json_out, "w") as f:
+                f.write(s + "\n")
+
+
+if __name__ == "__main__":
+    main()

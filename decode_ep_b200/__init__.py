@@ -1,0 +1,217 @@
+"""decode_ep_b200: EntroPack lossy weight compression with a fused sm_100a decode.
+
+This is a thin ctypes binding over ``libentropack.so`` (C ABI in ``include/entropack.h``). Every
+step of compression and decode runs in that library: the host encoder on the CPU, the decode in
+the CUDA kernel. This module only moves arguments. PyTorch provides device memory and streams.
+There is no CPU fallback. If the library is missing or cannot load, the import fails loudly.
+
+API, after the EntroPack README (quick-start and Config sections):
+
+    cfg = EntroPackLossyConfig(target_bpp=3.5)
+    c = compress(tensor, cfg)                  # CompressedTensor; c.actual_bpp counts metadata
+    w = decompress(c)                          # CUDA tensor, same shape and dtype
+    decompress_into(c, out, stream=None)       # hot path: preallocated output, async on a stream
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass, field
+
+import torch
+
+from . import build as _build
+
+__all__ = ["EntroPackLossyConfig", "CompressedTensor", "EntroPackError", "compress", "decompress",
+           "decompress_into", "decode_coords", "device_status", "blob_info", "lib"]
+
+EP_BF16, EP_FP16, EP_FP32, EP_FP8_E4M3, EP_INT8 = 1, 2, 3, 4, 5
+_TORCH_TO_EP = {torch.bfloat16: EP_BF16, torch.float16: EP_FP16, torch.float32: EP_FP32,
+                torch.float8_e4m3fn: EP_FP8_E4M3, torch.int8: EP_INT8}
+_EP_TO_TORCH = {v: k for k, v in _TORCH_TO_EP.items()}
+HEADER_BYTES = 64
+
+
+class EntroPackError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+class _Options(ctypes.Structure):
+    _fields_ = [("rounds_per_tile", ctypes.c_uint32), ("sample_coords", ctypes.c_uint32),
+                ("bisection_iters", ctypes.c_uint32), ("threads", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libentropack.so. The library is built in-tree if it is missing or out of date."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB
+        if not os.path.exists(path) or _build.stale():
+            path = _build.build()
+        L = ctypes.CDLL(path)
+        c = ctypes
+        L.ep_options_default.argtypes = [c.POINTER(_Options)]
+        L.ep_compress.argtypes = [c.c_void_p, c.c_int, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_double,
+                                  c.POINTER(_Options), c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
+                                  c.POINTER(c.c_double)]
+        L.ep_blob_free.argtypes = [c.c_void_p]
+        L.ep_blob_info.argtypes = [c.c_void_p, c.c_size_t, c.POINTER(c.c_int), c.POINTER(c.c_int64),
+                                   c.POINTER(c.c_int64), c.POINTER(c.c_double)]
+        for name in ("ep_decompress_into", "ep_decode_coords_into"):
+            getattr(L, name).argtypes = [c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p, c.c_size_t, c.c_void_p]
+        L.ep_decompress.argtypes = [c.c_void_p, c.c_void_p, c.c_size_t, c.POINTER(c.c_void_p), c.c_void_p]
+        L.ep_get_device_status.argtypes = [c.c_void_p, c.POINTER(c.c_int32)]
+        L.ep_status_string.restype = c.c_char_p
+        L.ep_status_string.argtypes = [c.c_int]
+        L.ep_last_error.restype = c.c_char_p
+        for name in ("ep_compress", "ep_blob_info", "ep_decompress_into", "ep_decode_coords_into", "ep_decompress",
+                     "ep_get_device_status"):
+            getattr(L, name).restype = c.c_int
+        _lib = L
+    return _lib
+
+
+def _check(st: int, what: str) -> None:
+    if st != 0:
+        L = lib()
+        msg = L.ep_last_error().decode() or L.ep_status_string(st).decode()
+        raise EntroPackError(st, f"{what}: {msg} (status {st})")
+
+
+@dataclass
+class EntroPackLossyConfig:
+    """Lossy EntroPack configuration (README, Config table).
+
+    target_bpp: finite, in [0.001, 11]. Fractional values are allowed. It counts metadata.
+    rounds_per_tile: G. A tile is 32 lanes x G rounds x 8 coordinates (default 4096 coordinates).
+    """
+    target_bpp: float
+    rounds_per_tile: int = 16
+    sample_coords: int = 1 << 18
+    bisection_iters: int = 40
+    threads: int = 0
+
+    def _options(self) -> _Options:
+        return _Options(self.rounds_per_tile, self.sample_coords, self.bisection_iters, self.threads)
+
+
+@dataclass
+class CompressedTensor:
+    """A compressed 2-D tensor: the blob bytes plus a cached device copy per CUDA device."""
+    blob: bytes
+    shape: tuple
+    dtype: torch.dtype
+    actual_bpp: float
+    _device_blobs: dict = field(default_factory=dict, repr=False)
+
+    @property
+    def header(self) -> bytes:
+        return self.blob[:HEADER_BYTES]
+
+    @property
+    def compressed_bits(self) -> int:
+        return 8 * len(self.blob)
+
+    def device_blob(self, device=None) -> torch.Tensor:
+        """The blob as a uint8 CUDA tensor (cached). cudaMalloc alignment (256 B) meets the 16 B rule."""
+        dev = torch.device("cuda", torch.cuda.current_device() if device is None else torch.device(device).index)
+        t = self._device_blobs.get(dev.index)
+        if t is None:
+            host = torch.frombuffer(bytearray(self.blob), dtype=torch.uint8)
+            t = host.to(dev)
+            self._device_blobs[dev.index] = t
+        return t
+
+    def state_dict(self) -> dict:
+        return {"blob": torch.frombuffer(bytearray(self.blob), dtype=torch.uint8)}
+
+    @staticmethod
+    def from_blob(blob: bytes) -> "CompressedTensor":
+        info = blob_info(blob)
+        return CompressedTensor(bytes(blob), (info["rows"], info["cols"]), _EP_TO_TORCH[info["dtype"]],
+                                info["actual_bpp"])
+
+
+def blob_info(blob: bytes) -> dict:
+    """Full host validation of a blob (header, tables, offsets, CRC) and its description."""
+    c = ctypes
+    dt, M, N, bpp = c.c_int(), c.c_int64(), c.c_int64(), c.c_double()
+    _check(lib().ep_blob_info(blob, len(blob), c.byref(dt), c.byref(M), c.byref(N), c.byref(bpp)), "blob_info")
+    return {"dtype": dt.value, "rows": M.value, "cols": N.value, "actual_bpp": bpp.value}
+
+
+def compress(tensor: torch.Tensor, config: EntroPackLossyConfig | float) -> CompressedTensor:
+    """Lossy compression of a 2-D tensor (CPU or CUDA). The library runs rate control and encoding."""
+    if not isinstance(config, EntroPackLossyConfig):
+        config = EntroPackLossyConfig(float(config))
+    if tensor.dim() != 2:
+        raise EntroPackError(-3, "compress: EntroPack lossy mode takes 2-D tensors only")
+    if tensor.dtype not in _TORCH_TO_EP:
+        raise EntroPackError(-2, f"compress: unsupported dtype {tensor.dtype}")
+    t = tensor if tensor.stride(1) == 1 else tensor.contiguous()
+    rows, cols = t.shape
+    blob_p, nbytes, actual = ctypes.c_void_p(), ctypes.c_size_t(), ctypes.c_double()
+    opt = config._options()
+    if t.is_cuda:
+        with torch.cuda.device(t.device):
+            torch.cuda.current_stream().synchronize()
+            st = lib().ep_compress(t.data_ptr(), 1, _TORCH_TO_EP[t.dtype], rows, cols, t.stride(0),
+                                   float(config.target_bpp), ctypes.byref(opt), ctypes.byref(blob_p),
+                                   ctypes.byref(nbytes), ctypes.byref(actual))
+    else:
+        st = lib().ep_compress(t.data_ptr(), 0, _TORCH_TO_EP[t.dtype], rows, cols, t.stride(0),
+                               float(config.target_bpp), ctypes.byref(opt), ctypes.byref(blob_p),
+                               ctypes.byref(nbytes), ctypes.byref(actual))
+    _check(st, "compress")
+    try:
+        blob = ctypes.string_at(blob_p.value, nbytes.value)
+    finally:
+        lib().ep_blob_free(blob_p)
+    return CompressedTensor(blob, (rows, cols), tensor.dtype, actual.value)
+
+
+def _stream_ptr(stream) -> int | None:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def decompress_into(compressed: CompressedTensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+    """Fused decode into a preallocated CUDA tensor (contiguous, the blob's dtype and shape).
+    Asynchronous on ``stream`` (default: the current stream). It allocates nothing and does not
+    synchronise."""
+    if not out.is_cuda or not out.is_contiguous() or out.dtype != compressed.dtype:
+        raise EntroPackError(-9, "decompress_into: out must be a contiguous CUDA tensor of the blob's dtype")
+    dblob = compressed.device_blob(out.device)
+    _check(lib().ep_decompress_into(compressed.header, dblob.data_ptr(), len(compressed.blob), out.data_ptr(),
+                                    out.numel() * out.element_size(), _stream_ptr(stream)), "decompress_into")
+    return out
+
+
+def decompress(compressed: CompressedTensor, config=None, device=None, stream=None) -> torch.Tensor:
+    """Decode to a new CUDA tensor of the original shape and dtype (README, quick-start section)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    out = torch.empty(compressed.shape, dtype=compressed.dtype, device=dev)
+    return decompress_into(compressed, out, stream)
+
+
+def decode_coords(compressed: CompressedTensor, device=None, stream=None) -> torch.Tensor:
+    """Lattice coordinates z = 2v (int32, shape of the tensor) as the CUDA decode produces them."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    out = torch.empty(compressed.shape, dtype=torch.int32, device=dev)
+    dblob = compressed.device_blob(dev)
+    _check(lib().ep_decode_coords_into(compressed.header, dblob.data_ptr(), len(compressed.blob), out.data_ptr(),
+                                       out.numel() * 4, _stream_ptr(stream)), "decode_coords")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronises the stream, then reads and clears the device status word (EP_DEV_* bits)."""
+    flags = ctypes.c_int32()
+    _check(lib().ep_get_device_status(_stream_ptr(stream), ctypes.byref(flags)), "device_status")
+    return flags.value

@@ -1,0 +1,575 @@
+// Host encoder of the EPK1 blob: ep_compress. This runs once per tensor and is not the hot path.
+//
+// The steps follow the EntroPack pages (arXiv 2609.34185):
+//   - Each row is normalised by its own scale s_row (paper page abstract; modelscope summary).
+//   - Each 8-wide group is quantised to the nearest E8 point at one global resolution alpha.
+//   - Alpha comes from bisection on log2(alpha) against a storage estimate taken on a sample of
+//     rows, so the full stream is never re-encoded (paper page abstract; techmoon article).
+//   - The coordinates are rANS-coded under 17 conditional 12-bit tables, in independent tiles of
+//     32 interleaved lanes (abstract; modelscope summary).
+// All floating point is IEEE double/binary32, round-to-nearest, with no FMA contraction. The
+// build passes -ffp-contract=off, so every estimate and every quantisation decision is a fixed
+// function of the input, whatever the thread count.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdlib>
+#include <functional>
+#include <thread>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "capi_internal.h"
+#include "entropack.h"
+#include "epk_format.h"
+
+namespace epk {
+namespace {
+
+// ------------------------------------------------------------------------------- threads
+
+void parallel_for(int64_t n, int threads, const std::function<void(int64_t, int64_t, int)>& fn) {
+    if (n <= 0) return;
+    int nt = int(std::min<int64_t>(threads, n));
+    if (nt <= 1) { fn(0, n, 0); return; }
+    int64_t chunk = std::max<int64_t>(1, n / (int64_t(nt) * 16));
+    std::atomic<int64_t> next{0};
+    std::vector<std::thread> pool;
+    pool.reserve(nt);
+    for (int t = 0; t < nt; ++t)
+        pool.emplace_back([&, t] {
+            for (;;) {
+                int64_t b = next.fetch_add(chunk);
+                if (b >= n) break;
+                fn(b, std::min(n, b + chunk), t);
+            }
+        });
+    for (auto& th : pool) th.join();
+}
+
+// ---------------------------------------------------------------------- number formats
+
+float bf16_bits_to_float(uint16_t h) {
+    uint32_t u = uint32_t(h) << 16;
+    float f;
+    std::memcpy(&f, &u, 4);
+    return f;
+}
+
+uint16_t float_to_bf16_rne(float f) {
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    uint32_t rounding = 0x7FFFu + ((u >> 16) & 1u);  // ties go to the even upper half
+    return uint16_t((u + rounding) >> 16);           // inputs here are finite and non-negative
+}
+
+float half_bits_to_float(uint16_t h) {
+    int e = (h >> 10) & 31, m = h & 1023;
+    float mag;
+    if (e == 31) mag = m ? NAN : INFINITY;
+    else if (e == 0) mag = std::ldexp(float(m), -24);
+    else mag = std::ldexp(float(1024 + m), e - 25);
+    return (h & 0x8000) ? -mag : mag;
+}
+
+float e4m3_bits_to_float(uint8_t c) {
+    int e = (c >> 3) & 15, m = c & 7;
+    float mag;
+    if (e == 15 && m == 7) mag = NAN;
+    else if (e == 0) mag = std::ldexp(float(m), -9);
+    else mag = std::ldexp(float(8 + m), e - 10);
+    return (c & 0x80) ? -mag : mag;
+}
+
+// Reads rows of a strided row-major container tensor as binary32.
+struct Source {
+    const uint8_t* base;
+    int dtype;
+    int64_t N, stride;  // elements
+    float e4m3[256];
+
+    Source(const void* p, int dt, int64_t n, int64_t st) : base(static_cast<const uint8_t*>(p)), dtype(dt), N(n), stride(st) {
+        for (int i = 0; i < 256; ++i) e4m3[i] = e4m3_bits_to_float(uint8_t(i));
+    }
+    void row(int64_t i, float* out) const {
+        const uint8_t* r = base + i * stride * elem_bytes(dtype);
+        switch (dtype) {
+            case EP_BF16: { const uint16_t* q = reinterpret_cast<const uint16_t*>(r); for (int64_t j = 0; j < N; ++j) out[j] = bf16_bits_to_float(q[j]); break; }
+            case EP_FP16: { const uint16_t* q = reinterpret_cast<const uint16_t*>(r); for (int64_t j = 0; j < N; ++j) out[j] = half_bits_to_float(q[j]); break; }
+            case EP_FP32: std::memcpy(out, r, sizeof(float) * size_t(N)); break;
+            case EP_FP8_E4M3: for (int64_t j = 0; j < N; ++j) out[j] = e4m3[r[j]]; break;
+            case EP_INT8: { const int8_t* q = reinterpret_cast<const int8_t*>(r); for (int64_t j = 0; j < N; ++j) out[j] = float(q[j]); break; }
+        }
+    }
+};
+
+// ------------------------------------------------------------------------------ lattice
+
+// Nearest point of D8 (integer vectors with even sum), after Conway and Sloane's D_n decoder:
+// round each coordinate half away from zero. If the sum is odd, re-round the coordinate that is
+// furthest from its rounded value (lowest index on ties) in the other direction.
+inline void nearest_d8(const double* x, int64_t* f) {
+    int64_t sum = 0;
+    int worst = 0;
+    double werr = -1.0;
+    for (int k = 0; k < 8; ++k) {
+        f[k] = int64_t(std::round(x[k]));
+        sum += f[k];
+        double e = std::fabs(x[k] - double(f[k]));
+        if (e > werr) { werr = e; worst = k; }
+    }
+    if (sum & 1) f[worst] += (x[worst] - double(f[worst]) >= 0.0) ? 1 : -1;
+}
+
+// Nearest E8 = D8 ∪ (D8 + 1/2) point. Writes the coset bit and the coded integers t[8]:
+// t_i = u_i for i < 7, and t_7 = h, where u_7 = 2h + (Σ_{i<7} u_i mod 2).
+inline int e8_code(const double* x, int32_t* t) {
+    int64_t a[8], c[8];
+    double xh[8];
+    nearest_d8(x, a);
+    for (int k = 0; k < 8; ++k) xh[k] = x[k] - 0.5;
+    nearest_d8(xh, c);
+    double d0 = 0.0, d1 = 0.0;
+    for (int k = 0; k < 8; ++k) {
+        double e0 = x[k] - double(a[k]);
+        double e1 = x[k] - (double(c[k]) + 0.5);
+        d0 += e0 * e0;
+        d1 += e1 * e1;
+    }
+    const int64_t* u = (d0 <= d1) ? a : c;
+    int64_t s = 0;
+    for (int i = 0; i < 7; ++i) { t[i] = int32_t(u[i]); s += u[i]; }
+    t[7] = int32_t((u[7] - (s & 1)) / 2);
+    return d0 <= d1 ? 0 : 1;
+}
+
+inline int32_t hi_of(int32_t t, int r) { return t >> r; }  // arithmetic shift = floor division by 2^r
+inline int idx_of(int32_t hi) { return (hi >= -31 && hi <= 31) ? hi + 31 : kEscIdx; }
+inline int cls_of(int32_t hi, int b) {
+    int32_t m = hi >= 0 ? hi : -hi - b;
+    return m < 3 ? int(m) : 3;
+}
+
+// Context and table symbol of each of the 8 positions of one group.
+inline void group_syms(int b, const int32_t* t, int r, uint8_t* ctx, uint8_t* sym, int32_t* hi) {
+    for (int i = 0; i < 8; ++i) hi[i] = hi_of(t[i], r);
+    ctx[0] = 0;
+    sym[0] = uint8_t(64 * b + idx_of(hi[0]));
+    for (int i = 1; i < 8; ++i) {
+        ctx[i] = uint8_t((i < 7 ? 1 : 9) + 4 * b + cls_of(hi[i - 1], b));
+        sym[i] = uint8_t(idx_of(hi[i]));
+    }
+}
+
+int raw_bits_for(float alpha) {
+    int r = 0;
+    while (r < 12 && 8.0 * double(int64_t(1) << r) < double(alpha)) ++r;
+    return r;
+}
+
+// ------------------------------------------------------------------------------ tables
+
+using Counts = std::vector<uint64_t>;  // [17][128]
+
+// 12-bit normalisation: f = max(1, floor(4096 n_s / n)) for present symbols. The rounding gap is
+// closed at the largest frequency, or in steps of whole units when there is too much. A single
+// present symbol gets 4096.
+void normalize(const uint64_t* cnt, int A, uint32_t* f) {
+    uint64_t total = 0;
+    int present = 0;
+    for (int s = 0; s < A; ++s) { total += cnt[s]; present += cnt[s] != 0; f[s] = 0; }
+    if (!present) return;
+    if (present == 1) { for (int s = 0; s < A; ++s) if (cnt[s]) f[s] = kProbScale; return; }
+    int64_t sum = 0;
+    for (int s = 0; s < A; ++s) {
+        if (!cnt[s]) continue;
+        uint64_t q = cnt[s] * uint64_t(kProbScale) / total;
+        f[s] = q ? uint32_t(q) : 1u;
+        sum += f[s];
+    }
+    int64_t d = int64_t(kProbScale) - sum;
+    while (d) {
+        int best = -1;
+        for (int s = 0; s < A; ++s) if (f[s] && (best < 0 || f[s] > f[best])) best = s;
+        if (d > 0) { f[best] += uint32_t(d); d = 0; }
+        else {
+            int64_t take = std::min<int64_t>(-d, int64_t(f[best]) - 1);
+            f[best] -= uint32_t(take);
+            d += take;
+        }
+    }
+}
+
+struct Tables {
+    uint32_t f[kNumCtx][128];
+    uint32_t cum[kNumCtx][128];
+    int lo[kNumCtx], cnt[kNumCtx];
+    uint64_t nsym = 0;
+
+    void build(const Counts& c) {
+        nsym = 0;
+        for (int k = 0; k < kNumCtx; ++k) {
+            int A = k == 0 ? 128 : 64;
+            normalize(&c[size_t(k) * 128], A, f[k]);
+            for (int s = A; s < 128; ++s) f[k][s] = 0;
+            int first = -1, last = -1;
+            for (int s = 0; s < A; ++s) if (c[size_t(k) * 128 + s]) { if (first < 0) first = s; last = s; }
+            lo[k] = first < 0 ? 0 : first;
+            cnt[k] = first < 0 ? 0 : last - first + 1;
+            nsym += uint64_t(cnt[k]);
+            uint32_t acc = 0;
+            for (int s = 0; s < 128; ++s) { cum[k][s] = acc; acc += f[k][s]; }
+        }
+    }
+    uint64_t serialized_bytes() const { return 2 * kNumCtx + (12 * nsym + 7) / 8; }
+    void serialize(uint8_t* out) const {
+        for (int k = 0; k < kNumCtx; ++k) { out[k] = uint8_t(lo[k]); out[kNumCtx + k] = uint8_t(cnt[k]); }
+        uint8_t* bits = out + 2 * kNumCtx;
+        uint64_t pos = 0;
+        for (int k = 0; k < kNumCtx; ++k)
+            for (int s = lo[k]; s < lo[k] + cnt[k]; ++s, pos += 12) {
+                uint32_t v = cnt[k] == 1 ? 0u : f[k][s];
+                uint32_t word = v << (pos & 7);  // 12 + 7 bits fit in three bytes
+                bits[pos >> 3] |= uint8_t(word);
+                bits[(pos >> 3) + 1] |= uint8_t(word >> 8);
+                if (word >> 16) bits[(pos >> 3) + 2] |= uint8_t(word >> 16);
+            }
+    }
+};
+
+// ------------------------------------------------------------------------------ encoder
+
+struct Encoder {
+    const Source& src;
+    int64_t M, N, NG, gpr;
+    int G, threads;
+    uint32_t T;
+    std::vector<uint16_t> sbits;
+    std::vector<float> s;
+
+    Encoder(const Source& sc, int64_t m, int64_t n, int g, int th)
+        : src(sc), M(m), N(n), NG(m * n / 8), gpr(n / 8), G(g), threads(th) {
+        T = uint32_t((NG + 32 * int64_t(G) - 1) / (32 * int64_t(G)));
+    }
+
+    // Row scales (root mean square in double, index order → binary32 → BF16) and max |w|/s.
+    // Returns false on a non-finite input.
+    bool scales(double& amax) {
+        sbits.assign(size_t(M), 0);
+        s.assign(size_t(M), 0.f);
+        std::vector<double> tmax(size_t(std::max(threads, 1)), 0.0);
+        std::atomic<bool> finite{true};
+        parallel_for(M, threads, [&](int64_t b, int64_t e, int t) {
+            std::vector<float> w(static_cast<size_t>(N));
+            for (int64_t i = b; i < e; ++i) {
+                src.row(i, w.data());
+                double acc = 0.0;
+                for (int64_t j = 0; j < N; ++j) {
+                    if (!std::isfinite(w[j])) { finite = false; return; }
+                    acc += double(w[j]) * double(w[j]);
+                }
+                float rms = float(std::sqrt(acc / double(N)));
+                sbits[size_t(i)] = float_to_bf16_rne(rms);
+                s[size_t(i)] = bf16_bits_to_float(sbits[size_t(i)]);
+                if (s[size_t(i)] != 0.f)
+                    for (int64_t j = 0; j < N; ++j) tmax[size_t(t)] = std::max(tmax[size_t(t)], std::fabs(double(w[j])) / double(s[size_t(i)]));
+            }
+        });
+        amax = *std::max_element(tmax.begin(), tmax.end());
+        return finite;
+    }
+
+    // Quantises one row (already converted) at alpha: coded integers t and coset bits per group.
+    void quantize_row(const float* w, int64_t i, float alpha, int32_t* t, uint8_t* b) const {
+        double sd = double(s[size_t(i)]), ad = double(alpha);
+        double x[8];
+        for (int64_t q = 0; q < gpr; ++q) {
+            for (int k = 0; k < 8; ++k) x[k] = (sd == 0.0) ? 0.0 : (ad * double(w[q * 8 + k])) / sd;
+            b[q] = uint8_t(e8_code(x, t + 8 * q));
+        }
+    }
+
+    // Storage estimate in bytes from the row sample (same definition the format fixes).
+    double estimate(float alpha, uint32_t sample_coords) const {
+        int64_t Rs = std::min<int64_t>(M, (int64_t(sample_coords) + N - 1) / N);
+        int r = raw_bits_for(alpha);
+        int nt = std::max(1, threads);
+        std::vector<Counts> counts(size_t(nt), Counts(size_t(kNumCtx) * 128, 0));
+        std::vector<uint64_t> esc(size_t(nt), 0);
+        parallel_for(Rs, threads, [&](int64_t b, int64_t e, int th) {
+            std::vector<float> w(static_cast<size_t>(N));
+            std::vector<int32_t> t(static_cast<size_t>(N));
+            std::vector<uint8_t> cb(static_cast<size_t>(gpr));
+            Counts& c = counts[size_t(th)];
+            for (int64_t k = b; k < e; ++k) {
+                int64_t row = (k * M) / Rs;
+                src.row(row, w.data());
+                quantize_row(w.data(), row, alpha, t.data(), cb.data());
+                for (int64_t q = 0; q < gpr; ++q) {
+                    uint8_t ctx[8], sym[8];
+                    int32_t hi[8];
+                    group_syms(cb[size_t(q)], &t[size_t(q * 8)], r, ctx, sym, hi);
+                    for (int i = 0; i < 8; ++i) {
+                        c[size_t(ctx[i]) * 128 + sym[i]]++;
+                        esc[size_t(th)] += idx_of(hi[i]) == kEscIdx;
+                    }
+                }
+            }
+        });
+        Counts total(size_t(kNumCtx) * 128, 0);
+        uint64_t n_esc = 0;
+        for (int th = 0; th < nt; ++th) {
+            for (size_t k = 0; k < total.size(); ++k) total[k] += counts[size_t(th)][k];
+            n_esc += esc[size_t(th)];
+        }
+        Tables tab;
+        tab.build(total);
+        double bits = 0.0;
+        for (int k = 0; k < kNumCtx; ++k)
+            for (int sy = tab.lo[k]; sy < tab.lo[k] + tab.cnt[k]; ++sy) {
+                uint64_t n = total[size_t(k) * 128 + sy];
+                if (n) bits += double(n) * (12.0 - std::log2(double(tab.f[k][sy])));
+            }
+        double ng_s = double(Rs * gpr);
+        bits += 16.0 * double(n_esc) + 8.0 * double(r) * ng_s;
+        double bits_full = bits * double(NG) / ng_s;
+        double meta = double(kHeaderBytes + pad16(2 * uint64_t(M)) + pad16(tab.serialized_bytes()) +
+                             pad16(4 * (uint64_t(T) + 1)) + uint64_t(T) * (128 - 32 + 8));
+        return meta + std::ceil(bits_full / 8.0);
+    }
+};
+
+// One tile's bytes: states, raw section, reversed word stream, zero padding.
+struct TileBytes {
+    std::vector<uint8_t> bytes;
+    bool has_esc = false;
+};
+
+void encode_tile(const std::vector<int32_t>& tq, const std::vector<uint8_t>& bq, int64_t g0, int64_t ng, int r,
+                 const Tables& tab, TileBytes& out) {
+    uint32_t x[kLanes];
+    for (auto& v : x) v = kRansL;
+    std::vector<uint16_t> words;
+    words.reserve(size_t(ng) * 4);
+    int64_t R = (ng + 31) / 32;
+    bool has_esc = false;
+    uint8_t ctx[kLanes][8], sym[kLanes][8];
+    int32_t hi[kLanes][8];
+    for (int64_t k = R - 1; k >= 0; --k) {
+        int nl = int(std::min<int64_t>(32, ng - 32 * k));
+        for (int L = 0; L < nl; ++L) {
+            int64_t g = g0 + 32 * k + L;
+            group_syms(bq[size_t(g)], &tq[size_t(g * 8)], r, ctx[L], sym[L], hi[L]);
+        }
+        for (int i = 7; i >= 0; --i) {
+            for (int L = nl - 1; L >= 0; --L)
+                if (idx_of(hi[L][i]) == kEscIdx) {
+                    words.push_back(uint16_t(int16_t(hi[L][i])));
+                    has_esc = true;
+                }
+            for (int L = nl - 1; L >= 0; --L) {
+                uint32_t f = tab.f[ctx[L][i]][sym[L][i]], c = tab.cum[ctx[L][i]][sym[L][i]];
+                uint32_t xv = x[L];
+                if (uint64_t(xv) >= (uint64_t(f) << 20)) { words.push_back(uint16_t(xv)); xv >>= 16; }
+                x[L] = (xv / f) * kProbScale + (xv % f) + c;
+            }
+        }
+    }
+    uint64_t raw = pad4(uint64_t(ng) * uint64_t(r));
+    uint64_t size = pad16(128 + raw + 2 * uint64_t(words.size()));
+    out.bytes.assign(size_t(size), 0);
+    uint8_t* p = out.bytes.data();
+    for (int L = 0; L < kLanes; ++L) wr32(p + 4 * L, x[L]);
+    if (r > 0) {
+        uint8_t* rp = p + 128;
+        const uint32_t mask = (1u << r) - 1u;
+        for (int64_t q = 0; q < ng; ++q) {
+            // 8 fields of r bits, LSB-first, starting at bit 8rq (byte rq)
+            uint64_t acc_lo = 0, acc_hi = 0;  // up to 96 bits
+            for (int i = 0; i < 8; ++i) {
+                uint32_t lo = uint32_t(tq[size_t((g0 + q) * 8 + i)]) & mask;
+                int pos = i * r;
+                if (pos < 64) {
+                    acc_lo |= uint64_t(lo) << pos;
+                    if (pos + r > 64) acc_hi |= uint64_t(lo) >> (64 - pos);
+                } else {
+                    acc_hi |= uint64_t(lo) << (pos - 64);
+                }
+            }
+            uint8_t* dst = rp + q * r;
+            for (int byte = 0; byte < r; ++byte)
+                dst[byte] = byte < 8 ? uint8_t(acc_lo >> (8 * byte)) : uint8_t(acc_hi >> (8 * (byte - 8)));
+        }
+    }
+    uint8_t* sp = p + 128 + raw;
+    size_t n = words.size();
+    for (size_t i = 0; i < n; ++i) wr16(sp + 2 * i, words[n - 1 - i]);
+    out.has_esc = has_esc;
+}
+
+}  // namespace
+}  // namespace epk
+
+using namespace epk;
+
+extern "C" void ep_options_default(ep_options* opt) {
+    if (!opt) return;
+    opt->rounds_per_tile = 16;
+    opt->sample_coords = 1u << 18;
+    opt->bisection_iters = 40;
+    opt->threads = 0;
+}
+
+extern "C" ep_status ep_compress(const void* data, int is_device, ep_dtype dt, int64_t rows, int64_t cols,
+                                 int64_t row_stride, double target_bpp, const ep_options* opt_in,
+                                 uint8_t** blob_out, size_t* blob_bytes, double* actual_bpp) {
+    clear_error();
+    if (!data || !blob_out || !blob_bytes) return fail(EP_ERR_ARG, "ep_compress: NULL argument");
+    if (!elem_bytes(int(dt))) return fail(EP_ERR_DTYPE, "ep_compress: unknown dtype %d", int(dt));
+    if (rows < 1 || cols < 8 || cols % 8 != 0 || rows > 0xFFFFFFFFll || cols > 0xFFFFFFFFll ||
+        (rows * cols) / 8 > 0xFFFFFFFFll)
+        return fail(EP_ERR_SHAPE, "ep_compress: need a 2-D tensor with rows >= 1 and cols a positive multiple of 8 (got %lld x %lld)",
+                    (long long)rows, (long long)cols);
+    if (row_stride < cols) return fail(EP_ERR_ARG, "ep_compress: row_stride %lld < cols", (long long)row_stride);
+    if (!(target_bpp >= 0.001 && target_bpp <= 11.0))
+        return fail(EP_ERR_TARGET, "ep_compress: target_bpp must be finite and in [0.001, 11]");
+    ep_options opt;
+    ep_options_default(&opt);
+    if (opt_in) opt = *opt_in;
+    if (opt.rounds_per_tile < 1 || opt.rounds_per_tile > uint32_t(kMaxG) || opt.sample_coords < 1 ||
+        opt.bisection_iters > 200)
+        return fail(EP_ERR_ARG, "ep_compress: bad options");
+    int threads = opt.threads > 0 ? opt.threads : int(std::max(1u, std::thread::hardware_concurrency()));
+
+    // Device input: one copy to the host, rows packed.
+    std::vector<uint8_t> staged;
+    const void* host = data;
+    int64_t stride = row_stride;
+    int es = elem_bytes(int(dt));
+    if (is_device) {
+        staged.resize(size_t(rows * cols * es));
+        cudaError_t e = cudaMemcpy2D(staged.data(), size_t(cols * es), data, size_t(row_stride * es), size_t(cols * es),
+                                     size_t(rows), cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return fail(EP_ERR_CUDA, "ep_compress: cudaMemcpy2D: %s", cudaGetErrorString(e));
+        host = staged.data();
+        stride = cols;
+    }
+
+    try {
+        Source src(host, int(dt), cols, stride);
+        Encoder enc(src, rows, cols, int(opt.rounds_per_tile), threads);
+        double amax = 0.0;
+        if (!enc.scales(amax)) return fail(EP_ERR_NONFINITE, "ep_compress: NaN or Inf in the input");
+
+        // Rate control: bisection on log2(alpha); the cap keeps |x| <= 2^22 so 2v is exact in binary32.
+        double lo = -12.0, hi = 15.0;
+        if (amax > 0.0) hi = std::min(hi, 22.0 - std::log2(amax));
+        if (hi < lo) hi = lo;
+        double budget = target_bpp * double(rows) * double(cols);
+        for (uint32_t it = 0; it < opt.bisection_iters; ++it) {
+            double mid = 0.5 * (lo + hi);
+            float a = float(std::exp2(mid));
+            if (8.0 * enc.estimate(a, opt.sample_coords) <= budget) lo = mid; else hi = mid;
+        }
+        float alpha = float(std::exp2(lo));
+
+        // Quantise the whole tensor once.
+        int64_t NG = enc.NG, gpr = enc.gpr;
+        std::vector<int32_t> tq(size_t(NG) * 8);
+        std::vector<uint8_t> bq(static_cast<size_t>(NG));
+        std::vector<int64_t> tabs(size_t(std::max(threads, 1)), 0);
+        parallel_for(rows, threads, [&](int64_t b, int64_t e, int th) {
+            std::vector<float> w(static_cast<size_t>(cols));
+            for (int64_t i = b; i < e; ++i) {
+                src.row(i, w.data());
+                enc.quantize_row(w.data(), i, alpha, &tq[size_t(i * gpr * 8)], &bq[size_t(i * gpr)]);
+                for (int64_t j = i * gpr * 8; j < (i + 1) * gpr * 8; ++j) {
+                    int64_t v = tq[size_t(j)], a = v >= 0 ? v : -v - 1;
+                    tabs[size_t(th)] = std::max(tabs[size_t(th)], a);
+                }
+            }
+        });
+        int64_t tmax = *std::max_element(tabs.begin(), tabs.end());
+        int r = raw_bits_for(alpha);
+        while (r < 12 && tmax >= (int64_t(1) << (15 + r))) ++r;
+        if (tmax >= (int64_t(1) << (15 + r))) return fail(EP_ERR_ARG, "ep_compress: value range too wide to code");
+
+        // Tables fitted on the whole tensor.
+        int nt = std::max(threads, 1);
+        std::vector<Counts> counts(size_t(nt), Counts(size_t(kNumCtx) * 128, 0));
+        parallel_for(NG, threads, [&](int64_t b, int64_t e, int th) {
+            Counts& c = counts[size_t(th)];
+            uint8_t ctx[8], sym[8];
+            int32_t hv[8];
+            for (int64_t g = b; g < e; ++g) {
+                group_syms(bq[size_t(g)], &tq[size_t(g * 8)], r, ctx, sym, hv);
+                for (int i = 0; i < 8; ++i) c[size_t(ctx[i]) * 128 + sym[i]]++;
+            }
+        });
+        Counts total(size_t(kNumCtx) * 128, 0);
+        for (auto& c : counts) for (size_t k = 0; k < total.size(); ++k) total[k] += c[k];
+        Tables tab;
+        tab.build(total);
+
+        // Tiles, in parallel.
+        uint32_t T = enc.T;
+        int64_t per_tile = 32 * int64_t(opt.rounds_per_tile);
+        std::vector<TileBytes> tiles(T);
+        parallel_for(T, threads, [&](int64_t b, int64_t e, int) {
+            for (int64_t j = b; j < e; ++j) {
+                int64_t g0 = j * per_tile, ng = std::min(per_tile, NG - g0);
+                encode_tile(tq, bq, g0, ng, r, tab, tiles[size_t(j)]);
+            }
+        });
+        std::vector<uint64_t> start(size_t(T) + 1, 0);
+        for (uint32_t j = 0; j < T; ++j) start[j + 1] = start[j] + tiles[j].bytes.size();
+        if (start[T] / 16 >= 0x80000000ull) return fail(EP_ERR_SHAPE, "ep_compress: payload too large");
+
+        uint64_t off_scales = kHeaderBytes;
+        uint64_t off_tables = off_scales + pad16(2 * uint64_t(rows));
+        uint64_t off_offsets = off_tables + pad16(tab.serialized_bytes());
+        uint64_t off_payload = off_offsets + pad16(4 * (uint64_t(T) + 1));
+        uint64_t total_bytes = off_payload + start[T];
+        if (off_payload > 0xFFFFFFFFull) return fail(EP_ERR_SHAPE, "ep_compress: metadata too large");
+        uint8_t* blob = static_cast<uint8_t*>(std::calloc(size_t(total_bytes), 1));
+        if (!blob) return fail(EP_ERR_NOMEM, "ep_compress: cannot allocate %llu bytes", (unsigned long long)total_bytes);
+
+        std::memcpy(blob, "EPK1", 4);
+        wr16(blob + 4, 1);
+        blob[6] = uint8_t(dt);
+        blob[7] = uint8_t(r);
+        wr32(blob + 8, uint32_t(rows));
+        wr32(blob + 12, uint32_t(cols));
+        uint32_t abits;
+        std::memcpy(&abits, &alpha, 4);
+        wr32(blob + 16, abits);
+        wr16(blob + 20, opt.rounds_per_tile);
+        blob[22] = kLanes;
+        wr32(blob + 24, T);
+        wr32(blob + 28, uint32_t(off_scales));
+        wr32(blob + 32, uint32_t(off_tables));
+        wr32(blob + 36, uint32_t(off_offsets));
+        wr32(blob + 40, uint32_t(off_payload));
+        wr64(blob + 48, total_bytes);
+        for (int64_t i = 0; i < rows; ++i) wr16(blob + off_scales + 2 * i, enc.sbits[size_t(i)]);
+        tab.serialize(blob + off_tables);
+        for (uint32_t j = 0; j < T; ++j)
+            wr32(blob + off_offsets + 4ull * j, uint32_t(start[j] / 16) | (tiles[j].has_esc ? 0x80000000u : 0u));
+        wr32(blob + off_offsets + 4ull * T, uint32_t(start[T] / 16));
+        parallel_for(T, threads, [&](int64_t b, int64_t e, int) {
+            for (int64_t j = b; j < e; ++j)
+                std::memcpy(blob + off_payload + start[size_t(j)], tiles[size_t(j)].bytes.data(), tiles[size_t(j)].bytes.size());
+        });
+        wr32(blob + 56, crc32(blob, off_payload));  // the crc field is still zero here
+
+        *blob_out = blob;
+        *blob_bytes = size_t(total_bytes);
+        if (actual_bpp) *actual_bpp = 8.0 * double(total_bytes) / (double(rows) * double(cols));
+        return EP_OK;
+    } catch (const std::bad_alloc&) {
+        return fail(EP_ERR_NOMEM, "ep_compress: out of host memory");
+    }
+}
+
+extern "C" void ep_blob_free(uint8_t* blob) { std::free(blob); }

@@ -1,0 +1,164 @@
+/*
+ * entropack.h: the C ABI of libentropack, a B200-native (sm_100a) EntroPack codec.
+ *
+ * EntroPack (arXiv 2609.34185, "EntroPack: Fast and Accurate Entropy-Coded Weight Compression at
+ * Arbitrary Bitrates") compresses a 2-D weight matrix at any target bits per parameter. It
+ * normalises each row, quantises 8-wide groups to the E8 lattice at one global resolution alpha,
+ * and rANS-codes the lattice coordinates under a conditional model. The coded coordinates sit in
+ * independently decodable tiles. (Paper page abstract; modelscope summary.)
+ *
+ * Decode is the hot path. One sm_100a kernel turns the tiles back into a dense matrix in the
+ * requested container. It runs symbol decode, the arithmetic inverse of the lattice map and the
+ * per-row rescale by s_row/alpha as one fused pass, with no symbol tensor and no codebook in
+ * between (modelscope summary). The Python API of the pages is compress(tensor, config) ->
+ * object with actual_bpp, and decompress(object) -> tensor of the same shape and dtype
+ * (README, quick-start section). This header is the same interface as plain C.
+ *
+ * Conventions:
+ *   - Every call returns an ep_status. Nothing throws. Out-parameters are written only on EP_OK.
+ *     ep_last_error() gives a thread-local message for the last failure.
+ *   - Layout: row-major, shape (rows, cols). A group is 8 consecutive columns of one row, so cols
+ *     must be a multiple of 8 (EP_ERR_SHAPE otherwise).
+ *   - Blob: a flat little-endian byte string (format "EPK1"). It describes itself fully, so it can
+ *     be stored as it is, for example as a uint8 tensor in a state_dict.
+ *   - Ownership: the library owns the blob returned by ep_compress until ep_blob_free. The caller
+ *     owns every device buffer and every stream. Decode calls are asynchronous on the caller's
+ *     stream.
+ *   - Threads: every call is thread-safe. Decode calls on different streams may run concurrently.
+ */
+#ifndef ENTROPACK_H
+#define ENTROPACK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Container dtypes, for the input of ep_compress and the output of decode. Storage bitrate is
+ * independent of the container (paper page abstract). */
+typedef enum {
+    EP_BF16 = 1,
+    EP_FP16 = 2,
+    EP_FP32 = 3,
+    EP_FP8_E4M3 = 4, /* OCP e4m3; decode saturates to +-448 */
+    EP_INT8 = 5      /* decode rounds half to even, then clamps to [-128, 127] */
+} ep_dtype;
+
+typedef enum {
+    EP_OK = 0,
+    EP_ERR_ARG = -1,       /* NULL pointer, bad option, or value range too wide to code */
+    EP_ERR_DTYPE = -2,     /* unknown container dtype */
+    EP_ERR_SHAPE = -3,     /* not 2-D with rows >= 1, cols >= 8, cols % 8 == 0, or too large */
+    EP_ERR_TARGET = -4,    /* target_bpp not finite or outside [0.001, 11] (README, Config table) */
+    EP_ERR_NONFINITE = -5, /* NaN or Inf in the input */
+    EP_ERR_CORRUPT = -6,   /* malformed blob, caught on the host */
+    EP_ERR_CUDA = -7,      /* a CUDA runtime call failed; ep_last_error() names it */
+    EP_ERR_NOMEM = -8,     /* host or device allocation failed */
+    EP_ERR_BUFFER = -9     /* destination too small or misaligned, or blob shorter than its header says */
+} ep_status;
+
+/* Bits of the device status word: set by the decode kernel, read by ep_get_device_status. */
+#define EP_DEV_CORRUPT_TILE 1u  /* a tile's final rANS states or its word count did not check out */
+#define EP_DEV_BAD_OFFSETS 2u   /* a tile offset points outside the payload */
+#define EP_DEV_BAD_TABLES 4u    /* a frequency table does not sum to 4096 */
+
+/* Encoder options. Start from ep_options_default(). */
+typedef struct {
+    uint32_t rounds_per_tile; /* G: a tile holds 32 * G * 8 coordinates. Range 1..1024, default 16 (4096) */
+    uint32_t sample_coords;   /* rate-control sample: about this many coordinates of whole rows. Default 2^18 */
+    uint32_t bisection_iters; /* bisection steps on log2(alpha). Default 40 */
+    int32_t threads;          /* encoder threads; 0 = all hardware threads */
+} ep_options;
+
+void ep_options_default(ep_options* opt);
+
+/*
+ * ep_compress: lossy compression of one 2-D tensor to a blob.
+ *
+ * data        rows x cols elements of container dtype dt; row i starts at element i*row_stride.
+ *             is_device != 0 means a CUDA device pointer, which is copied to the host once.
+ * target_bpp  target storage in bits per parameter, metadata included. Must be finite and in
+ *             [0.001, 11] (README, quick-start section and Config table). The resolution is chosen
+ *             by bisection on log2(alpha), against a storage estimate taken from a sample of rows.
+ *             The full tensor is never encoded twice (paper page abstract). Below the metadata floor
+ *             the smallest alpha is used, and *actual_bpp is reported above the target.
+ * opt         NULL means the defaults.
+ * blob        receives a malloc'd buffer, released by ep_blob_free; *blob_bytes is its size.
+ * actual_bpp  8 * blob_bytes / (rows * cols), metadata included (README, quick-start section).
+ * Errors: EP_ERR_ARG, EP_ERR_DTYPE, EP_ERR_SHAPE, EP_ERR_TARGET, EP_ERR_NONFINITE, EP_ERR_NOMEM,
+ *         EP_ERR_CUDA (device input).
+ */
+ep_status ep_compress(const void* data, int is_device, ep_dtype dt, int64_t rows, int64_t cols,
+                      int64_t row_stride, double target_bpp, const ep_options* opt, uint8_t** blob,
+                      size_t* blob_bytes, double* actual_bpp);
+
+/* Releases a blob returned by ep_compress. NULL is accepted. */
+void ep_blob_free(uint8_t* blob);
+
+/*
+ * ep_blob_info: full host-side validation of a blob, then its description.
+ * Checks the header, the section layout, the frequency tables, the tile offsets and the CRC-32 of
+ * the metadata. Every out-pointer may be NULL. Errors: EP_ERR_ARG, EP_ERR_CORRUPT.
+ */
+ep_status ep_blob_info(const uint8_t* blob, size_t blob_bytes, ep_dtype* dt, int64_t* rows, int64_t* cols,
+                       double* actual_bpp);
+
+/*
+ * ep_decompress_into: fused decode of a blob into a caller-owned device buffer. This is the hot path.
+ *
+ * host_hdr    host copy of at least the first 64 bytes of the blob (the header). The launch geometry
+ *             comes from it, with no device-to-host traffic.
+ * dev_blob    device copy of the whole blob, 16-byte aligned, blob_bytes long. Caller-owned, and
+ *             read only.
+ * dst         device buffer of rows*cols elements of the blob's container dtype, 16-byte aligned,
+ *             row-major. dst_bytes is its size. Only those rows*cols elements are written.
+ * cuda_stream cudaStream_t to launch on; NULL means the legacy default stream.
+ *
+ * The call validates the header on the host, launches one kernel and returns. It allocates nothing
+ * and does not synchronise. Host-detectable errors come back at once: EP_ERR_ARG, EP_ERR_CORRUPT
+ * (bad header), EP_ERR_BUFFER (dst too small or misaligned, blob_bytes too short), EP_ERR_CUDA
+ * (launch failure). Payload corruption is found by the kernel itself: it checks every tile's final
+ * rANS states and word count, and bounds every read to the tile. It then sets bits of the device
+ * status word (see ep_get_device_status) instead of faulting. A corrupt tile's outputs are
+ * unspecified.
+ */
+ep_status ep_decompress_into(const uint8_t* host_hdr, const void* dev_blob, size_t blob_bytes, void* dst,
+                             size_t dst_bytes, void* cuda_stream);
+
+/*
+ * ep_decompress: the same decode, into a device buffer that the call allocates with cudaMallocAsync
+ * on cuda_stream. *dst receives the pointer, and the caller frees it (cudaFreeAsync or cudaFree).
+ * Errors: as ep_decompress_into, plus EP_ERR_NOMEM.
+ */
+ep_status ep_decompress(const uint8_t* host_hdr, const void* dev_blob, size_t blob_bytes, void** dst,
+                        void* cuda_stream);
+
+/*
+ * ep_decode_coords_into: test and inspection entry. It runs the same decode, but stores the lattice
+ * coordinates instead of rescaled values: z = 2v as int32, rows*cols of them, row-major, where v is
+ * the decoded E8 point (v = u + b/2). dst_z must be 16-byte aligned, with dst_bytes >= 4*rows*cols.
+ * Errors as ep_decompress_into.
+ */
+ep_status ep_decode_coords_into(const uint8_t* host_hdr, const void* dev_blob, size_t blob_bytes,
+                                int32_t* dst_z, size_t dst_bytes, void* cuda_stream);
+
+/*
+ * ep_get_device_status: synchronises cuda_stream, then reads and clears the device status word of the
+ * current device. That word is the OR of the EP_DEV_* bits that the decode kernels set since the last
+ * read. Errors: EP_ERR_ARG, EP_ERR_CUDA.
+ */
+ep_status ep_get_device_status(void* cuda_stream, int32_t* flags);
+
+/* Static English text for a status code. */
+const char* ep_status_string(ep_status st);
+
+/* Message for the calling thread's last failed call ("" if none). Valid until that thread's next call. */
+const char* ep_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ENTROPACK_H */

@@ -1,0 +1,260 @@
+"""GPU parity: the sm_100a decode (called through the C ABI) against the CPU oracle, on the same blobs.
+
+The decode has to be bit-exact on two things:
+- the lattice coordinates (z = 2v, from ep_decode_coords_into);
+- the container values (ep_decompress_into). The reconstruction is fl32(v · fl32(s_row/α)),
+  then the container rounding. Both sides compute it in IEEE binary32, so the bar is identity
+  rather than the 1-ulp tolerance a looser reading of the rescale would need.
+
+The blobs come from the product host encoder. A separate CPU test shows that encoder is
+byte-identical to the oracle encoder.
+
+Sizes:
+- Small fuzz and edge cases, plus full-size tensors of every workload: 256², 3072² with
+  outliers, each DiT-like layer shape, the 4096² bitrate sweep, and the 8192x28672 FP8/INT8
+  codes.
+- When the oracle would be slow, it decodes a sample of tiles (tiles are independent) and
+  those are compared. The sample always includes the first tile and the ragged last one.
+"""
+import ctypes
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+import decode_ep_b200 as ep  # noqa: E402
+
+NP_BITS = {torch.bfloat16: np.uint16, torch.float16: np.uint16, torch.float32: np.float32,
+           torch.float8_e4m3fn: np.uint8, torch.int8: np.int8}
+
+
+def gpu_bits(t: torch.Tensor) -> np.ndarray:
+    t = t.cpu()
+    if t.dtype in (torch.bfloat16, torch.float16):
+        return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
+    return t.numpy()
+
+
+def status_clean():
+    assert ep.device_status() == 0
+
+
+def check_full(orc, c: ep.CompressedTensor):
+    want, zwant = orc.decompress(c.blob, with_coords=True)
+    got = gpu_bits(ep.decompress(c))
+    z = ep.decode_coords(c).cpu().numpy()
+    status_clean()
+    assert np.array_equal(z, zwant), "lattice coordinates differ"
+    if got.dtype == np.float32:
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    else:
+        assert np.array_equal(got, want)
+
+
+def check_sampled(orc, c: ep.CompressedTensor, n_tiles=24, seed=0):
+    info = orc.blob_info(c.blob)
+    T = info["num_tiles"]
+    got = gpu_bits(ep.decompress(c))
+    z = ep.decode_coords(c).cpu().numpy()
+    status_clean()
+    rng = np.random.default_rng(seed)
+    tiles = sorted(set([0, T - 1] + list(rng.integers(0, T, size=min(n_tiles, T)))))
+    want = np.zeros(c.shape, NP_BITS[c.dtype])
+    zwant = np.zeros(c.shape, np.int32)
+    mask = np.zeros(c.shape, bool)
+    per_tile = 32 * info["G"] * 8
+    flat = mask.reshape(-1)
+    for j in tiles:
+        orc.decode_tiles(c.blob, int(j), int(j) + 1, want, zwant)
+        flat[j * per_tile: (j + 1) * per_tile] = True
+    assert np.array_equal(z[mask], zwant[mask])
+    if got.dtype == np.float32:
+        assert np.array_equal(got[mask].view(np.uint32), want[mask].view(np.uint32))
+    else:
+        assert np.array_equal(got[mask], want[mask])
+    return tiles
+
+
+# ------------------------------------------------------------------- small and edge cases
+
+EDGE = [
+    ("quickstart", lambda: synth.quickstart_256(), 3.5, 16),
+    ("outliers_esc", lambda: synth.lognormal_rows_with_outliers(n=256, seed=11, outlier_frac=2e-3, outlier_mult=40.0), 4.0, 16),
+    ("fp16_raw_bits", lambda: synth.gaussian(128, 128, seed=8, container="fp16"), 9.0, 16),
+    ("ragged_1_group_tile", lambda: synth.gaussian(129, 8, seed=3, container="bf16"), 3.0, 2),
+    ("one_row", lambda: synth.gaussian(1, 8, seed=4, container="bf16"), 5.0, 1),
+    ("narrow_rows", lambda: synth.gaussian(3000, 8, seed=13, container="bf16"), 4.0, 16),
+    ("fp8", lambda: synth.fp8_codes(64, 512, seed=3), 5.0, 16),
+    ("int8", lambda: synth.int8_codes(64, 512, seed=4), 3.0, 16),
+    ("fp32_11bpp", lambda: synth.gaussian(96, 64, seed=5, container="fp32"), 11.0, 16),
+    ("all_zero", lambda: torch.zeros(64, 64, dtype=torch.bfloat16), 2.0, 16),
+    ("below_floor", lambda: synth.gaussian(64, 64, seed=3, container="bf16"), 0.001, 16),
+    ("G1024", lambda: synth.gaussian(200, 96, seed=9, container="bf16"), 2.5, 1024),
+    ("G1", lambda: synth.gaussian(40, 64, seed=10, container="fp16"), 6.0, 1),
+]
+
+
+@pytest.mark.parametrize("name,maker,target,G", EDGE, ids=[e[0] for e in EDGE])
+def test_parity_edge_cases(orc, name, maker, target, G):
+    c = ep.compress(maker(), ep.EntroPackLossyConfig(target, rounds_per_tile=G))
+    check_full(orc, c)
+
+
+def test_parity_r12_extremes(orc):
+    g = torch.Generator().manual_seed(6)
+    w = torch.randn(40, 8, generator=g)
+    c = ep.compress(w, ep.EntroPackLossyConfig(11.0, rounds_per_tile=1))
+    check_full(orc, c)
+    # int16-range escapes at r = 0 come from the oracle encoder with a forced alpha
+    w2 = torch.randn(64, 4096, generator=g) * 1e-3
+    w2[:, 7] = 1.0
+    w2[::2, 9] = -1.0
+    blob, _ = orc.compress(w2.numpy(), 3, 3.0, 16, 450.0)
+    check_full(orc, ep.CompressedTensor.from_blob(blob))
+
+
+def test_parity_random_fuzz(orc):
+    rng = np.random.default_rng(2024)
+    for it in range(30):
+        M = int(rng.integers(1, 300)); N = 8 * int(rng.integers(1, 80))
+        cont = ["bf16", "fp16", "fp32"][it % 3]
+        w = synth.gaussian(M, N, seed=1000 + it, container=cont, std=float(rng.uniform(0.001, 3)))
+        target = float(rng.uniform(0.3, 11.0))
+        G = int(rng.choice([1, 2, 3, 16, 40]))
+        check_full(orc, ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G)))
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def test_parity_quickstart_256(orc):
+    c = ep.compress(synth.quickstart_256(), 3.5)
+    assert abs(c.actual_bpp - 3.5) <= 0.05
+    out = ep.decompress(c)
+    assert out.shape == (256, 256) and out.dtype == torch.bfloat16
+    check_full(orc, c)
+
+
+def test_parity_3072_lognormal_outliers(orc):
+    c = ep.compress(synth.lognormal_rows_with_outliers(), 4.0)
+    assert c.actual_bpp <= 4.05
+    check_full(orc, c)
+
+
+@pytest.mark.parametrize("i", [0, 4, 6, 7, 272, 273, 274])
+def test_parity_dit_layer_shapes(orc, i):
+    """One layer of every distinct shape of the 276-layer DiT-like set, at 4 bpp."""
+    w = synth.dit_layer(i)
+    c = ep.compress(w, 4.0)
+    assert c.actual_bpp <= 4.05
+    if w.numel() <= 16_000_000:
+        check_full(orc, c)
+    else:
+        check_sampled(orc, c, n_tiles=200)
+
+
+def test_parity_bitrate_sweep_4096(orc):
+    base = synth.gaussian(4096, 4096, seed=2, container="fp32")
+    for cont in ("bf16", "fp16", "fp32"):
+        w = base.to(synth.CONTAINERS[cont])
+        prev = None
+        for target in (0.5, 1.0, 2.3, 3.0, 5.0, 6.0, 8.0, 11.0):
+            c = ep.compress(w, target)
+            assert abs(c.actual_bpp - target) <= 0.05
+            check_sampled(orc, c, n_tiles=12, seed=int(target * 10))
+            y = ep.decompress(c).float()
+            err = float((y - w.cuda().float()).norm() / w.cuda().float().norm())
+            if prev is not None:
+                assert err <= prev + 1e-7
+            prev = err
+
+
+@pytest.mark.parametrize("kind", ["fp8", "int8"])
+def test_parity_llm_prefill_containers(orc, kind):
+    if kind == "fp8":
+        w, target = synth.fp8_codes(), 5.0
+    else:
+        w, target = synth.int8_codes(), 3.0
+    c = ep.compress(w, target)
+    assert abs(c.actual_bpp - target) <= 0.05
+    check_sampled(orc, c, n_tiles=48)
+
+
+# -------------------------------------------------------------------- faults, made on the host
+
+def test_corrupt_payload_sets_status_not_fault(orc):
+    c = ep.compress(synth.gaussian(512, 512, seed=3, container="bf16"), 4.0)
+    off_payload = int.from_bytes(c.blob[40:44], "little")
+    rng = np.random.default_rng(1)
+    hits = 0
+    for _ in range(12):
+        bad = bytearray(c.blob)
+        for _ in range(4):
+            pos = int(rng.integers(off_payload + 128, len(bad)))
+            bad[pos] ^= 0xFF
+        cc = ep.CompressedTensor(bytes(bad), c.shape, c.dtype, c.actual_bpp)
+        ep.decompress(cc)
+        st = ep.device_status()
+        hits += bool(st & 1)
+    assert hits >= 11
+    # the GPU keeps working after corrupt input
+    check_full(orc, c)
+
+
+def test_corrupt_offsets_and_tables_flags(orc):
+    c = ep.compress(synth.gaussian(512, 512, seed=4, container="bf16"), 4.0)
+    hdr = c.blob[:64]
+    off_tables = int.from_bytes(hdr[32:36], "little")
+    off_offsets = int.from_bytes(hdr[36:40], "little")
+    bad = bytearray(c.blob)
+    bad[off_offsets + 4 * 5: off_offsets + 4 * 5 + 4] = (0x7FFFFFF0).to_bytes(4, "little")
+    ep.decompress(ep.CompressedTensor(bytes(bad), c.shape, c.dtype, 0))
+    assert ep.device_status() & 2
+    bad = bytearray(c.blob)
+    bad[off_tables + 17 + 3] = 200     # cnt beyond the alphabet
+    bad[off_tables + 40] ^= 0x5A       # and a damaged frequency
+    ep.decompress(ep.CompressedTensor(bytes(bad), c.shape, c.dtype, 0))
+    assert ep.device_status() != 0
+    check_full(orc, c)
+
+
+def test_host_side_errors():
+    c = ep.compress(synth.quickstart_256(), 3.5)
+    out = torch.empty(255, 256, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ep.EntroPackError) as e:
+        ep.decompress_into(c, out)
+    assert e.value.status == -9
+    with pytest.raises(ep.EntroPackError):
+        ep.decompress_into(c, torch.empty(256, 256, dtype=torch.float16, device="cuda"))
+
+
+def test_streams_and_allocating_entry(orc):
+    c = ep.compress(synth.dit_layer(9, shape=(512, 1024)), 4.0)
+    s = torch.cuda.Stream()
+    out = torch.empty(c.shape, dtype=c.dtype, device="cuda")
+    with torch.cuda.stream(s):
+        ep.decompress_into(c, out, stream=s)
+    s.synchronize()
+    ref = ep.decompress(c)
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    # ep_decompress allocates the output itself (cudaMallocAsync on the stream)
+    from cuda.bindings import runtime as rt
+    L = ep.lib()
+    ptr = ctypes.c_void_p()
+    dblob = c.device_blob()
+    st = L.ep_decompress(c.header, dblob.data_ptr(), len(c.blob), ctypes.byref(ptr), None)
+    assert st == 0 and ptr.value
+    host = np.empty(c.shape, np.uint16)
+    err, = rt.cudaMemcpy(host.ctypes.data, ptr.value, host.nbytes, rt.cudaMemcpyKind.cudaMemcpyDeviceToHost)
+    assert err == rt.cudaError_t.cudaSuccess
+    assert rt.cudaFree(ptr.value)[0] == rt.cudaError_t.cudaSuccess
+    assert np.array_equal(host, gpu_bits(ref))

@@ -1,0 +1,137 @@
+"""CPU-only checks of the product library (no GPU calls).
+
+Covered here:
+- libentropack.so loads and exports every function that include/entropack.h declares;
+- the host encoder (product) and the oracle encoder are independent implementations of the same
+  format, and they produce byte-identical blobs;
+- the host validator accepts every good blob and rejects corrupted ones;
+- the C ABI returns the documented status codes for bad input (README, Config table: the target
+  range; 2-D only).
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def ep():
+    import decode_ep_b200 as m
+    m.lib()
+    return m
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "entropack.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ep_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol(ep):
+    names = declared_functions()
+    assert len(names) >= 10
+    L = ctypes.CDLL(ep.lib()._name)
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/entropack.h but not exported"
+
+
+def test_library_is_sm100a_build(ep):
+    import decode_ep_b200.build as b
+    assert "arch=compute_100a,code=sm_100a" in " ".join(b.ARCH)
+    assert os.path.dirname(ep.lib()._name) == os.path.join(ROOT, "decode_ep_b200")
+
+
+CASES = [
+    ("quickstart", lambda: synth.quickstart_256(), 3.5, 16),
+    ("outliers", lambda: synth.lognormal_rows_with_outliers(n=256, seed=11, outlier_frac=2e-3, outlier_mult=40.0), 4.0, 16),
+    ("fp16_raw_bits", lambda: synth.gaussian(128, 128, seed=8, container="fp16"), 9.0, 16),
+    ("ragged_1_group_tile", lambda: synth.gaussian(129, 8, seed=3, container="bf16"), 3.0, 2),
+    ("fp8", lambda: synth.fp8_codes(64, 512, seed=3), 5.0, 16),
+    ("int8", lambda: synth.int8_codes(64, 512, seed=4), 3.0, 16),
+    ("fp32_11bpp", lambda: synth.gaussian(96, 64, seed=5, container="fp32"), 11.0, 16),
+    ("all_zero", lambda: torch.zeros(64, 64, dtype=torch.bfloat16), 2.0, 16),
+    ("below_floor", lambda: synth.gaussian(64, 64, seed=3, container="bf16"), 0.001, 16),
+    ("dit_like", lambda: synth.dit_layer(3, shape=(512, 256)), 4.0, 16),
+    ("G1024", lambda: synth.gaussian(200, 96, seed=9, container="bf16"), 2.5, 1024),
+]
+
+
+@pytest.mark.parametrize("name,maker,target,G", CASES, ids=[c[0] for c in CASES])
+def test_host_encoder_matches_oracle_bytes(ep, orc, name, maker, target, G):
+    w = maker()
+    ob, obpp = orc.compress(synth.container_bits(w), synth.dtype_code(w), target, G)
+    c = ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G))
+    assert c.blob == ob
+    assert c.actual_bpp == pytest.approx(obpp)
+    info = ep.blob_info(c.blob)
+    assert (info["rows"], info["cols"]) == tuple(w.shape)
+    assert orc.blob_info(c.blob)["num_tiles"] >= 1
+
+
+def test_host_encoder_thread_count_does_not_change_the_blob(ep):
+    w = synth.dit_layer(5, shape=(300, 512))
+    blobs = {ep.compress(w, ep.EntroPackLossyConfig(3.7, threads=t)).blob for t in (1, 3, 8)}
+    assert len(blobs) == 1
+
+
+def test_strided_input(ep):
+    base = synth.gaussian(64, 96, seed=12, container="bf16")
+    view = base[:, 16:80]
+    assert view.stride(0) == 96
+    a = ep.compress(view, 3.0).blob
+    b = ep.compress(view.contiguous(), 3.0).blob
+    assert a == b
+
+
+def test_status_codes(ep):
+    w = synth.gaussian(16, 16, seed=1, container="bf16")
+    for bad in (0.0009, 11.0001, float("nan"), float("inf")):
+        with pytest.raises(ep.EntroPackError) as e:
+            ep.compress(w, bad)
+        assert e.value.status == -4
+    with pytest.raises(ep.EntroPackError) as e:
+        ep.compress(torch.zeros(4, 12, dtype=torch.bfloat16), 3.0)
+    assert e.value.status == -3
+    with pytest.raises(ep.EntroPackError) as e:
+        ep.compress(torch.zeros(4, 4, 8, dtype=torch.bfloat16), 3.0)
+    assert e.value.status == -3
+    x = torch.zeros(8, 16)
+    x[3, 3] = float("inf")
+    with pytest.raises(ep.EntroPackError) as e:
+        ep.compress(x, 3.0)
+    assert e.value.status == -5
+    L = ep.lib()
+    assert L.ep_status_string(-6) == b"corrupt blob"
+
+
+def test_validator_rejects_corruption(ep):
+    c = ep.compress(synth.quickstart_256(), 3.5)
+    ep.blob_info(c.blob)
+    bad = bytearray(c.blob); bad[100] ^= 4          # scale byte: CRC
+    with pytest.raises(ep.EntroPackError) as e:
+        ep.blob_info(bytes(bad))
+    assert e.value.status == -6
+    with pytest.raises(ep.EntroPackError):
+        ep.blob_info(c.blob[:-16])
+    with pytest.raises(ep.EntroPackError):
+        ep.blob_info(b"EPK1" + b"\0" * 60)
+
+
+def test_decode_rejects_bad_arguments_without_launching(ep):
+    """Host-side checks of ep_decompress_into run before any CUDA call."""
+    c = ep.compress(synth.quickstart_256(), 3.5)
+    L = ep.lib()
+    hdr = c.header
+    fake_dev = 0x10000  # never dereferenced: every case fails on the host first
+    assert L.ep_decompress_into(hdr, fake_dev, len(c.blob) - 16, fake_dev, 1 << 20, None) == -9  # blob size
+    assert L.ep_decompress_into(hdr, fake_dev + 8, len(c.blob), fake_dev, 1 << 20, None) == -9  # alignment
+    assert L.ep_decompress_into(hdr, fake_dev, len(c.blob), fake_dev, 1000, None) == -9         # dst too small
+    assert L.ep_decompress_into(b"EPK2" + hdr[4:], fake_dev, len(c.blob), fake_dev, 1 << 20, None) == -6
+    assert L.ep_decompress_into(None, fake_dev, len(c.blob), fake_dev, 1 << 20, None) == -1
