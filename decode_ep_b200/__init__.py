@@ -23,8 +23,8 @@ import torch
 
 from . import build as _build
 
-__all__ = ["EntroPackLossyConfig", "CompressedTensor", "EntroPackError", "compress", "decompress",
-           "decompress_into", "decode_coords", "device_status", "blob_info", "lib"]
+__all__ = ["EntroPackLossyConfig", "CompressedTensor", "EntroPackError", "LayerBatch", "compress", "decompress",
+           "decompress_into", "decompress_many", "decode_coords", "device_status", "blob_info", "lib"]
 
 EP_BF16, EP_FP16, EP_FP32, EP_FP8_E4M3, EP_INT8 = 1, 2, 3, 4, 5
 _TORCH_TO_EP = {torch.bfloat16: EP_BF16, torch.float16: EP_FP16, torch.float32: EP_FP32,
@@ -66,12 +66,15 @@ def lib() -> ctypes.CDLL:
         for name in ("ep_decompress_into", "ep_decode_coords_into"):
             getattr(L, name).argtypes = [c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p, c.c_size_t, c.c_void_p]
         L.ep_decompress.argtypes = [c.c_void_p, c.c_void_p, c.c_size_t, c.POINTER(c.c_void_p), c.c_void_p]
+        L.ep_decompress_many.argtypes = [c.c_int, c.POINTER(c.c_char_p), c.POINTER(c.c_void_p),
+                                         c.POINTER(c.c_size_t), c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
+                                         c.c_void_p]
         L.ep_get_device_status.argtypes = [c.c_void_p, c.POINTER(c.c_int32)]
         L.ep_status_string.restype = c.c_char_p
         L.ep_status_string.argtypes = [c.c_int]
         L.ep_last_error.restype = c.c_char_p
         for name in ("ep_compress", "ep_blob_info", "ep_decompress_into", "ep_decode_coords_into", "ep_decompress",
-                     "ep_get_device_status"):
+                     "ep_get_device_status", "ep_decompress_many"):
             getattr(L, name).restype = c.c_int
         _lib = L
     return _lib
@@ -191,6 +194,38 @@ def decompress_into(compressed: CompressedTensor, out: torch.Tensor, stream=None
     _check(lib().ep_decompress_into(compressed.header, dblob.data_ptr(), len(compressed.blob), out.data_ptr(),
                                     out.numel() * out.element_size(), _stream_ptr(stream)), "decompress_into")
     return out
+
+
+class LayerBatch:
+    """A fixed list of (compressed tensor, output tensor) pairs, marshalled once. Each call to
+    ``run()`` is one ``ep_decompress_many`` call: the whole sequence of fused decodes, chained with
+    programmatic dependent launch, on one stream."""
+
+    def __init__(self, pairs, stream=None):
+        c = ctypes
+        self.pairs = list(pairs)
+        n = len(self.pairs)
+        for comp, out in self.pairs:
+            if not out.is_cuda or not out.is_contiguous() or out.dtype != comp.dtype:
+                raise EntroPackError(-9, "LayerBatch: outputs must be contiguous CUDA tensors of the blobs' dtypes")
+        self._keep = [comp.device_blob(out.device) for comp, out in self.pairs]
+        self.n = n
+        self.hdrs = (c.c_char_p * n)(*[comp.header for comp, _ in self.pairs])
+        self.blobs = (c.c_void_p * n)(*[d.data_ptr() for d in self._keep])
+        self.sizes = (c.c_size_t * n)(*[len(comp.blob) for comp, _ in self.pairs])
+        self.dsts = (c.c_void_p * n)(*[out.data_ptr() for _, out in self.pairs])
+        self.dst_sizes = (c.c_size_t * n)(*[out.numel() * out.element_size() for _, out in self.pairs])
+        self.stream = stream
+
+    def run(self, stream=None) -> None:
+        s = _stream_ptr(stream if stream is not None else self.stream)
+        _check(lib().ep_decompress_many(self.n, self.hdrs, self.blobs, self.sizes, self.dsts, self.dst_sizes, s),
+               "decompress_many")
+
+
+def decompress_many(pairs, stream=None) -> None:
+    """Decodes each compressed tensor into its output tensor, in order, with one C call."""
+    LayerBatch(pairs, stream).run()
 
 
 def decompress(compressed: CompressedTensor, config=None, device=None, stream=None) -> torch.Tensor:

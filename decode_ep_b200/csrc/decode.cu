@@ -3,17 +3,23 @@
 // arithmetic inverse of the lattice map and the per-row rescale are fused with the symbol decode
 // (modelscope paper page, summary; paper page abstract).
 //
-// Kernel shape: a persistent grid with one 1024-thread CTA per SM.
-//   - Each CTA first expands the blob's 17 twelve-bit frequency tables into shared memory. Every
-//     context gets a block: a 4096-entry slot -> symbol byte table, then one 16-byte record per
-//     symbol {f, -cum, next context block, value}. The next-context pointer and the reconstructed
-//     value are baked into the record. The hot loop therefore spends two shared loads per
-//     coordinate and does no extra arithmetic for the context chain.
-//   - Each warp then decodes whole tiles. Lane L owns the groups 32k + L of the tile. After every
-//     symbol step the lanes that must refill take the next 16-bit words of the shared stream in
-//     lane order, found with a warp ballot and a popcount prefix.
-//   - Each lane reconstructs its 8 values and writes them with one 16-byte store (BF16/FP16), so a
-//     warp writes 512 contiguous bytes.
+// Kernel shape: a persistent grid with one 1024-thread CTA per SM (32 warps).
+//   - Tables. Each CTA first expands the blob's 17 twelve-bit frequency tables into shared
+//     memory. Every context gets a block: a 4096-entry slot -> symbol byte table, then one
+//     16-byte record per symbol {f, -cum, next context block, value}. The next-context pointer
+//     and the reconstructed value are baked into the record, so the hot loop spends two shared
+//     loads per coordinate and does no extra arithmetic for the context chain.
+//   - Tiles. Each warp decodes whole tiles. Lane L owns the groups 32k + L of the tile. After
+//     every symbol step, the lanes that must refill take the next 16-bit words of the shared
+//     stream in lane order, found with a warp ballot and a popcount prefix.
+//   - Stream staging. The words come from a 2 KB per-warp ring in shared memory. Asynchronous
+//     16-byte copies (cp.async, one 512-byte chunk per round, up to 3 chunks ahead) fill it, so
+//     no refill waits on DRAM.
+//   - Stores. Each lane reconstructs its 8 values and writes them with one 16-byte store
+//     (BF16/FP16), so a warp writes 512 contiguous bytes.
+//   - Layer sequences. Successive launches are chained with programmatic dependent launch. A
+//     kernel builds its tables and fills its first rings while the previous kernel drains, and it
+//     waits on the grid dependency only before its first store.
 // The loop is bound by integer issue and shared-memory bandwidth, not by tensor cores: decode has
 // no dense contraction.
 #include <cuda_bf16.h>
@@ -32,16 +38,34 @@ namespace dev {
 
 constexpr int kWarps = 32;
 constexpr int kThreads = kWarps * 32;
+constexpr uint32_t kFullMask = 0xFFFFFFFFu;
+
+// Tables: per context a 4096-byte slot -> symbol table, then 16-byte records.
 constexpr uint32_t kLutBytes = 4096;
 constexpr uint32_t kStartBlock = kLutBytes + 128 * 16;  // START: 128 symbols (coset bit x 64)
 constexpr uint32_t kCtxBlock = kLutBytes + 64 * 16;     // other contexts: 64 symbols
 constexpr uint32_t kPos7Shift = 8 * kCtxBlock;          // contexts 9..16 sit 8 blocks after 1..8
 constexpr uint32_t kTablesBytes = kStartBlock + 16 * kCtxBlock;
-constexpr uint32_t kCumBytes = (kNumCtx * 129 * 4 + 15) & ~15u;
-constexpr uint32_t kSmemBytes = kTablesBytes + kCumBytes;
-constexpr uint32_t kFullMask = 0xFFFFFFFFu;
-// Words one round can take in the table-only fast path: 8 positions x 32 lanes, one refill each.
-constexpr uint32_t kFastRoundWords = 8 * 32;
+
+// Per-warp stream rings.
+constexpr uint32_t kRingBytes = 2048;
+constexpr uint32_t kChunkBytes = 512;  // one 16-byte copy per lane
+constexpr uint32_t kRingChunks = kRingBytes / kChunkBytes;
+constexpr uint32_t kRingsBytes = kWarps * kRingBytes;
+
+// Dynamic shared memory: [alignment pad up to 2 KB][rings][tables]. The table-build scratch lives in
+// the ring area, which is free until decoding starts.
+constexpr uint32_t kSmemBytes = kRingBytes + kRingsBytes + kTablesBytes;
+constexpr uint32_t kScratchCum = 0;                               // u32 [17][129]
+constexpr uint32_t kScratchBytes = kScratchCum + 8784;            // table bytes, <= 2048
+constexpr uint32_t kScratchTableCap = 2048;
+constexpr uint32_t kScratchBucket = kScratchBytes + kScratchTableCap;  // u8 [17][64]
+constexpr uint32_t kScratchMeta = kScratchBucket + 17 * 64;       // u32 lo, cnt, bit [17] each
+static_assert(kScratchMeta + 3 * 17 * 4 <= kRingsBytes, "table-build scratch must fit the ring area");
+
+// Words one round can take: 8 positions x 32 lanes, one refill each, plus as many ESC words.
+constexpr uint32_t kRoundWords = 8 * 32;
+constexpr uint32_t kRoundWordsEsc = 2 * kRoundWords;
 
 __host__ __device__ constexpr uint32_t block_of(int c) {
     return c == 0 ? 0u : kStartBlock + uint32_t(c - 1) * kCtxBlock;
@@ -62,27 +86,59 @@ struct Params {
 
 __device__ int g_status;
 
+// ------------------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint32_t ld_shared_u16(uint32_t addr) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+// 16-byte asynchronous copy global -> shared; bytes past `src_bytes` (0..16) are zero-filled and
+// not read.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // ------------------------------------------------------------------------- table expansion
 
-__device__ void build_tables(const Params& p, uint8_t* smem) {
-    __shared__ uint32_t s_lo[kNumCtx], s_cnt[kNumCtx], s_bit[kNumCtx];
-    uint32_t* cum = reinterpret_cast<uint32_t*>(smem + kTablesBytes);  // [17][129]
-    const uint8_t* tb = p.blob + p.off_tables;
+__device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch) {
+    uint32_t* cum = reinterpret_cast<uint32_t*>(scratch + kScratchCum);  // [17][129]
+    uint8_t* tbytes = scratch + kScratchBytes;
+    uint8_t* bucket = scratch + kScratchBucket;                          // symbol at slot 64k
+    uint32_t* s_lo = reinterpret_cast<uint32_t*>(scratch + kScratchMeta);
+    uint32_t* s_cnt = s_lo + kNumCtx;
+    uint32_t* s_bit = s_cnt + kNumCtx;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    if (tid < kNumCtx) {
-        s_lo[tid] = tb[tid];
-        s_cnt[tid] = tb[kNumCtx + tid];
-    }
+    // Stage the serialised tables (about 2 KB at most) with one coalesced pass.
+    const uint32_t tlen = p.tables_len < kScratchTableCap ? p.tables_len : kScratchTableCap;
+    const uint8_t* tb = p.blob + p.off_tables;
+    for (uint32_t i = tid; i < tlen; i += kThreads) tbytes[i] = __ldg(tb + i);
+    for (uint32_t i = tid; i < kNumCtx * 64; i += kThreads) bucket[i] = 0;
     __syncthreads();
-    if (tid == 0) {
-        uint32_t acc = 0;
-        for (int c = 0; c < kNumCtx; ++c) { s_bit[c] = acc; acc += 12 * s_cnt[c]; }
+    if (warp == 0) {
+        uint32_t lo = 0, cnt = 0;
+        if (lane < kNumCtx) { lo = tbytes[lane]; cnt = tbytes[kNumCtx + lane]; }
+        uint32_t bits = 12 * cnt, incl = bits;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            uint32_t v = __shfl_up_sync(kFullMask, incl, d);
+            if (lane >= d) incl += v;
+        }
+        if (lane < kNumCtx) { s_lo[lane] = lo; s_cnt[lane] = cnt; s_bit[lane] = incl - bits; }
     }
     __syncthreads();
 
     // Frequencies, indexed by symbol (zero outside [lo, lo + cnt)).
-    const uint32_t bits_len = p.tables_len > 2 * kNumCtx ? p.tables_len - 2 * kNumCtx : 0;
+    const uint32_t bits_len = tlen > 2 * kNumCtx ? tlen - 2 * kNumCtx : 0;
     for (int i = tid; i < kNumCtx * 128; i += kThreads) {
         int c = i >> 7, s = i & 127, A = c == 0 ? 128 : 64;
         uint32_t lo = s_lo[c], cnt = s_cnt[c], f = 0;
@@ -91,8 +147,9 @@ __device__ void build_tables(const Params& p, uint8_t* smem) {
                 f = kProbScale;
             } else {
                 uint32_t bit = s_bit[c] + 12 * (uint32_t(s) - lo), byte = bit >> 3, w = 0;
+#pragma unroll
                 for (int k = 0; k < 3; ++k)
-                    if (byte + k < bits_len) w |= uint32_t(tb[2 * kNumCtx + byte + k]) << (8 * k);
+                    if (byte + k < bits_len) w |= uint32_t(tbytes[2 * kNumCtx + byte + k]) << (8 * k);
                 f = (w >> (bit & 7)) & 0xFFFu;
             }
         }
@@ -124,8 +181,9 @@ __device__ void build_tables(const Params& p, uint8_t* smem) {
     }
     __syncthreads();
 
-    // Records: {f, -cum, next block, value}. The value is v = hi + b/2 for positions 0..6 and
-    // 2h + b/2 for position 7 (u7 = 2h + parity is completed in the decode loop).
+    // Records {f, -cum, next block, value}, and the symbol at every 64th slot. The value is
+    // v = hi + b/2 for positions 0..6 and 2h + b/2 for position 7 (u7 = 2h + parity is completed in
+    // the decode loop).
     for (int i = tid; i < kNumCtx * 128; i += kThreads) {
         int c = i >> 7, s = i & 127, A = c == 0 ? 128 : 64;
         if (s >= A) continue;
@@ -143,31 +201,34 @@ __device__ void build_tables(const Params& p, uint8_t* smem) {
         } else {
             val = float(2 * hi) + 0.5f * float(b);
         }
-        uint4 rec = make_uint4(f, 0u - cc[s], next, __float_as_uint(val));
-        *reinterpret_cast<uint4*>(smem + block_of(c) + kLutBytes + 16 * s) = rec;
+        *reinterpret_cast<uint4*>(tables + block_of(c) + kLutBytes + 16 * s) =
+            make_uint4(f, 0u - cc[s], next, __float_as_uint(val));
+        if (f) {
+            uint32_t k0 = (cc[s] + 63) >> 6, k1 = (cc[s] + f + 63) >> 6;
+            for (uint32_t k = k0; k < k1 && k < 64; ++k) bucket[c * 64 + k] = uint8_t(s);
+        }
     }
+    __syncthreads();
 
-    // Slot -> symbol bytes, 16 slots per thread: the largest s with cum[s] <= slot (symbols with f = 0
-    // share their successor's cum and are skipped).
+    // Slot -> symbol bytes, 16 slots per thread. Start from the symbol of the chunk's 64-slot bucket
+    // and step past boundaries; zero-frequency symbols share their successor's cum and are skipped.
     for (int i = tid; i < kNumCtx * 256; i += kThreads) {
         int c = i >> 8, A = c == 0 ? 128 : 64;
         uint32_t slot0 = uint32_t(i & 255) * 16;
         const uint32_t* cc = cum + c * 129;
-        int lo = 0, hi = A - 1;
-        while (lo < hi) {
-            int mid = (lo + hi + 1) >> 1;
-            if (cc[mid] <= slot0) lo = mid; else hi = mid - 1;
-        }
-        int s = lo;
+        int s = bucket[c * 64 + (slot0 >> 6)];
+        s = s < A ? s : A - 1;
+        uint32_t nb = cc[s + 1];
         uint32_t out[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             uint32_t slot = slot0 + j;
-            while (s + 1 < A && cc[s + 1] <= slot) ++s;
+            while (slot >= nb && s + 1 < A) { ++s; nb = cc[s + 1]; }
             out[j >> 2] |= uint32_t(s) << (8 * (j & 3));
         }
-        *reinterpret_cast<uint4*>(smem + block_of(c) + slot0) = make_uint4(out[0], out[1], out[2], out[3]);
+        *reinterpret_cast<uint4*>(tables + block_of(c) + slot0) = make_uint4(out[0], out[1], out[2], out[3]);
     }
+    __syncthreads();
 }
 
 // ------------------------------------------------------------------------------- stores
@@ -217,8 +278,9 @@ __device__ __forceinline__ void store_group(void* dst, uint32_t g, const float* 
     }
 }
 
-// Per-lane state of the row of the current group; c_row = fl32(s_row / alpha) is recomputed only
-// when the row changes.
+// ------------------------------------------------------------------------- per-warp state
+
+// Row of the lane's current group. c_row = fl32(s_row / alpha) is recomputed only when the row changes.
 struct RowCursor {
     uint32_t row, col, cached_row;
     float c_row;
@@ -237,118 +299,123 @@ struct RowCursor {
     }
 };
 
+// The tile's u16 word stream, read either from the warp's shared ring (all but ragged rounds) or
+// straight from global memory with a bounds check. `pb` is the byte position of the next word in
+// ring coordinates (lead + 2 * words consumed).
+struct RingWords {
+    uint32_t base;  // shared address of the warp's ring, kRingBytes-aligned
+    __device__ __forceinline__ uint32_t at(uint32_t pb) const { return ld_shared_u16(((pb) & (kRingBytes - 1)) | base); }
+};
+struct GlobalWords {
+    const uint8_t* ring0;  // global address that ring coordinate 0 mirrors
+    uint32_t lo, hi;       // valid ring coordinates of the stream: [lo, hi)
+    __device__ __forceinline__ uint32_t at(uint32_t pb) const {
+        return (pb >= lo && pb + 2 <= hi) ? uint32_t(__ldg(reinterpret_cast<const uint16_t*>(ring0 + pb))) : 0u;
+    }
+};
+
+struct TileState {
+    uint32_t x;   // rANS state of this lane
+    uint32_t pb;  // ring coordinate of the next stream word
+};
+
 // ------------------------------------------------------------------------------ one round
 
-// Fast round: all 32 lanes hold a group, the tile has no ESC, r = 0, and a full round of reads stays
-// inside the payload, so no read needs a bounds check.
-template <int MODE>
-__device__ __forceinline__ void round_fast(const Params& p, const uint8_t* smem, const uint16_t* words,
-                                           const uint16_t* scales, uint32_t& x, uint32_t& pos, uint32_t g,
-                                           uint32_t lt_mask, RowCursor& rc) {
+// Decodes one round (8 coordinates per lane). ESC: the tile holds escapes (check every position).
+// RAW: r > 0 raw low bits. PARTIAL: some lanes hold no group.
+template <int MODE, bool ESC, bool RAW, bool PARTIAL, class Words>
+__device__ __forceinline__ void decode_round(const Params& p, const uint8_t* tables, const Words& words,
+                                             const uint8_t* rawsec, uint32_t raw_avail, const uint16_t* scales,
+                                             TileState& st, uint32_t q, bool active, uint32_t g, uint32_t lt_mask,
+                                             RowCursor& rc) {
+    constexpr bool SIMPLE = !ESC && !RAW;  // values straight from the records
     float v[8];
-    uint32_t B = 0, par = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        if (i == 7) B += kPos7Shift;
-        const uint32_t slot = x & (kProbScale - 1);
-        const uint32_t sym = smem[B + slot];
-        const uint4 rec = *reinterpret_cast<const uint4*>(smem + B + kLutBytes + 16 * sym);
-        x = rec.x * (x >> kProbBits) + slot + rec.y;  // f * (x >> 12) + slot - cum
-        const bool need = x < kRansL;
-        const uint32_t m = __ballot_sync(kFullMask, need);
-        if (need) x = (x << 16) | uint32_t(__ldg(words + pos + __popc(m & lt_mask)));
-        pos += __popc(m);
-        if (i < 7) par ^= sym;
-        v[i] = __uint_as_float(rec.w);
-        B = rec.z;
-    }
-    // u_i = idx_i - 31 flips parity against idx_i; seven flips make pi = 1 when the idx parity is even.
-    if (!(par & 1u)) v[7] += 1.0f;
-    const float c = rc.scale(p, scales);
-    float y[8];
-    int32_t z[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        y[i] = __fmul_rn(v[i], c);
-        if constexpr (MODE == kCoords) z[i] = __float2int_rn(v[i] * 2.0f);
-    }
-    store_group<MODE>(p.dst, g, y, z);
-}
-
-// General round: partial rounds, ESC words, raw low bits and bounded stream reads.
-template <int MODE>
-__device__ __noinline__ void round_general(const Params& p, const uint8_t* smem, const uint16_t* words,
-                                           uint32_t nwords, const uint8_t* rawsec, uint32_t raw_avail,
-                                           const uint16_t* scales, uint32_t& x, uint32_t& pos, uint32_t q,
-                                           bool active, uint32_t g, uint32_t lt_mask, RowCursor& rc) {
-    const int r = p.r;
-    // The group's 8r raw bits start at byte q*r of the raw section; load a 96-bit window.
-    uint32_t win0 = 0, win1 = 0, win2 = 0;
-    if (r > 0 && active) {
-        uint32_t o = q * uint32_t(r), a = o & ~3u, sh = (o & 3u) * 8;
-        uint32_t w[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            w[j] = (a + 4 * j + 4 <= raw_avail) ? __ldg(reinterpret_cast<const uint32_t*>(rawsec + a) + j) : 0u;
-        win0 = __funnelshift_r(w[0], w[1], sh);
-        win1 = __funnelshift_r(w[1], w[2], sh);
-        win2 = __funnelshift_r(w[2], w[3], sh);
-    }
-    const uint32_t rmask = (1u << r) - 1u;
-    uint32_t B = 0, b = 0;
     int32_t t[8];
+    uint32_t B = 0, par = 0, b = 0;
+    uint32_t win0 = 0, win1 = 0, win2 = 0;
+    if constexpr (RAW) {
+        // The group's 8r raw bits start at byte q*r of the raw section; load a 96-bit window.
+        if (active) {
+            const int r = p.r;
+            uint32_t o = q * uint32_t(r), a = o & ~3u, sh = (o & 3u) * 8;
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                w[j] = (a + 4 * j + 4 <= raw_avail) ? __ldg(reinterpret_cast<const uint32_t*>(rawsec + a) + j) : 0u;
+            win0 = __funnelshift_r(w[0], w[1], sh);
+            win1 = __funnelshift_r(w[1], w[2], sh);
+            win2 = __funnelshift_r(w[2], w[3], sh);
+        }
+    }
+    uint32_t x = st.x, pb = st.pb;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         if (i == 7) B += kPos7Shift;
         uint32_t sym = 0;
         uint4 rec = make_uint4(0, 0, 0, 0);
-        if (active) {
+        if (!PARTIAL || active) {
             const uint32_t slot = x & (kProbScale - 1);
-            sym = smem[B + slot];
-            rec = *reinterpret_cast<const uint4*>(smem + B + kLutBytes + 16 * sym);
-            x = rec.x * (x >> kProbBits) + slot + rec.y;
+            sym = tables[B + slot];
+            rec = *reinterpret_cast<const uint4*>(tables + B + kLutBytes + 16 * sym);
+            x = rec.x * (x >> kProbBits) + slot + rec.y;  // f * (x >> 12) + slot - cum
         }
-        const bool need = active && x < kRansL;
+        const bool need = (!PARTIAL || active) && x < kRansL;
         const uint32_t m = __ballot_sync(kFullMask, need);
-        if (need) {
-            uint32_t wi = pos + __popc(m & lt_mask);
-            x = (x << 16) | (wi < nwords ? uint32_t(__ldg(words + wi)) : 0u);
-        }
-        pos += __popc(m);
-        const uint32_t idx = sym & 63u;
-        int32_t hi = int32_t(idx) - 31;
-        const bool esc = active && idx == uint32_t(kEscIdx);
-        const uint32_t me = __ballot_sync(kFullMask, esc);
-        if (me) {
-            if (esc) {
-                uint32_t wi = pos + __popc(me & lt_mask);
-                hi = int32_t(int16_t(wi < nwords ? __ldg(words + wi) : 0));
+        const uint32_t w = words.at(pb + 2 * __popc(m & lt_mask));
+        x = need ? (x << 16) | w : x;
+        pb += 2 * __popc(m);
+        if constexpr (SIMPLE) {
+            if (i < 7) par ^= sym;
+            v[i] = __uint_as_float(rec.w);
+        } else {
+            const uint32_t idx = sym & 63u;
+            int32_t hi = int32_t(idx) - 31;
+            if constexpr (ESC) {
+                const bool esc = (!PARTIAL || active) && idx == uint32_t(kEscIdx);
+                const uint32_t me = __ballot_sync(kFullMask, esc);
+                if (me) {
+                    const uint32_t e = words.at(pb + 2 * __popc(me & lt_mask));
+                    if (esc) hi = int32_t(int16_t(e));
+                    pb += 2 * __popc(me);
+                }
             }
-            pos += __popc(me);
+            if (i == 0) b = sym >> 6;
+            int32_t lo = 0;
+            if constexpr (RAW) {
+                const uint32_t bp = uint32_t(i) * uint32_t(p.r), sel = bp >> 5, sh = bp & 31;
+                const uint32_t wa = sel == 0 ? win0 : (sel == 1 ? win1 : win2);
+                const uint32_t wb = sel == 0 ? win1 : win2;
+                lo = int32_t(__funnelshift_r(wa, wb, sh) & ((1u << p.r) - 1u));
+            }
+            t[i] = hi * (1 << p.r) + lo;
         }
-        if (i == 0) b = sym >> 6;
-        int32_t lo = 0;
-        if (r > 0) {
-            uint32_t bp = uint32_t(i) * uint32_t(r), sel = bp >> 5, sh = bp & 31;
-            uint32_t wa = sel == 0 ? win0 : (sel == 1 ? win1 : win2);
-            uint32_t wb = sel == 0 ? win1 : win2;
-            lo = int32_t(__funnelshift_r(wa, wb, sh) & rmask);
-        }
-        t[i] = hi * (1 << r) + lo;
         B = rec.z;
     }
-    if (!active) return;
-    int32_t s7 = 0;
-#pragma unroll
-    for (int i = 0; i < 7; ++i) s7 += t[i];
+    st.x = x;
+    st.pb = pb;
+    if (PARTIAL && !active) return;
+
     const float c = rc.scale(p, scales);
     float y[8];
     int32_t z[8];
+    if constexpr (SIMPLE) {
+        // u_i = idx_i - 31 flips parity against idx_i; seven flips make pi = 1 when the idx parity is even.
+        if (!(par & 1u)) v[7] += 1.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        int32_t u = i < 7 ? t[i] : 2 * t[7] + (s7 & 1);
-        z[i] = 2 * u + int32_t(b);
-        y[i] = __fmul_rn(__int2float_rn(z[i]) * 0.5f, c);
+        for (int i = 0; i < 8; ++i) {
+            y[i] = __fmul_rn(v[i], c);
+            if constexpr (MODE == kCoords) z[i] = __float2int_rn(v[i] * 2.0f);
+        }
+    } else {
+        int32_t s7 = 0;
+#pragma unroll
+        for (int i = 0; i < 7; ++i) s7 += t[i];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int32_t u = i < 7 ? t[i] : 2 * t[7] + (s7 & 1);
+            z[i] = 2 * u + int32_t(b);
+            y[i] = __fmul_rn(__int2float_rn(z[i]) * 0.5f, c);
+        }
     }
     store_group<MODE>(p.dst, g, y, z);
 }
@@ -357,9 +424,15 @@ __device__ __noinline__ void round_general(const Params& p, const uint8_t* smem,
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    build_tables(p, smem);
-    __syncthreads();
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    // Rings must be kRingBytes-aligned in the shared window so that ring addresses are (offset | base).
+    const uint32_t raw_base = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + ((kRingBytes - (raw_base & (kRingBytes - 1))) & (kRingBytes - 1));
+    uint8_t* rings = smem;
+    uint8_t* tables = smem + kRingsBytes;
+
+    grid_dependents_launch();  // lets the next launch of a sequence start its prologue early
+    build_tables(p, tables, rings);
 
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt_mask = (1u << lane) - 1u;
@@ -367,6 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
     const uint32_t* toff = reinterpret_cast<const uint32_t*>(p.blob + p.off_offsets);
     const uint8_t* payload = p.blob + p.off_payload;
     const uint32_t per_tile = 32 * p.G;
+    const RingWords ring{smem_addr(rings + warp * kRingBytes)};
+    bool waited = false;
 
     for (uint32_t tile = blockIdx.x * kWarps + warp; tile < p.T; tile += gridDim.x * kWarps) {
         const uint32_t e0 = __ldg(toff + tile), e1 = __ldg(toff + tile + 1);
@@ -374,43 +449,85 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
         const uint32_t g0 = tile * per_tile;
         const uint32_t ng = min(per_tile, p.NG - g0);
         const uint32_t raw = (ng * uint32_t(p.r) + 3u) & ~3u;
-        if (end < start || end > p.payload_bytes || end - start < 128ull + raw || end - start > 0xFFFFFFF0ull) {
+        if (end < start || end > p.payload_bytes || end - start < 128ull + raw || end - start > 0x7FFFFFF0ull) {
             if (lane == 0) atomicOr(&g_status, int(EP_DEV_BAD_OFFSETS));
             continue;
         }
         const uint8_t* tp = payload + start;
         const uint32_t tile_bytes = uint32_t(end - start);
-        uint32_t x = __ldg(reinterpret_cast<const uint32_t*>(tp) + lane);
-        const uint16_t* words = reinterpret_cast<const uint16_t*>(tp + 128 + raw);
-        const uint32_t nwords = (tile_bytes - 128 - raw) / 2;
-        uint32_t pos = 0;
-        const bool fast_tile = !(e0 >> 31) && p.r == 0;
-        // The fast round reads without bounds checks. It is allowed while a whole round of reads stays
-        // inside the payload: reading past this tile into the next is harmless (the end-of-tile check
-        // catches it), reading past the blob is not.
-        const uint64_t words_to_payload_end = (p.payload_bytes - start - 128 - raw) / 2;
-        const uint32_t fast_limit = words_to_payload_end > 0xFFFFFFFFull ? 0xFFFFFFFFu : uint32_t(words_to_payload_end);
+        TileState st;
+        st.x = __ldg(reinterpret_cast<const uint32_t*>(tp) + lane);
+
+        // Ring coordinate 0 mirrors tile byte A0 (16-byte aligned); the stream starts at ring
+        // coordinate `lead`.
+        const uint32_t s0 = 128 + raw, a0 = s0 & ~15u, lead = s0 - a0;
+        const uint32_t span = tile_bytes - a0;  // ring coordinates that hold tile bytes
+        const uint32_t chunks = (span + kChunkBytes - 1) / kChunkBytes;
+        st.pb = lead;
+        const GlobalWords gwords{tp + a0, lead, span};
+        const uint8_t* src0 = tp + a0 + 16 * lane;
+        auto issue = [&](uint32_t c) {
+            const uint32_t off = c * kChunkBytes + 16 * lane;
+            const uint32_t n = off < span ? min(16u, span - off) : 0u;
+            cp_async16(ring.base + (off & (kRingBytes - 1)), n ? src0 + c * kChunkBytes : tp, n);
+        };
+        // Prologue: three chunks in flight, one commit group each.
+        uint32_t issued = 0, h0 = 0, h1 = 0, h2 = 0;
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+            if (issued < chunks) { issue(issued); ++issued; }
+            cp_async_commit();
+            h2 = h1; h1 = h0; h0 = issued;
+        }
 
         RowCursor rc;
         rc.row = (g0 + lane) / p.gpr;
         rc.col = (g0 + lane) - rc.row * p.gpr;
         rc.cached_row = 0xFFFFFFFFu;
         rc.c_row = 0.f;
+        const bool esc_tile = e0 >> 31;
+        const bool raw_tile = p.r > 0;
+        const uint32_t round_bytes = 2 * (esc_tile ? kRoundWordsEsc : kRoundWords);
 
         const uint32_t R = (ng + 31) / 32;
         for (uint32_t k = 0; k < R; ++k) {
+            // One more chunk if its ring slot is free (the chunk it replaces lies wholly behind pb).
+            if (issued < chunks && issued <= st.pb / kChunkBytes + (kRingChunks - 1)) { issue(issued); ++issued; }
+            cp_async_commit();
+            h2 = h1; h1 = h0; h0 = issued;
+            cp_async_wait<2>();  // chunks [0, h2) have landed
+            uint32_t ready = h2 == chunks ? 0xFFFFFFFFu : h2 * kChunkBytes;
+            if (st.pb + round_bytes > ready) {
+                cp_async_wait<0>();
+                ready = issued == chunks ? 0xFFFFFFFFu : issued * kChunkBytes;
+            }
+            __syncwarp();
+            if (!waited) { grid_dependency_wait(); waited = true; }  // first store of this warp follows
+
             const uint32_t q = 32 * k + lane, g = g0 + q;
             const bool full = 32 * k + 32 <= ng;
-            if (fast_tile && full && pos <= fast_limit - kFastRoundWords && fast_limit >= kFastRoundWords)
-                round_fast<MODE>(p, smem, words, scales, x, pos, g, lt_mask, rc);
-            else
-                round_general<MODE>(p, smem, words, nwords, tp + 128, tile_bytes - 128, scales, x, pos, q, q < ng, g,
-                                    lt_mask, rc);
+            const bool in_ring = st.pb + round_bytes <= ready;
+            const uint8_t* rawsec = tp + 128;
+            const uint32_t raw_avail = tile_bytes - 128;
+            if (full && in_ring) {
+                if (!esc_tile && !raw_tile)
+                    decode_round<MODE, false, false, false>(p, tables, ring, rawsec, raw_avail, scales, st, q, true, g, lt_mask, rc);
+                else if (!raw_tile)
+                    decode_round<MODE, true, false, false>(p, tables, ring, rawsec, raw_avail, scales, st, q, true, g, lt_mask, rc);
+                else
+                    decode_round<MODE, true, true, false>(p, tables, ring, rawsec, raw_avail, scales, st, q, true, g, lt_mask, rc);
+            } else {
+                decode_round<MODE, true, true, true>(p, tables, gwords, rawsec, raw_avail, scales, st, q, q < ng, g, lt_mask, rc);
+            }
             rc.advance(p.gpr);
         }
-        const bool ok = __all_sync(kFullMask, x == kRansL) && pos <= nwords && nwords - pos <= 7;
+        cp_async_wait<0>();  // the ring is reused by this warp's next tile
+        __syncwarp();
+        const uint32_t used = st.pb - lead, cap = span - lead;  // bytes of stream read / present
+        const bool ok = __all_sync(kFullMask, st.x == kRansL) && used <= cap && cap - used <= 14;
         if (!ok && lane == 0) atomicOr(&g_status, int(EP_DEV_CORRUPT_TILE));
     }
+    if (!waited) grid_dependency_wait();
 }
 
 }  // namespace dev
@@ -427,7 +544,7 @@ std::mutex g_dev_mu;
 DeviceInfo g_dev[64];
 
 template <int MODE>
-ep_status launch_mode(const dev::Params& p, cudaStream_t stream, int device) {
+ep_status launch_mode(const dev::Params& p, cudaStream_t stream, int device, bool chained) {
     {
         std::lock_guard<std::mutex> lk(g_dev_mu);
         DeviceInfo& d = g_dev[device];
@@ -441,14 +558,24 @@ ep_status launch_mode(const dev::Params& p, cudaStream_t stream, int device) {
     uint32_t want = (p.T + dev::kWarps - 1) / dev::kWarps;
     uint32_t grid = want < uint32_t(g_dev[device].sms) ? want : uint32_t(g_dev[device].sms);
     if (grid == 0) grid = 1;
-    dev::decode_kernel<MODE><<<grid, dev::kThreads, dev::kSmemBytes, stream>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(dev::kThreads);
+    cfg.dynamicSmemBytes = dev::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = chained ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, dev::decode_kernel<MODE>, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(EP_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
     return EP_OK;
 }
 
 ep_status launch_decode(const uint8_t* host_hdr, const void* dev_blob, size_t blob_bytes, void* dst, size_t dst_bytes,
-                        int mode, void* stream_ptr) {
+                        int mode, void* stream_ptr, bool chained) {
     if (!host_hdr || !dev_blob || !dst) return fail(EP_ERR_ARG, "decode: NULL argument");
     Header h;
     if (!parse_header(host_hdr, h)) return fail(EP_ERR_CORRUPT, "decode: malformed EPK1 header");
@@ -488,12 +615,12 @@ ep_status launch_decode(const uint8_t* host_hdr, const void* dev_blob, size_t bl
     p.payload_bytes = h.total - h.off_payload;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
     switch (mode) {
-        case dev::kBF16: return launch_mode<dev::kBF16>(p, stream, device);
-        case dev::kFP16: return launch_mode<dev::kFP16>(p, stream, device);
-        case dev::kFP32: return launch_mode<dev::kFP32>(p, stream, device);
-        case dev::kFP8: return launch_mode<dev::kFP8>(p, stream, device);
-        case dev::kINT8: return launch_mode<dev::kINT8>(p, stream, device);
-        case dev::kCoords: return launch_mode<dev::kCoords>(p, stream, device);
+        case dev::kBF16: return launch_mode<dev::kBF16>(p, stream, device, chained);
+        case dev::kFP16: return launch_mode<dev::kFP16>(p, stream, device, chained);
+        case dev::kFP32: return launch_mode<dev::kFP32>(p, stream, device, chained);
+        case dev::kFP8: return launch_mode<dev::kFP8>(p, stream, device, chained);
+        case dev::kINT8: return launch_mode<dev::kINT8>(p, stream, device, chained);
+        case dev::kCoords: return launch_mode<dev::kCoords>(p, stream, device, chained);
     }
     return fail(EP_ERR_DTYPE, "decode: unknown dtype %d", mode);
 }
@@ -509,13 +636,36 @@ extern "C" ep_status ep_decompress_into(const uint8_t* host_hdr, const void* dev
     if (!host_hdr) return fail(EP_ERR_ARG, "decode: NULL header");
     Header h;
     if (!parse_header(host_hdr, h)) return fail(EP_ERR_CORRUPT, "decode: malformed EPK1 header");
-    return launch_decode(host_hdr, dev_blob, blob_bytes, dst, dst_bytes, h.dtype, cuda_stream);
+    return launch_decode(host_hdr, dev_blob, blob_bytes, dst, dst_bytes, h.dtype, cuda_stream, false);
+}
+
+extern "C" ep_status ep_decompress_many(int count, const uint8_t* const* host_hdrs, const void* const* dev_blobs,
+                                        const size_t* blob_bytes, void* const* dsts, const size_t* dst_bytes,
+                                        void* cuda_stream) {
+    clear_error();
+    if (count < 0 || (count > 0 && (!host_hdrs || !dev_blobs || !blob_bytes || !dsts || !dst_bytes)))
+        return fail(EP_ERR_ARG, "ep_decompress_many: bad arguments");
+    // Validate every header before launching anything, so a failure launches nothing.
+    for (int i = 0; i < count; ++i) {
+        Header h;
+        if (!host_hdrs[i] || !parse_header(host_hdrs[i], h))
+            return fail(EP_ERR_CORRUPT, "ep_decompress_many: blob %d has a malformed header", i);
+        if (h.total != blob_bytes[i]) return fail(EP_ERR_BUFFER, "ep_decompress_many: blob %d size mismatch", i);
+    }
+    for (int i = 0; i < count; ++i) {
+        Header h;
+        parse_header(host_hdrs[i], h);
+        ep_status st = launch_decode(host_hdrs[i], dev_blobs[i], blob_bytes[i], dsts[i], dst_bytes[i], h.dtype,
+                                     cuda_stream, i > 0);
+        if (st != EP_OK) return st;
+    }
+    return EP_OK;
 }
 
 extern "C" ep_status ep_decode_coords_into(const uint8_t* host_hdr, const void* dev_blob, size_t blob_bytes,
                                            int32_t* dst_z, size_t dst_bytes, void* cuda_stream) {
     clear_error();
-    return launch_decode(host_hdr, dev_blob, blob_bytes, dst_z, dst_bytes, dev::kCoords, cuda_stream);
+    return launch_decode(host_hdr, dev_blob, blob_bytes, dst_z, dst_bytes, dev::kCoords, cuda_stream, false);
 }
 
 extern "C" ep_status ep_decompress(const uint8_t* host_hdr, const void* dev_blob, size_t blob_bytes, void** dst,
@@ -529,7 +679,7 @@ extern "C" ep_status ep_decompress(const uint8_t* host_hdr, const void* dev_blob
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     cudaError_t e = cudaMallocAsync(&out, bytes, stream);
     if (e != cudaSuccess) return fail(EP_ERR_NOMEM, "cudaMallocAsync(%zu): %s", bytes, cudaGetErrorString(e));
-    ep_status st = launch_decode(host_hdr, dev_blob, blob_bytes, out, bytes, h.dtype, cuda_stream);
+    ep_status st = launch_decode(host_hdr, dev_blob, blob_bytes, out, bytes, h.dtype, cuda_stream, false);
     if (st != EP_OK) {
         cudaFreeAsync(out, stream);
         return st;

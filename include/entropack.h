@@ -128,6 +128,23 @@ ep_status ep_decompress_into(const uint8_t* host_hdr, const void* dev_blob, size
                              size_t dst_bytes, void* cuda_stream);
 
 /*
+ * ep_decompress_many: decodes `count` blobs in order on one stream: blob i into dsts[i], with the
+ * argument rules of ep_decompress_into for each one. This is the layer-sequence form of the hot
+ * path, for example all linear layers of a model before a forward pass.
+ *
+ * The first launch is ordered after earlier work on the stream as usual. Each later launch is a
+ * programmatic dependent launch of the one before it: it may expand its frequency tables and
+ * prefetch its first tiles while the previous decode drains, and it stores nothing until that
+ * decode has finished. Overlapping dsts are therefore written in order. One requirement follows
+ * from the early reads: no blob in the list may be written by the decodes listed before it.
+ * Every header is validated before anything launches, so an error launches nothing.
+ * Errors: as ep_decompress_into, for the first failing blob.
+ */
+ep_status ep_decompress_many(int count, const uint8_t* const* host_hdrs, const void* const* dev_blobs,
+                             const size_t* blob_bytes, void* const* dsts, const size_t* dst_bytes,
+                             void* cuda_stream);
+
+/*
  * ep_decompress: the same decode, into a device buffer that the call allocates with cudaMallocAsync
  * on cuda_stream. *dst receives the pointer, and the caller frees it (cudaFreeAsync or cudaFree).
  * Errors: as ep_decompress_into, plus EP_ERR_NOMEM.

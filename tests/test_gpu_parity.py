@@ -258,3 +258,33 @@ def test_streams_and_allocating_entry(orc):
     assert err == rt.cudaError_t.cudaSuccess
     assert rt.cudaFree(ptr.value)[0] == rt.cudaError_t.cudaSuccess
     assert np.array_equal(host, gpu_bits(ref))
+
+
+def test_decompress_many_matches_single_decodes(orc):
+    """The layer-sequence entry (programmatic dependent launches) gives the same bytes as one-by-one
+    decodes. The last output is one buffer shared by several layers, written in list order."""
+    comps = [ep.compress(synth.dit_layer(i, shape=shp), 4.0)
+             for i, shp in enumerate([(384, 256), (1024, 512), (64, 3840), (3840, 64), (1536, 256)])]
+    comps.append(ep.compress(synth.fp8_codes(256, 512, seed=5), 5.0))
+    comps.append(ep.compress(synth.gaussian(300, 200, seed=6, container="fp32"), 7.0))
+    outs = [torch.empty(c.shape, dtype=c.dtype, device="cuda") for c in comps]
+    batch = ep.LayerBatch(list(zip(comps, outs)))
+    for _ in range(3):
+        batch.run()
+    status_clean()
+    for c, o in zip(comps, outs):
+        want = orc.decompress(c.blob)
+        got = gpu_bits(o)
+        if got.dtype == np.float32:
+            assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+        else:
+            assert np.array_equal(got, want)
+    # one reused buffer: after the sequence it holds the last layer that wrote it
+    shared = torch.empty(1024 * 512, dtype=torch.bfloat16, device="cuda")
+    bf = [c for c in comps if c.dtype == torch.bfloat16]
+    views = [shared[: c.shape[0] * c.shape[1]].view(c.shape) for c in bf]
+    ep.decompress_many(list(zip(bf, views)))
+    torch.cuda.synchronize()
+    status_clean()
+    last = bf[-1]
+    assert np.array_equal(gpu_bits(views[-1]), orc.decompress(last.blob))
