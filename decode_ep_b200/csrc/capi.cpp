@@ -73,7 +73,7 @@ ep_status validate_blob(const uint8_t* p, uint64_t bytes) {
             sum += v;
             fmax = v > fmax ? v : fmax;
         }
-        if (cnt == 1 && sum != 0) return fail(EP_ERR_CORRUPT, "context %d: lone symbol must store 0", c);
+        if (cnt == 1) return fail(EP_ERR_CORRUPT, "context %d: a single symbol must be stored as 4095 + 1", c);
         if (cnt >= 2 && (sum != kProbScale || fmax > kProbScale - 1))
             return fail(EP_ERR_CORRUPT, "context %d: frequencies do not sum to 4096", c);
     }

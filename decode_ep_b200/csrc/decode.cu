@@ -4,19 +4,22 @@
 // (modelscope paper page, summary; paper page abstract).
 //
 // Kernel shape: a persistent grid with one 1024-thread CTA per SM (32 warps).
-//   - Tables. Each CTA first expands the blob's 17 twelve-bit frequency tables into shared
-//     memory. Every context gets a block: a 4096-entry slot -> symbol byte table, then one
-//     16-byte record per symbol {f, -cum, next context block, value}. The next-context pointer
-//     and the reconstructed value are baked into the record, so the hot loop spends two shared
-//     loads per coordinate and does no extra arithmetic for the context chain.
-//   - Tiles. Each warp decodes whole tiles. Lane L owns the groups 32k + L of the tile. After
-//     every symbol step, the lanes that must refill take the next 16-bit words of the shared
-//     stream in lane order, found with a warp ballot and a popcount prefix.
+//   - Tables. Each CTA first expands the blob's 9 twelve-bit frequency tables into fused 32-bit
+//     decode entries in shared memory: 9 contexts x 4096 slots, 144 KB. One entry holds
+//       f (bits 0-11), a value field (bits 12-18 or 12-19), the magnitude class of the decoded
+//       coordinate (bit 19, which picks the next context) and slot - cum (bits 20-31).
+//     A symbol step is therefore one random 4-byte shared load and a handful of integer operations.
+//     There are no symbol, record or codebook tables.
+//   - Tiles. Each warp decodes whole tiles. Lane L owns the groups 32k + L of the tile. After every
+//     symbol step, the lanes that must refill take the next 16-bit words of the shared stream in
+//     lane order, found with a warp ballot and a popcount prefix.
 //   - Stream staging. The words come from a 2 KB per-warp ring in shared memory. Asynchronous
 //     16-byte copies (cp.async, one 512-byte chunk per round, up to 3 chunks ahead) fill it, so
 //     no refill waits on DRAM.
-//   - Stores. Each lane reconstructs its 8 values and writes them with one 16-byte store
-//     (BF16/FP16), so a warp writes 512 contiguous bytes.
+//   - Values. v = hi + b/2 is rebuilt with no conversion instruction. The value field is ORed into
+//     the mantissa of 1.5 * 2^22, a float whose last-place unit is 1/2, and the bias is subtracted.
+//     Each lane then writes its 8 values with one 16-byte store (BF16/FP16), so a warp writes 512
+//     contiguous bytes.
 //   - Layer sequences. Successive launches are chained with programmatic dependent launch. A
 //     kernel builds its tables and fills its first rings while the previous kernel drains, and it
 //     waits on the grid dependency only before its first store.
@@ -40,12 +43,14 @@ constexpr int kWarps = 32;
 constexpr int kThreads = kWarps * 32;
 constexpr uint32_t kFullMask = 0xFFFFFFFFu;
 
-// Tables: per context a 4096-byte slot -> symbol table, then 16-byte records.
-constexpr uint32_t kLutBytes = 4096;
-constexpr uint32_t kStartBlock = kLutBytes + 128 * 16;  // START: 128 symbols (coset bit x 64)
-constexpr uint32_t kCtxBlock = kLutBytes + 64 * 16;     // other contexts: 64 symbols
-constexpr uint32_t kPos7Shift = 8 * kCtxBlock;          // contexts 9..16 sit 8 blocks after 1..8
-constexpr uint32_t kTablesBytes = kStartBlock + 16 * kCtxBlock;
+// Fused decode tables: 4096 four-byte entries per context. Blocks: contexts 1..8 at (c-1) * 16 KB,
+// so (b, class) selects a block by bits 14 (class) and 15 (b), with +64 KB for position 7; START at
+// 128 KB.
+constexpr uint32_t kCtxBytes = 4096 * 4;
+constexpr uint32_t kPos7Offset = 4 * kCtxBytes;
+constexpr uint32_t kStartOffset = 8 * kCtxBytes;
+constexpr uint32_t kTablesBytes = 9 * kCtxBytes;
+__host__ __device__ constexpr uint32_t block_of(int c) { return c == 0 ? kStartOffset : uint32_t(c - 1) * kCtxBytes; }
 
 // Per-warp stream rings.
 constexpr uint32_t kRingBytes = 2048;
@@ -56,20 +61,22 @@ constexpr uint32_t kRingsBytes = kWarps * kRingBytes;
 // Dynamic shared memory: [alignment pad up to 2 KB][rings][tables]. The table-build scratch lives in
 // the ring area, which is free until decoding starts.
 constexpr uint32_t kSmemBytes = kRingBytes + kRingsBytes + kTablesBytes;
-constexpr uint32_t kScratchCum = 0;                               // u32 [17][129]
-constexpr uint32_t kScratchBytes = kScratchCum + 8784;            // table bytes, <= 2048
+constexpr uint32_t kScratchCum = 0;                                    // u32 [9][129]
+constexpr uint32_t kScratchBytes = 4656;                               // serialised tables, <= 2048
 constexpr uint32_t kScratchTableCap = 2048;
-constexpr uint32_t kScratchBucket = kScratchBytes + kScratchTableCap;  // u8 [17][64]
-constexpr uint32_t kScratchMeta = kScratchBucket + 17 * 64;       // u32 lo, cnt, bit [17] each
-static_assert(kScratchMeta + 3 * 17 * 4 <= kRingsBytes, "table-build scratch must fit the ring area");
+constexpr uint32_t kScratchBucket = kScratchBytes + kScratchTableCap;  // u8 [9][64]
+constexpr uint32_t kScratchMeta = kScratchBucket + kNumCtx * 64;       // u32 lo, cnt, bit [9] each
+static_assert(kScratchCum + kNumCtx * 129 * 4 <= kScratchBytes, "scratch overlap");
+static_assert(kScratchMeta + 3 * kNumCtx * 4 <= kRingsBytes, "table-build scratch must fit the ring area");
 
 // Words one round can take: 8 positions x 32 lanes, one refill each, plus as many ESC words.
 constexpr uint32_t kRoundWords = 8 * 32;
 constexpr uint32_t kRoundWordsEsc = 2 * kRoundWords;
 
-__host__ __device__ constexpr uint32_t block_of(int c) {
-    return c == 0 ? 0u : kStartBlock + uint32_t(c - 1) * kCtxBlock;
-}
+// 1.5 * 2^22: binary32 with a last-place unit of 1/2. ORing a field F < 2^22 into its mantissa gives
+// 1.5 * 2^22 + F/2 exactly.
+constexpr uint32_t kHalfMagic = 0x4AC00000u;
+constexpr float kHalfMagicF = 6291456.0f;
 
 enum Mode { kBF16 = 1, kFP16 = 2, kFP32 = 3, kFP8 = 4, kINT8 = 5, kCoords = 6 };
 
@@ -96,6 +103,11 @@ __device__ __forceinline__ uint32_t ld_shared_u16(uint32_t addr) {
     asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
     return v;
 }
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
 // 16-byte asynchronous copy global -> shared; bytes past `src_bytes` (0..16) are zero-filled and
 // not read.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -109,8 +121,28 @@ __device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddep
 
 // ------------------------------------------------------------------------- table expansion
 
+// Magnitude class of a coded coordinate: 1 when m = floor(|v|), taken on hi, is at least 2.
+__device__ __forceinline__ uint32_t mag_class(int hi, int b) {
+    int m = hi >= 0 ? hi : -hi - b;
+    return m >= 2 ? 1u : 0u;
+}
+
+// The fused entry of symbol `sym` of context c, for a slot that lies `bias` past the symbol's cum.
+__device__ __forceinline__ uint32_t fused_entry(int c, int sym, uint32_t f, uint32_t bias) {
+    int b = c == 0 ? (sym >> 6) : (c <= 4 ? (c - 1) >> 1 : (c - 5) >> 1);
+    int idx = sym & 63, hi = idx - 31;
+    uint32_t field, cls = 0;
+    if (c <= 4) {
+        field = uint32_t(2 * idx + b);                                // v = hi + b/2
+        cls = idx == kEscIdx ? 1u : mag_class(hi, b);                 // an escape has |hi| >= 32
+    } else {
+        field = uint32_t(4 * idx + b);                                // 2h + b/2 (parity added later)
+    }
+    return (f & 0xFFFu) | (field << 12) | (cls << 19) | (bias << 20);
+}
+
 __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch) {
-    uint32_t* cum = reinterpret_cast<uint32_t*>(scratch + kScratchCum);  // [17][129]
+    uint32_t* cum = reinterpret_cast<uint32_t*>(scratch + kScratchCum);  // [9][129]
     uint8_t* tbytes = scratch + kScratchBytes;
     uint8_t* bucket = scratch + kScratchBucket;                          // symbol at slot 64k
     uint32_t* s_lo = reinterpret_cast<uint32_t*>(scratch + kScratchMeta);
@@ -118,7 +150,7 @@ __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch)
     uint32_t* s_bit = s_cnt + kNumCtx;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // Stage the serialised tables (about 2 KB at most) with one coalesced pass.
+    // Stage the serialised tables (under 1 KB for valid blobs) with one coalesced pass.
     const uint32_t tlen = p.tables_len < kScratchTableCap ? p.tables_len : kScratchTableCap;
     const uint8_t* tb = p.blob + p.off_tables;
     for (uint32_t i = tid; i < tlen; i += kThreads) tbytes[i] = __ldg(tb + i);
@@ -143,15 +175,11 @@ __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch)
         int c = i >> 7, s = i & 127, A = c == 0 ? 128 : 64;
         uint32_t lo = s_lo[c], cnt = s_cnt[c], f = 0;
         if (uint32_t(s) >= lo && uint32_t(s) < lo + cnt && s < A) {
-            if (cnt == 1) {
-                f = kProbScale;
-            } else {
-                uint32_t bit = s_bit[c] + 12 * (uint32_t(s) - lo), byte = bit >> 3, w = 0;
+            uint32_t bit = s_bit[c] + 12 * (uint32_t(s) - lo), byte = bit >> 3, w = 0;
 #pragma unroll
-                for (int k = 0; k < 3; ++k)
-                    if (byte + k < bits_len) w |= uint32_t(tbytes[2 * kNumCtx + byte + k]) << (8 * k);
-                f = (w >> (bit & 7)) & 0xFFFu;
-            }
+            for (int k = 0; k < 3; ++k)
+                if (byte + k < bits_len) w |= uint32_t(tbytes[2 * kNumCtx + byte + k]) << (8 * k);
+            f = (w >> (bit & 7)) & 0xFFFu;
         }
         cum[c * 129 + s] = f;
     }
@@ -175,34 +203,18 @@ __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch)
         cc[4 * lane + 3] = ex + f0 + f1 + f2;
         if (lane == 31) {
             cc[128] = incl;
-            bool ok = s_cnt[warp] == 0 ? incl == 0 : incl == kProbScale;
+            bool ok = s_cnt[warp] == 0 ? incl == 0 : (incl == kProbScale && s_cnt[warp] >= 2);
             if (!ok && blockIdx.x == 0) atomicOr(&g_status, int(EP_DEV_BAD_TABLES));
         }
     }
     __syncthreads();
 
-    // Records {f, -cum, next block, value}, and the symbol at every 64th slot. The value is
-    // v = hi + b/2 for positions 0..6 and 2h + b/2 for position 7 (u7 = 2h + parity is completed in
-    // the decode loop).
+    // The symbol at every 64th slot.
     for (int i = tid; i < kNumCtx * 128; i += kThreads) {
         int c = i >> 7, s = i & 127, A = c == 0 ? 128 : 64;
         if (s >= A) continue;
         const uint32_t* cc = cum + c * 129;
         uint32_t f = cc[s + 1] - cc[s];
-        int b = c == 0 ? (s >> 6) : (c <= 8 ? (c - 1) >> 2 : (c - 9) >> 2);
-        int idx = s & 63, hi = idx - 31;
-        uint32_t next = 0;
-        float val;
-        if (c <= 8) {
-            int m = hi >= 0 ? hi : -hi - b;
-            int cls = idx == kEscIdx ? 3 : (m < 3 ? m : 3);
-            next = block_of(1 + 4 * b + cls);
-            val = float(hi) + 0.5f * float(b);
-        } else {
-            val = float(2 * hi) + 0.5f * float(b);
-        }
-        *reinterpret_cast<uint4*>(tables + block_of(c) + kLutBytes + 16 * s) =
-            make_uint4(f, 0u - cc[s], next, __float_as_uint(val));
         if (f) {
             uint32_t k0 = (cc[s] + 63) >> 6, k1 = (cc[s] + f + 63) >> 6;
             for (uint32_t k = k0; k < k1 && k < 64; ++k) bucket[c * 64 + k] = uint8_t(s);
@@ -210,23 +222,25 @@ __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch)
     }
     __syncthreads();
 
-    // Slot -> symbol bytes, 16 slots per thread. Start from the symbol of the chunk's 64-slot bucket
-    // and step past boundaries; zero-frequency symbols share their successor's cum and are skipped.
+    // Fused entries, 16 slots per thread. Start from the symbol of the chunk's 64-slot bucket and step
+    // past boundaries; zero-frequency symbols share their successor's cum and are skipped.
     for (int i = tid; i < kNumCtx * 256; i += kThreads) {
         int c = i >> 8, A = c == 0 ? 128 : 64;
         uint32_t slot0 = uint32_t(i & 255) * 16;
         const uint32_t* cc = cum + c * 129;
         int s = bucket[c * 64 + (slot0 >> 6)];
         s = s < A ? s : A - 1;
-        uint32_t nb = cc[s + 1];
-        uint32_t out[4] = {0, 0, 0, 0};
+        uint32_t lo = cc[s], nb = cc[s + 1];
+        uint32_t out[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             uint32_t slot = slot0 + j;
-            while (slot >= nb && s + 1 < A) { ++s; nb = cc[s + 1]; }
-            out[j >> 2] |= uint32_t(s) << (8 * (j & 3));
+            while (slot >= nb && s + 1 < A) { ++s; lo = nb; nb = cc[s + 1]; }
+            out[j] = fused_entry(c, s, nb - lo, slot - lo);
         }
-        *reinterpret_cast<uint4*>(tables + block_of(c) + slot0) = make_uint4(out[0], out[1], out[2], out[3]);
+        uint4* dst = reinterpret_cast<uint4*>(tables + block_of(c) + 4 * slot0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(out[4 * j], out[4 * j + 1], out[4 * j + 2], out[4 * j + 3]);
     }
     __syncthreads();
 }
@@ -304,7 +318,7 @@ struct RowCursor {
 // ring coordinates (lead + 2 * words consumed).
 struct RingWords {
     uint32_t base;  // shared address of the warp's ring, kRingBytes-aligned
-    __device__ __forceinline__ uint32_t at(uint32_t pb) const { return ld_shared_u16(((pb) & (kRingBytes - 1)) | base); }
+    __device__ __forceinline__ uint32_t at(uint32_t pb) const { return ld_shared_u16((pb & (kRingBytes - 1)) | base); }
 };
 struct GlobalWords {
     const uint8_t* ring0;  // global address that ring coordinate 0 mirrors
@@ -321,101 +335,126 @@ struct TileState {
 
 // ------------------------------------------------------------------------------ one round
 
-// Decodes one round (8 coordinates per lane). ESC: the tile holds escapes (check every position).
-// RAW: r > 0 raw low bits. PARTIAL: some lanes hold no group.
-template <int MODE, bool ESC, bool RAW, bool PARTIAL, class Words>
-__device__ __forceinline__ void decode_round(const Params& p, const uint8_t* tables, const Words& words,
-                                             const uint8_t* rawsec, uint32_t raw_avail, const uint16_t* scales,
-                                             TileState& st, uint32_t q, bool active, uint32_t g, uint32_t lt_mask,
-                                             RowCursor& rc) {
-    constexpr bool SIMPLE = !ESC && !RAW;  // values straight from the records
-    float v[8];
-    int32_t t[8];
-    uint32_t B = 0, par = 0, b = 0;
-    uint32_t win0 = 0, win1 = 0, win2 = 0;
-    if constexpr (RAW) {
-        // The group's 8r raw bits start at byte q*r of the raw section; load a 96-bit window.
-        if (active) {
-            const int r = p.r;
-            uint32_t o = q * uint32_t(r), a = o & ~3u, sh = (o & 3u) * 8;
-            uint32_t w[4];
+// One symbol step: the fused entry for the current context block B, the state update and the
+// refill from the shared word stream. Returns the entry.
+template <bool PARTIAL, class Words>
+__device__ __forceinline__ uint32_t symbol_step(uint32_t B, const Words& words, uint32_t& x, uint32_t& pb,
+                                                bool active, uint32_t lt_mask) {
+    uint32_t e = 0;
+    if (!PARTIAL || active) {
+        e = ld_shared_u32(B + ((x & (kProbScale - 1)) << 2));
+        x = (e & 0xFFFu) * (x >> kProbBits) + (e >> 20);  // f * (x >> 12) + slot - cum
+    }
+    const bool need = (!PARTIAL || active) && x < kRansL;
+    const uint32_t m = __ballot_sync(kFullMask, need);
+    const uint32_t w = words.at(pb + 2 * __popc(m & lt_mask));
+    x = need ? (x << 16) | w : x;
+    pb += 2 * __popc(m);
+    return e;
+}
+
+// Fast round: every lane holds a group, the tile has no escapes and no raw bits. Values come from
+// the entries' value fields.
+template <int MODE>
+__device__ __forceinline__ void round_fast(const Params& p, uint32_t t0, const RingWords& words, const uint16_t* scales,
+                                           TileState& st, uint32_t g, uint32_t lt_mask, RowCursor& rc) {
+    uint32_t x = st.x, pb = st.pb;
+    uint32_t e[8];
+    e[0] = symbol_step<false>(t0 + kStartOffset, words, x, pb, true, lt_mask);
+    const uint32_t gbase = t0 + ((e[0] << 3) & 0x8000u);  // coset bit (entry bit 12) -> block bit 15
+    uint32_t par = e[0];
+    uint32_t B = gbase + ((e[0] >> 5) & 0x4000u);         // class bit (entry bit 19) -> block bit 14
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                w[j] = (a + 4 * j + 4 <= raw_avail) ? __ldg(reinterpret_cast<const uint32_t*>(rawsec + a) + j) : 0u;
-            win0 = __funnelshift_r(w[0], w[1], sh);
-            win1 = __funnelshift_r(w[1], w[2], sh);
-            win2 = __funnelshift_r(w[2], w[3], sh);
+    for (int i = 1; i < 8; ++i) {
+        e[i] = symbol_step<false>(B, words, x, pb, true, lt_mask);
+        if (i < 7) {
+            par ^= e[i];
+            B = gbase + (i == 6 ? kPos7Offset : 0u) + ((e[i] >> 5) & 0x4000u);
         }
     }
-    uint32_t x = st.x, pb = st.pb;
+    st.x = x;
+    st.pb = pb;
+
+    // Entry bit 13 is the parity of idx; u_i = idx_i - 31 flips it, and seven flips make
+    // pi = 1 - (XOR of the idx parities).
+    const uint32_t two_pi = (~par >> 12) & 2u;
+    const float c = rc.scale(p, scales);
+    float y[8];
+    int32_t z[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        if (i == 7) B += kPos7Shift;
-        uint32_t sym = 0;
-        uint4 rec = make_uint4(0, 0, 0, 0);
-        if (!PARTIAL || active) {
-            const uint32_t slot = x & (kProbScale - 1);
-            sym = tables[B + slot];
-            rec = *reinterpret_cast<const uint4*>(tables + B + kLutBytes + 16 * sym);
-            x = rec.x * (x >> kProbBits) + slot + rec.y;  // f * (x >> 12) + slot - cum
+        float v;
+        if (i < 7) v = __uint_as_float(((e[i] >> 12) & 0x7Fu) | kHalfMagic) - (kHalfMagicF + 31.0f);
+        else v = __uint_as_float((((e[7] >> 12) & 0xFFu) | kHalfMagic) + two_pi) - (kHalfMagicF + 62.0f);
+        y[i] = __fmul_rn(v, c);
+        if constexpr (MODE == kCoords) z[i] = __float2int_rn(v * 2.0f);
+    }
+    store_group<MODE>(p.dst, g, y, z);
+}
+
+// General round: escapes, raw low bits and ragged rounds (PARTIAL: some lanes hold no group).
+template <int MODE, bool PARTIAL, class Words>
+__device__ __forceinline__ void round_general(const Params& p, uint32_t t0, const Words& words, const uint8_t* rawsec,
+                                              uint32_t raw_avail, const uint16_t* scales, TileState& st, uint32_t q,
+                                              bool active, uint32_t g, uint32_t lt_mask, RowCursor& rc) {
+    const int r = p.r;
+    // The group's 8r raw bits start at byte q*r of the raw section; load a 96-bit window.
+    uint32_t win0 = 0, win1 = 0, win2 = 0;
+    if (r > 0 && active) {
+        uint32_t o = q * uint32_t(r), a = o & ~3u, sh = (o & 3u) * 8;
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            w[j] = (a + 4 * j + 4 <= raw_avail) ? __ldg(reinterpret_cast<const uint32_t*>(rawsec + a) + j) : 0u;
+        win0 = __funnelshift_r(w[0], w[1], sh);
+        win1 = __funnelshift_r(w[1], w[2], sh);
+        win2 = __funnelshift_r(w[2], w[3], sh);
+    }
+    uint32_t x = st.x, pb = st.pb;
+    uint32_t B = t0 + kStartOffset, gbase = t0, b = 0;
+    int32_t t[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t e = symbol_step<PARTIAL>(B, words, x, pb, active, lt_mask);
+        // idx: entry bits 13-18 (field 2 idx + b) for positions 0..6, bits 14-19 (4 idx + b) for 7.
+        const uint32_t idx = i < 7 ? (e >> 13) & 63u : (e >> 14) & 63u;
+        int32_t hi = int32_t(idx) - 31;
+        const bool esc = (!PARTIAL || active) && idx == uint32_t(kEscIdx);
+        const uint32_t me = __ballot_sync(kFullMask, esc);
+        if (me) {
+            const uint32_t ew = words.at(pb + 2 * __popc(me & lt_mask));
+            if (esc) hi = int32_t(int16_t(ew));
+            pb += 2 * __popc(me);
         }
-        const bool need = (!PARTIAL || active) && x < kRansL;
-        const uint32_t m = __ballot_sync(kFullMask, need);
-        const uint32_t w = words.at(pb + 2 * __popc(m & lt_mask));
-        x = need ? (x << 16) | w : x;
-        pb += 2 * __popc(m);
-        if constexpr (SIMPLE) {
-            if (i < 7) par ^= sym;
-            v[i] = __uint_as_float(rec.w);
-        } else {
-            const uint32_t idx = sym & 63u;
-            int32_t hi = int32_t(idx) - 31;
-            if constexpr (ESC) {
-                const bool esc = (!PARTIAL || active) && idx == uint32_t(kEscIdx);
-                const uint32_t me = __ballot_sync(kFullMask, esc);
-                if (me) {
-                    const uint32_t e = words.at(pb + 2 * __popc(me & lt_mask));
-                    if (esc) hi = int32_t(int16_t(e));
-                    pb += 2 * __popc(me);
-                }
-            }
-            if (i == 0) b = sym >> 6;
-            int32_t lo = 0;
-            if constexpr (RAW) {
-                const uint32_t bp = uint32_t(i) * uint32_t(p.r), sel = bp >> 5, sh = bp & 31;
-                const uint32_t wa = sel == 0 ? win0 : (sel == 1 ? win1 : win2);
-                const uint32_t wb = sel == 0 ? win1 : win2;
-                lo = int32_t(__funnelshift_r(wa, wb, sh) & ((1u << p.r) - 1u));
-            }
-            t[i] = hi * (1 << p.r) + lo;
+        if (i == 0) {
+            b = (e >> 12) & 1u;
+            gbase = t0 + (b << 15);
         }
-        B = rec.z;
+        int32_t lo = 0;
+        if (r > 0) {
+            const uint32_t bp = uint32_t(i) * uint32_t(r), sel = bp >> 5, sh = bp & 31;
+            const uint32_t wa = sel == 0 ? win0 : (sel == 1 ? win1 : win2);
+            const uint32_t wb = sel == 0 ? win1 : win2;
+            lo = int32_t(__funnelshift_r(wa, wb, sh) & ((1u << r) - 1u));
+        }
+        t[i] = hi * (1 << r) + lo;
+        if (i < 7) B = gbase + (i == 6 ? kPos7Offset : 0u) + ((e >> 5) & 0x4000u);
     }
     st.x = x;
     st.pb = pb;
     if (PARTIAL && !active) return;
 
+    int32_t s7 = 0;
+#pragma unroll
+    for (int i = 0; i < 7; ++i) s7 += t[i];
     const float c = rc.scale(p, scales);
     float y[8];
     int32_t z[8];
-    if constexpr (SIMPLE) {
-        // u_i = idx_i - 31 flips parity against idx_i; seven flips make pi = 1 when the idx parity is even.
-        if (!(par & 1u)) v[7] += 1.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            y[i] = __fmul_rn(v[i], c);
-            if constexpr (MODE == kCoords) z[i] = __float2int_rn(v[i] * 2.0f);
-        }
-    } else {
-        int32_t s7 = 0;
-#pragma unroll
-        for (int i = 0; i < 7; ++i) s7 += t[i];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int32_t u = i < 7 ? t[i] : 2 * t[7] + (s7 & 1);
-            z[i] = 2 * u + int32_t(b);
-            y[i] = __fmul_rn(__int2float_rn(z[i]) * 0.5f, c);
-        }
+    for (int i = 0; i < 8; ++i) {
+        const int32_t u = i < 7 ? t[i] : 2 * t[7] + (s7 & 1);
+        z[i] = 2 * u + int32_t(b);
+        y[i] = __fmul_rn(__int2float_rn(z[i]) * 0.5f, c);
     }
     store_group<MODE>(p.dst, g, y, z);
 }
@@ -430,6 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
     uint8_t* smem = smem_raw + ((kRingBytes - (raw_base & (kRingBytes - 1))) & (kRingBytes - 1));
     uint8_t* rings = smem;
     uint8_t* tables = smem + kRingsBytes;
+    const uint32_t t0 = smem_addr(tables);
 
     grid_dependents_launch();  // lets the next launch of a sequence start its prologue early
     build_tables(p, tables, rings);
@@ -458,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
         TileState st;
         st.x = __ldg(reinterpret_cast<const uint32_t*>(tp) + lane);
 
-        // Ring coordinate 0 mirrors tile byte A0 (16-byte aligned); the stream starts at ring
+        // Ring coordinate 0 mirrors tile byte a0 (16-byte aligned); the stream starts at ring
         // coordinate `lead`.
         const uint32_t s0 = 128 + raw, a0 = s0 & ~15u, lead = s0 - a0;
         const uint32_t span = tile_bytes - a0;  // ring coordinates that hold tile bytes
@@ -485,9 +525,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
         rc.col = (g0 + lane) - rc.row * p.gpr;
         rc.cached_row = 0xFFFFFFFFu;
         rc.c_row = 0.f;
-        const bool esc_tile = e0 >> 31;
-        const bool raw_tile = p.r > 0;
-        const uint32_t round_bytes = 2 * (esc_tile ? kRoundWordsEsc : kRoundWords);
+        const bool simple = !(e0 >> 31) && p.r == 0;
+        const uint32_t round_bytes = 2 * ((e0 >> 31) ? kRoundWordsEsc : kRoundWords);
+        const uint8_t* rawsec = tp + 128;
+        const uint32_t raw_avail = tile_bytes - 128;
 
         const uint32_t R = (ng + 31) / 32;
         for (uint32_t k = 0; k < R; ++k) {
@@ -507,17 +548,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
             const uint32_t q = 32 * k + lane, g = g0 + q;
             const bool full = 32 * k + 32 <= ng;
             const bool in_ring = st.pb + round_bytes <= ready;
-            const uint8_t* rawsec = tp + 128;
-            const uint32_t raw_avail = tile_bytes - 128;
             if (full && in_ring) {
-                if (!esc_tile && !raw_tile)
-                    decode_round<MODE, false, false, false>(p, tables, ring, rawsec, raw_avail, scales, st, q, true, g, lt_mask, rc);
-                else if (!raw_tile)
-                    decode_round<MODE, true, false, false>(p, tables, ring, rawsec, raw_avail, scales, st, q, true, g, lt_mask, rc);
+                if (simple)
+                    round_fast<MODE>(p, t0, ring, scales, st, g, lt_mask, rc);
                 else
-                    decode_round<MODE, true, true, false>(p, tables, ring, rawsec, raw_avail, scales, st, q, true, g, lt_mask, rc);
+                    round_general<MODE, false>(p, t0, ring, rawsec, raw_avail, scales, st, q, true, g, lt_mask, rc);
             } else {
-                decode_round<MODE, true, true, true>(p, tables, gwords, rawsec, raw_avail, scales, st, q, q < ng, g, lt_mask, rc);
+                round_general<MODE, true>(p, t0, gwords, rawsec, raw_avail, scales, st, q, q < ng, g, lt_mask, rc);
             }
             rc.advance(p.gpr);
         }

@@ -1,6 +1,6 @@
 // Internal constants and the host-side header reader of the EPK1 blob, used by the host encoder,
 // the C ABI and the decode launcher. The byte layout:
-//   header (64 B) | scales M x bf16 | tables: lo[17], cnt[17], 12-bit frequencies packed LSB-first |
+//   header (64 B) | scales M x bf16 | tables: lo[9], cnt[9], 12-bit frequencies packed LSB-first |
 //   tile offsets (T+1) x u32 (start/16 | has_esc<<31) | payload: per tile 32 x u32 states,
 //   raw low bits (groups*r bytes, padded to 4), u16 word stream, zero padding to 16.
 // Every section starts 16-byte aligned; all fields are little-endian.
@@ -14,7 +14,7 @@ namespace epk {
 
 constexpr uint32_t kHeaderBytes = 64;
 constexpr int kLanes = 32;
-constexpr int kNumCtx = 17;
+constexpr int kNumCtx = 9;
 constexpr int kProbBits = 12;
 constexpr uint32_t kProbScale = 1u << kProbBits;  // 4096
 constexpr uint32_t kRansL = 1u << 16;             // state lower bound; 16-bit refills
@@ -77,8 +77,8 @@ inline bool parse_header(const uint8_t* p, Header& h) {
     uint64_t per_tile = 32ull * uint64_t(h.G);
     if (h.T != (h.groups() + per_tile - 1) / per_tile) return false;
     if (h.off_scales != kHeaderBytes || h.off_tables != h.off_scales + pad16(2ull * h.M)) return false;
-    // The tables section is at least pad16(34) bytes: the decode kernel reads lo[17] and cnt[17] unchecked.
-    if (h.off_offsets < h.off_tables + 48 || (h.off_offsets & 15) ||
+    // The tables section is at least pad16(18) bytes: the decode kernel reads lo[9] and cnt[9] unchecked.
+    if (h.off_offsets < h.off_tables + 32 || (h.off_offsets & 15) ||
         h.off_payload != h.off_offsets + pad16(4ull * (uint64_t(h.T) + 1)) || h.off_payload > h.total)
         return false;
     return true;

@@ -5,7 +5,7 @@
 //   - Each 8-wide group is quantised to the nearest E8 point at one global resolution alpha.
 //   - Alpha comes from bisection on log2(alpha) against a storage estimate taken on a sample of
 //     rows, so the full stream is never re-encoded (paper page abstract; techmoon article).
-//   - The coordinates are rANS-coded under 17 conditional 12-bit tables, in independent tiles of
+//   - The coordinates are rANS-coded under 9 conditional 12-bit tables, in independent tiles of
 //     32 interleaved lanes (abstract; modelscope summary).
 // All floating point is IEEE double/binary32, round-to-nearest, with no FMA contraction. The
 // build passes -ffp-contract=off, so every estimate and every quantisation decision is a fixed
@@ -146,9 +146,10 @@ inline int e8_code(const double* x, int32_t* t) {
 
 inline int32_t hi_of(int32_t t, int r) { return t >> r; }  // arithmetic shift = floor division by 2^r
 inline int idx_of(int32_t hi) { return (hi >= -31 && hi <= 31) ? hi + 31 : kEscIdx; }
+// Magnitude class: 1 when m = floor(|v|), taken on hi, is at least 2.
 inline int cls_of(int32_t hi, int b) {
     int32_t m = hi >= 0 ? hi : -hi - b;
-    return m < 3 ? int(m) : 3;
+    return m >= 2 ? 1 : 0;
 }
 
 // Context and table symbol of each of the 8 positions of one group.
@@ -157,7 +158,7 @@ inline void group_syms(int b, const int32_t* t, int r, uint8_t* ctx, uint8_t* sy
     ctx[0] = 0;
     sym[0] = uint8_t(64 * b + idx_of(hi[0]));
     for (int i = 1; i < 8; ++i) {
-        ctx[i] = uint8_t((i < 7 ? 1 : 9) + 4 * b + cls_of(hi[i - 1], b));
+        ctx[i] = uint8_t((i < 7 ? 1 : 5) + 2 * b + cls_of(hi[i - 1], b));
         sym[i] = uint8_t(idx_of(hi[i]));
     }
 }
@@ -173,14 +174,19 @@ int raw_bits_for(float alpha) {
 using Counts = std::vector<uint64_t>;  // [17][128]
 
 // 12-bit normalisation: f = max(1, floor(4096 n_s / n)) for present symbols. The rounding gap is
-// closed at the largest frequency, or in steps of whole units when there is too much. A single
-// present symbol gets 4096.
+// closed at the largest frequency, or in steps of whole units when there is too much. No f exceeds
+// 4095: a single present symbol gets 4095, and its neighbour (s + 1, or s - 1 at the alphabet's
+// end) gets 1.
 void normalize(const uint64_t* cnt, int A, uint32_t* f) {
     uint64_t total = 0;
     int present = 0;
     for (int s = 0; s < A; ++s) { total += cnt[s]; present += cnt[s] != 0; f[s] = 0; }
     if (!present) return;
-    if (present == 1) { for (int s = 0; s < A; ++s) if (cnt[s]) f[s] = kProbScale; return; }
+    if (present == 1) {
+        for (int s = 0; s < A; ++s)
+            if (cnt[s]) { f[s] = kProbScale - 1; f[s + 1 < A ? s + 1 : s - 1] = 1; }
+        return;
+    }
     int64_t sum = 0;
     for (int s = 0; s < A; ++s) {
         if (!cnt[s]) continue;
@@ -214,7 +220,7 @@ struct Tables {
             normalize(&c[size_t(k) * 128], A, f[k]);
             for (int s = A; s < 128; ++s) f[k][s] = 0;
             int first = -1, last = -1;
-            for (int s = 0; s < A; ++s) if (c[size_t(k) * 128 + s]) { if (first < 0) first = s; last = s; }
+            for (int s = 0; s < A; ++s) if (f[k][s]) { if (first < 0) first = s; last = s; }
             lo[k] = first < 0 ? 0 : first;
             cnt[k] = first < 0 ? 0 : last - first + 1;
             nsym += uint64_t(cnt[k]);
@@ -229,7 +235,7 @@ struct Tables {
         uint64_t pos = 0;
         for (int k = 0; k < kNumCtx; ++k)
             for (int s = lo[k]; s < lo[k] + cnt[k]; ++s, pos += 12) {
-                uint32_t v = cnt[k] == 1 ? 0u : f[k][s];
+                uint32_t v = f[k][s];
                 uint32_t word = v << (pos & 7);  // 12 + 7 bits fit in three bytes
                 bits[pos >> 3] |= uint8_t(word);
                 bits[(pos >> 3) + 1] |= uint8_t(word >> 8);

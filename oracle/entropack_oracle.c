@@ -16,7 +16,7 @@
  *  - decode = symbol decode, arithmetic inverse of the lattice map, per-row
  *    rescale, with no symbol tensor or codebook — modelscope summary.
  * Every detail the pages leave open is read as the format document states
- * (E8 = D8 ∪ D8+½, 17 contexts of 12-bit tables conditioned on the coset bit
+ * (E8 = D8 ∪ D8+½, 9 contexts of 12-bit tables conditioned on the coset bit
  * and the previous coordinate's magnitude class, 32-lane interleaved rANS).
  */
 #include "entropack_oracle.h"
@@ -29,7 +29,7 @@ enum { OK = 0, E_ARG = -1, E_DTYPE = -2, E_SHAPE = -3, E_TARGET = -4, E_NONFINIT
        E_CORRUPT = -6, E_NOMEM = -8 };
 
 #define LANES 32
-#define NCTX 17
+#define NCTX 9
 #define PROB_BITS 12
 #define PROB_SCALE 4096u
 #define RANS_L 65536u
@@ -239,19 +239,24 @@ static int64_t floor_shift(int64_t t, int r) { return (t >= 0) ? (t >> r) : -((-
 
 static int sym_index(int64_t hi) { return (hi >= -31 && hi <= 31) ? (int)(hi + 31) : ESC_IDX; }
 
+/* Magnitude class of a coded coordinate: 1 when m = ⌊|v|⌋ (taken on hi) is at least 2, else 0. */
 static int mag_class(int64_t hi, int b) {
     int64_t m = (hi >= 0) ? hi : -hi - b;
-    return m < 3 ? (int)m : 3;
+    return m >= 2 ? 1 : 0;
 }
 
-/* Context of position i, given the previous position's hi and the coset bit. */
+/* Context of position i, given the previous position's hi and the coset bit:
+ * START for position 0, 1 + 2b + class for positions 1..6, 5 + 2b + class for position 7. */
 static int context_of(int i, int64_t hi_prev, int b) {
     if (i == 0) return 0;
-    return (i < 7 ? 1 : 9) + 4 * b + mag_class(hi_prev, b);
+    return (i < 7 ? 1 : 5) + 2 * b + mag_class(hi_prev, b);
 }
 
 /* --------------------------------------------------- frequency normalisation */
 
+/* n is the alphabet size. Every present symbol gets f >= 1 and no f exceeds 4095: a context with
+ * a single present symbol s gives it 4095 and its neighbour (s + 1, or s - 1 at the end of the
+ * alphabet) the remaining 1. */
 int orc_normalize(const uint64_t* counts, int n, uint32_t* f) {
     uint64_t total = 0;
     int present = 0;
@@ -259,7 +264,11 @@ int orc_normalize(const uint64_t* counts, int n, uint32_t* f) {
     for (int s = 0; s < n; s++) f[s] = 0;
     if (present == 0) return OK;
     if (present == 1) {
-        for (int s = 0; s < n; s++) if (counts[s]) f[s] = PROB_SCALE;
+        for (int s = 0; s < n; s++)
+            if (counts[s]) {
+                f[s] = PROB_SCALE - 1;
+                f[s + 1 < n ? s + 1 : s - 1] = 1;
+            }
         return OK;
     }
     int64_t sum = 0;
@@ -298,8 +307,8 @@ static void model_from_counts(uint64_t counts[NCTX][128], Model* m) {
     memset(m, 0, sizeof(*m));
     for (int c = 0; c < NCTX; c++) {
         int A = ctx_alphabet(c), lo = -1, hi = -1;
-        for (int s = 0; s < A; s++) if (counts[c][s]) { if (lo < 0) lo = s; hi = s; }
         orc_normalize(counts[c], A, m->f[c]);
+        for (int s = 0; s < A; s++) if (m->f[c][s]) { if (lo < 0) lo = s; hi = s; }
         m->lo[c] = lo < 0 ? 0 : lo;
         m->cnt[c] = lo < 0 ? 0 : hi - lo + 1;
         uint32_t acc = 0;
@@ -320,7 +329,7 @@ static void write_tables(const Model* m, uint8_t* out) {
     for (int c = 0; c < NCTX; c++) { out[c] = (uint8_t)m->lo[c]; out[NCTX + c] = (uint8_t)m->cnt[c]; }
     for (int c = 0; c < NCTX; c++) {
         for (int s = m->lo[c]; s < m->lo[c] + m->cnt[c]; s++) {
-            uint32_t v = (m->cnt[c] == 1) ? 0 : m->f[c][s];
+            uint32_t v = m->f[c][s];
             for (int k = 0; k < 12; k++, bit++)
                 if ((v >> k) & 1) bits[bit >> 3] |= (uint8_t)(1u << (bit & 7));
         }
@@ -352,8 +361,7 @@ static int read_tables(const uint8_t* in, uint64_t avail, Model* m, uint64_t* us
             total += v;
         }
         if (m->cnt[c] == 1) {
-            if (total != 0) return E_CORRUPT;
-            m->f[c][m->lo[c]] = PROB_SCALE;
+            return E_CORRUPT; /* a lone symbol is stored as 4095 + 1 */
         } else if (m->cnt[c] >= 2) {
             if (total != PROB_SCALE) return E_CORRUPT;
             for (int s = m->lo[c]; s < m->lo[c] + m->cnt[c]; s++)
