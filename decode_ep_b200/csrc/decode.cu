@@ -348,7 +348,8 @@ __device__ __forceinline__ uint32_t symbol_step(uint32_t B, const Words& words, 
     const bool need = (!PARTIAL || active) && x < kRansL;
     const uint32_t m = __ballot_sync(kFullMask, need);
     const uint32_t w = words.at(pb + 2 * __popc(m & lt_mask));
-    x = need ? (x << 16) | w : x;
+    // x = need ? (x << 16) | w : x, as one byte permute: bytes (w0, w1, x0, x1) or x unchanged.
+    x = __byte_perm(x, w, need ? 0x1054u : 0x3210u);
     pb += 2 * __popc(m);
     return e;
 }
@@ -483,7 +484,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
     const RingWords ring{smem_addr(rings + warp * kRingBytes)};
     bool waited = false;
 
-    for (uint32_t tile = blockIdx.x * kWarps + warp; tile < p.T; tile += gridDim.x * kWarps) {
+    // Tiles are dealt round-robin over the CTAs first, so that consecutive tiles land on different SMs
+    // and a partial last wave is spread over the whole GPU: tile = (k * kWarps + warp) * grid + block.
+    for (uint32_t slot = warp;; slot += kWarps) {
+        const uint32_t tile = slot * gridDim.x + blockIdx.x;
+        if (tile >= p.T) break;
         const uint32_t e0 = __ldg(toff + tile), e1 = __ldg(toff + tile + 1);
         const uint64_t start = uint64_t(e0 & 0x7FFFFFFFu) * 16, end = uint64_t(e1 & 0x7FFFFFFFu) * 16;
         const uint32_t g0 = tile * per_tile;
@@ -592,8 +597,8 @@ ep_status launch_mode(const dev::Params& p, cudaStream_t stream, int device, boo
             d.configured[MODE] = true;
         }
     }
-    uint32_t want = (p.T + dev::kWarps - 1) / dev::kWarps;
-    uint32_t grid = want < uint32_t(g_dev[device].sms) ? want : uint32_t(g_dev[device].sms);
+    // One CTA per SM, or one per tile when there are fewer tiles than SMs.
+    uint32_t grid = p.T < uint32_t(g_dev[device].sms) ? p.T : uint32_t(g_dev[device].sms);
     if (grid == 0) grid = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
