@@ -66,8 +66,10 @@ constexpr uint32_t kScratchBytes = 4656;                               // serial
 constexpr uint32_t kScratchTableCap = 2048;
 constexpr uint32_t kScratchBucket = kScratchBytes + kScratchTableCap;  // u8 [9][64]
 constexpr uint32_t kScratchMeta = kScratchBucket + kNumCtx * 64;       // u32 lo, cnt, bit [9] each
+constexpr uint32_t kScratchTmpl = kScratchMeta + 112;                   // u32 [9][128] entry templates
 static_assert(kScratchCum + kNumCtx * 129 * 4 <= kScratchBytes, "scratch overlap");
-static_assert(kScratchMeta + 3 * kNumCtx * 4 <= kRingsBytes, "table-build scratch must fit the ring area");
+static_assert(3 * kNumCtx * 4 <= 112, "scratch overlap");
+static_assert(kScratchTmpl + kNumCtx * 128 * 4 <= kRingsBytes, "table-build scratch must fit the ring area");
 
 // Words one round can take: 8 positions x 32 lanes, one refill each, plus as many ESC words.
 constexpr uint32_t kRoundWords = 8 * 32;
@@ -86,7 +88,7 @@ struct Params {
     uint32_t gpr;  // groups per row, N / 8
     uint32_t T, G, NG, M;
     int r;
-    float alpha;
+    float alpha, inv_alpha;  // inv_alpha = RN(1 / alpha), computed on the host
     uint32_t off_scales, off_tables, off_offsets, off_payload, tables_len;
     uint64_t payload_bytes;
 };
@@ -116,6 +118,17 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+// (a0, a1) - k, then times c: two binary32 values per instruction (packed f32x2, sm_100).
+__device__ __forceinline__ void sub_mul_f32x2(float a0, float a1, float k, float c, float& y0, float& y1) {
+    uint64_t a, kk, cc, r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(kk) : "f"(k));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(cc) : "f"(c));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(kk));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(r), "l"(cc));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(r));
+}
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
 
@@ -127,8 +140,8 @@ __device__ __forceinline__ uint32_t mag_class(int hi, int b) {
     return m >= 2 ? 1u : 0u;
 }
 
-// The fused entry of symbol `sym` of context c, for a slot that lies `bias` past the symbol's cum.
-__device__ __forceinline__ uint32_t fused_entry(int c, int sym, uint32_t f, uint32_t bias) {
+// The fused entry of symbol `sym` of context c without its slot - cum field (bits 20-31).
+__device__ __forceinline__ uint32_t entry_template(int c, int sym, uint32_t f) {
     int b = c == 0 ? (sym >> 6) : (c <= 4 ? (c - 1) >> 1 : (c - 5) >> 1);
     int idx = sym & 63, hi = idx - 31;
     uint32_t field, cls = 0;
@@ -138,13 +151,14 @@ __device__ __forceinline__ uint32_t fused_entry(int c, int sym, uint32_t f, uint
     } else {
         field = uint32_t(4 * idx + b);                                // 2h + b/2 (parity added later)
     }
-    return (f & 0xFFFu) | (field << 12) | (cls << 19) | (bias << 20);
+    return (f & 0xFFFu) | (field << 12) | (cls << 19);
 }
 
 __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch) {
     uint32_t* cum = reinterpret_cast<uint32_t*>(scratch + kScratchCum);  // [9][129]
     uint8_t* tbytes = scratch + kScratchBytes;
     uint8_t* bucket = scratch + kScratchBucket;                          // symbol at slot 64k
+    uint32_t* tmpl = reinterpret_cast<uint32_t*>(scratch + kScratchTmpl);  // [9][128]
     uint32_t* s_lo = reinterpret_cast<uint32_t*>(scratch + kScratchMeta);
     uint32_t* s_cnt = s_lo + kNumCtx;
     uint32_t* s_bit = s_cnt + kNumCtx;
@@ -209,12 +223,13 @@ __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch)
     }
     __syncthreads();
 
-    // The symbol at every 64th slot.
+    // Entry templates, and the symbol at every 64th slot.
     for (int i = tid; i < kNumCtx * 128; i += kThreads) {
         int c = i >> 7, s = i & 127, A = c == 0 ? 128 : 64;
         if (s >= A) continue;
         const uint32_t* cc = cum + c * 129;
         uint32_t f = cc[s + 1] - cc[s];
+        tmpl[i] = entry_template(c, s, f);
         if (f) {
             uint32_t k0 = (cc[s] + 63) >> 6, k1 = (cc[s] + f + 63) >> 6;
             for (uint32_t k = k0; k < k1 && k < 64; ++k) bucket[c * 64 + k] = uint8_t(s);
@@ -222,21 +237,28 @@ __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch)
     }
     __syncthreads();
 
-    // Fused entries, 16 slots per thread. Start from the symbol of the chunk's 64-slot bucket and step
-    // past boundaries; zero-frequency symbols share their successor's cum and are skipped.
+    // Fused entries, 16 slots per thread. Start from the symbol of the chunk's 64-slot bucket. Most chunks
+    // lie inside one symbol (entry j = template + (slot0 + j - cum) << 20); the others step past each
+    // boundary, skipping zero-frequency symbols, which share their successor's cum.
     for (int i = tid; i < kNumCtx * 256; i += kThreads) {
         int c = i >> 8, A = c == 0 ? 128 : 64;
         uint32_t slot0 = uint32_t(i & 255) * 16;
         const uint32_t* cc = cum + c * 129;
+        const uint32_t* tc = tmpl + c * 128;
         int s = bucket[c * 64 + (slot0 >> 6)];
         s = s < A ? s : A - 1;
         uint32_t lo = cc[s], nb = cc[s + 1];
         uint32_t out[16];
+        if (slot0 >= lo && slot0 + 15 < nb) {
+            const uint32_t e0 = tc[s] + ((slot0 - lo) << 20);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            uint32_t slot = slot0 + j;
-            while (slot >= nb && s + 1 < A) { ++s; lo = nb; nb = cc[s + 1]; }
-            out[j] = fused_entry(c, s, nb - lo, slot - lo);
+            for (int j = 0; j < 16; ++j) out[j] = e0 + (uint32_t(j) << 20);
+        } else {
+            for (int j = 0; j < 16; ++j) {
+                uint32_t slot = slot0 + j;
+                while (slot >= nb && s + 1 < A) { ++s; lo = nb; nb = cc[s + 1]; }
+                out[j] = tc[s] + ((slot - lo) << 20);
+            }
         }
         uint4* dst = reinterpret_cast<uint4*>(tables + block_of(c) + 4 * slot0);
 #pragma unroll
@@ -299,17 +321,27 @@ struct RowCursor {
     uint32_t row, col, cached_row;
     float c_row;
 
+    // s / alpha correctly rounded: q0 = s * RN(1/alpha) corrected once with the exact residual
+    // s - alpha * q0 (Markstein). This matches IEEE division for every bf16 s >= 2^-96 with a quotient
+    // in [2^-96, 2^96] (checked exhaustively over all such s for thousands of alphas). Anything else,
+    // zero rows included, takes the IEEE division.
     __device__ __forceinline__ float scale(const Params& p, const uint16_t* scales) {
         if (row != cached_row) {
             cached_row = row;
-            float s = __uint_as_float(uint32_t(__ldg(scales + row)) << 16);
-            c_row = __fdiv_rn(s, p.alpha);
+            const float s = __uint_as_float(uint32_t(__ldg(scales + row)) << 16);
+            const float q0 = __fmul_rn(s, p.inv_alpha);
+            const float q = __fmaf_rn(__fmaf_rn(-p.alpha, q0, s), p.inv_alpha, q0);
+            c_row = (s >= 0x1p-96f && q >= 0x1p-96f && q <= 0x1p96f) ? q : __fdiv_rn(s, p.alpha);
         }
         return c_row;
     }
     __device__ __forceinline__ void advance(uint32_t gpr) {  // next round: 32 groups further
         col += 32;
-        while (col >= gpr) { col -= gpr; ++row; }
+        if (col >= gpr) {
+            col -= gpr;
+            ++row;
+            while (col >= gpr) { col -= gpr; ++row; }  // rows narrower than 32 groups
+        }
     }
 };
 
@@ -380,15 +412,18 @@ __device__ __forceinline__ void round_fast(const Params& p, uint32_t t0, const R
     // pi = 1 - (XOR of the idx parities).
     const uint32_t two_pi = (~par >> 12) & 2u;
     const float c = rc.scale(p, scales);
-    float y[8];
+    float m[8], y[8];
     int32_t z[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        float v;
-        if (i < 7) v = __uint_as_float(((e[i] >> 12) & 0x7Fu) | kHalfMagic) - (kHalfMagicF + 31.0f);
-        else v = __uint_as_float((((e[7] >> 12) & 0xFFu) | kHalfMagic) + two_pi) - (kHalfMagicF + 62.0f);
-        y[i] = __fmul_rn(v, c);
-        if constexpr (MODE == kCoords) z[i] = __float2int_rn(v * 2.0f);
+    for (int i = 0; i < 7; ++i) m[i] = __uint_as_float(((e[i] >> 12) & 0x7Fu) | kHalfMagic);  // 1.5*2^22 + idx + b/2
+    m[7] = __uint_as_float((((e[7] >> 12) & 0xFFu) | kHalfMagic) + two_pi);                  // 1.5*2^22 + 2 idx + b/2 + pi
+    // v = m - (1.5*2^22 + 31) for positions 0..6 and m - (1.5*2^22 + 62) for 7: exact; y = v * c_row.
+    m[7] -= 31.0f;  // exact: m[7] is an integer or half-integer near 1.5*2^22
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) sub_mul_f32x2(m[i], m[i + 1], kHalfMagicF + 31.0f, c, y[i], y[i + 1]);
+    if constexpr (MODE == kCoords) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) z[i] = __float2int_rn((m[i] - (kHalfMagicF + 31.0f)) * 2.0f);
     }
     store_group<MODE>(p.dst, g, y, z);
 }
@@ -516,13 +551,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
             const uint32_t n = off < span ? min(16u, span - off) : 0u;
             cp_async16(ring.base + (off & (kRingBytes - 1)), n ? src0 + c * kChunkBytes : tp, n);
         };
-        // Prologue: three chunks in flight, one commit group each.
-        uint32_t issued = 0, h0 = 0, h1 = 0, h2 = 0;
-#pragma unroll
-        for (int c = 0; c < 3; ++c) {
-            if (issued < chunks) { issue(issued); ++issued; }
-            cp_async_commit();
-            h2 = h1; h1 = h0; h0 = issued;
+
+        // Pull the first 4 KB of this warp's next tile toward L2 while this one decodes.
+        {
+            const uint32_t next = tile + kWarps * gridDim.x;
+            if (next < p.T && lane < 32) {
+                const uint64_t ns = uint64_t(__ldg(toff + next) & 0x7FFFFFFFu) * 16 + 128ull * lane;
+                if (ns < p.payload_bytes) prefetch_l2(payload + ns);
+            }
         }
 
         RowCursor rc;
@@ -531,40 +567,67 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
         rc.cached_row = 0xFFFFFFFFu;
         rc.c_row = 0.f;
         const bool simple = !(e0 >> 31) && p.r == 0;
-        const uint32_t round_bytes = 2 * ((e0 >> 31) ? kRoundWordsEsc : kRoundWords);
         const uint8_t* rawsec = tp + 128;
         const uint32_t raw_avail = tile_bytes - 128;
-
         const uint32_t R = (ng + 31) / 32;
-        for (uint32_t k = 0; k < R; ++k) {
-            // One more chunk if its ring slot is free (the chunk it replaces lies wholly behind pb).
-            if (issued < chunks && issued <= st.pb / kChunkBytes + (kRingChunks - 1)) { issue(issued); ++issued; }
+
+        if (simple && chunks <= kRingChunks) {
+            // The whole stream fits the ring: one batch of copies, then rounds with no ring bookkeeping.
+            for (uint32_t c = 0; c < chunks; ++c) issue(c);
             cp_async_commit();
-            h2 = h1; h1 = h0; h0 = issued;
-            cp_async_wait<2>();  // chunks [0, h2) have landed
-            uint32_t ready = h2 == chunks ? 0xFFFFFFFFu : h2 * kChunkBytes;
-            if (st.pb + round_bytes > ready) {
-                cp_async_wait<0>();
-                ready = issued == chunks ? 0xFFFFFFFFu : issued * kChunkBytes;
-            }
+            cp_async_wait<0>();
             __syncwarp();
             if (!waited) { grid_dependency_wait(); waited = true; }  // first store of this warp follows
-
-            const uint32_t q = 32 * k + lane, g = g0 + q;
-            const bool full = 32 * k + 32 <= ng;
-            const bool in_ring = st.pb + round_bytes <= ready;
-            if (full && in_ring) {
-                if (simple)
-                    round_fast<MODE>(p, t0, ring, scales, st, g, lt_mask, rc);
-                else
-                    round_general<MODE, false>(p, t0, ring, rawsec, raw_avail, scales, st, q, true, g, lt_mask, rc);
-            } else {
-                round_general<MODE, true>(p, t0, gwords, rawsec, raw_avail, scales, st, q, q < ng, g, lt_mask, rc);
+            const uint32_t Rf = ng / 32;
+            uint32_t g = g0 + lane;
+            for (uint32_t k = 0; k < Rf; ++k, g += 32) {
+                round_fast<MODE>(p, t0, ring, scales, st, g, lt_mask, rc);
+                rc.advance(p.gpr);
             }
-            rc.advance(p.gpr);
+            if (Rf < R) {
+                const uint32_t q = 32 * Rf + lane;
+                round_general<MODE, true>(p, t0, gwords, rawsec, raw_avail, scales, st, q, q < ng, g0 + q, lt_mask, rc);
+            }
+        } else {
+            // Rolling ring: three 512-byte chunks in flight, one more per round while the ring has room.
+            uint32_t issued = 0, h0 = 0, h1 = 0, h2 = 0;
+#pragma unroll
+            for (int c = 0; c < 3; ++c) {
+                if (issued < chunks) { issue(issued); ++issued; }
+                cp_async_commit();
+                h2 = h1; h1 = h0; h0 = issued;
+            }
+            const uint32_t round_bytes = 2 * ((e0 >> 31) ? kRoundWordsEsc : kRoundWords);
+            for (uint32_t k = 0; k < R; ++k) {
+                // One more chunk if its ring slot is free (the chunk it replaces lies wholly behind pb).
+                if (issued < chunks && issued <= st.pb / kChunkBytes + (kRingChunks - 1)) { issue(issued); ++issued; }
+                cp_async_commit();
+                h2 = h1; h1 = h0; h0 = issued;
+                cp_async_wait<2>();  // chunks [0, h2) have landed
+                uint32_t ready = h2 == chunks ? 0xFFFFFFFFu : h2 * kChunkBytes;
+                if (st.pb + round_bytes > ready) {
+                    cp_async_wait<0>();
+                    ready = issued == chunks ? 0xFFFFFFFFu : issued * kChunkBytes;
+                }
+                __syncwarp();
+                if (!waited) { grid_dependency_wait(); waited = true; }  // first store of this warp follows
+
+                const uint32_t q = 32 * k + lane, g = g0 + q;
+                const bool full = 32 * k + 32 <= ng;
+                const bool in_ring = st.pb + round_bytes <= ready;
+                if (full && in_ring) {
+                    if (simple)
+                        round_fast<MODE>(p, t0, ring, scales, st, g, lt_mask, rc);
+                    else
+                        round_general<MODE, false>(p, t0, ring, rawsec, raw_avail, scales, st, q, true, g, lt_mask, rc);
+                } else {
+                    round_general<MODE, true>(p, t0, gwords, rawsec, raw_avail, scales, st, q, q < ng, g, lt_mask, rc);
+                }
+                rc.advance(p.gpr);
+            }
+            cp_async_wait<0>();  // the ring is reused by this warp's next tile
+            __syncwarp();
         }
-        cp_async_wait<0>();  // the ring is reused by this warp's next tile
-        __syncwarp();
         const uint32_t used = st.pb - lead, cap = span - lead;  // bytes of stream read / present
         const bool ok = __all_sync(kFullMask, st.x == kRansL) && used <= cap && cap - used <= 14;
         if (!ok && lane == 0) atomicOr(&g_status, int(EP_DEV_CORRUPT_TILE));
@@ -649,6 +712,7 @@ ep_status launch_decode(const uint8_t* host_hdr, const void* dev_blob, size_t bl
     p.M = h.M;
     p.r = h.r;
     p.alpha = h.alpha;
+    p.inv_alpha = 1.0f / h.alpha;  // IEEE binary32 division: RN(1 / alpha)
     p.off_scales = h.off_scales;
     p.off_tables = h.off_tables;
     p.off_offsets = h.off_offsets;
