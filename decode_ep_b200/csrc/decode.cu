@@ -58,18 +58,17 @@ constexpr uint32_t kChunkBytes = 512;  // one 16-byte copy per lane
 constexpr uint32_t kRingChunks = kRingBytes / kChunkBytes;
 constexpr uint32_t kRingsBytes = kWarps * kRingBytes;
 
-// Dynamic shared memory: [alignment pad up to 2 KB][rings][tables]. The table-build scratch lives in
-// the ring area, which is free until decoding starts.
-constexpr uint32_t kSmemBytes = kRingBytes + kRingsBytes + kTablesBytes;
-constexpr uint32_t kScratchCum = 0;                                    // u32 [9][129]
-constexpr uint32_t kScratchBytes = 4656;                               // serialised tables, <= 2048
-constexpr uint32_t kScratchTableCap = 2048;
-constexpr uint32_t kScratchBucket = kScratchBytes + kScratchTableCap;  // u8 [9][64]
-constexpr uint32_t kScratchMeta = kScratchBucket + kNumCtx * 64;       // u32 lo, cnt, bit [9] each
-constexpr uint32_t kScratchTmpl = kScratchMeta + 112;                   // u32 [9][128] entry templates
+// Dynamic shared memory: [alignment pad up to 2 KB][rings][tables][table-build scratch]. The scratch
+// is its own region so that the first tile's stream copies can be in flight during the build.
+constexpr uint32_t kScratchCum = 0;                                      // u32 [9][129]
+constexpr uint32_t kScratchBytes = 4656;                                 // serialised tables
+constexpr uint32_t kScratchTableCap = 1024;                              // a valid blob's tables take < 1 KB
+constexpr uint32_t kScratchBucket = kScratchBytes + kScratchTableCap;    // u8 [9][64]: symbol at slot 64k
+constexpr uint32_t kScratchTmpl = kScratchBucket + kNumCtx * 64;         // u32 [9][128]: entry templates
+constexpr uint32_t kScratchSize = kScratchTmpl + kNumCtx * 128 * 4;
 static_assert(kScratchCum + kNumCtx * 129 * 4 <= kScratchBytes, "scratch overlap");
-static_assert(3 * kNumCtx * 4 <= 112, "scratch overlap");
-static_assert(kScratchTmpl + kNumCtx * 128 * 4 <= kRingsBytes, "table-build scratch must fit the ring area");
+constexpr uint32_t kSmemBytes = kRingBytes + kRingsBytes + kTablesBytes + kScratchSize;
+static_assert(kSmemBytes <= 227 * 1024, "exceeds the per-block shared memory of sm_100");
 
 // Words one round can take: 8 positions x 32 lanes, one refill each, plus as many ESC words.
 constexpr uint32_t kRoundWords = 8 * 32;
@@ -155,114 +154,95 @@ __device__ __forceinline__ uint32_t entry_template(int c, int sym, uint32_t f) {
 }
 
 __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch) {
-    uint32_t* cum = reinterpret_cast<uint32_t*>(scratch + kScratchCum);  // [9][129]
+    uint32_t* cum = reinterpret_cast<uint32_t*>(scratch + kScratchCum);    // [9][129]
     uint8_t* tbytes = scratch + kScratchBytes;
-    uint8_t* bucket = scratch + kScratchBucket;                          // symbol at slot 64k
+    uint8_t* bucket = scratch + kScratchBucket;                            // symbol at slot 64k
     uint32_t* tmpl = reinterpret_cast<uint32_t*>(scratch + kScratchTmpl);  // [9][128]
-    uint32_t* s_lo = reinterpret_cast<uint32_t*>(scratch + kScratchMeta);
-    uint32_t* s_cnt = s_lo + kNumCtx;
-    uint32_t* s_bit = s_cnt + kNumCtx;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // Stage the serialised tables (under 1 KB for valid blobs) with one coalesced pass.
+    // Stage the serialised tables with one coalesced pass.
     const uint32_t tlen = p.tables_len < kScratchTableCap ? p.tables_len : kScratchTableCap;
     const uint8_t* tb = p.blob + p.off_tables;
-    for (uint32_t i = tid; i < tlen; i += kThreads) tbytes[i] = __ldg(tb + i);
+    for (uint32_t i = tid; i < kScratchTableCap; i += kThreads) tbytes[i] = i < tlen ? __ldg(tb + i) : 0;
     for (uint32_t i = tid; i < kNumCtx * 64; i += kThreads) bucket[i] = 0;
     __syncthreads();
-    if (warp == 0) {
-        uint32_t lo = 0, cnt = 0;
-        if (lane < kNumCtx) { lo = tbytes[lane]; cnt = tbytes[kNumCtx + lane]; }
-        uint32_t bits = 12 * cnt, incl = bits;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            uint32_t v = __shfl_up_sync(kFullMask, incl, d);
-            if (lane >= d) incl += v;
-        }
-        if (lane < kNumCtx) { s_lo[lane] = lo; s_cnt[lane] = cnt; s_bit[lane] = incl - bits; }
-    }
-    __syncthreads();
 
-    // Frequencies, indexed by symbol (zero outside [lo, lo + cnt)).
-    const uint32_t bits_len = tlen > 2 * kNumCtx ? tlen - 2 * kNumCtx : 0;
-    for (int i = tid; i < kNumCtx * 128; i += kThreads) {
-        int c = i >> 7, s = i & 127, A = c == 0 ? 128 : 64;
-        uint32_t lo = s_lo[c], cnt = s_cnt[c], f = 0;
-        if (uint32_t(s) >= lo && uint32_t(s) < lo + cnt && s < A) {
-            uint32_t bit = s_bit[c] + 12 * (uint32_t(s) - lo), byte = bit >> 3, w = 0;
-#pragma unroll
-            for (int k = 0; k < 3; ++k)
-                if (byte + k < bits_len) w |= uint32_t(tbytes[2 * kNumCtx + byte + k]) << (8 * k);
-            f = (w >> (bit & 7)) & 0xFFFu;
-        }
-        cum[c * 129 + s] = f;
-    }
-    __syncthreads();
-
-    // Exclusive prefix sums, one warp per context (4 symbols per lane).
+    // One warp per context: unpack the 12-bit frequencies (4 symbols per lane), prefix-sum them,
+    // write cum, the entry templates and the symbol at every 64th slot.
     if (warp < kNumCtx) {
-        uint32_t* cc = cum + warp * 129;
-        uint32_t f0 = cc[4 * lane], f1 = cc[4 * lane + 1], f2 = cc[4 * lane + 2], f3 = cc[4 * lane + 3];
-        uint32_t sum = f0 + f1 + f2 + f3, incl = sum;
+        const int c = warp, A = c == 0 ? 128 : 64;
+        const uint32_t lo = tbytes[c], cnt = tbytes[kNumCtx + c];
+        uint32_t bit0 = 0;
+        for (int k = 0; k < c; ++k) bit0 += 12 * tbytes[kNumCtx + k];
+        const uint32_t bits_len = tlen > 2 * kNumCtx ? tlen - 2 * kNumCtx : 0;
+        uint32_t f[4], sum = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t sym = 4 * lane + j;
+            f[j] = 0;
+            if (sym >= lo && sym < lo + cnt && int(sym) < A) {
+                const uint32_t bit = bit0 + 12 * (sym - lo), byte = bit >> 3;
+                uint32_t w = 0;
+#pragma unroll
+                for (int k = 0; k < 3; ++k)
+                    if (byte + k < bits_len) w |= uint32_t(tbytes[2 * kNumCtx + byte + k]) << (8 * k);
+                f[j] = (w >> (bit & 7)) & 0xFFFu;
+            }
+            sum += f[j];
+        }
+        uint32_t incl = sum;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
-            uint32_t v = __shfl_up_sync(kFullMask, incl, d);
+            const uint32_t v = __shfl_up_sync(kFullMask, incl, d);
             if (lane >= d) incl += v;
         }
-        uint32_t ex = incl - sum;
-        __syncwarp();
-        cc[4 * lane] = ex;
-        cc[4 * lane + 1] = ex + f0;
-        cc[4 * lane + 2] = ex + f0 + f1;
-        cc[4 * lane + 3] = ex + f0 + f1 + f2;
+        uint32_t acc = incl - sum;
+        uint32_t* cc = cum + c * 129;
+        for (int j = 0; j < 4; ++j) {
+            const int sym = 4 * lane + j;
+            cc[sym] = acc;
+            tmpl[c * 128 + sym] = entry_template(c, sym, f[j]);
+            if (f[j]) {
+                const uint32_t k0 = (acc + 63) >> 6, k1 = (acc + f[j] + 63) >> 6;
+                for (uint32_t k = k0; k < k1 && k < 64; ++k) bucket[c * 64 + k] = uint8_t(sym);
+            }
+            acc += f[j];
+        }
         if (lane == 31) {
             cc[128] = incl;
-            bool ok = s_cnt[warp] == 0 ? incl == 0 : (incl == kProbScale && s_cnt[warp] >= 2);
+            const bool ok = cnt == 0 ? incl == 0 : (incl == kProbScale && cnt >= 2);
             if (!ok && blockIdx.x == 0) atomicOr(&g_status, int(EP_DEV_BAD_TABLES));
         }
     }
     __syncthreads();
 
-    // Entry templates, and the symbol at every 64th slot.
-    for (int i = tid; i < kNumCtx * 128; i += kThreads) {
-        int c = i >> 7, s = i & 127, A = c == 0 ? 128 : 64;
-        if (s >= A) continue;
-        const uint32_t* cc = cum + c * 129;
-        uint32_t f = cc[s + 1] - cc[s];
-        tmpl[i] = entry_template(c, s, f);
-        if (f) {
-            uint32_t k0 = (cc[s] + 63) >> 6, k1 = (cc[s] + f + 63) >> 6;
-            for (uint32_t k = k0; k < k1 && k < 64; ++k) bucket[c * 64 + k] = uint8_t(s);
-        }
-    }
-    __syncthreads();
-
-    // Fused entries, 16 slots per thread. Start from the symbol of the chunk's 64-slot bucket. Most chunks
-    // lie inside one symbol (entry j = template + (slot0 + j - cum) << 20); the others step past each
-    // boundary, skipping zero-frequency symbols, which share their successor's cum.
-    for (int i = tid; i < kNumCtx * 256; i += kThreads) {
-        int c = i >> 8, A = c == 0 ? 128 : 64;
-        uint32_t slot0 = uint32_t(i & 255) * 16;
+    // Fused entries, 4 slots per thread. Consecutive threads fill consecutive slots, so a warp's
+    // 16-byte stores cover 512 contiguous bytes with no bank conflict. Each thread starts from the
+    // symbol of its 64-slot bucket. Most chunks lie inside one symbol:
+    // entry j = template + (slot0 + j - cum) << 20. The rest step past each boundary and skip
+    // zero-frequency symbols, which share their successor's cum.
+    for (int i = tid; i < kNumCtx * 1024; i += kThreads) {
+        const int c = i >> 10, A = c == 0 ? 128 : 64;
+        const uint32_t slot0 = uint32_t(i & 1023) * 4;
         const uint32_t* cc = cum + c * 129;
         const uint32_t* tc = tmpl + c * 128;
         int s = bucket[c * 64 + (slot0 >> 6)];
         s = s < A ? s : A - 1;
         uint32_t lo = cc[s], nb = cc[s + 1];
-        uint32_t out[16];
-        if (slot0 >= lo && slot0 + 15 < nb) {
-            const uint32_t e0 = tc[s] + ((slot0 - lo) << 20);
+        uint32_t out[4];
+        if (slot0 >= lo && slot0 + 3 < nb) {
+            const uint32_t e = tc[s] + ((slot0 - lo) << 20);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) out[j] = e0 + (uint32_t(j) << 20);
+            for (int j = 0; j < 4; ++j) out[j] = e + (uint32_t(j) << 20);
         } else {
-            for (int j = 0; j < 16; ++j) {
-                uint32_t slot = slot0 + j;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t slot = slot0 + j;
                 while (slot >= nb && s + 1 < A) { ++s; lo = nb; nb = cc[s + 1]; }
                 out[j] = tc[s] + ((slot - lo) << 20);
             }
         }
-        uint4* dst = reinterpret_cast<uint4*>(tables + block_of(c) + 4 * slot0);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(out[4 * j], out[4 * j + 1], out[4 * j + 2], out[4 * j + 3]);
+        *reinterpret_cast<uint4*>(tables + block_of(c) + 4 * slot0) = make_uint4(out[0], out[1], out[2], out[3]);
     }
     __syncthreads();
 }
@@ -495,6 +475,46 @@ __device__ __forceinline__ void round_general(const Params& p, uint32_t t0, cons
     store_group<MODE>(p.dst, g, y, z);
 }
 
+// ------------------------------------------------------------------------------ tiles
+
+// Geometry of one tile, from its payload offsets. Returns false when the offsets are malformed.
+struct TileGeom {
+    uint64_t start;                  // payload byte offset of the tile
+    uint32_t tile_bytes, g0, ng;     // size, first group, groups held
+    uint32_t a0, lead, span, chunks;  // ring coordinate 0 mirrors tile byte a0; the stream starts at `lead`
+    bool esc, simple, fast_fit;      // escapes present; no escapes and r = 0; simple and the stream fits the ring
+};
+
+__device__ __forceinline__ bool tile_geometry(const Params& p, const uint32_t* toff, uint32_t tile, uint32_t per_tile,
+                                              TileGeom& tg) {
+    const uint32_t e0 = __ldg(toff + tile), e1 = __ldg(toff + tile + 1);
+    const uint64_t start = uint64_t(e0 & 0x7FFFFFFFu) * 16, end = uint64_t(e1 & 0x7FFFFFFFu) * 16;
+    tg.g0 = tile * per_tile;
+    tg.ng = min(per_tile, p.NG - tg.g0);
+    const uint32_t raw = (tg.ng * uint32_t(p.r) + 3u) & ~3u;
+    if (end < start || end > p.payload_bytes || end - start < 128ull + raw || end - start > 0x7FFFFFF0ull) return false;
+    tg.start = start;
+    tg.tile_bytes = uint32_t(end - start);
+    const uint32_t s0 = 128 + raw;
+    tg.a0 = s0 & ~15u;
+    tg.lead = s0 - tg.a0;
+    tg.span = tg.tile_bytes - tg.a0;
+    tg.chunks = (tg.span + kChunkBytes - 1) / kChunkBytes;
+    tg.esc = e0 >> 31;
+    tg.simple = !tg.esc && p.r == 0;
+    tg.fast_fit = tg.simple && tg.chunks <= kRingChunks;
+    return true;
+}
+
+// Lane L's 16-byte share of ring chunk c of the tile (zero-filled past the tile's end).
+__device__ __forceinline__ void issue_chunk(const uint8_t* payload, const TileGeom& tg, uint32_t c, uint32_t ring_base,
+                                            uint32_t lane) {
+    const uint32_t off = c * kChunkBytes + 16 * lane;
+    const uint32_t n = off < tg.span ? min(16u, tg.span - off) : 0u;
+    const uint8_t* tp = payload + tg.start;
+    cp_async16(ring_base + (off & (kRingBytes - 1)), n ? tp + tg.a0 + off : tp, n);
+}
+
 // ---------------------------------------------------------------------------------- kernel
 
 template <int MODE>
@@ -505,10 +525,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
     uint8_t* smem = smem_raw + ((kRingBytes - (raw_base & (kRingBytes - 1))) & (kRingBytes - 1));
     uint8_t* rings = smem;
     uint8_t* tables = smem + kRingsBytes;
+    uint8_t* scratch = tables + kTablesBytes;
     const uint32_t t0 = smem_addr(tables);
-
-    grid_dependents_launch();  // lets the next launch of a sequence start its prologue early
-    build_tables(p, tables, rings);
 
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt_mask = (1u << lane) - 1u;
@@ -517,123 +535,131 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
     const uint8_t* payload = p.blob + p.off_payload;
     const uint32_t per_tile = 32 * p.G;
     const RingWords ring{smem_addr(rings + warp * kRingBytes)};
-    bool waited = false;
+
+    grid_dependents_launch();  // lets the next launch of a sequence start its prologue early
 
     // Tiles are dealt round-robin over the CTAs first, so that consecutive tiles land on different SMs
     // and a partial last wave is spread over the whole GPU: tile = (k * kWarps + warp) * grid + block.
-    for (uint32_t slot = warp;; slot += kWarps) {
+    // The copies of the warp's first tile are issued before the table build, which hides them.
+    uint32_t slot = warp;
+    bool first_issued = false;
+    {
+        const uint32_t tile = slot * gridDim.x + blockIdx.x;
+        if (tile < p.T) {
+            TileGeom tg;
+            if (tile_geometry(p, toff, tile, per_tile, tg) && tg.fast_fit) {
+                for (uint32_t c = 0; c < tg.chunks; ++c) issue_chunk(payload, tg, c, ring.base, lane);
+                cp_async_commit();
+                first_issued = true;
+            }
+        }
+    }
+    build_tables(p, tables, scratch);
+    grid_dependency_wait();  // stores below may overwrite what the previous launch of a sequence wrote
+
+    for (;; slot += kWarps) {
         const uint32_t tile = slot * gridDim.x + blockIdx.x;
         if (tile >= p.T) break;
-        const uint32_t e0 = __ldg(toff + tile), e1 = __ldg(toff + tile + 1);
-        const uint64_t start = uint64_t(e0 & 0x7FFFFFFFu) * 16, end = uint64_t(e1 & 0x7FFFFFFFu) * 16;
-        const uint32_t g0 = tile * per_tile;
-        const uint32_t ng = min(per_tile, p.NG - g0);
-        const uint32_t raw = (ng * uint32_t(p.r) + 3u) & ~3u;
-        if (end < start || end > p.payload_bytes || end - start < 128ull + raw || end - start > 0x7FFFFFF0ull) {
+        TileGeom tg;
+        if (!tile_geometry(p, toff, tile, per_tile, tg)) {
             if (lane == 0) atomicOr(&g_status, int(EP_DEV_BAD_OFFSETS));
+            first_issued = false;
             continue;
         }
-        const uint8_t* tp = payload + start;
-        const uint32_t tile_bytes = uint32_t(end - start);
+        const uint8_t* tp = payload + tg.start;
         TileState st;
         st.x = __ldg(reinterpret_cast<const uint32_t*>(tp) + lane);
-
-        // Ring coordinate 0 mirrors tile byte a0 (16-byte aligned); the stream starts at ring
-        // coordinate `lead`.
-        const uint32_t s0 = 128 + raw, a0 = s0 & ~15u, lead = s0 - a0;
-        const uint32_t span = tile_bytes - a0;  // ring coordinates that hold tile bytes
-        const uint32_t chunks = (span + kChunkBytes - 1) / kChunkBytes;
-        st.pb = lead;
-        const GlobalWords gwords{tp + a0, lead, span};
-        const uint8_t* src0 = tp + a0 + 16 * lane;
-        auto issue = [&](uint32_t c) {
-            const uint32_t off = c * kChunkBytes + 16 * lane;
-            const uint32_t n = off < span ? min(16u, span - off) : 0u;
-            cp_async16(ring.base + (off & (kRingBytes - 1)), n ? src0 + c * kChunkBytes : tp, n);
-        };
+        st.pb = tg.lead;
+        const GlobalWords gwords{tp + tg.a0, tg.lead, tg.span};
 
         // Pull the first 4 KB of this warp's next tile toward L2 while this one decodes.
         {
             const uint32_t next = tile + kWarps * gridDim.x;
-            if (next < p.T && lane < 32) {
+            if (next < p.T) {
                 const uint64_t ns = uint64_t(__ldg(toff + next) & 0x7FFFFFFFu) * 16 + 128ull * lane;
                 if (ns < p.payload_bytes) prefetch_l2(payload + ns);
             }
         }
 
         RowCursor rc;
-        rc.row = (g0 + lane) / p.gpr;
-        rc.col = (g0 + lane) - rc.row * p.gpr;
+        rc.row = (tg.g0 + lane) / p.gpr;
+        rc.col = (tg.g0 + lane) - rc.row * p.gpr;
         rc.cached_row = 0xFFFFFFFFu;
         rc.c_row = 0.f;
-        const bool simple = !(e0 >> 31) && p.r == 0;
         const uint8_t* rawsec = tp + 128;
-        const uint32_t raw_avail = tile_bytes - 128;
-        const uint32_t R = (ng + 31) / 32;
+        const uint32_t raw_avail = tg.tile_bytes - 128;
+        const uint32_t R = (tg.ng + 31) / 32;
 
-        if (simple && chunks <= kRingChunks) {
+        if (tg.fast_fit) {
             // The whole stream fits the ring: one batch of copies, then rounds with no ring bookkeeping.
-            for (uint32_t c = 0; c < chunks; ++c) issue(c);
-            cp_async_commit();
+            if (!first_issued) {
+                for (uint32_t c = 0; c < tg.chunks; ++c) issue_chunk(payload, tg, c, ring.base, lane);
+                cp_async_commit();
+            }
+            first_issued = false;
             cp_async_wait<0>();
             __syncwarp();
-            if (!waited) { grid_dependency_wait(); waited = true; }  // first store of this warp follows
-            const uint32_t Rf = ng / 32;
-            uint32_t g = g0 + lane;
+            const uint32_t Rf = tg.ng / 32;
+            uint32_t g = tg.g0 + lane;
             for (uint32_t k = 0; k < Rf; ++k, g += 32) {
                 round_fast<MODE>(p, t0, ring, scales, st, g, lt_mask, rc);
                 rc.advance(p.gpr);
             }
             if (Rf < R) {
                 const uint32_t q = 32 * Rf + lane;
-                round_general<MODE, true>(p, t0, gwords, rawsec, raw_avail, scales, st, q, q < ng, g0 + q, lt_mask, rc);
+                round_general<MODE, true>(p, t0, gwords, rawsec, raw_avail, scales, st, q, q < tg.ng, tg.g0 + q,
+                                          lt_mask, rc);
             }
         } else {
             // Rolling ring: three 512-byte chunks in flight, one more per round while the ring has room.
+            first_issued = false;
             uint32_t issued = 0, h0 = 0, h1 = 0, h2 = 0;
 #pragma unroll
             for (int c = 0; c < 3; ++c) {
-                if (issued < chunks) { issue(issued); ++issued; }
+                if (issued < tg.chunks) { issue_chunk(payload, tg, issued, ring.base, lane); ++issued; }
                 cp_async_commit();
                 h2 = h1; h1 = h0; h0 = issued;
             }
-            const uint32_t round_bytes = 2 * ((e0 >> 31) ? kRoundWordsEsc : kRoundWords);
+            const uint32_t round_bytes = 2 * (tg.esc ? kRoundWordsEsc : kRoundWords);
             for (uint32_t k = 0; k < R; ++k) {
                 // One more chunk if its ring slot is free (the chunk it replaces lies wholly behind pb).
-                if (issued < chunks && issued <= st.pb / kChunkBytes + (kRingChunks - 1)) { issue(issued); ++issued; }
+                if (issued < tg.chunks && issued <= st.pb / kChunkBytes + (kRingChunks - 1)) {
+                    issue_chunk(payload, tg, issued, ring.base, lane);
+                    ++issued;
+                }
                 cp_async_commit();
                 h2 = h1; h1 = h0; h0 = issued;
                 cp_async_wait<2>();  // chunks [0, h2) have landed
-                uint32_t ready = h2 == chunks ? 0xFFFFFFFFu : h2 * kChunkBytes;
+                uint32_t ready = h2 == tg.chunks ? 0xFFFFFFFFu : h2 * kChunkBytes;
                 if (st.pb + round_bytes > ready) {
                     cp_async_wait<0>();
-                    ready = issued == chunks ? 0xFFFFFFFFu : issued * kChunkBytes;
+                    ready = issued == tg.chunks ? 0xFFFFFFFFu : issued * kChunkBytes;
                 }
                 __syncwarp();
-                if (!waited) { grid_dependency_wait(); waited = true; }  // first store of this warp follows
-
-                const uint32_t q = 32 * k + lane, g = g0 + q;
-                const bool full = 32 * k + 32 <= ng;
+                const uint32_t q = 32 * k + lane, g = tg.g0 + q;
+                const bool full = 32 * k + 32 <= tg.ng;
                 const bool in_ring = st.pb + round_bytes <= ready;
                 if (full && in_ring) {
-                    if (simple)
+                    if (tg.simple)
                         round_fast<MODE>(p, t0, ring, scales, st, g, lt_mask, rc);
                     else
                         round_general<MODE, false>(p, t0, ring, rawsec, raw_avail, scales, st, q, true, g, lt_mask, rc);
                 } else {
-                    round_general<MODE, true>(p, t0, gwords, rawsec, raw_avail, scales, st, q, q < ng, g, lt_mask, rc);
+                    round_general<MODE, true>(p, t0, gwords, rawsec, raw_avail, scales, st, q, q < tg.ng, g, lt_mask,
+                                              rc);
                 }
                 rc.advance(p.gpr);
             }
             cp_async_wait<0>();  // the ring is reused by this warp's next tile
             __syncwarp();
         }
-        const uint32_t used = st.pb - lead, cap = span - lead;  // bytes of stream read / present
+        const uint32_t used = st.pb - tg.lead, cap = tg.span - tg.lead;  // bytes of stream read / present
         const bool ok = __all_sync(kFullMask, st.x == kRansL) && used <= cap && cap - used <= 14;
         if (!ok && lane == 0) atomicOr(&g_status, int(EP_DEV_CORRUPT_TILE));
     }
-    if (!waited) grid_dependency_wait();
+    if (first_issued) cp_async_wait<0>();
 }
+
 
 }  // namespace dev
 
