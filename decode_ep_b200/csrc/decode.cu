@@ -63,8 +63,7 @@ constexpr uint32_t kRingsBytes = kWarps * kRingBytes;
 constexpr uint32_t kScratchCum = 0;                                      // u32 [9][129]
 constexpr uint32_t kScratchBytes = 4656;                                 // serialised tables
 constexpr uint32_t kScratchTableCap = 1024;                              // a valid blob's tables take < 1 KB
-constexpr uint32_t kScratchBucket = kScratchBytes + kScratchTableCap;    // u8 [9][64]: symbol at slot 64k
-constexpr uint32_t kScratchTmpl = kScratchBucket + kNumCtx * 64;         // u32 [9][128]: entry templates
+constexpr uint32_t kScratchTmpl = kScratchBytes + kScratchTableCap;      // u32 [9][128]: entry templates
 constexpr uint32_t kScratchSize = kScratchTmpl + kNumCtx * 128 * 4;
 static_assert(kScratchCum + kNumCtx * 129 * 4 <= kScratchBytes, "scratch overlap");
 constexpr uint32_t kSmemBytes = kRingBytes + kRingsBytes + kTablesBytes + kScratchSize;
@@ -156,7 +155,6 @@ __device__ __forceinline__ uint32_t entry_template(int c, int sym, uint32_t f) {
 __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch) {
     uint32_t* cum = reinterpret_cast<uint32_t*>(scratch + kScratchCum);    // [9][129]
     uint8_t* tbytes = scratch + kScratchBytes;
-    uint8_t* bucket = scratch + kScratchBucket;                            // symbol at slot 64k
     uint32_t* tmpl = reinterpret_cast<uint32_t*>(scratch + kScratchTmpl);  // [9][128]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -164,11 +162,10 @@ __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch)
     const uint32_t tlen = p.tables_len < kScratchTableCap ? p.tables_len : kScratchTableCap;
     const uint8_t* tb = p.blob + p.off_tables;
     for (uint32_t i = tid; i < kScratchTableCap; i += kThreads) tbytes[i] = i < tlen ? __ldg(tb + i) : 0;
-    for (uint32_t i = tid; i < kNumCtx * 64; i += kThreads) bucket[i] = 0;
     __syncthreads();
 
     // One warp per context: unpack the 12-bit frequencies (4 symbols per lane), prefix-sum them,
-    // write cum, the entry templates and the symbol at every 64th slot.
+    // write cum and the entry templates.
     if (warp < kNumCtx) {
         const int c = warp, A = c == 0 ? 128 : 64;
         const uint32_t lo = tbytes[c], cnt = tbytes[kNumCtx + c];
@@ -202,10 +199,6 @@ __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch)
             const int sym = 4 * lane + j;
             cc[sym] = acc;
             tmpl[c * 128 + sym] = entry_template(c, sym, f[j]);
-            if (f[j]) {
-                const uint32_t k0 = (acc + 63) >> 6, k1 = (acc + f[j] + 63) >> 6;
-                for (uint32_t k = k0; k < k1 && k < 64; ++k) bucket[c * 64 + k] = uint8_t(sym);
-            }
             acc += f[j];
         }
         if (lane == 31) {
@@ -216,33 +209,54 @@ __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch)
     }
     __syncthreads();
 
-    // Fused entries, 4 slots per thread. Consecutive threads fill consecutive slots, so a warp's
-    // 16-byte stores cover 512 contiguous bytes with no bank conflict. Each thread starts from the
-    // symbol of its 64-slot bucket. Most chunks lie inside one symbol:
-    // entry j = template + (slot0 + j - cum) << 20. The rest step past each boundary and skip
-    // zero-frequency symbols, which share their successor's cum.
-    for (int i = tid; i < kNumCtx * 1024; i += kThreads) {
-        const int c = i >> 10, A = c == 0 ? 128 : 64;
-        const uint32_t slot0 = uint32_t(i & 1023) * 4;
+    // Fused entries. The 9 blocks are contiguous in memory (contexts 1..8, then START), so the tables
+    // are one run of 9 x 4096 entries. Each thread writes 36 consecutive entries (1024 x 36 = 36864).
+    // It finds the symbol at its first slot with a 7-step binary search over cum, then walks its slots
+    // with the next boundary in a register; zero-frequency symbols share their successor's cum and are
+    // stepped over. The entries go out as 16-byte stores: lane stride 144 B = 36 words, and 36 = 4
+    // (mod 32), so the 8 lanes of a quarter-warp hit all 32 banks once.
+    {
+        constexpr uint32_t kPer = kNumCtx * 4096 / kThreads;
+        static_assert(kPer * kThreads == kNumCtx * 4096 && kPer % 4 == 0, "fill geometry");
+        const uint32_t gfirst = uint32_t(tid) * kPer;
+        uint32_t blk = gfirst >> 12;                         // memory block: contexts 1..8, then START
+        int c = blk == 8 ? 0 : int(blk) + 1, A = c == 0 ? 128 : 64;
         const uint32_t* cc = cum + c * 129;
         const uint32_t* tc = tmpl + c * 128;
-        int s = bucket[c * 64 + (slot0 >> 6)];
-        s = s < A ? s : A - 1;
-        uint32_t lo = cc[s], nb = cc[s + 1];
-        uint32_t out[4];
-        if (slot0 >= lo && slot0 + 3 < nb) {
-            const uint32_t e = tc[s] + ((slot0 - lo) << 20);
+        uint32_t slot = gfirst & 4095u;
+        int s = 0;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) out[j] = e + (uint32_t(j) << 20);
-        } else {
+        for (int step = 64; step >= 1; step >>= 1)           // largest s < A with cum[s] <= slot
+            if (s + step < A && cc[s + step] <= slot) s += step;
+        uint32_t lo = cc[s], nb = cc[s + 1], tv = tc[s];
+        uint4* dst = reinterpret_cast<uint4*>(tables + 4 * gfirst);
+        for (uint32_t q = 0; q < kPer / 4; ++q) {
+            uint32_t out[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const uint32_t slot = slot0 + j;
-                while (slot >= nb && s + 1 < A) { ++s; lo = nb; nb = cc[s + 1]; }
-                out[j] = tc[s] + ((slot - lo) << 20);
+                if (slot == 4096) {                          // the run crosses into the next block
+                    ++blk;
+                    c = blk == 8 ? 0 : int(blk) + 1;
+                    A = c == 0 ? 128 : 64;
+                    cc = cum + c * 129;
+                    tc = tmpl + c * 128;
+                    slot = 0;
+                    s = 0;
+                    lo = cc[0];
+                    nb = cc[1];
+                    tv = tc[0];
+                }
+                while (slot >= nb && s + 1 < A) {
+                    ++s;
+                    lo = nb;
+                    nb = cc[s + 1];
+                    tv = tc[s];
+                }
+                out[j] = tv + ((slot - lo) << 20);
+                ++slot;
             }
+            dst[q] = make_uint4(out[0], out[1], out[2], out[3]);
         }
-        *reinterpret_cast<uint4*>(tables + block_of(c) + 4 * slot0) = make_uint4(out[0], out[1], out[2], out[3]);
     }
     __syncthreads();
 }
