@@ -66,7 +66,11 @@ constexpr uint32_t kScratchTableCap = 1024;                              // a va
 constexpr uint32_t kScratchTmpl = kScratchBytes + kScratchTableCap;      // u32 [9][128]: entry templates
 constexpr uint32_t kScratchSize = kScratchTmpl + kNumCtx * 128 * 4;
 static_assert(kScratchCum + kNumCtx * 129 * 4 <= kScratchBytes, "scratch overlap");
-constexpr uint32_t kSmemBytes = kRingBytes + kRingsBytes + kTablesBytes + kScratchSize;
+// The table region starts on a 32 KB boundary of the shared window. Every (b, position family) base is
+// then a multiple of 32 KB, and the class bit selects +16 KB with one OR. Rings fill the gap in front
+// of the tables, and the rest go after them: the request covers any starting offset.
+constexpr uint32_t kTableAlign = 32 * 1024;
+constexpr uint32_t kSmemBytes = kTablesBytes + kRingsBytes + kScratchSize + 2 * kRingBytes;
 static_assert(kSmemBytes <= 227 * 1024, "exceeds the per-block shared memory of sm_100");
 
 // Words one round can take: 8 positions x 32 lanes, one refill each, plus as many ESC words.
@@ -312,31 +316,37 @@ __device__ __forceinline__ void store_group(void* dst, uint32_t g, const float* 
 
 // Row of the lane's current group. c_row = fl32(s_row / alpha) is recomputed only when the row changes.
 struct RowCursor {
-    uint32_t row, col, cached_row;
+    uint32_t row, col;
     float c_row;
 
     // s / alpha correctly rounded: q0 = s * RN(1/alpha) corrected once with the exact residual
     // s - alpha * q0 (Markstein). This matches IEEE division for every bf16 s >= 2^-96 with a quotient
     // in [2^-96, 2^96] (checked exhaustively over all such s for thousands of alphas). Anything else,
     // zero rows included, takes the IEEE division.
-    __device__ __forceinline__ float scale(const Params& p, const uint16_t* scales) {
-        if (row != cached_row) {
-            cached_row = row;
-            const float s = __uint_as_float(uint32_t(__ldg(scales + row)) << 16);
-            const float q0 = __fmul_rn(s, p.inv_alpha);
-            const float q = __fmaf_rn(__fmaf_rn(-p.alpha, q0, s), p.inv_alpha, q0);
-            c_row = (s >= 0x1p-96f && q >= 0x1p-96f && q <= 0x1p96f) ? q : __fdiv_rn(s, p.alpha);
-        }
-        return c_row;
+    __device__ __forceinline__ void load_scale(const Params& p, const uint16_t* scales) {
+        if (row >= p.M) return;  // lanes past the last group
+        const float s = __uint_as_float(uint32_t(__ldg(scales + row)) << 16);
+        const float q0 = __fmul_rn(s, p.inv_alpha);
+        const float q = __fmaf_rn(__fmaf_rn(-p.alpha, q0, s), p.inv_alpha, q0);
+        c_row = (s >= 0x1p-96f && q >= 0x1p-96f && q <= 0x1p96f) ? q : __fdiv_rn(s, p.alpha);
     }
-    __device__ __forceinline__ void advance(uint32_t gpr) {  // next round: 32 groups further
+    __device__ __forceinline__ void start(const Params& p, const uint16_t* scales, uint32_t g) {
+        row = g / p.gpr;
+        col = g - row * p.gpr;
+        c_row = 0.f;
+        load_scale(p, scales);
+    }
+    // Next round: 32 groups further. The scale is reloaded only when the row changes.
+    __device__ __forceinline__ void advance(const Params& p, const uint16_t* scales) {
         col += 32;
-        if (col >= gpr) {
-            col -= gpr;
+        if (col >= p.gpr) {
+            col -= p.gpr;
             ++row;
-            while (col >= gpr) { col -= gpr; ++row; }  // rows narrower than 32 groups
+            while (col >= p.gpr) { col -= p.gpr; ++row; }  // rows narrower than 32 groups
+            load_scale(p, scales);
         }
     }
+    __device__ __forceinline__ float scale() const { return c_row; }
 };
 
 // The tile's u16 word stream, read either from the warp's shared ring (all but ragged rounds) or
@@ -388,15 +398,16 @@ __device__ __forceinline__ void round_fast(const Params& p, uint32_t t0, const R
     uint32_t x = st.x, pb = st.pb;
     uint32_t e[8];
     e[0] = symbol_step<false>(t0 + kStartOffset, words, x, pb, true, lt_mask);
-    const uint32_t gbase = t0 + ((e[0] << 3) & 0x8000u);  // coset bit (entry bit 12) -> block bit 15
+    const uint32_t gbase = t0 + ((e[0] << 3) & 0x8000u);  // coset bit (entry bit 12) -> +32 KB
+    const uint32_t gbase7 = gbase + kPos7Offset;
     uint32_t par = e[0];
-    uint32_t B = gbase + ((e[0] >> 5) & 0x4000u);         // class bit (entry bit 19) -> block bit 14
+    uint32_t B = gbase | ((e[0] >> 5) & 0x4000u);         // class bit (entry bit 19) -> block bit 14
 #pragma unroll
     for (int i = 1; i < 8; ++i) {
         e[i] = symbol_step<false>(B, words, x, pb, true, lt_mask);
         if (i < 7) {
             par ^= e[i];
-            B = gbase + (i == 6 ? kPos7Offset : 0u) + ((e[i] >> 5) & 0x4000u);
+            B = (i == 6 ? gbase7 : gbase) | ((e[i] >> 5) & 0x4000u);
         }
     }
     st.x = x;
@@ -405,7 +416,7 @@ __device__ __forceinline__ void round_fast(const Params& p, uint32_t t0, const R
     // Entry bit 13 is the parity of idx; u_i = idx_i - 31 flips it, and seven flips make
     // pi = 1 - (XOR of the idx parities).
     const uint32_t two_pi = (~par >> 12) & 2u;
-    const float c = rc.scale(p, scales);
+    const float c = rc.scale();
     float m[8], y[8];
     int32_t z[8];
 #pragma unroll
@@ -468,7 +479,7 @@ __device__ __forceinline__ void round_general(const Params& p, uint32_t t0, cons
             lo = int32_t(__funnelshift_r(wa, wb, sh) & ((1u << r) - 1u));
         }
         t[i] = hi * (1 << r) + lo;
-        if (i < 7) B = gbase + (i == 6 ? kPos7Offset : 0u) + ((e >> 5) & 0x4000u);
+        if (i < 7) B = (gbase + (i == 6 ? kPos7Offset : 0u)) | ((e >> 5) & 0x4000u);
     }
     st.x = x;
     st.pb = pb;
@@ -477,7 +488,7 @@ __device__ __forceinline__ void round_general(const Params& p, uint32_t t0, cons
     int32_t s7 = 0;
 #pragma unroll
     for (int i = 0; i < 7; ++i) s7 += t[i];
-    const float c = rc.scale(p, scales);
+    const float c = rc.scale();
     float y[8];
     int32_t z[8];
 #pragma unroll
@@ -536,10 +547,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // Rings must be kRingBytes-aligned in the shared window so that ring addresses are (offset | base).
     const uint32_t raw_base = smem_addr(smem_raw);
-    uint8_t* smem = smem_raw + ((kRingBytes - (raw_base & (kRingBytes - 1))) & (kRingBytes - 1));
-    uint8_t* rings = smem;
-    uint8_t* tables = smem + kRingsBytes;
-    uint8_t* scratch = tables + kTablesBytes;
+    const uint32_t tbl_pad = (kTableAlign - (raw_base & (kTableAlign - 1))) & (kTableAlign - 1);
+    uint8_t* tables = smem_raw + tbl_pad;
+    const uint32_t gap_lead = (kRingBytes - (raw_base & (kRingBytes - 1))) & (kRingBytes - 1);
+    const uint32_t gap_rings = tbl_pad >= gap_lead ? (tbl_pad - gap_lead) / kRingBytes : 0u;
+    const uint32_t rings_before = gap_rings < uint32_t(kWarps) ? gap_rings : uint32_t(kWarps);
+    uint8_t* rings_after = tables + kTablesBytes;
+    uint8_t* scratch = rings_after + (kWarps - rings_before) * kRingBytes;
     const uint32_t t0 = smem_addr(tables);
 
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -548,7 +562,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
     const uint32_t* toff = reinterpret_cast<const uint32_t*>(p.blob + p.off_offsets);
     const uint8_t* payload = p.blob + p.off_payload;
     const uint32_t per_tile = 32 * p.G;
-    const RingWords ring{smem_addr(rings + warp * kRingBytes)};
+    const RingWords ring{smem_addr(warp < rings_before ? smem_raw + gap_lead + warp * kRingBytes
+                                                       : rings_after + (warp - rings_before) * kRingBytes)};
 
     grid_dependents_launch();  // lets the next launch of a sequence start its prologue early
 
@@ -596,10 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
         }
 
         RowCursor rc;
-        rc.row = (tg.g0 + lane) / p.gpr;
-        rc.col = (tg.g0 + lane) - rc.row * p.gpr;
-        rc.cached_row = 0xFFFFFFFFu;
-        rc.c_row = 0.f;
+        rc.start(p, scales, tg.g0 + lane);
         const uint8_t* rawsec = tp + 128;
         const uint32_t raw_avail = tg.tile_bytes - 128;
         const uint32_t R = (tg.ng + 31) / 32;
@@ -617,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
             uint32_t g = tg.g0 + lane;
             for (uint32_t k = 0; k < Rf; ++k, g += 32) {
                 round_fast<MODE>(p, t0, ring, scales, st, g, lt_mask, rc);
-                rc.advance(p.gpr);
+                rc.advance(p, scales);
             }
             if (Rf < R) {
                 const uint32_t q = 32 * Rf + lane;
@@ -662,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
                     round_general<MODE, true>(p, t0, gwords, rawsec, raw_avail, scales, st, q, q < tg.ng, g, lt_mask,
                                               rc);
                 }
-                rc.advance(p.gpr);
+                rc.advance(p, scales);
             }
             cp_async_wait<0>();  // the ring is reused by this warp's next tile
             __syncwarp();
