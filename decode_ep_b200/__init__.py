@@ -92,10 +92,12 @@ class EntroPackLossyConfig:
     """Lossy EntroPack configuration (README, Config table).
 
     target_bpp: finite, in [0.001, 11]. Fractional values are allowed. It counts metadata.
-    rounds_per_tile: G. A tile is 32 lanes x G rounds x 8 coordinates (default 4096 coordinates).
+    rounds_per_tile: G. A tile is 32 lanes x G rounds x 8 coordinates. 0 (the default) means automatic:
+    16 (4096 coordinates), or, for tensors of at least half a wave of tiles on a 148-SM B200, the G in
+    [12, 24] that fills whole waves.
     """
     target_bpp: float
-    rounds_per_tile: int = 16
+    rounds_per_tile: int = 0
     sample_coords: int = 1 << 18
     bisection_iters: int = 40
     threads: int = 0

@@ -414,6 +414,19 @@ void encode_tile(const std::vector<int32_t>& tq, const std::vector<uint8_t>& bq,
     out.has_esc = has_esc;
 }
 
+// Tile rounds G for a tensor of NG groups. The decode runs one tile per warp at a time, on 148 SMs x
+// 32 warps of a B200. With fixed 16-round tiles, a tensor's last wave of tiles can be nearly empty: it
+// then runs at the latency of a lone tile. For tensors that fill at least half a wave, G is chosen in
+// [12, 24] so that the tiles fill a whole number of waves. Smaller tensors keep G = 16.
+uint32_t auto_rounds_per_tile(int64_t NG) {
+    const double slots = 148.0 * 32.0;
+    const double t16 = std::ceil(double(NG) / 512.0);
+    if (t16 < 0.5 * slots) return 16;
+    const double waves = std::max(1.0, std::floor(t16 / slots + 0.25));
+    const double g = std::ceil(double(NG) / (32.0 * slots * waves));
+    return uint32_t(std::min(24.0, std::max(12.0, g)));
+}
+
 }  // namespace
 }  // namespace epk
 
@@ -421,7 +434,7 @@ using namespace epk;
 
 extern "C" void ep_options_default(ep_options* opt) {
     if (!opt) return;
-    opt->rounds_per_tile = 16;
+    opt->rounds_per_tile = 0;  // automatic
     opt->sample_coords = 1u << 18;
     opt->bisection_iters = 40;
     opt->threads = 0;
@@ -443,6 +456,7 @@ extern "C" ep_status ep_compress(const void* data, int is_device, ep_dtype dt, i
     ep_options opt;
     ep_options_default(&opt);
     if (opt_in) opt = *opt_in;
+    if (opt.rounds_per_tile == 0) opt.rounds_per_tile = auto_rounds_per_tile(rows * cols / 8);
     if (opt.rounds_per_tile < 1 || opt.rounds_per_tile > uint32_t(kMaxG) || opt.sample_coords < 1 ||
         opt.bisection_iters > 200)
         return fail(EP_ERR_ARG, "ep_compress: bad options");

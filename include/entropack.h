@@ -66,7 +66,11 @@ typedef enum {
 
 /* Encoder options. Start from ep_options_default(). */
 typedef struct {
-    uint32_t rounds_per_tile; /* G: a tile holds 32 * G * 8 coordinates. Range 1..1024, default 16 (4096) */
+    uint32_t rounds_per_tile; /* G: a tile holds 32 * G * 8 coordinates. Range 1..1024, or 0 (the default)
+                                 for automatic: 16 (4096 coordinates) unless the tensor fills at least half a
+                                 wave of 16-round tiles on a 148-SM B200 (148 x 32 warps). It then takes the
+                                 G in [12, 24] that fills whole waves, which spares the decode a
+                                 near-empty last wave. */
     uint32_t sample_coords;   /* rate-control sample: about this many coordinates of whole rows. Default 2^18 */
     uint32_t bisection_iters; /* bisection steps on log2(alpha). Default 40 */
     int32_t threads;          /* encoder threads; 0 = all hardware threads */
