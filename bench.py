@@ -282,7 +282,7 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "u32+f32", "data": "synthetic",
         "config": {"workload": "dit276_bf16_4bpp", "layers": len(layers), "params": n_params,
                    "target_bpp": args.target_bpp, "actual_bpp": round(8 * blob_bytes / n_params, 4),
-                   "container": "bf16", "rounds_per_tile": 16, "blob_bytes": blob_bytes,
+                   "container": "bf16", "rounds_per_tile": "auto (12..24 by shape)", "blob_bytes": blob_bytes,
                    "output": f"one reused {2 * max_numel / 1e6:.1f} MB buffer",
                    "l2": "inputs larger than L2 (blobs %.2f GB read per step)" % (blob_bytes / 1e9),
                    "parallelism": f"replicas x{world}",
