@@ -6,10 +6,11 @@
 // Kernel shape: a persistent grid with one 1024-thread CTA per SM (32 warps).
 //   - Tables. Each CTA first expands the blob's 9 twelve-bit frequency tables into fused 32-bit
 //     decode entries in shared memory: 9 contexts x 4096 slots, 144 KB. One entry holds
-//       f (bits 0-11), a value field (bits 12-18 or 12-19), the magnitude class of the decoded
-//       coordinate (bit 19, which picks the next context) and slot - cum (bits 20-31).
+//       a value field (bits 0-6; 0-7 at position 7), the magnitude class of the decoded coordinate
+//       (bit 7, which picks the next context), f (bits 8-19) and slot - cum (bits 20-31).
 //     A symbol step is therefore one random 4-byte shared load and a handful of integer operations.
-//     There are no symbol, record or codebook tables.
+//     There are no symbol, record or codebook tables. The field sits at the bottom of the entry, so
+//     one AND-OR gives the value's float bits.
 //   - Tiles. Each warp decodes whole tiles. Lane L owns the groups 32k + L of the tile. After every
 //     symbol step, the lanes that must refill take the next 16-bit words of the shared stream in
 //     lane order, found with a warp ballot and a popcount prefix.
@@ -63,7 +64,7 @@ constexpr uint32_t kRingsBytes = kWarps * kRingBytes;
 constexpr uint32_t kScratchCum = 0;                                      // u32 [9][129]
 constexpr uint32_t kScratchBytes = 4656;                                 // serialised tables
 constexpr uint32_t kScratchTableCap = 1024;                              // a valid blob's tables take < 1 KB
-constexpr uint32_t kScratchTmpl = kScratchBytes + kScratchTableCap;      // u32 [9][128]: entry templates
+constexpr uint32_t kScratchTmpl = kScratchBytes + kScratchTableCap;      // u32 [9][128]: D = template - cum
 constexpr uint32_t kScratchSize = kScratchTmpl + kNumCtx * 128 * 4;
 static_assert(kScratchCum + kNumCtx * 129 * 4 <= kScratchBytes, "scratch overlap");
 // The table region starts on a 32 KB boundary of the shared window. Every (b, position family) base is
@@ -91,6 +92,9 @@ struct Params {
     uint32_t T, G, NG, M;
     int r;
     float alpha, inv_alpha;  // inv_alpha = RN(1 / alpha), computed on the host
+    // Multipliers kept out of the compiler's sight (2, 4, -4096, 128), so that the products below are
+    // issued as integer multiply-adds instead of ALU shifts: the loop saturates the ALU pipe first.
+    uint32_t k2, k4, kneg4096, k128;
     uint32_t off_scales, off_tables, off_offsets, off_payload, tables_len;
     uint64_t payload_bytes;
 };
@@ -153,23 +157,36 @@ __device__ __forceinline__ uint32_t entry_template(int c, int sym, uint32_t f) {
     } else {
         field = uint32_t(4 * idx + b);                                // 2h + b/2 (parity added later)
     }
-    return (f & 0xFFFu) | (field << 12) | (cls << 19);
+    return ((f & 0xFFFu) << 8) | (c <= 4 ? (cls << 7) | field : field);
 }
 
+// Expands the serialised tables into the fused entries. The entry of slot t in a context is
+// D[s] + (t << 20), where s is the symbol owning the slot (cum[s] <= t < cum[s] + f[s]) and
+// D[s] = template[s] - (cum[s] << 20); D is never 0, since f >= 1 sits in bits 8-19. Three passes, no
+// branching per slot:
+//   1. zero the 144 KB and stage the serialised bytes;
+//   2. one warp per context unpacks the 12-bit frequencies, prefix-sums them and drops D[s] at slot
+//      cum[s] of every symbol with f > 0 (the marker);
+//   3. each thread takes 36 consecutive entries of the 9 x 4096, starts from the marker in force at its
+//      first slot (a 7-step binary search over cum) and carries markers forward: entry = D + (slot << 20).
 __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch) {
     uint32_t* cum = reinterpret_cast<uint32_t*>(scratch + kScratchCum);    // [9][129]
     uint8_t* tbytes = scratch + kScratchBytes;
-    uint32_t* tmpl = reinterpret_cast<uint32_t*>(scratch + kScratchTmpl);  // [9][128]
+    uint32_t* dval = reinterpret_cast<uint32_t*>(scratch + kScratchTmpl);  // [9][128]: D[s]
+    uint32_t* t32 = reinterpret_cast<uint32_t*>(tables);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // Stage the serialised tables with one coalesced pass.
+    // Pass 1.
+    {
+        uint4* t4 = reinterpret_cast<uint4*>(tables);
+        for (uint32_t i = tid; i < kTablesBytes / 16; i += kThreads) t4[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
     const uint32_t tlen = p.tables_len < kScratchTableCap ? p.tables_len : kScratchTableCap;
     const uint8_t* tb = p.blob + p.off_tables;
     for (uint32_t i = tid; i < kScratchTableCap; i += kThreads) tbytes[i] = i < tlen ? __ldg(tb + i) : 0;
     __syncthreads();
 
-    // One warp per context: unpack the 12-bit frequencies (4 symbols per lane), prefix-sum them,
-    // write cum and the entry templates.
+    // Pass 2: 4 symbols per lane.
     if (warp < kNumCtx) {
         const int c = warp, A = c == 0 ? 128 : 64;
         const uint32_t lo = tbytes[c], cnt = tbytes[kNumCtx + c];
@@ -199,10 +216,13 @@ __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch)
         }
         uint32_t acc = incl - sum;
         uint32_t* cc = cum + c * 129;
+        uint32_t* block = t32 + block_of(c) / 4;
         for (int j = 0; j < 4; ++j) {
             const int sym = 4 * lane + j;
+            const uint32_t d = entry_template(c, sym, f[j]) - (acc << 20);
             cc[sym] = acc;
-            tmpl[c * 128 + sym] = entry_template(c, sym, f[j]);
+            dval[c * 128 + sym] = d;
+            if (f[j] != 0 && acc < kProbScale) block[acc] = d;
             acc += f[j];
         }
         if (lane == 31) {
@@ -213,53 +233,36 @@ __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch)
     }
     __syncthreads();
 
-    // Fused entries. The 9 blocks are contiguous in memory (contexts 1..8, then START), so the tables
-    // are one run of 9 x 4096 entries. Each thread writes 36 consecutive entries (1024 x 36 = 36864).
-    // It finds the symbol at its first slot with a 7-step binary search over cum, then walks its slots
-    // with the next boundary in a register; zero-frequency symbols share their successor's cum and are
-    // stepped over. The entries go out as 16-byte stores: lane stride 144 B = 36 words, and 36 = 4
-    // (mod 32), so the 8 lanes of a quarter-warp hit all 32 banks once.
+    // Pass 3. The 9 blocks are contiguous (contexts 1..8, then START): one run of 9 x 4096 entries.
+    // Lane stride 144 B = 36 words and 36 = 4 (mod 32), so the 8 lanes of a quarter-warp cover all 32
+    // banks once per 16-byte access.
     {
         constexpr uint32_t kPer = kNumCtx * 4096 / kThreads;
         static_assert(kPer * kThreads == kNumCtx * 4096 && kPer % 4 == 0, "fill geometry");
         const uint32_t gfirst = uint32_t(tid) * kPer;
-        uint32_t blk = gfirst >> 12;                         // memory block: contexts 1..8, then START
-        int c = blk == 8 ? 0 : int(blk) + 1, A = c == 0 ? 128 : 64;
+        const uint32_t blk = gfirst >> 12;                   // memory block: contexts 1..8, then START
+        const int c = blk == 8 ? 0 : int(blk) + 1, A = c == 0 ? 128 : 64;
         const uint32_t* cc = cum + c * 129;
-        const uint32_t* tc = tmpl + c * 128;
-        uint32_t slot = gfirst & 4095u;
+        const uint32_t slot0 = gfirst & 4095u;
         int s = 0;
 #pragma unroll
-        for (int step = 64; step >= 1; step >>= 1)           // largest s < A with cum[s] <= slot
-            if (s + step < A && cc[s + step] <= slot) s += step;
-        uint32_t lo = cc[s], nb = cc[s + 1], tv = tc[s];
-        uint4* dst = reinterpret_cast<uint4*>(tables + 4 * gfirst);
+        for (int step = 64; step >= 1; step >>= 1)           // largest s < A with cum[s] <= slot0
+            if (s + step < A && cc[s + step] <= slot0) s += step;
+        uint32_t d = dval[c * 128 + s];
+        uint4* run = reinterpret_cast<uint4*>(tables + 4 * gfirst);
+#pragma unroll 3
         for (uint32_t q = 0; q < kPer / 4; ++q) {
-            uint32_t out[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if (slot == 4096) {                          // the run crosses into the next block
-                    ++blk;
-                    c = blk == 8 ? 0 : int(blk) + 1;
-                    A = c == 0 ? 128 : 64;
-                    cc = cum + c * 129;
-                    tc = tmpl + c * 128;
-                    slot = 0;
-                    s = 0;
-                    lo = cc[0];
-                    nb = cc[1];
-                    tv = tc[0];
-                }
-                while (slot >= nb && s + 1 < A) {
-                    ++s;
-                    lo = nb;
-                    nb = cc[s + 1];
-                    tv = tc[s];
-                }
-                out[j] = tv + ((slot - lo) << 20);
-                ++slot;
-            }
-            dst[q] = make_uint4(out[0], out[1], out[2], out[3]);
+            uint4 v = run[q];
+            const uint32_t t = (gfirst + 4 * q) << 20;      // slot of v.x, in bits 20-31
+            d = v.x ? v.x : d;
+            v.x = d + t;
+            d = v.y ? v.y : d;
+            v.y = d + t + (1u << 20);
+            d = v.z ? v.z : d;
+            v.z = d + t + (2u << 20);
+            d = v.w ? v.w : d;
+            v.w = d + t + (3u << 20);
+            run[q] = v;
         }
     }
     __syncthreads();
@@ -379,7 +382,7 @@ __device__ __forceinline__ uint32_t symbol_step(uint32_t B, const Words& words, 
     uint32_t e = 0;
     if (!PARTIAL || active) {
         e = ld_shared_u32(B + ((x & (kProbScale - 1)) << 2));
-        x = (e & 0xFFFu) * (x >> kProbBits) + (e >> 20);  // f * (x >> 12) + slot - cum
+        x = ((e >> 8) & 0xFFFu) * (x >> kProbBits) + (e >> 20);  // f * (x >> 12) + slot - cum
     }
     const bool need = (!PARTIAL || active) && x < kRansL;
     const uint32_t m = __ballot_sync(kFullMask, need);
@@ -390,38 +393,54 @@ __device__ __forceinline__ uint32_t symbol_step(uint32_t B, const Words& words, 
     return e;
 }
 
-// Fast round: every lane holds a group, the tile has no escapes and no raw bits. Values come from
-// the entries' value fields.
-template <int MODE>
-__device__ __forceinline__ void round_fast(const Params& p, uint32_t t0, const RingWords& words, const uint16_t* scales,
-                                           TileState& st, uint32_t g, uint32_t lt_mask, RowCursor& rc) {
-    uint32_t x = st.x, pb = st.pb;
+// Symbol step of the fast rounds. The refill is a predicated byte permute; address arithmetic runs as
+// integer multiply-adds. WRAP = false: the whole stream sits in the warp's ring without wrapping and `pa` is the shared
+// address of the next word itself. WRAP = true: `pa` is a ring coordinate, taken modulo the ring.
+template <bool WRAP>
+__device__ __forceinline__ uint32_t symbol_step_fast(const Params& p, uint32_t B, uint32_t& x, uint32_t& pa,
+                                                     uint32_t ring_base, uint32_t lt_mask) {
+    const uint32_t q = x >> kProbBits;
+    const uint32_t e = ld_shared_u32((x + q * p.kneg4096) * p.k4 + B);  // B + 4 (x mod 4096)
+    x = ((e >> 8) & 0xFFFu) * q + (e >> 20);                     // f * (x >> 12) + slot - cum
+    const bool need = x < kRansL;
+    const uint32_t m = __ballot_sync(kFullMask, need);
+    const uint32_t wp = pa + __popc(m & lt_mask) * p.k2;
+    const uint32_t w = ld_shared_u16(WRAP ? (wp & (kRingBytes - 1)) | ring_base : wp);
+    if (need) x = __byte_perm(x, w, 0x1054u);                    // (x << 16) | w
+    pa += __popc(m) * p.k2;
+    return e;
+}
+
+// Fast round: every lane holds a group, the tile has no escapes and no raw bits, and the round's words
+// are in the ring. Values come from the entries' value fields.
+template <int MODE, bool WRAP>
+__device__ __forceinline__ void round_fast(const Params& p, uint32_t t0, uint32_t& x, uint32_t& pa, uint32_t ring_base,
+                                           uint32_t g, uint32_t lt_mask, const RowCursor& rc) {
     uint32_t e[8];
-    e[0] = symbol_step<false>(t0 + kStartOffset, words, x, pb, true, lt_mask);
-    const uint32_t gbase = t0 + ((e[0] << 3) & 0x8000u);  // coset bit (entry bit 12) -> +32 KB
+    e[0] = symbol_step_fast<WRAP>(p, t0 + kStartOffset, x, pa, ring_base, lt_mask);
+    // Entry bits 0 (coset bit b of START) and 7 (class) land on block bits 15 and 14.
+    const uint32_t gbase = t0 + ((e[0] << 15) & 0x8000u);
     const uint32_t gbase7 = gbase + kPos7Offset;
     uint32_t par = e[0];
-    uint32_t B = gbase | ((e[0] >> 5) & 0x4000u);         // class bit (entry bit 19) -> block bit 14
+    uint32_t B = gbase | ((e[0] << 7) & 0x4000u);
 #pragma unroll
     for (int i = 1; i < 8; ++i) {
-        e[i] = symbol_step<false>(B, words, x, pb, true, lt_mask);
+        e[i] = symbol_step_fast<WRAP>(p, B, x, pa, ring_base, lt_mask);
         if (i < 7) {
             par ^= e[i];
-            B = (i == 6 ? gbase7 : gbase) | ((e[i] >> 5) & 0x4000u);
+            B = (i == 6 ? gbase7 : gbase) | ((e[i] * p.k128) & 0x4000u);
         }
     }
-    st.x = x;
-    st.pb = pb;
 
-    // Entry bit 13 is the parity of idx; u_i = idx_i - 31 flips it, and seven flips make
+    // Entry bit 1 is the parity of idx; u_i = idx_i - 31 flips it, and seven flips make
     // pi = 1 - (XOR of the idx parities).
-    const uint32_t two_pi = (~par >> 12) & 2u;
+    const uint32_t two_pi = ~par & 2u;
     const float c = rc.scale();
     float m[8], y[8];
     int32_t z[8];
 #pragma unroll
-    for (int i = 0; i < 7; ++i) m[i] = __uint_as_float(((e[i] >> 12) & 0x7Fu) | kHalfMagic);  // 1.5*2^22 + idx + b/2
-    m[7] = __uint_as_float((((e[7] >> 12) & 0xFFu) | kHalfMagic) + two_pi);                  // 1.5*2^22 + 2 idx + b/2 + pi
+    for (int i = 0; i < 7; ++i) m[i] = __uint_as_float((e[i] & 0x7Fu) | kHalfMagic);         // 1.5*2^22 + idx + b/2
+    m[7] = __uint_as_float(((e[7] & 0xFFu) | kHalfMagic) + two_pi);                          // 1.5*2^22 + 2 idx + b/2 + pi
     // v = m - (1.5*2^22 + 31) for positions 0..6 and m - (1.5*2^22 + 62) for 7: exact; y = v * c_row.
     m[7] -= 31.0f;  // exact: m[7] is an integer or half-integer near 1.5*2^22
 #pragma unroll
@@ -457,8 +476,8 @@ __device__ __forceinline__ void round_general(const Params& p, uint32_t t0, cons
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const uint32_t e = symbol_step<PARTIAL>(B, words, x, pb, active, lt_mask);
-        // idx: entry bits 13-18 (field 2 idx + b) for positions 0..6, bits 14-19 (4 idx + b) for 7.
-        const uint32_t idx = i < 7 ? (e >> 13) & 63u : (e >> 14) & 63u;
+        // idx: entry bits 1-6 (field 2 idx + b) for positions 0..6, bits 2-7 (4 idx + b) for 7.
+        const uint32_t idx = i < 7 ? (e >> 1) & 63u : (e >> 2) & 63u;
         int32_t hi = int32_t(idx) - 31;
         const bool esc = (!PARTIAL || active) && idx == uint32_t(kEscIdx);
         const uint32_t me = __ballot_sync(kFullMask, esc);
@@ -468,7 +487,7 @@ __device__ __forceinline__ void round_general(const Params& p, uint32_t t0, cons
             pb += 2 * __popc(me);
         }
         if (i == 0) {
-            b = (e >> 12) & 1u;
+            b = e & 1u;
             gbase = t0 + (b << 15);
         }
         int32_t lo = 0;
@@ -479,7 +498,7 @@ __device__ __forceinline__ void round_general(const Params& p, uint32_t t0, cons
             lo = int32_t(__funnelshift_r(wa, wb, sh) & ((1u << r) - 1u));
         }
         t[i] = hi * (1 << r) + lo;
-        if (i < 7) B = (gbase + (i == 6 ? kPos7Offset : 0u)) | ((e >> 5) & 0x4000u);
+        if (i < 7) B = (gbase + (i == 6 ? kPos7Offset : 0u)) | ((e << 7) & 0x4000u);
     }
     st.x = x;
     st.pb = pb;
@@ -625,12 +644,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
             first_issued = false;
             cp_async_wait<0>();
             __syncwarp();
-            const uint32_t Rf = tg.ng / 32;
-            uint32_t g = tg.g0 + lane;
-            for (uint32_t k = 0; k < Rf; ++k, g += 32) {
-                round_fast<MODE>(p, t0, ring, scales, st, g, lt_mask, rc);
+            // pa: shared address of the next word. A valid stream ends inside the ring. A corrupt one is
+            // stopped at the first round boundary past the ring's end, so reads stay within 512 bytes of
+            // it, still inside the CTA's shared memory (the scratch region follows the last ring).
+            const uint32_t Rf = tg.ng / 32, pa_end = ring.base + kRingBytes;
+            uint32_t g = tg.g0 + lane, x = st.x, pa = ring.base + st.pb;
+            for (uint32_t k = 0; k < Rf && pa <= pa_end; ++k, g += 32) {
+                round_fast<MODE, false>(p, t0, x, pa, 0, g, lt_mask, rc);
                 rc.advance(p, scales);
             }
+            st.x = x;
+            st.pb = pa - ring.base;
             if (Rf < R) {
                 const uint32_t q = 32 * Rf + lane;
                 round_general<MODE, true>(p, t0, gwords, rawsec, raw_avail, scales, st, q, q < tg.ng, tg.g0 + q,
@@ -667,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
                 const bool in_ring = st.pb + round_bytes <= ready;
                 if (full && in_ring) {
                     if (tg.simple)
-                        round_fast<MODE>(p, t0, ring, scales, st, g, lt_mask, rc);
+                        round_fast<MODE, true>(p, t0, st.x, st.pb, ring.base, g, lt_mask, rc);
                     else
                         round_general<MODE, false>(p, t0, ring, rawsec, raw_avail, scales, st, q, true, g, lt_mask, rc);
                 } else {
@@ -765,6 +789,10 @@ ep_status launch_decode(const uint8_t* host_hdr, const void* dev_blob, size_t bl
     p.r = h.r;
     p.alpha = h.alpha;
     p.inv_alpha = 1.0f / h.alpha;  // IEEE binary32 division: RN(1 / alpha)
+    p.k2 = 2;
+    p.k4 = 4;
+    p.kneg4096 = 0xFFFFF000u;
+    p.k128 = 128;
     p.off_scales = h.off_scales;
     p.off_tables = h.off_tables;
     p.off_offsets = h.off_offsets;
