@@ -14,9 +14,10 @@
 //   - Tiles. Each warp decodes whole tiles. Lane L owns the groups 32k + L of the tile. After every
 //     symbol step, the lanes that must refill take the next 16-bit words of the shared stream in
 //     lane order, found with a warp ballot and a popcount prefix.
-//   - Stream staging. The words come from a 2 KB per-warp ring in shared memory. Asynchronous
-//     16-byte copies (cp.async, one 512-byte chunk per round, up to 3 chunks ahead) fill it, so
-//     no refill waits on DRAM.
+//   - Stream staging. The words come from a 2 KB per-warp ring in shared memory, filled by
+//     asynchronous 16-byte copies (cp.async) in 512-byte chunks, so no refill waits on DRAM. The first
+//     2 KB of a tile's stream (all of it, for most tiles at 4 bpp) land in one batch. A longer stream
+//     gets its next chunk copied into the slot that the rounds have left behind.
 //   - Values. v = hi + b/2 is rebuilt with no conversion instruction. The value field is ORed into
 //     the mantissa of 1.5 * 2^22, a float whose last-place unit is 1/2, and the bias is subtracted.
 //     Each lane then writes its 8 values with one 16-byte store (BF16/FP16), so a warp writes 512
@@ -526,7 +527,7 @@ struct TileGeom {
     uint64_t start;                  // payload byte offset of the tile
     uint32_t tile_bytes, g0, ng;     // size, first group, groups held
     uint32_t a0, lead, span, chunks;  // ring coordinate 0 mirrors tile byte a0; the stream starts at `lead`
-    bool esc, simple, fast_fit;      // escapes present; no escapes and r = 0; simple and the stream fits the ring
+    bool esc, simple;                // escapes present; no escapes and r = 0
 };
 
 __device__ __forceinline__ bool tile_geometry(const Params& p, const uint32_t* toff, uint32_t tile, uint32_t per_tile,
@@ -546,7 +547,6 @@ __device__ __forceinline__ bool tile_geometry(const Params& p, const uint32_t* t
     tg.chunks = (tg.span + kChunkBytes - 1) / kChunkBytes;
     tg.esc = e0 >> 31;
     tg.simple = !tg.esc && p.r == 0;
-    tg.fast_fit = tg.simple && tg.chunks <= kRingChunks;
     return true;
 }
 
@@ -595,8 +595,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
         const uint32_t tile = slot * gridDim.x + blockIdx.x;
         if (tile < p.T) {
             TileGeom tg;
-            if (tile_geometry(p, toff, tile, per_tile, tg) && tg.fast_fit) {
-                for (uint32_t c = 0; c < tg.chunks; ++c) issue_chunk(payload, tg, c, ring.base, lane);
+            if (tile_geometry(p, toff, tile, per_tile, tg)) {
+                const uint32_t first = min(tg.chunks, kRingChunks);
+                for (uint32_t c = 0; c < first; ++c) issue_chunk(payload, tg, c, ring.base, lane);
                 cp_async_commit();
                 first_issued = true;
             }
@@ -635,45 +636,59 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
         const uint32_t raw_avail = tg.tile_bytes - 128;
         const uint32_t R = (tg.ng + 31) / 32;
 
-        if (tg.fast_fit) {
-            // The whole stream fits the ring: one batch of copies, then rounds with no ring bookkeeping.
-            if (!first_issued) {
-                for (uint32_t c = 0; c < tg.chunks; ++c) issue_chunk(payload, tg, c, ring.base, lane);
-                cp_async_commit();
-            }
-            first_issued = false;
-            cp_async_wait<0>();
-            __syncwarp();
-            // pa: shared address of the next word. A valid stream ends inside the ring. A corrupt one is
-            // stopped at the first round boundary past the ring's end, so reads stay within 512 bytes of
-            // it, still inside the CTA's shared memory (the scratch region follows the last ring).
-            const uint32_t Rf = tg.ng / 32, pa_end = ring.base + kRingBytes;
+        // The first 2 KB of the stream (all of it for most tiles at 4 bpp) fill the ring in one batch.
+        const uint32_t first = min(tg.chunks, kRingChunks);
+        if (!first_issued) {
+            for (uint32_t c = 0; c < first; ++c) issue_chunk(payload, tg, c, ring.base, lane);
+            cp_async_commit();
+        }
+        first_issued = false;
+        cp_async_wait<0>();
+        __syncwarp();
+        uint32_t issued = first, k = 0;
+
+        if (tg.simple) {
+            // Fast rounds with no wrap: pa is the shared address of the next word. A round reads at most
+            // 512 bytes past pa. When the stream fits the ring, a valid stream ends inside it, and a corrupt
+            // one is stopped at the first round boundary past the ring's end: reads stay within 512 bytes
+            // of it, still inside the CTA's shared memory (the scratch region follows the last ring). A
+            // longer stream runs here while a round cannot reach the ring's end, and its next chunk is
+            // copied into the slot the rounds have left behind.
+            const uint32_t Rf = tg.ng / 32;
+            const uint32_t pa_lim = ring.base + (tg.chunks <= kRingChunks ? kRingBytes : kRingBytes - 2 * kRoundWords);
             uint32_t g = tg.g0 + lane, x = st.x, pa = ring.base + st.pb;
-            for (uint32_t k = 0; k < Rf && pa <= pa_end; ++k, g += 32) {
-                round_fast<MODE, false>(p, t0, x, pa, 0, g, lt_mask, rc);
-                rc.advance(p, scales);
+            if (tg.chunks <= kRingChunks) {
+                for (; k < Rf && pa <= pa_lim; ++k, g += 32) {
+                    round_fast<MODE, false>(p, t0, x, pa, 0, g, lt_mask, rc);
+                    rc.advance(p, scales);
+                }
+            } else {
+                for (; k < Rf && pa <= pa_lim; ++k, g += 32) {
+                    if (issued < tg.chunks && pa >= ring.base + (issued - (kRingChunks - 1)) * kChunkBytes) {
+                        __syncwarp();  // every lane is done reading the slot
+                        issue_chunk(payload, tg, issued, ring.base, lane);
+                        cp_async_commit();
+                        ++issued;
+                    }
+                    round_fast<MODE, false>(p, t0, x, pa, 0, g, lt_mask, rc);
+                    rc.advance(p, scales);
+                }
             }
             st.x = x;
             st.pb = pa - ring.base;
-            if (Rf < R) {
-                const uint32_t q = 32 * Rf + lane;
-                round_general<MODE, true>(p, t0, gwords, rawsec, raw_avail, scales, st, q, q < tg.ng, tg.g0 + q,
-                                          lt_mask, rc);
-            }
-        } else {
-            // Rolling ring: three 512-byte chunks in flight, one more per round while the ring has room.
-            first_issued = false;
-            uint32_t issued = 0, h0 = 0, h1 = 0, h2 = 0;
-#pragma unroll
-            for (int c = 0; c < 3; ++c) {
-                if (issued < tg.chunks) { issue_chunk(payload, tg, issued, ring.base, lane); ++issued; }
-                cp_async_commit();
-                h2 = h1; h1 = h0; h0 = issued;
-            }
+        }
+
+        if (k < R) {
+            // Rolling ring: tiles with escapes or raw bits, the last rounds of a stream longer than the
+            // ring, and the ragged last round. Up to three chunks in flight; one more per round while the
+            // chunk it replaces lies wholly behind pb.
+            cp_async_wait<0>();
+            __syncwarp();
+            uint32_t h0 = issued, h1 = issued, h2 = issued;
             const uint32_t round_bytes = 2 * (tg.esc ? kRoundWordsEsc : kRoundWords);
-            for (uint32_t k = 0; k < R; ++k) {
-                // One more chunk if its ring slot is free (the chunk it replaces lies wholly behind pb).
+            for (; k < R; ++k) {
                 if (issued < tg.chunks && issued <= st.pb / kChunkBytes + (kRingChunks - 1)) {
+                    __syncwarp();  // every lane is done reading the slot
                     issue_chunk(payload, tg, issued, ring.base, lane);
                     ++issued;
                 }
@@ -700,9 +715,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
                 }
                 rc.advance(p, scales);
             }
-            cp_async_wait<0>();  // the ring is reused by this warp's next tile
-            __syncwarp();
         }
+        cp_async_wait<0>();  // the ring is reused by this warp's next tile
+        __syncwarp();
         const uint32_t used = st.pb - tg.lead, cap = tg.span - tg.lead;  // bytes of stream read / present
         const bool ok = __all_sync(kFullMask, st.x == kRansL) && used <= cap && cap - used <= 14;
         if (!ok && lane == 0) atomicOr(&g_status, int(EP_DEV_CORRUPT_TILE));
