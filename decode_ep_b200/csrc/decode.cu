@@ -66,7 +66,8 @@ constexpr uint32_t kScratchCum = 0;                                      // u32 
 constexpr uint32_t kScratchBytes = 4656;                                 // serialised tables
 constexpr uint32_t kScratchTableCap = 1024;                              // a valid blob's tables take < 1 KB
 constexpr uint32_t kScratchTmpl = kScratchBytes + kScratchTableCap;      // u32 [9][128]: D = template - cum
-constexpr uint32_t kScratchSize = kScratchTmpl + kNumCtx * 128 * 4;
+constexpr uint32_t kScratchWsum = kScratchTmpl + kNumCtx * 128 * 4;      // u32 [32]: per-warp frequency sums
+constexpr uint32_t kScratchSize = kScratchWsum + 32 * 4;
 static_assert(kScratchCum + kNumCtx * 129 * 4 <= kScratchBytes, "scratch overlap");
 // The table region starts on a 32 KB boundary of the shared window. Every (b, position family) base is
 // then a multiple of 32 KB, and the class bit selects +16 KB with one OR. Rings fill the gap in front
@@ -166,8 +167,8 @@ __device__ __forceinline__ uint32_t entry_template(int c, int sym, uint32_t f) {
 // D[s] = template[s] - (cum[s] << 20); D is never 0, since f >= 1 sits in bits 8-19. Three passes, no
 // branching per slot:
 //   1. zero the 144 KB and stage the serialised bytes;
-//   2. one warp per context unpacks the 12-bit frequencies, prefix-sums them and drops D[s] at slot
-//      cum[s] of every symbol with f > 0 (the marker);
+//   2. one thread per symbol unpacks its 12-bit frequency; warp scans prefix-sum them into cum, and
+//      each symbol with f > 0 drops D[s] at slot cum[s] (the marker);
 //   3. each thread takes 36 consecutive entries of the 9 x 4096, starts from the marker in force at its
 //      first slot (a 7-step binary search over cum) and carries markers forward: entry = D + (slot << 20).
 __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch) {
@@ -187,47 +188,51 @@ __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch)
     for (uint32_t i = tid; i < kScratchTableCap; i += kThreads) tbytes[i] = i < tlen ? __ldg(tb + i) : 0;
     __syncthreads();
 
-    // Pass 2: 4 symbols per lane.
-    if (warp < kNumCtx) {
-        const int c = warp, A = c == 0 ? 128 : 64;
+    // Pass 2: one thread per symbol. Threads 0-127 hold START, then 64 threads (two warps) per context
+    // 1..8. A warp scan plus the sums of the context's earlier warps give cum.
+    uint32_t* wsum = reinterpret_cast<uint32_t*>(scratch + kScratchWsum);
+    const bool owner = tid < 128 + 8 * 64;
+    const int c = tid < 128 ? 0 : 1 + (tid - 128) / 64;
+    const int sym = tid < 128 ? tid : (tid - 128) & 63;
+    const int A = c == 0 ? 128 : 64;
+    uint32_t f = 0, incl = 0;
+    if (owner) {
         const uint32_t lo = tbytes[c], cnt = tbytes[kNumCtx + c];
         uint32_t bit0 = 0;
-        for (int k = 0; k < c; ++k) bit0 += 12 * tbytes[kNumCtx + k];
+#pragma unroll
+        for (int k = 0; k < kNumCtx - 1; ++k) bit0 += k < c ? 12u * tbytes[kNumCtx + k] : 0u;
         const uint32_t bits_len = tlen > 2 * kNumCtx ? tlen - 2 * kNumCtx : 0;
-        uint32_t f[4], sum = 0;
+        if (uint32_t(sym) >= lo && uint32_t(sym) < lo + cnt) {
+            const uint32_t bit = bit0 + 12 * (uint32_t(sym) - lo), byte = bit >> 3;
+            uint32_t w = 0;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t sym = 4 * lane + j;
-            f[j] = 0;
-            if (sym >= lo && sym < lo + cnt && int(sym) < A) {
-                const uint32_t bit = bit0 + 12 * (sym - lo), byte = bit >> 3;
-                uint32_t w = 0;
-#pragma unroll
-                for (int k = 0; k < 3; ++k)
-                    if (byte + k < bits_len) w |= uint32_t(tbytes[2 * kNumCtx + byte + k]) << (8 * k);
-                f[j] = (w >> (bit & 7)) & 0xFFFu;
-            }
-            sum += f[j];
+            for (int k = 0; k < 3; ++k)
+                if (byte + k < bits_len) w |= uint32_t(tbytes[2 * kNumCtx + byte + k]) << (8 * k);
+            f = (w >> (bit & 7)) & 0xFFFu;
         }
-        uint32_t incl = sum;
+        incl = f;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
             const uint32_t v = __shfl_up_sync(kFullMask, incl, d);
             if (lane >= d) incl += v;
         }
-        uint32_t acc = incl - sum;
+        if (lane == 31) wsum[warp] = incl;
+    }
+    __syncthreads();
+    if (owner) {
+        // Earlier warps of the same context: warps 0..3 hold START, warps 4+2(c-1) and 5+2(c-1) context c.
+        const int first = c == 0 ? 0 : 4 + 2 * (c - 1);
+        for (int w = first; w < warp; ++w) incl += wsum[w];
+        const uint32_t acc = incl - f;  // cum[sym]
+        const uint32_t d = entry_template(c, sym, f) - (acc << 20);
         uint32_t* cc = cum + c * 129;
-        uint32_t* block = t32 + block_of(c) / 4;
-        for (int j = 0; j < 4; ++j) {
-            const int sym = 4 * lane + j;
-            const uint32_t d = entry_template(c, sym, f[j]) - (acc << 20);
-            cc[sym] = acc;
-            dval[c * 128 + sym] = d;
-            if (f[j] != 0 && acc < kProbScale) block[acc] = d;
-            acc += f[j];
-        }
-        if (lane == 31) {
-            cc[128] = incl;
+        cc[sym] = acc;
+        dval[c * 128 + sym] = d;
+        if (f != 0 && acc < kProbScale) t32[block_of(c) / 4 + acc] = d;
+        if (sym == A - 1) {
+            cc[A] = incl;
+            if (A < 128) cc[128] = incl;
+            const uint32_t cnt = tbytes[kNumCtx + c];
             const bool ok = cnt == 0 ? incl == 0 : (incl == kProbScale && cnt >= 2);
             if (!ok && blockIdx.x == 0) atomicOr(&g_status, int(EP_DEV_BAD_TABLES));
         }
