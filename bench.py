@@ -14,6 +14,12 @@ N x params / max-over-ranks step time.
 
 --impl reference times the CPU oracle decoder on the host cores instead: a bounded sample of tiles
 from the same layers each step, with the same metric and unit. The other ranks exit without work.
+
+--workload names one of the single-tensor workloads instead (the 256x256 quick-start tensor, the
+3072x3072 lognormal-rows matrix with outliers, the 24-point bitrate sweep on a 4096x4096 Gaussian in
+BF16/FP16/FP32, and the 8192x28672 FP8 e4m3 and INT8 code matrices). Each tensor prints its own line:
+the median and best decode time with L2 flushed between steps, actual bpp, rel-L2, the roofline
+fraction, an end-to-end figure with host buffers, and the oracle's rate on all host cores and on one.
 """
 from __future__ import annotations
 
@@ -53,7 +59,11 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true",
                     help="profiling runs: skip rel-L2, the e2e pass and the CPU baseline")
-    ap.add_argument("--json-out", default="")
+    ap.add_argument("--json-out", default="", help="appends each printed JSON line to this file")
+    ap.add_argument("--workload", default="dit276_bf16_4bpp",
+                    choices=["dit276_bf16_4bpp", "quickstart256_bf16_3.5bpp", "lognormal3072_bf16_4bpp", "sweep4096",
+                             "fp8_8192x28672_5bpp", "int8_8192x28672_3bpp"],
+                    help="the default is the headline line; the others print one line per tensor")
     return ap.parse_args()
 
 
@@ -387,13 +397,15 @@ def oracle_decode_for(seconds, blobs, layers, plan, workers):
     """Decodes the planned tile runs on `workers` threads until `seconds` of wall time have passed.
     Returns (params decoded, elapsed seconds)."""
     import oracle
-    outs = {li: np.zeros(blobs[li].shape, np.uint16) for li in {p[0] for p in plan}}
+    used = {p[0] for p in plan}
+    outs = {li: np.zeros(blobs[li].shape, np.uint16) for li in used}
+    per_tile = {li: 256 * oracle.blob_info(blobs[li].blob)["G"] for li in used}  # 32 lanes x G rounds x 8
 
     def job(item):
         li, t0, t1 = item
         oracle.decode_tiles(blobs[li].blob, t0, t1, outs[li])
         _, _, M, N = layers[li]
-        return min(t1 * 4096, M * N) - t0 * 4096
+        return min(t1 * per_tile[li], M * N) - t0 * per_tile[li]
 
     done = 0
     t0 = time.perf_counter()
@@ -478,14 +490,168 @@ def run_reference(args):
     }
 
 
+# ------------------------------------------------------------------- single-tensor workloads
+
+def workload_items(name):
+    """(label, tensor factory, target bpp, rounds per tile) for the single-tensor workloads."""
+    if name == "quickstart256_bf16_3.5bpp":
+        return [("quickstart256_bf16_3.5bpp", synth.quickstart_256, 3.5, 16)]
+    if name == "lognormal3072_bf16_4bpp":
+        return [("lognormal3072_bf16_4bpp", synth.lognormal_rows_with_outliers, 4.0, 0)]
+    if name == "sweep4096":
+        return [(f"gauss4096_{c}_{t:g}bpp", (lambda c=c: synth.gaussian(4096, 4096, 2, container=c)), t, 0)
+                for c in ("bf16", "fp16", "fp32") for t in (0.5, 1.0, 2.3, 3.0, 5.0, 6.0, 8.0, 11.0)]
+    if name == "fp8_8192x28672_5bpp":
+        return [("fp8_8192x28672_5bpp", synth.fp8_codes, 5.0, 0)]
+    if name == "int8_8192x28672_3bpp":
+        return [("int8_8192x28672_3bpp", synth.int8_codes, 3.0, 0)]
+    raise SystemExit(f"unknown workload {name}")
+
+
+def oracle_rate(blob, shape, seconds, workers):
+    """Oracle decode rate (params/s) on `workers` threads over runs of 16 tiles, bounded by `seconds`."""
+    import oracle
+    info = oracle.blob_info(blob)
+    M, N, T, per = info["rows"], info["cols"], info["num_tiles"], 256 * info["G"]
+    out = np.zeros((M, N), oracle.NP_CONTAINER[info["dtype"]])
+    runs = [(t, min(T, t + 16)) for t in range(0, T, 16)]
+
+    def job(r):
+        oracle.decode_tiles(blob, r[0], r[1], out)
+        return min(r[1] * per, M * N) - r[0] * per
+
+    done, k, t0 = 0, 0, time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+        while time.perf_counter() - t0 < seconds:
+            batch = [runs[(k + j) % len(runs)] for j in range(2 * workers)]
+            k += len(batch)
+            done += sum(ex.map(job, batch))
+    return done / (time.perf_counter() - t0)
+
+
+def run_workload(args):
+    """One JSON line per tensor of a single-tensor workload. A step is one ep_decompress_into of the
+    tensor. Each timed step is bracketed by its own CUDA events, with a 256 MB write between steps that
+    flushes the 126 MB L2, so value = params / median step time."""
+    import decode_ep_b200 as ep
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    L = ep.lib()
+    stream = torch.cuda.current_stream(device)
+    sptr = stream.cuda_stream
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    peak, peak_kind = measured_hbm_peak()
+    lines = []
+    for label, make, target, G in workload_items(args.workload):
+        w = make()
+        t_enc = time.perf_counter()
+        c = ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G))
+        t_enc = time.perf_counter() - t_enc
+        M, N = c.shape
+        n_params = M * N
+        d = c.device_blob(device)
+        out = torch.empty((M, N), dtype=c.dtype, device=device)
+        out_bytes = out.numel() * out.element_size()
+
+        def launch():
+            st = L.ep_decompress_into(c.header, d.data_ptr(), len(c.blob), out.data_ptr(), out_bytes, sptr)
+            if st:
+                raise RuntimeError(L.ep_last_error().decode())
+
+        for _ in range(args.warmup):
+            launch()
+        torch.cuda.synchronize(device)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        with ClockSampler(local) as clk:
+            for a, b in evs:
+                flush.fill_(1)
+                a.record(stream)
+                launch()
+                b.record(stream)
+            torch.cuda.synchronize(device)
+        times = sorted(a.elapsed_time(b) for a, b in evs)
+        t = torch.tensor([statistics.median(times), times[0]], dtype=torch.float64, device=device)
+        if world > 1:
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        med, best = float(t[0]), float(t[1])
+        if ep.device_status(stream):
+            raise RuntimeError(f"{label}: device status set")
+        ref = w.to(device).double()
+        rel = float(((out.double() - ref) ** 2).sum().sqrt() / (ref ** 2).sum().sqrt().clamp_min(1e-300))
+        alg = len(c.blob) + out_bytes
+        achieved = alg / (med * 1e-3) / 1e9
+
+        # End to end through the C ABI with host buffers: upload, decode, read back, one stream.
+        e2e = None
+        if rank == 0:
+            hb = torch.frombuffer(bytearray(c.blob), dtype=torch.uint8).pin_memory()
+            ho = torch.empty((M, N), dtype=c.dtype).pin_memory()
+            stage = torch.empty(len(c.blob) + 256, dtype=torch.uint8, device=device)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            for rep in range(2):
+                a.record(stream)
+                for _ in range(3):
+                    stage[: hb.numel()].copy_(hb, non_blocking=True)
+                    L.ep_decompress_into(c.header, stage.data_ptr(), len(c.blob), out.data_ptr(), out_bytes, sptr)
+                    ho.copy_(out, non_blocking=True)
+                b.record(stream)
+                torch.cuda.synchronize(device)
+            ms = a.elapsed_time(b) / 3
+            e2e = {"value": round(world * n_params / (ms * 1e-3) / 1e9, 3), "unit": "Gparams/s",
+                   "h2d_bytes_per_step": len(c.blob), "d2h_bytes_per_step": out_bytes, "ms_per_step": round(ms, 4)}
+        cpu = None
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            import oracle
+            oracle.build()
+            cores = os.cpu_count() or 1
+            many = oracle_rate(c.blob, (M, N), args.cpu_seconds / 4, cores)
+            one = oracle_rate(c.blob, (M, N), args.cpu_seconds / 8, 1)
+            cpu = {"value": round(many / 1e9, 5), "unit": "Gparams/s", "cores": cores, "kind": "oracle",
+                   "single_thread_value": round(one / 1e9, 5),
+                   "sample": f"runs of 16 tiles of this blob, cycled, C oracle for {args.cpu_seconds / 4:.1f} s on "
+                             f"{cores} threads and {args.cpu_seconds / 8:.1f} s on 1"}
+        lines.append({
+            "metric": "decode Gparams/s and % of HBM roofline on 1 B200", "value": round(world * n_params / (med * 1e-3) / 1e9, 3),
+            "unit": "Gparams/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(med, 5), "best_ms": round(best, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "u32+f32", "data": "synthetic",
+            "config": {"workload": label, "shape": [M, N], "params": n_params, "container": str(c.dtype).replace("torch.", ""),
+                       "target_bpp": target, "actual_bpp": round(c.actual_bpp, 4),
+                       "rounds_per_tile": int.from_bytes(c.header[20:22], "little"),
+                       "rel_l2": round(rel, 6), "encode_s": round(t_enc, 3),
+                       "l2": "256 MB write between timed steps (L2 flushed)", "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": None, "peak_source": f"{peak_kind} copy bandwidth",
+                         "per_launch_algorithmic_bytes": alg},
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(), "gpu_launches": args.steps,
+        })
+        del ref, out, d
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return lines if rank == 0 else None
+
+
 def main():
     args = parse_args()
-    line = run_reference(args) if args.impl == "reference" else run_ours(args)
-    if line is not None:
+    if args.impl == "reference":
+        lines = [run_reference(args)]
+    elif args.workload == "dit276_bf16_4bpp":
+        lines = [run_ours(args)]
+    else:
+        lines = run_workload(args)
+    for line in lines or []:
+        if line is None:
+            continue
         s = json.dumps(line)
         print(s, flush=True)
         if args.json_out:
-            with open(args.json_out, "w") as f:
+            with open(args.json_out, "a") as f:
                 f.write(s + "\n")
 
 
