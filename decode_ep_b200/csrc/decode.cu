@@ -127,11 +127,11 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
-// (a0, a1) - k, then times c: two binary32 values per instruction (packed f32x2, sm_100).
-__device__ __forceinline__ void sub_mul_f32x2(float a0, float a1, float k, float c, float& y0, float& y1) {
+// (a0 - k0, a1 - k1), then times c: two binary32 values per instruction (packed f32x2, sm_100).
+__device__ __forceinline__ void sub_mul_f32x2(float a0, float a1, float k0, float k1, float c, float& y0, float& y1) {
     uint64_t a, kk, cc, r;
     asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
-    asm("mov.b64 %0, {%1, %1};" : "=l"(kk) : "f"(k));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(kk) : "f"(k0), "f"(k1));
     asm("mov.b64 %0, {%1, %1};" : "=l"(cc) : "f"(c));
     asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(kk));
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(r), "l"(cc));
@@ -417,11 +417,34 @@ __device__ __forceinline__ uint32_t symbol_step_fast(const Params& p, uint32_t B
     return e;
 }
 
-// Fast round: every lane holds a group, the tile has no escapes and no raw bits, and the round's words
-// are in the ring. Values come from the entries' value fields.
-template <int MODE, bool WRAP>
+// Raw low bits of group q: the r bytes at q*r of the tile's raw section, as the four aligned words that
+// cover them (zero past the section) and the bit offset of the first one.
+struct RawWindow {
+    uint32_t w[4], sh;
+    __device__ __forceinline__ void load(const uint8_t* rawsec, uint32_t raw_avail, uint32_t q, uint32_t r) {
+        const uint32_t o = q * r, a = o & ~3u;
+        sh = (o & 3u) * 8;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            w[j] = (a + 4 * j + 4 <= raw_avail) ? __ldg(reinterpret_cast<const uint32_t*>(rawsec + a) + j) : 0u;
+    }
+    // Bits [i r, i r + r) of the group's 8r-bit field, LSB first.
+    __device__ __forceinline__ uint32_t lo(int i, uint32_t r) const {
+        const uint32_t bp = uint32_t(i) * r + sh, sel = bp >> 5, s = bp & 31;
+        const uint32_t wa = sel == 0 ? w[0] : (sel == 1 ? w[1] : (sel == 2 ? w[2] : w[3]));
+        const uint32_t wb = sel == 0 ? w[1] : (sel == 1 ? w[2] : w[3]);
+        return __funnelshift_r(wa, wb, s) & ((1u << r) - 1u);
+    }
+};
+
+// Fast round: every lane holds a group, the tile has no escapes, and the round's words are in the ring.
+// Values come from the entries' value fields. RAW: the tile carries r >= 1 raw low bits per coordinate,
+// taken from `raw` (loaded a round ahead); then t = hi 2^r + lo and the parity of u_0..u_6 is that of
+// the lo's.
+template <int MODE, bool WRAP, bool RAW = false>
 __device__ __forceinline__ void round_fast(const Params& p, uint32_t t0, uint32_t& x, uint32_t& pa, uint32_t ring_base,
-                                           uint32_t g, uint32_t lt_mask, const RowCursor& rc) {
+                                           uint32_t g, uint32_t lt_mask, const RowCursor& rc,
+                                           const RawWindow* raw = nullptr) {
     uint32_t e[8];
     e[0] = symbol_step_fast<WRAP>(p, t0 + kStartOffset, x, pa, ring_base, lt_mask);
     // Entry bits 0 (coset bit b of START) and 7 (class) land on block bits 15 and 14.
@@ -438,22 +461,45 @@ __device__ __forceinline__ void round_fast(const Params& p, uint32_t t0, uint32_
         }
     }
 
-    // Entry bit 1 is the parity of idx; u_i = idx_i - 31 flips it, and seven flips make
-    // pi = 1 - (XOR of the idx parities).
-    const uint32_t two_pi = ~par & 2u;
     const float c = rc.scale();
     float m[8], y[8];
     int32_t z[8];
+    float K, K7;
+    if constexpr (!RAW) {
+        // Entry bit 1 is the parity of idx; u_i = idx_i - 31 flips it, and seven flips make
+        // pi = 1 - (XOR of the idx parities).
+        const uint32_t two_pi = ~par & 2u;
 #pragma unroll
-    for (int i = 0; i < 7; ++i) m[i] = __uint_as_float((e[i] & 0x7Fu) | kHalfMagic);         // 1.5*2^22 + idx + b/2
-    m[7] = __uint_as_float(((e[7] & 0xFFu) | kHalfMagic) + two_pi);                          // 1.5*2^22 + 2 idx + b/2 + pi
-    // v = m - (1.5*2^22 + 31) for positions 0..6 and m - (1.5*2^22 + 62) for 7: exact; y = v * c_row.
-    m[7] -= 31.0f;  // exact: m[7] is an integer or half-integer near 1.5*2^22
+        for (int i = 0; i < 7; ++i) m[i] = __uint_as_float((e[i] & 0x7Fu) | kHalfMagic);     // 1.5*2^22 + idx + b/2
+        m[7] = __uint_as_float(((e[7] & 0xFFu) | kHalfMagic) + two_pi);                      // 1.5*2^22 + 2 idx + b/2 + pi
+        // v = m - (1.5*2^22 + 31) for positions 0..6 and m - (1.5*2^22 + 62) for 7: exact.
+        K = kHalfMagicF + 31.0f;
+        K7 = kHalfMagicF + 62.0f;
+    } else {
+        // m_i = 1.5*2^22 + idx 2^r + lo + b/2 (i < 7); m_7 = 1.5*2^22 + 2 (idx 2^r + lo_7) + pi + b/2, with
+        // pi = XOR of the lo's lowest bits. v = m - (1.5*2^22 + 31 2^r) or m - (1.5*2^22 + 62 2^r): exact,
+        // since every field stays below 2^22 for r <= 12.
+        const uint32_t r = uint32_t(p.r);
+        uint32_t lpar = 0;
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) sub_mul_f32x2(m[i], m[i + 1], kHalfMagicF + 31.0f, c, y[i], y[i + 1]);
+        for (int i = 0; i < 7; ++i) {
+            const uint32_t lo = raw->lo(i, r);
+            lpar ^= lo;
+            m[i] = __uint_as_float(kHalfMagic + ((e[i] & 0x7Eu) << r) + (lo << 1) + (e[i] & 1u));
+        }
+        const uint32_t lo7 = raw->lo(7, r);
+        m[7] = __uint_as_float(kHalfMagic + ((e[7] & 0xFCu) << r) + (lo7 << 2) + ((lpar & 1u) << 1) + (e[7] & 1u));
+        const float sc = float(1u << r);
+        K = kHalfMagicF + 31.0f * sc;
+        K7 = kHalfMagicF + 62.0f * sc;
+    }
+    // y = v * c_row, two coordinates per instruction.
+#pragma unroll
+    for (int i = 0; i < 6; i += 2) sub_mul_f32x2(m[i], m[i + 1], K, K, c, y[i], y[i + 1]);
+    sub_mul_f32x2(m[6], m[7], K, K7, c, y[6], y[7]);
     if constexpr (MODE == kCoords) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) z[i] = __float2int_rn((m[i] - (kHalfMagicF + 31.0f)) * 2.0f);
+        for (int i = 0; i < 8; ++i) z[i] = __float2int_rn((m[i] - (i < 7 ? K : K7)) * 2.0f);
     }
     store_group<MODE>(p.dst, g, y, z);
 }
@@ -532,7 +578,7 @@ struct TileGeom {
     uint64_t start;                  // payload byte offset of the tile
     uint32_t tile_bytes, g0, ng;     // size, first group, groups held
     uint32_t a0, lead, span, chunks;  // ring coordinate 0 mirrors tile byte a0; the stream starts at `lead`
-    bool esc, simple;                // escapes present; no escapes and r = 0
+    bool esc, simple, raw;           // escapes present; no escapes and r = 0; no escapes and r > 0
 };
 
 __device__ __forceinline__ bool tile_geometry(const Params& p, const uint32_t* toff, uint32_t tile, uint32_t per_tile,
@@ -552,6 +598,7 @@ __device__ __forceinline__ bool tile_geometry(const Params& p, const uint32_t* t
     tg.chunks = (tg.span + kChunkBytes - 1) / kChunkBytes;
     tg.esc = e0 >> 31;
     tg.simple = !tg.esc && p.r == 0;
+    tg.raw = !tg.esc && p.r > 0;
     return true;
 }
 
@@ -562,6 +609,49 @@ __device__ __forceinline__ void issue_chunk(const uint8_t* payload, const TileGe
     const uint32_t n = off < tg.span ? min(16u, tg.span - off) : 0u;
     const uint8_t* tp = payload + tg.start;
     cp_async16(ring_base + (off & (kRingBytes - 1)), n ? tp + tg.a0 + off : tp, n);
+}
+
+// Fast rounds with no wrap, for tiles without escapes (RAW: with r >= 1 raw low bits). pa is the shared
+// address of the next word, and a round reads at most 512 bytes past it. When the stream fits the ring,
+// a valid stream ends inside it, and a corrupt one is stopped at the first round boundary past the ring's
+// end: reads stay within 512 bytes of it, still inside the CTA's shared memory (the scratch region
+// follows the last ring). A longer stream runs here while a round cannot reach the ring's end, and its
+// next chunk is copied into the slot the rounds have left behind. The raw window of the next round is
+// loaded while the current one decodes. Returns the number of rounds done.
+template <int MODE, bool RAW>
+__device__ __forceinline__ uint32_t fast_rounds(const Params& p, uint32_t t0, const TileGeom& tg, const uint8_t* payload,
+                                                uint32_t ring_base, uint32_t lane, uint32_t lt_mask,
+                                                const uint16_t* scales, RowCursor& rc, TileState& st, uint32_t& issued,
+                                                const uint8_t* rawsec, uint32_t raw_avail) {
+    const uint32_t Rf = tg.ng / 32, r = uint32_t(p.r);
+    const uint32_t pa_lim = ring_base + (tg.chunks <= kRingChunks ? kRingBytes : kRingBytes - 2 * kRoundWords);
+    uint32_t k = 0, g = tg.g0 + lane, x = st.x, pa = ring_base + st.pb;
+    RawWindow cur, nxt;
+    if (RAW) cur.load(rawsec, raw_avail, lane, r);
+    if (tg.chunks <= kRingChunks) {
+        for (; k < Rf && pa <= pa_lim; ++k, g += 32) {
+            if (RAW) nxt.load(rawsec, raw_avail, 32 * (k + 1) + lane, r);
+            round_fast<MODE, false, RAW>(p, t0, x, pa, 0, g, lt_mask, rc, &cur);
+            rc.advance(p, scales);
+            if (RAW) cur = nxt;
+        }
+    } else {
+        for (; k < Rf && pa <= pa_lim; ++k, g += 32) {
+            if (issued < tg.chunks && pa >= ring_base + (issued - (kRingChunks - 1)) * kChunkBytes) {
+                __syncwarp();  // every lane is done reading the slot
+                issue_chunk(payload, tg, issued, ring_base, lane);
+                cp_async_commit();
+                ++issued;
+            }
+            if (RAW) nxt.load(rawsec, raw_avail, 32 * (k + 1) + lane, r);
+            round_fast<MODE, false, RAW>(p, t0, x, pa, 0, g, lt_mask, rc, &cur);
+            rc.advance(p, scales);
+            if (RAW) cur = nxt;
+        }
+    }
+    st.x = x;
+    st.pb = pa - ring_base;
+    return k;
 }
 
 // ---------------------------------------------------------------------------------- kernel
@@ -652,35 +742,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
         __syncwarp();
         uint32_t issued = first, k = 0;
 
-        if (tg.simple) {
-            // Fast rounds with no wrap: pa is the shared address of the next word. A round reads at most
-            // 512 bytes past pa. When the stream fits the ring, a valid stream ends inside it, and a corrupt
-            // one is stopped at the first round boundary past the ring's end: reads stay within 512 bytes
-            // of it, still inside the CTA's shared memory (the scratch region follows the last ring). A
-            // longer stream runs here while a round cannot reach the ring's end, and its next chunk is
-            // copied into the slot the rounds have left behind.
-            const uint32_t Rf = tg.ng / 32;
-            const uint32_t pa_lim = ring.base + (tg.chunks <= kRingChunks ? kRingBytes : kRingBytes - 2 * kRoundWords);
-            uint32_t g = tg.g0 + lane, x = st.x, pa = ring.base + st.pb;
-            if (tg.chunks <= kRingChunks) {
-                for (; k < Rf && pa <= pa_lim; ++k, g += 32) {
-                    round_fast<MODE, false>(p, t0, x, pa, 0, g, lt_mask, rc);
-                    rc.advance(p, scales);
-                }
-            } else {
-                for (; k < Rf && pa <= pa_lim; ++k, g += 32) {
-                    if (issued < tg.chunks && pa >= ring.base + (issued - (kRingChunks - 1)) * kChunkBytes) {
-                        __syncwarp();  // every lane is done reading the slot
-                        issue_chunk(payload, tg, issued, ring.base, lane);
-                        cp_async_commit();
-                        ++issued;
-                    }
-                    round_fast<MODE, false>(p, t0, x, pa, 0, g, lt_mask, rc);
-                    rc.advance(p, scales);
-                }
-            }
-            st.x = x;
-            st.pb = pa - ring.base;
+        if (!tg.esc) {
+            k = tg.raw ? fast_rounds<MODE, true>(p, t0, tg, payload, ring.base, lane, lt_mask, scales, rc, st, issued,
+                                                 rawsec, raw_avail)
+                       : fast_rounds<MODE, false>(p, t0, tg, payload, ring.base, lane, lt_mask, scales, rc, st, issued,
+                                                  rawsec, raw_avail);
         }
 
         if (k < R) {
@@ -710,10 +776,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
                 const bool full = 32 * k + 32 <= tg.ng;
                 const bool in_ring = st.pb + round_bytes <= ready;
                 if (full && in_ring) {
-                    if (tg.simple)
+                    if (tg.simple) {
                         round_fast<MODE, true>(p, t0, st.x, st.pb, ring.base, g, lt_mask, rc);
-                    else
+                    } else if (!tg.esc) {
+                        RawWindow rw;
+                        rw.load(rawsec, raw_avail, q, uint32_t(p.r));
+                        round_fast<MODE, true, true>(p, t0, st.x, st.pb, ring.base, g, lt_mask, rc, &rw);
+                    } else {
                         round_general<MODE, false>(p, t0, ring, rawsec, raw_avail, scales, st, q, true, g, lt_mask, rc);
+                    }
                 } else {
                     round_general<MODE, true>(p, t0, gwords, rawsec, raw_avail, scales, st, q, q < tg.ng, g, lt_mask,
                                               rc);
