@@ -153,6 +153,21 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(rows)}
 
 
+def max_over_ranks(values, device):
+    """Element-wise maximum of `values` over the ranks of the process group (identity without one).
+    Every rank must call it at the same point, with the same number of values."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized() and torch.distributed.get_world_size() > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def weak_scaling_value(world, params_per_rank, ms_per_step):
+    """Whole-job Gparams/s when every rank decodes `params_per_rank` parameters per step and the
+    slowest rank takes `ms_per_step`."""
+    return world * params_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
 # --------------------------------------------------------------------------------- workload
 
 def layer_list(n_layers: int):
@@ -252,13 +267,11 @@ def run_ours(args):
     status = ep.device_status(stream)
     if status:
         raise RuntimeError(f"device status {status} after the timed region")
-    t = torch.tensor([ms_total], dtype=torch.float64, device=device)
+    (ms_max,) = max_over_ranks([ms_total], device)
     if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         torch.distributed.barrier()
-    ms_max = float(t.item())
     ms_per_step = ms_max / args.steps
-    value = world * n_params / (ms_per_step * 1e-3) / 1e9
+    value = weak_scaling_value(world, n_params, ms_per_step)
 
     # Roofline of the decode kernel: algorithmic bytes (blob read once + container written once)
     # over the summed per-launch event durations of one pass.
@@ -576,10 +589,7 @@ def run_workload(args):
                 b.record(stream)
             torch.cuda.synchronize(device)
         times = sorted(a.elapsed_time(b) for a, b in evs)
-        t = torch.tensor([statistics.median(times), times[0]], dtype=torch.float64, device=device)
-        if world > 1:
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        med, best = float(t[0]), float(t[1])
+        med, best = max_over_ranks([statistics.median(times), times[0]], device)
         if ep.device_status(stream):
             raise RuntimeError(f"{label}: device status set")
         ref = w.to(device).double()
@@ -617,7 +627,7 @@ def run_workload(args):
                    "sample": f"runs of 16 tiles of this blob, cycled, C oracle for {args.cpu_seconds / 4:.1f} s on "
                              f"{cores} threads and {args.cpu_seconds / 8:.1f} s on 1"}
         lines.append({
-            "metric": "decode Gparams/s and % of HBM roofline on 1 B200", "value": round(world * n_params / (med * 1e-3) / 1e9, 3),
+            "metric": "decode Gparams/s and % of HBM roofline on 1 B200", "value": round(weak_scaling_value(world, n_params, med), 3),
             "unit": "Gparams/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(med, 5), "best_ms": round(best, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "u32+f32", "data": "synthetic",
