@@ -21,11 +21,14 @@
 #include <cuda_runtime.h>
 
 #include "capi_internal.h"
+#include "encoder_common.h"
 #include "entropack.h"
 #include "epk_format.h"
 
 namespace epk {
 namespace {
+
+using namespace enc;
 
 // ------------------------------------------------------------------------------- threads
 
@@ -49,20 +52,6 @@ void parallel_for(int64_t n, int threads, const std::function<void(int64_t, int6
 }
 
 // ---------------------------------------------------------------------- number formats
-
-float bf16_bits_to_float(uint16_t h) {
-    uint32_t u = uint32_t(h) << 16;
-    float f;
-    std::memcpy(&f, &u, 4);
-    return f;
-}
-
-uint16_t float_to_bf16_rne(float f) {
-    uint32_t u;
-    std::memcpy(&u, &f, 4);
-    uint32_t rounding = 0x7FFFu + ((u >> 16) & 1u);  // ties go to the even upper half
-    return uint16_t((u + rounding) >> 16);           // inputs here are finite and non-negative
-}
 
 float half_bits_to_float(uint16_t h) {
     int e = (h >> 10) & 31, m = h & 1023;
@@ -163,86 +152,7 @@ inline void group_syms(int b, const int32_t* t, int r, uint8_t* ctx, uint8_t* sy
     }
 }
 
-int raw_bits_for(float alpha) {
-    int r = 0;
-    while (r < 12 && 8.0 * double(int64_t(1) << r) < double(alpha)) ++r;
-    return r;
-}
-
 // ------------------------------------------------------------------------------ tables
-
-using Counts = std::vector<uint64_t>;  // [17][128]
-
-// 12-bit normalisation: f = max(1, floor(4096 n_s / n)) for present symbols. The rounding gap is
-// closed at the largest frequency, or in steps of whole units when there is too much. No f exceeds
-// 4095: a single present symbol gets 4095, and its neighbour (s + 1, or s - 1 at the alphabet's
-// end) gets 1.
-void normalize(const uint64_t* cnt, int A, uint32_t* f) {
-    uint64_t total = 0;
-    int present = 0;
-    for (int s = 0; s < A; ++s) { total += cnt[s]; present += cnt[s] != 0; f[s] = 0; }
-    if (!present) return;
-    if (present == 1) {
-        for (int s = 0; s < A; ++s)
-            if (cnt[s]) { f[s] = kProbScale - 1; f[s + 1 < A ? s + 1 : s - 1] = 1; }
-        return;
-    }
-    int64_t sum = 0;
-    for (int s = 0; s < A; ++s) {
-        if (!cnt[s]) continue;
-        uint64_t q = cnt[s] * uint64_t(kProbScale) / total;
-        f[s] = q ? uint32_t(q) : 1u;
-        sum += f[s];
-    }
-    int64_t d = int64_t(kProbScale) - sum;
-    while (d) {
-        int best = -1;
-        for (int s = 0; s < A; ++s) if (f[s] && (best < 0 || f[s] > f[best])) best = s;
-        if (d > 0) { f[best] += uint32_t(d); d = 0; }
-        else {
-            int64_t take = std::min<int64_t>(-d, int64_t(f[best]) - 1);
-            f[best] -= uint32_t(take);
-            d += take;
-        }
-    }
-}
-
-struct Tables {
-    uint32_t f[kNumCtx][128];
-    uint32_t cum[kNumCtx][128];
-    int lo[kNumCtx], cnt[kNumCtx];
-    uint64_t nsym = 0;
-
-    void build(const Counts& c) {
-        nsym = 0;
-        for (int k = 0; k < kNumCtx; ++k) {
-            int A = k == 0 ? 128 : 64;
-            normalize(&c[size_t(k) * 128], A, f[k]);
-            for (int s = A; s < 128; ++s) f[k][s] = 0;
-            int first = -1, last = -1;
-            for (int s = 0; s < A; ++s) if (f[k][s]) { if (first < 0) first = s; last = s; }
-            lo[k] = first < 0 ? 0 : first;
-            cnt[k] = first < 0 ? 0 : last - first + 1;
-            nsym += uint64_t(cnt[k]);
-            uint32_t acc = 0;
-            for (int s = 0; s < 128; ++s) { cum[k][s] = acc; acc += f[k][s]; }
-        }
-    }
-    uint64_t serialized_bytes() const { return 2 * kNumCtx + (12 * nsym + 7) / 8; }
-    void serialize(uint8_t* out) const {
-        for (int k = 0; k < kNumCtx; ++k) { out[k] = uint8_t(lo[k]); out[kNumCtx + k] = uint8_t(cnt[k]); }
-        uint8_t* bits = out + 2 * kNumCtx;
-        uint64_t pos = 0;
-        for (int k = 0; k < kNumCtx; ++k)
-            for (int s = lo[k]; s < lo[k] + cnt[k]; ++s, pos += 12) {
-                uint32_t v = f[k][s];
-                uint32_t word = v << (pos & 7);  // 12 + 7 bits fit in three bytes
-                bits[pos >> 3] |= uint8_t(word);
-                bits[(pos >> 3) + 1] |= uint8_t(word >> 8);
-                if (word >> 16) bits[(pos >> 3) + 2] |= uint8_t(word >> 16);
-            }
-    }
-};
 
 // ------------------------------------------------------------------------------ encoder
 
@@ -329,20 +239,7 @@ struct Encoder {
             for (size_t k = 0; k < total.size(); ++k) total[k] += counts[size_t(th)][k];
             n_esc += esc[size_t(th)];
         }
-        Tables tab;
-        tab.build(total);
-        double bits = 0.0;
-        for (int k = 0; k < kNumCtx; ++k)
-            for (int sy = tab.lo[k]; sy < tab.lo[k] + tab.cnt[k]; ++sy) {
-                uint64_t n = total[size_t(k) * 128 + sy];
-                if (n) bits += double(n) * (12.0 - std::log2(double(tab.f[k][sy])));
-            }
-        double ng_s = double(Rs * gpr);
-        bits += 16.0 * double(n_esc) + 8.0 * double(r) * ng_s;
-        double bits_full = bits * double(NG) / ng_s;
-        double meta = double(kHeaderBytes + pad16(2 * uint64_t(M)) + pad16(tab.serialized_bytes()) +
-                             pad16(4 * (uint64_t(T) + 1)) + uint64_t(T) * (128 - 32 + 8));
-        return meta + std::ceil(bits_full / 8.0);
+        return estimate_from_counts(total, n_esc, r, Rs, gpr, NG, M, T);
     }
 };
 
@@ -412,19 +309,6 @@ void encode_tile(const std::vector<int32_t>& tq, const std::vector<uint8_t>& bq,
     size_t n = words.size();
     for (size_t i = 0; i < n; ++i) wr16(sp + 2 * i, words[n - 1 - i]);
     out.has_esc = has_esc;
-}
-
-// Tile rounds G for a tensor of NG groups. The decode runs one tile per warp at a time, on 148 SMs x
-// 32 warps of a B200. With fixed 16-round tiles, a tensor's last wave of tiles can be nearly empty: it
-// then runs at the latency of a lone tile. For tensors that fill at least half a wave, G is chosen in
-// [12, 24] so that the tiles fill a whole number of waves. Smaller tensors keep G = 16.
-uint32_t auto_rounds_per_tile(int64_t NG) {
-    const double slots = 148.0 * 32.0;
-    const double t16 = std::ceil(double(NG) / 512.0);
-    if (t16 < 0.5 * slots) return 16;
-    const double waves = std::max(1.0, std::floor(t16 / slots + 0.25));
-    const double g = std::ceil(double(NG) / (32.0 * slots * waves));
-    return uint32_t(std::min(24.0, std::max(12.0, g)));
 }
 
 }  // namespace
@@ -546,42 +430,20 @@ extern "C" ep_status ep_compress(const void* data, int is_device, ep_dtype dt, i
         for (uint32_t j = 0; j < T; ++j) start[j + 1] = start[j] + tiles[j].bytes.size();
         if (start[T] / 16 >= 0x80000000ull) return fail(EP_ERR_SHAPE, "ep_compress: payload too large");
 
-        uint64_t off_scales = kHeaderBytes;
-        uint64_t off_tables = off_scales + pad16(2 * uint64_t(rows));
-        uint64_t off_offsets = off_tables + pad16(tab.serialized_bytes());
-        uint64_t off_payload = off_offsets + pad16(4 * (uint64_t(T) + 1));
-        uint64_t total_bytes = off_payload + start[T];
-        if (off_payload > 0xFFFFFFFFull) return fail(EP_ERR_SHAPE, "ep_compress: metadata too large");
-        uint8_t* blob = static_cast<uint8_t*>(std::calloc(size_t(total_bytes), 1));
-        if (!blob) return fail(EP_ERR_NOMEM, "ep_compress: cannot allocate %llu bytes", (unsigned long long)total_bytes);
-
-        std::memcpy(blob, "EPK1", 4);
-        wr16(blob + 4, 1);
-        blob[6] = uint8_t(dt);
-        blob[7] = uint8_t(r);
-        wr32(blob + 8, uint32_t(rows));
-        wr32(blob + 12, uint32_t(cols));
-        uint32_t abits;
-        std::memcpy(&abits, &alpha, 4);
-        wr32(blob + 16, abits);
-        wr16(blob + 20, opt.rounds_per_tile);
-        blob[22] = kLanes;
-        wr32(blob + 24, T);
-        wr32(blob + 28, uint32_t(off_scales));
-        wr32(blob + 32, uint32_t(off_tables));
-        wr32(blob + 36, uint32_t(off_offsets));
-        wr32(blob + 40, uint32_t(off_payload));
-        wr64(blob + 48, total_bytes);
-        for (int64_t i = 0; i < rows; ++i) wr16(blob + off_scales + 2 * i, enc.sbits[size_t(i)]);
-        tab.serialize(blob + off_tables);
-        for (uint32_t j = 0; j < T; ++j)
-            wr32(blob + off_offsets + 4ull * j, uint32_t(start[j] / 16) | (tiles[j].has_esc ? 0x80000000u : 0u));
-        wr32(blob + off_offsets + 4ull * T, uint32_t(start[T] / 16));
+        const BlobLayout L = blob_layout(rows, tab, T, start[T]);
+        if (L.off_payload > 0xFFFFFFFFull) return fail(EP_ERR_SHAPE, "ep_compress: metadata too large");
+        uint8_t* blob = static_cast<uint8_t*>(std::calloc(size_t(L.total), 1));
+        if (!blob) return fail(EP_ERR_NOMEM, "ep_compress: cannot allocate %llu bytes", (unsigned long long)L.total);
+        std::vector<uint8_t> esc(T);
+        for (uint32_t j = 0; j < T; ++j) esc[j] = tiles[j].has_esc;
+        write_metadata(blob, L, dt, r, rows, cols, alpha, opt.rounds_per_tile, T, enc.sbits.data(), tab, start.data(),
+                       esc.data());
         parallel_for(T, threads, [&](int64_t b, int64_t e, int) {
             for (int64_t j = b; j < e; ++j)
-                std::memcpy(blob + off_payload + start[size_t(j)], tiles[size_t(j)].bytes.data(), tiles[size_t(j)].bytes.size());
+                std::memcpy(blob + L.off_payload + start[size_t(j)], tiles[size_t(j)].bytes.data(), tiles[size_t(j)].bytes.size());
         });
-        wr32(blob + 56, crc32(blob, off_payload));  // the crc field is still zero here
+        finish_crc(blob, L);
+        const uint64_t total_bytes = L.total;
 
         *blob_out = blob;
         *blob_bytes = size_t(total_bytes);
