@@ -60,6 +60,9 @@ def lib() -> ctypes.CDLL:
         L.ep_compress.argtypes = [c.c_void_p, c.c_int, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_double,
                                   c.POINTER(_Options), c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
                                   c.POINTER(c.c_double)]
+        L.ep_compress_cuda.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_double,
+                                       c.POINTER(_Options), c.c_void_p, c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
+                                       c.POINTER(c.c_double)]
         L.ep_blob_free.argtypes = [c.c_void_p]
         L.ep_blob_info.argtypes = [c.c_void_p, c.c_size_t, c.POINTER(c.c_int), c.POINTER(c.c_int64),
                                    c.POINTER(c.c_int64), c.POINTER(c.c_double)]
@@ -73,7 +76,7 @@ def lib() -> ctypes.CDLL:
         L.ep_status_string.restype = c.c_char_p
         L.ep_status_string.argtypes = [c.c_int]
         L.ep_last_error.restype = c.c_char_p
-        for name in ("ep_compress", "ep_blob_info", "ep_decompress_into", "ep_decode_coords_into", "ep_decompress",
+        for name in ("ep_compress", "ep_compress_cuda", "ep_blob_info", "ep_decompress_into", "ep_decode_coords_into", "ep_decompress",
                      "ep_get_device_status", "ep_decompress_many"):
             getattr(L, name).restype = c.c_int
         _lib = L
@@ -95,12 +98,16 @@ class EntroPackLossyConfig:
     rounds_per_tile: G. A tile is 32 lanes x G rounds x 8 coordinates. 0 (the default) means automatic:
     16 (4096 coordinates), or, for tensors of at least half a wave of tiles on a 148-SM B200, the G in
     [12, 24] that fills whole waves.
+    encoder: "host" runs the multithreaded host encoder (ep_compress; CUDA inputs are copied to the host
+    once). "cuda" runs the GPU encoder (ep_compress_cuda) on a CUDA input, on the current stream. Both
+    write the same blob bytes.
     """
     target_bpp: float
     rounds_per_tile: int = 0
     sample_coords: int = 1 << 18
     bisection_iters: int = 40
     threads: int = 0
+    encoder: str = "host"
 
     def _options(self) -> _Options:
         return _Options(self.rounds_per_tile, self.sample_coords, self.bisection_iters, self.threads)
@@ -163,7 +170,16 @@ def compress(tensor: torch.Tensor, config: EntroPackLossyConfig | float) -> Comp
     rows, cols = t.shape
     blob_p, nbytes, actual = ctypes.c_void_p(), ctypes.c_size_t(), ctypes.c_double()
     opt = config._options()
-    if t.is_cuda:
+    if config.encoder not in ("host", "cuda"):
+        raise EntroPackError(-1, f"compress: unknown encoder {config.encoder!r}")
+    if config.encoder == "cuda":
+        if not t.is_cuda:
+            raise EntroPackError(-1, "compress: the cuda encoder takes a CUDA tensor")
+        with torch.cuda.device(t.device):
+            st = lib().ep_compress_cuda(t.data_ptr(), _TORCH_TO_EP[t.dtype], rows, cols, t.stride(0),
+                                        float(config.target_bpp), ctypes.byref(opt), torch.cuda.current_stream().cuda_stream,
+                                        ctypes.byref(blob_p), ctypes.byref(nbytes), ctypes.byref(actual))
+    elif t.is_cuda:
         with torch.cuda.device(t.device):
             torch.cuda.current_stream().synchronize()
             st = lib().ep_compress(t.data_ptr(), 1, _TORCH_TO_EP[t.dtype], rows, cols, t.stride(0),

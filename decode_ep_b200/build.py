@@ -11,13 +11,16 @@ import os
 import shutil
 import subprocess
 import sys
+import tempfile
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libentropack.so")
 SOURCES = ["decode.cu", "host_encoder.cpp", "capi.cpp"]
-HEADERS = ["epk_format.h", "capi_internal.h"]
+# Compiled on their own with --fmad=false: the CUDA encoder must round every double operation alone.
+NOFMA_SOURCES = ["gpu_encoder.cu"]
+HEADERS = ["epk_format.h", "capi_internal.h", "encoder_common.h", "lattice_code.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -32,22 +35,30 @@ def stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(ROOT, "include", "entropack.h")]
+    deps = [os.path.join(CSRC, f) for f in SOURCES + NOFMA_SOURCES + HEADERS] + [os.path.join(ROOT, "include", "entropack.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not stale():
         return LIB
-    cmd = [nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-shared",
-           "-Xcompiler", "-fPIC,-ffp-contract=off,-O3",
-           "-I", os.path.join(ROOT, "include"), "-I", CSRC,
-           *[os.path.join(CSRC, f) for f in SOURCES],
-           "-o", LIB + ".tmp", "-lpthread"]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
+    common = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC,-ffp-contract=off,-O3",
+              "-I", os.path.join(ROOT, "include"), "-I", CSRC]
+    with tempfile.TemporaryDirectory() as tmp:
+        objs = []
+        for f in NOFMA_SOURCES:
+            obj = os.path.join(tmp, f + ".o")
+            cmd = [nvcc(), *common, "--fmad=false", "-c", os.path.join(CSRC, f), "-o", obj]
+            if verbose:
+                print(" ".join(cmd), file=sys.stderr)
+            subprocess.run(cmd, check=True)
+            objs.append(obj)
+        cmd = [nvcc(), *common, "-shared", *[os.path.join(CSRC, f) for f in SOURCES], *objs,
+               "-o", LIB + ".tmp", "-lpthread"]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+            print(" ".join(cmd), file=sys.stderr)
+        subprocess.run(cmd, check=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

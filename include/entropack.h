@@ -98,7 +98,29 @@ ep_status ep_compress(const void* data, int is_device, ep_dtype dt, int64_t rows
                       int64_t row_stride, double target_bpp, const ep_options* opt, uint8_t** blob,
                       size_t* blob_bytes, double* actual_bpp);
 
-/* Releases a blob returned by ep_compress. NULL is accepted. */
+/*
+ * ep_compress_cuda: the same compression run on the GPU, for a tensor already in device memory. It
+ * writes the same blob bytes as ep_compress for the same input and options: row scales, every probe
+ * of the rate-control bisection, the quantisation and the rANS tiles run as kernels, and the host
+ * fits the 12-bit tables and takes the storage estimate with the host encoder's code (paper page
+ * abstract: sampled storage estimates, independently decodable tiles).
+ *
+ * dev_data    CUDA device pointer to rows x cols elements of dtype dt; row i starts at element
+ *             i*row_stride. Read only.
+ * cuda_stream cudaStream_t for every kernel and copy; NULL means the legacy default stream. The call
+ *             synchronises this stream several times and returns when the blob is complete.
+ * opt         NULL means the defaults; opt->threads is ignored.
+ * Other arguments and the ownership of *blob as for ep_compress (release with ep_blob_free).
+ * Device scratch (about 10 bytes per parameter) comes from cudaMallocAsync on the stream and is
+ * released before the call returns.
+ * Errors: as ep_compress; EP_ERR_ARG also when dev_data is not device memory; EP_ERR_CUDA for a failed
+ *         allocation, launch or copy.
+ */
+ep_status ep_compress_cuda(const void* dev_data, ep_dtype dt, int64_t rows, int64_t cols, int64_t row_stride,
+                           double target_bpp, const ep_options* opt, void* cuda_stream, uint8_t** blob,
+                           size_t* blob_bytes, double* actual_bpp);
+
+/* Releases a blob returned by ep_compress or ep_compress_cuda. NULL is accepted. */
 void ep_blob_free(uint8_t* blob);
 
 /*
