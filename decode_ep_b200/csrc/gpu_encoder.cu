@@ -66,12 +66,14 @@ __device__ __forceinline__ uint16_t bf16_rne(float f) {
 }
 
 // Row scales: s_row = bf16(fl32(sqrt(Σ w² / N))), the sum in double and index order, then the largest
-// |w| / s over rows with s != 0. One thread per row.
+// |w| / s over rows with s != 0. A correctly rounded division is monotonic, so the largest quotient is
+// the quotient of the largest |w|: one division per row. One thread per row.
 __global__ void row_scales_kernel(Src src, int64_t M, uint16_t* sbits, float* s_out, unsigned long long* amax_bits,
                                   int* nonfinite) {
     const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= M) return;
     double acc = 0.0;
+    float wmax = 0.f;
     for (int64_t j = 0; j < src.N; ++j) {
         const float w = load_w(src, i, j);
         if (!isfinite(w)) {
@@ -79,15 +81,14 @@ __global__ void row_scales_kernel(Src src, int64_t M, uint16_t* sbits, float* s_
             return;
         }
         acc = __dadd_rn(acc, __dmul_rn(double(w), double(w)));
+        wmax = fmaxf(wmax, fabsf(w));
     }
     const float rms = __double2float_rn(__dsqrt_rn(__ddiv_rn(acc, double(src.N))));
     const uint16_t sb = bf16_rne(rms);
     const float s = __uint_as_float(uint32_t(sb) << 16);
     sbits[i] = sb;
     s_out[i] = s;
-    double m = 0.0;
-    if (s != 0.f)
-        for (int64_t j = 0; j < src.N; ++j) m = fmax(m, __ddiv_rn(fabs(double(load_w(src, i, j))), double(s)));
+    const double m = s != 0.f ? __ddiv_rn(double(wmax), double(s)) : 0.0;
     atomicMax(amax_bits, static_cast<unsigned long long>(__double_as_longlong(m)));  // m >= 0: bits order as values
 }
 
@@ -119,9 +120,22 @@ __device__ __forceinline__ void flush_hist(const unsigned int* h, unsigned long 
         if (h[k]) atomicAdd(&counts[k], static_cast<unsigned long long>(h[k]));
 }
 
-// Counts of the row sample at alpha: rows floor(k M / Rs), k < Rs, every group of each.
-__global__ void sample_counts_kernel(Src src, int64_t M, int64_t gpr, int64_t Rs, const float* s, float alpha, int r,
+// Rate-control probes evaluated in one launch: blockIdx.y picks the probe.
+constexpr int kProbeDepth = 4;                         // bisection steps resolved per launch
+constexpr int kMaxProbes = (1 << kProbeDepth) - 1;     // every midpoint those steps can visit
+struct Probes {
+    float alpha[kMaxProbes];
+    int r[kMaxProbes];
+};
+
+// Counts of the row sample at probe blockIdx.y's alpha: rows floor(k M / Rs), k < Rs, every group of
+// each. counts and n_esc_out hold one histogram and one escape count per probe.
+__global__ void sample_counts_kernel(Src src, int64_t M, int64_t gpr, int64_t Rs, const float* s, Probes pr,
                                      unsigned long long* counts, unsigned long long* n_esc_out) {
+    const float alpha = pr.alpha[blockIdx.y];
+    const int r = pr.r[blockIdx.y];
+    counts += size_t(blockIdx.y) * kHistBins;
+    n_esc_out += blockIdx.y;
     __shared__ unsigned int h[kHistBins];
     for (int k = threadIdx.x; k < kHistBins; k += blockDim.x) h[k] = 0;
     __syncthreads();
@@ -367,34 +381,57 @@ extern "C" ep_status ep_compress_cuda(const void* dev_data, ep_dtype dt, int64_t
         double amax;
         std::memcpy(&amax, &hsmall[0], 8);
 
-        // Rate control: the same bisection as the host encoder, with the sample counted on the GPU.
+        // Rate control: the same bisection as the host encoder, with the sample counted on the GPU. One
+        // launch counts the sample at every midpoint the next kProbeDepth steps can visit (the nodes of a
+        // depth-kProbeDepth subtree, heap order: child 2n+1 when the estimate fits, 2n+2 when not). The
+        // host then takes the steps one by one, estimating only the nodes on the path taken, so lo and hi
+        // follow the exact sequence of the one-probe-per-step bisection.
         const int64_t Rs = std::min<int64_t>(M, (int64_t(opt.sample_coords) + N - 1) / N);
+        DevBuf d_pcounts;
+        EPK_CUDA(d_pcounts.alloc(sizeof(unsigned long long) * (genc::kHistBins + 1) * genc::kMaxProbes, st));
+        unsigned long long* pcounts = d_pcounts.as<unsigned long long>();
+        unsigned long long* pesc = pcounts + size_t(genc::kHistBins) * genc::kMaxProbes;
+        std::vector<unsigned long long> hcounts(size_t(genc::kHistBins + 1) * genc::kMaxProbes);
         Counts counts(size_t(genc::kHistBins));
-        auto estimate = [&](float a, double& est) -> ep_status {
-            const int r = raw_bits_for(a);
-            EPK_CUDA(cudaMemsetAsync(d_counts.p, 0, sizeof(unsigned long long) * genc::kHistBins, st));
-            EPK_CUDA(cudaMemsetAsync(small + 1, 0, 8, st));
-            genc::sample_counts_kernel<<<blocks_for(Rs * gpr, 256), 256, 0, st>>>(
-                src, M, gpr, Rs, d_s.as<float>(), a, r, d_counts.as<unsigned long long>(), small + 1);
-            EPK_CUDA(cudaGetLastError());
-            unsigned long long n_esc = 0;
-            EPK_CUDA(cudaMemcpyAsync(counts.data(), d_counts.p, sizeof(unsigned long long) * genc::kHistBins,
-                                     cudaMemcpyDeviceToHost, st));
-            EPK_CUDA(cudaMemcpyAsync(&n_esc, small + 1, 8, cudaMemcpyDeviceToHost, st));
-            EPK_CUDA(cudaStreamSynchronize(st));
-            est = estimate_from_counts(counts, n_esc, r, Rs, gpr, NG, M, T);
-            return EP_OK;
-        };
         double lo = -12.0, hi = 15.0;
         if (amax > 0.0) hi = std::min(hi, 22.0 - std::log2(amax));
         if (hi < lo) hi = lo;
         const double budget = target_bpp * double(rows) * double(cols);
-        for (uint32_t it = 0; it < opt.bisection_iters; ++it) {
-            const double mid = 0.5 * (lo + hi);
-            double est = 0.0;
-            const ep_status es = estimate(float(std::exp2(mid)), est);
-            if (es != EP_OK) return es;
-            if (8.0 * est <= budget) lo = mid; else hi = mid;
+        for (uint32_t it = 0; it < opt.bisection_iters;) {
+            const int depth = int(std::min<uint32_t>(genc::kProbeDepth, opt.bisection_iters - it));
+            const int nodes = (1 << depth) - 1;
+            double nlo[genc::kMaxProbes], nhi[genc::kMaxProbes], nmid[genc::kMaxProbes];
+            genc::Probes pr;
+            nlo[0] = lo;
+            nhi[0] = hi;
+            for (int n = 0; n < nodes; ++n) {
+                nmid[n] = 0.5 * (nlo[n] + nhi[n]);
+                pr.alpha[n] = float(std::exp2(nmid[n]));
+                pr.r[n] = raw_bits_for(pr.alpha[n]);
+                if (2 * n + 2 < nodes) {
+                    nlo[2 * n + 1] = nmid[n], nhi[2 * n + 1] = nhi[n];  // the estimate fits: lo = mid
+                    nlo[2 * n + 2] = nlo[n], nhi[2 * n + 2] = nmid[n];  // it does not: hi = mid
+                }
+            }
+            EPK_CUDA(cudaMemsetAsync(pcounts, 0, sizeof(unsigned long long) * genc::kHistBins * nodes, st));
+            EPK_CUDA(cudaMemsetAsync(pesc, 0, sizeof(unsigned long long) * genc::kMaxProbes, st));
+            genc::sample_counts_kernel<<<dim3(blocks_for(Rs * gpr, 256), unsigned(nodes)), 256, 0, st>>>(
+                src, M, gpr, Rs, d_s.as<float>(), pr, pcounts, pesc);
+            EPK_CUDA(cudaGetLastError());
+            EPK_CUDA(cudaMemcpyAsync(hcounts.data(), pcounts, sizeof(unsigned long long) * genc::kHistBins * nodes,
+                                     cudaMemcpyDeviceToHost, st));
+            EPK_CUDA(cudaMemcpyAsync(hcounts.data() + size_t(genc::kHistBins) * genc::kMaxProbes, pesc,
+                                     sizeof(unsigned long long) * nodes, cudaMemcpyDeviceToHost, st));
+            EPK_CUDA(cudaStreamSynchronize(st));
+            for (int n = 0, step = 0; step < depth; ++step) {
+                std::copy(hcounts.begin() + size_t(n) * genc::kHistBins, hcounts.begin() + size_t(n + 1) * genc::kHistBins,
+                          counts.begin());
+                const double est = estimate_from_counts(counts, hcounts[size_t(genc::kHistBins) * genc::kMaxProbes + n],
+                                                        pr.r[n], Rs, gpr, NG, M, T);
+                if (8.0 * est <= budget) { lo = nmid[n]; n = 2 * n + 1; }
+                else { hi = nmid[n]; n = 2 * n + 2; }
+            }
+            it += uint32_t(depth);
         }
         const float alpha = float(std::exp2(lo));
 
