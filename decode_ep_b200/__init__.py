@@ -63,6 +63,10 @@ def lib() -> ctypes.CDLL:
         L.ep_compress_cuda.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_double,
                                        c.POINTER(_Options), c.c_void_p, c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
                                        c.POINTER(c.c_double)]
+        L.ep_compress_cuda_noalloc.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_double,
+                                               c.POINTER(_Options), c.c_void_p, c.c_void_p, c.c_size_t,
+                                               c.POINTER(c.c_size_t), c.POINTER(c.c_double)]
+        L.ep_compress_cuda_noalloc.restype = c.c_int
         L.ep_blob_free.argtypes = [c.c_void_p]
         L.ep_blob_info.argtypes = [c.c_void_p, c.c_size_t, c.POINTER(c.c_int), c.POINTER(c.c_int64),
                                    c.POINTER(c.c_int64), c.POINTER(c.c_double)]
@@ -195,6 +199,30 @@ def compress(tensor: torch.Tensor, config: EntroPackLossyConfig | float) -> Comp
     finally:
         lib().ep_blob_free(blob_p)
     return CompressedTensor(blob, (rows, cols), tensor.dtype, actual.value)
+
+
+def compress_cuda_noalloc(tensor: torch.Tensor, config: EntroPackLossyConfig | float) -> CompressedTensor:
+    """ep_compress_cuda_noalloc on a CUDA tensor: the CUDA encoder with its device scratch in the
+    library's fixed 64 MiB area (tensors up to about 4.5 M parameters), on the current stream."""
+    if not isinstance(config, EntroPackLossyConfig):
+        config = EntroPackLossyConfig(float(config))
+    if tensor.dim() != 2 or not tensor.is_cuda:
+        raise EntroPackError(-1, "compress_cuda_noalloc: takes a 2-D CUDA tensor")
+    if tensor.dtype not in _TORCH_TO_EP:
+        raise EntroPackError(-2, f"compress_cuda_noalloc: unsupported dtype {tensor.dtype}")
+    t = tensor if tensor.stride(1) == 1 else tensor.contiguous()
+    rows, cols = t.shape
+    cap = 8 * rows * cols + 2 * rows + 4096
+    buf = (ctypes.c_uint8 * cap)()
+    nbytes, actual = ctypes.c_size_t(), ctypes.c_double()
+    opt = config._options()
+    with torch.cuda.device(t.device):
+        st = lib().ep_compress_cuda_noalloc(t.data_ptr(), _TORCH_TO_EP[t.dtype], rows, cols, t.stride(0),
+                                            float(config.target_bpp), ctypes.byref(opt),
+                                            torch.cuda.current_stream().cuda_stream, buf, cap, ctypes.byref(nbytes),
+                                            ctypes.byref(actual))
+    _check(st, "compress_cuda_noalloc")
+    return CompressedTensor(ctypes.string_at(buf, nbytes.value), (rows, cols), tensor.dtype, actual.value)
 
 
 def _stream_ptr(stream) -> int | None:

@@ -20,6 +20,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "capi_internal.h"
@@ -520,5 +521,247 @@ extern "C" ep_status ep_compress_cuda(const void* dev_data, ep_dtype dt, int64_t
         return EP_OK;
     } catch (const std::bad_alloc&) {
         return fail(EP_ERR_NOMEM, "ep_compress_cuda: out of host memory");
+    }
+}
+
+// --------------------------------------------------------- variant with static device scratch
+
+namespace epk {
+namespace genc {
+
+// Fixed device scratch of ep_compress_cuda_noalloc: 64 MiB per device, zero at module load. With
+// lazy module loading it is reserved when this file's kernels are first used.
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+}  // namespace genc
+
+namespace {
+
+struct StaticScratch {
+    std::mutex mu;  // one call at a time per device: the area has no owner beyond the call
+    void* addr = nullptr;
+    bool resolved = false;
+};
+StaticScratch g_static[64];
+
+// Bump carving of the static area, 256-byte aligned. With base == nullptr it only sums the sizes.
+struct Carve {
+    unsigned char* base;
+    size_t used = 0;
+    template <class T>
+    T* take(size_t bytes) {
+        const size_t o = (used + 255) & ~size_t(255);
+        used = o + (bytes ? bytes : 1);
+        return base ? reinterpret_cast<T*>(base + o) : nullptr;
+    }
+};
+
+}  // namespace
+}  // namespace epk
+
+extern "C" ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt, int64_t rows, int64_t cols,
+                                              int64_t row_stride, double target_bpp, const ep_options* opt_in,
+                                              void* cuda_stream, uint8_t* blob, size_t blob_capacity,
+                                              size_t* blob_bytes, double* actual_bpp) {
+    clear_error();
+    if (!dev_data || !blob || !blob_bytes) return fail(EP_ERR_ARG, "ep_compress_cuda_noalloc: NULL argument");
+    if (!elem_bytes(int(dt))) return fail(EP_ERR_DTYPE, "ep_compress_cuda_noalloc: unknown dtype %d", int(dt));
+    if (rows < 1 || cols < 8 || cols % 8 != 0 || rows > 0xFFFFFFFFll || cols > 0xFFFFFFFFll ||
+        (rows * cols) / 8 > 0xFFFFFFFFll)
+        return fail(EP_ERR_SHAPE, "ep_compress_cuda_noalloc: need a 2-D tensor with rows >= 1 and cols a positive multiple of 8");
+    if (row_stride < cols) return fail(EP_ERR_ARG, "ep_compress_cuda_noalloc: row_stride %lld < cols", (long long)row_stride);
+    if (!(target_bpp >= 0.001 && target_bpp <= 11.0))
+        return fail(EP_ERR_TARGET, "ep_compress_cuda_noalloc: target_bpp must be finite and in [0.001, 11]");
+    ep_options opt;
+    ep_options_default(&opt);
+    if (opt_in) opt = *opt_in;
+    if (opt.rounds_per_tile == 0) opt.rounds_per_tile = auto_rounds_per_tile(rows * cols / 8);
+    if (opt.rounds_per_tile < 1 || opt.rounds_per_tile > uint32_t(kMaxG) || opt.sample_coords < 1 ||
+        opt.bisection_iters > 200)
+        return fail(EP_ERR_ARG, "ep_compress_cuda_noalloc: bad options");
+    cudaPointerAttributes pa;
+    if (cudaPointerGetAttributes(&pa, dev_data) != cudaSuccess || pa.type != cudaMemoryTypeDevice) {
+        cudaGetLastError();
+        return fail(EP_ERR_ARG, "ep_compress_cuda_noalloc: the input is not device memory");
+    }
+    const int64_t M = rows, N = cols, NG = M * N / 8, gpr = N / 8;
+    const int G = int(opt.rounds_per_tile);
+    const uint32_t T = uint32_t((NG + 32 * int64_t(G) - 1) / (32 * int64_t(G)));
+    const int64_t per_tile = 32 * int64_t(G);
+
+    // Scratch plan (the same buffers as ep_compress_cuda); the payload is sized for r = 12, its largest.
+    uint64_t payload_cap = 0;
+    for (uint32_t j = 0; j < T; ++j) {
+        const int64_t ng = std::min(per_tile, NG - int64_t(j) * per_tile);
+        payload_cap += pad16(128 + pad4(uint64_t(ng) * 12) + 2 * 16 * uint64_t(ng));
+    }
+    auto plan = [&](Carve& c, uint16_t** sb, float** s, unsigned long long** small, unsigned long long** counts,
+                    unsigned long long** pcounts, int32_t** tq, uint8_t** bq, uint32_t** tabs, uint16_t** words,
+                    uint32_t** states, uint32_t** nw, uint8_t** esc, uint64_t** start, uint8_t** payload) {
+        *sb = c.take<uint16_t>(size_t(M) * 2);
+        *s = c.take<float>(size_t(M) * 4);
+        *small = c.take<unsigned long long>(64);
+        *counts = c.take<unsigned long long>(sizeof(unsigned long long) * genc::kHistBins);
+        *pcounts = c.take<unsigned long long>(sizeof(unsigned long long) * (genc::kHistBins + 1) * genc::kMaxProbes);
+        *tq = c.take<int32_t>(size_t(NG) * 32);
+        *bq = c.take<uint8_t>(size_t(NG));
+        *tabs = c.take<uint32_t>(2 * sizeof(uint32_t) * genc::kHistBins);
+        *words = c.take<uint16_t>(size_t(T) * 16 * size_t(per_tile) * 2);
+        *states = c.take<uint32_t>(size_t(T) * 128);
+        *nw = c.take<uint32_t>(size_t(T) * 4);
+        *esc = c.take<uint8_t>(size_t(T));
+        *start = c.take<uint64_t>(sizeof(uint64_t) * (size_t(T) + 1));
+        *payload = c.take<uint8_t>(size_t(payload_cap));
+    };
+    uint16_t* d_sbits; float* d_s; unsigned long long *small, *d_counts, *pcounts; int32_t* d_tq; uint8_t* d_bq;
+    uint32_t* d_tabs; uint16_t* d_words; uint32_t *d_states, *d_nwords; uint8_t* d_esc; uint64_t* d_start;
+    uint8_t* d_payload;
+    {
+        Carve dry{nullptr};
+        plan(dry, &d_sbits, &d_s, &small, &d_counts, &pcounts, &d_tq, &d_bq, &d_tabs, &d_words, &d_states, &d_nwords,
+             &d_esc, &d_start, &d_payload);
+        if (dry.used > genc::kStaticScratchBytes)
+            return fail(EP_ERR_ARG, "ep_compress_cuda_noalloc: this tensor needs %llu bytes of device scratch; the static area holds %llu",
+                        (unsigned long long)dry.used, (unsigned long long)genc::kStaticScratchBytes);
+    }
+
+    int device = 0;
+    EPK_CUDA(cudaGetDevice(&device));
+    if (device < 0 || device >= 64) return fail(EP_ERR_CUDA, "ep_compress_cuda_noalloc: device %d out of range", device);
+    StaticScratch& ss = g_static[device];
+    std::lock_guard<std::mutex> lock(ss.mu);
+    if (!ss.resolved) {  // once per device, with that device current
+        EPK_CUDA(cudaGetSymbolAddress(&ss.addr, genc::g_static_scratch));
+        ss.resolved = true;
+    }
+    Carve carve{static_cast<unsigned char*>(ss.addr)};
+    plan(carve, &d_sbits, &d_s, &small, &d_counts, &pcounts, &d_tq, &d_bq, &d_tabs, &d_words, &d_states, &d_nwords,
+         &d_esc, &d_start, &d_payload);
+    unsigned long long* pesc = pcounts + size_t(genc::kHistBins) * genc::kMaxProbes;
+
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    const genc::Src src{static_cast<const uint8_t*>(dev_data), int(dt), N, row_stride};
+    try {
+        EPK_CUDA(cudaMemsetAsync(small, 0, 64, st));
+        genc::row_scales_kernel<<<blocks_for(M, 128), 128, 0, st>>>(src, M, d_sbits, d_s, small,
+                                                                    reinterpret_cast<int*>(small + 3));
+        EPK_CUDA(cudaGetLastError());
+        std::vector<uint16_t> sbits(static_cast<size_t>(M));
+        unsigned long long hsmall[4];
+        EPK_CUDA(cudaMemcpyAsync(sbits.data(), d_sbits, size_t(M) * 2, cudaMemcpyDeviceToHost, st));
+        EPK_CUDA(cudaMemcpyAsync(hsmall, small, sizeof(hsmall), cudaMemcpyDeviceToHost, st));
+        EPK_CUDA(cudaStreamSynchronize(st));
+        if (int(hsmall[3])) return fail(EP_ERR_NONFINITE, "ep_compress_cuda_noalloc: NaN or Inf in the input");
+        double amax;
+        std::memcpy(&amax, &hsmall[0], 8);
+
+        // Rate control, four bisection steps per launch, exactly as ep_compress_cuda.
+        const int64_t Rs = std::min<int64_t>(M, (int64_t(opt.sample_coords) + N - 1) / N);
+        std::vector<unsigned long long> hcounts(size_t(genc::kHistBins + 1) * genc::kMaxProbes);
+        Counts counts(size_t(genc::kHistBins));
+        double lo = -12.0, hi = 15.0;
+        if (amax > 0.0) hi = std::min(hi, 22.0 - std::log2(amax));
+        if (hi < lo) hi = lo;
+        const double budget = target_bpp * double(rows) * double(cols);
+        for (uint32_t it = 0; it < opt.bisection_iters;) {
+            const int depth = int(std::min<uint32_t>(genc::kProbeDepth, opt.bisection_iters - it));
+            const int nodes = (1 << depth) - 1;
+            double nlo[genc::kMaxProbes], nhi[genc::kMaxProbes], nmid[genc::kMaxProbes];
+            genc::Probes pr;
+            nlo[0] = lo;
+            nhi[0] = hi;
+            for (int n = 0; n < nodes; ++n) {
+                nmid[n] = 0.5 * (nlo[n] + nhi[n]);
+                pr.alpha[n] = float(std::exp2(nmid[n]));
+                pr.r[n] = raw_bits_for(pr.alpha[n]);
+                if (2 * n + 2 < nodes) {
+                    nlo[2 * n + 1] = nmid[n], nhi[2 * n + 1] = nhi[n];
+                    nlo[2 * n + 2] = nlo[n], nhi[2 * n + 2] = nmid[n];
+                }
+            }
+            EPK_CUDA(cudaMemsetAsync(pcounts, 0, sizeof(unsigned long long) * genc::kHistBins * nodes, st));
+            EPK_CUDA(cudaMemsetAsync(pesc, 0, sizeof(unsigned long long) * genc::kMaxProbes, st));
+            genc::sample_counts_kernel<<<dim3(blocks_for(Rs * gpr, 256), unsigned(nodes)), 256, 0, st>>>(
+                src, M, gpr, Rs, d_s, pr, pcounts, pesc);
+            EPK_CUDA(cudaGetLastError());
+            EPK_CUDA(cudaMemcpyAsync(hcounts.data(), pcounts, sizeof(unsigned long long) * genc::kHistBins * nodes,
+                                     cudaMemcpyDeviceToHost, st));
+            EPK_CUDA(cudaMemcpyAsync(hcounts.data() + size_t(genc::kHistBins) * genc::kMaxProbes, pesc,
+                                     sizeof(unsigned long long) * nodes, cudaMemcpyDeviceToHost, st));
+            EPK_CUDA(cudaStreamSynchronize(st));
+            for (int n = 0, step = 0; step < depth; ++step) {
+                std::copy(hcounts.begin() + size_t(n) * genc::kHistBins, hcounts.begin() + size_t(n + 1) * genc::kHistBins,
+                          counts.begin());
+                const double est = estimate_from_counts(counts, hcounts[size_t(genc::kHistBins) * genc::kMaxProbes + n],
+                                                        pr.r[n], Rs, gpr, NG, M, T);
+                if (8.0 * est <= budget) { lo = nmid[n]; n = 2 * n + 1; }
+                else { hi = nmid[n]; n = 2 * n + 2; }
+            }
+            it += uint32_t(depth);
+        }
+        const float alpha = float(std::exp2(lo));
+
+        // Quantisation, raw bits, tables.
+        EPK_CUDA(cudaMemsetAsync(small + 2, 0, 8, st));
+        genc::quantize_kernel<<<blocks_for(NG, 256), 256, 0, st>>>(src, NG, gpr, d_s, alpha, d_tq, d_bq, small + 2);
+        EPK_CUDA(cudaGetLastError());
+        unsigned long long tmax_u = 0;
+        EPK_CUDA(cudaMemcpyAsync(&tmax_u, small + 2, 8, cudaMemcpyDeviceToHost, st));
+        EPK_CUDA(cudaStreamSynchronize(st));
+        const int64_t tmax = int64_t(tmax_u);
+        int r = raw_bits_for(alpha);
+        while (r < 12 && tmax >= (int64_t(1) << (15 + r))) ++r;
+        if (tmax >= (int64_t(1) << (15 + r))) return fail(EP_ERR_ARG, "ep_compress_cuda_noalloc: value range too wide to code");
+        EPK_CUDA(cudaMemsetAsync(d_counts, 0, sizeof(unsigned long long) * genc::kHistBins, st));
+        genc::full_counts_kernel<<<std::min<unsigned>(blocks_for(NG, 256), 148u * 8u), 256, 0, st>>>(d_tq, d_bq, NG, r,
+                                                                                                   d_counts);
+        EPK_CUDA(cudaGetLastError());
+        EPK_CUDA(cudaMemcpyAsync(counts.data(), d_counts, sizeof(unsigned long long) * genc::kHistBins,
+                                 cudaMemcpyDeviceToHost, st));
+        EPK_CUDA(cudaStreamSynchronize(st));
+        Tables tab;
+        tab.build(counts);
+
+        // Tiles.
+        EPK_CUDA(cudaMemcpyAsync(d_tabs, tab.f, sizeof(uint32_t) * genc::kHistBins, cudaMemcpyHostToDevice, st));
+        EPK_CUDA(cudaMemcpyAsync(d_tabs + genc::kHistBins, tab.cum, sizeof(uint32_t) * genc::kHistBins,
+                                 cudaMemcpyHostToDevice, st));
+        genc::encode_tiles_kernel<<<blocks_for(T, 8), 256, 0, st>>>(d_tq, d_bq, NG, T, G, r, d_tabs,
+                                                                   d_tabs + genc::kHistBins, d_words, d_states,
+                                                                   d_nwords, d_esc);
+        EPK_CUDA(cudaGetLastError());
+        std::vector<uint32_t> nwords(T);
+        std::vector<uint8_t> esc(T);
+        EPK_CUDA(cudaMemcpyAsync(nwords.data(), d_nwords, size_t(T) * 4, cudaMemcpyDeviceToHost, st));
+        EPK_CUDA(cudaMemcpyAsync(esc.data(), d_esc, size_t(T), cudaMemcpyDeviceToHost, st));
+        EPK_CUDA(cudaStreamSynchronize(st));
+        std::vector<uint64_t> start(size_t(T) + 1, 0);
+        for (uint32_t j = 0; j < T; ++j) {
+            const int64_t ng = std::min(per_tile, NG - int64_t(j) * per_tile);
+            start[j + 1] = start[j] + pad16(128 + pad4(uint64_t(ng) * uint64_t(r)) + 2 * uint64_t(nwords[j]));
+        }
+        if (start[T] / 16 >= 0x80000000ull) return fail(EP_ERR_SHAPE, "ep_compress_cuda_noalloc: payload too large");
+        const BlobLayout L = blob_layout(rows, tab, T, start[T]);
+        if (L.total > blob_capacity)
+            return fail(EP_ERR_BUFFER, "ep_compress_cuda_noalloc: the blob takes %llu bytes, the buffer holds %llu",
+                        (unsigned long long)L.total, (unsigned long long)blob_capacity);
+
+        // Payload in the static area (zeroed first: padding bytes stay zero), then into the caller's buffer.
+        EPK_CUDA(cudaMemcpyAsync(d_start, start.data(), sizeof(uint64_t) * (size_t(T) + 1), cudaMemcpyHostToDevice, st));
+        EPK_CUDA(cudaMemsetAsync(d_payload, 0, size_t(start[T]), st));
+        genc::assemble_kernel<<<blocks_for(T, 8), 256, 0, st>>>(d_payload, d_start, d_states, d_words, d_nwords, d_tq,
+                                                              NG, T, G, r);
+        EPK_CUDA(cudaGetLastError());
+        std::memset(blob, 0, size_t(L.off_payload));
+        EPK_CUDA(cudaMemcpyAsync(blob + L.off_payload, d_payload, size_t(start[T]), cudaMemcpyDeviceToHost, st));
+        EPK_CUDA(cudaStreamSynchronize(st));
+        write_metadata(blob, L, dt, r, rows, cols, alpha, uint32_t(G), T, sbits.data(), tab, start.data(), esc.data());
+        finish_crc(blob, L);
+        *blob_bytes = size_t(L.total);
+        if (actual_bpp) *actual_bpp = 8.0 * double(L.total) / (double(rows) * double(cols));
+        return EP_OK;
+    } catch (const std::bad_alloc&) {
+        return fail(EP_ERR_NOMEM, "ep_compress_cuda_noalloc: out of host memory");
     }
 }

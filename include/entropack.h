@@ -120,6 +120,29 @@ ep_status ep_compress_cuda(const void* dev_data, ep_dtype dt, int64_t rows, int6
                            double target_bpp, const ep_options* opt, void* cuda_stream, uint8_t** blob,
                            size_t* blob_bytes, double* actual_bpp);
 
+/*
+ * ep_compress_cuda_noalloc: ep_compress_cuda with no device allocation. The pages have no counterpart
+ * to this entry point: it exists for callers that must not allocate device memory (no cudaMalloc,
+ * cudaMallocAsync, cudaFree or cudaFreeAsync happens in it). It runs the same kernels and writes the
+ * same blob bytes as ep_compress_cuda.
+ *
+ * Scratch     every device buffer is carved from one fixed 64 MiB array in device memory (a static
+ *             __device__ array of the library, one per device, reserved when the encoder's kernels are
+ *             first loaded). That bounds the tensor to about 4.5 M parameters (for example 2048 x 2048);
+ *             a larger request is rejected with EP_ERR_ARG before any work. Counters and the payload
+ *             area are zeroed by each call.
+ * blob        caller-owned host buffer of blob_capacity bytes; the blob is written there and *blob_bytes
+ *             receives its size. 8*rows*cols + 2*rows + 4096 bytes always suffice; a smaller buffer that
+ *             cannot hold the blob gives EP_ERR_BUFFER.
+ * Races       the array is shared by every call on a device in the process. Calls on one device are
+ *             serialised by a lock held for the whole call, and each call synchronises cuda_stream before
+ *             it returns, so no two calls use the array at once. Other processes have their own array.
+ * Other arguments and errors as ep_compress_cuda.
+ */
+ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt, int64_t rows, int64_t cols, int64_t row_stride,
+                                   double target_bpp, const ep_options* opt, void* cuda_stream, uint8_t* blob,
+                                   size_t blob_capacity, size_t* blob_bytes, double* actual_bpp);
+
 /* Releases a blob returned by ep_compress or ep_compress_cuda. NULL is accepted. */
 void ep_blob_free(uint8_t* blob);
 
