@@ -62,7 +62,7 @@ def parse_args():
     ap.add_argument("--json-out", default="", help="appends each printed JSON line to this file")
     ap.add_argument("--workload", default="dit276_bf16_4bpp",
                     choices=["dit276_bf16_4bpp", "quickstart256_bf16_3.5bpp", "lognormal3072_bf16_4bpp", "sweep4096",
-                             "fp8_8192x28672_5bpp", "int8_8192x28672_3bpp"],
+                             "fp8_8192x28672_5bpp", "int8_8192x28672_3bpp", "dit276_gemm_overhead"],
                     help="the default is the headline line; the others print one line per tensor")
     return ap.parse_args()
 
@@ -567,6 +567,112 @@ def oracle_rate(blob, shape, seconds, workers):
     return done / (time.perf_counter() - t0)
 
 
+def run_gemm_overhead(args, tokens=4096):
+    """Decode overhead against the layer GEMMs of a prefill-sized forward pass (the pages measure it as
+    the denoising-step time with compressed vs BF16 weights; that needs the real model, so this times
+    the proxy: the 276 layer GEMMs y = x W^T on `tokens` synthetic activations, in layer order).
+      gemm:      BF16 weights resident, GEMMs only (cuBLAS through torch.matmul);
+      serial:    each layer decoded into one reused buffer, then its GEMM;
+      overlap:   layer i+1 decodes on a second stream into the other of two buffers while GEMM i runs.
+    value = serial / gemm - 1 (the overhead); the overlap figure is reported beside it."""
+    import decode_ep_b200 as ep
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    layers = layer_list(args.layers)
+    ws = [synth.dit_layer(i, shape=(M, N)).to(device) for i, _, M, N in layers]
+    streams_enc = [torch.cuda.Stream(device) for _ in range(4)]
+
+    def enc(k):
+        with torch.cuda.stream(streams_enc[k % 4]):
+            return ep.compress(ws[k], ep.EntroPackLossyConfig(args.target_bpp, encoder="cuda"))
+
+    with cf.ThreadPoolExecutor(max_workers=4) as ex:
+        blobs = list(ex.map(enc, range(len(layers))))
+    torch.cuda.synchronize(device)
+    resident = [ep.decompress(c, device=device) for c in blobs]  # what the GEMM-only pass reads
+    del ws
+    g = torch.Generator(device=device).manual_seed(7)
+    xs = {N: torch.randn(tokens, N, generator=g, device=device, dtype=torch.bfloat16) for _, _, _, N in layers}
+    max_numel = max(M * N for _, _, M, N in layers)
+    y = torch.empty(tokens * max(M for _, _, M, _ in layers), dtype=torch.bfloat16, device=device)
+    wbuf = [torch.empty(max_numel, dtype=torch.bfloat16, device=device) for _ in range(2)]
+    main = torch.cuda.current_stream(device)
+    side = torch.cuda.Stream(device)
+
+    def gemm(k, w):
+        _, _, M, N = layers[k]
+        torch.matmul(xs[N], w.reshape(-1)[: M * N].view(M, N).t(), out=y[: tokens * M].view(tokens, M))
+
+    def step_gemm():
+        for k in range(len(layers)):
+            gemm(k, resident[k])
+
+    def step_serial():
+        for k, c in enumerate(blobs):
+            out = wbuf[0][: c.shape[0] * c.shape[1]].view(c.shape)
+            ep.decompress_into(c, out, main)
+            gemm(k, out)
+
+    def step_overlap():
+        done = [torch.cuda.Event(), torch.cuda.Event()]   # GEMM that last read wbuf[b] is done
+        ready = [torch.cuda.Event(), torch.cuda.Event()]  # decode into wbuf[b] is done
+        first = [True, True]
+
+        def decode(k):
+            b = k & 1
+            c = blobs[k]
+            with torch.cuda.stream(side):
+                if not first[b]:
+                    side.wait_event(done[b])
+                first[b] = False
+                ep.decompress_into(c, wbuf[b][: c.shape[0] * c.shape[1]].view(c.shape), side)
+                ready[b].record(side)
+
+        decode(0)
+        for k in range(len(layers)):
+            if k + 1 < len(layers):
+                decode(k + 1)
+            b = k & 1
+            main.wait_event(ready[b])
+            gemm(k, wbuf[b])
+            done[b].record(main)
+        main.wait_stream(side)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(device)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(main)
+        for _ in range(args.steps):
+            fn()
+        b.record(main)
+        torch.cuda.synchronize(device)
+        return a.elapsed_time(b) / args.steps
+
+    with ClockSampler(local) as clk:
+        ms_gemm = timed(step_gemm)
+        ms_serial = timed(step_serial)
+        ms_overlap = timed(step_overlap)
+    if ep.device_status(main):
+        raise RuntimeError("device status set")
+    flops = 2.0 * tokens * sum(M * N for _, _, M, N in layers)
+    return {
+        "metric": "decode overhead on the 276 layer GEMMs of a 4096-token prefill (serial decode+GEMM / GEMM - 1)",
+        "value": round(100.0 * (ms_serial / ms_gemm - 1.0), 2), "unit": "%", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_serial, 3), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 GEMM; u32+f32 decode", "data": "synthetic",
+        "config": {"workload": "dit276_gemm_overhead", "tokens": tokens, "layers": len(layers),
+                   "target_bpp": args.target_bpp, "gemm_tflops": round(flops / (ms_gemm * 1e-3) / 1e12, 1),
+                   "ms_gemm_only": round(ms_gemm, 3), "ms_decode_then_gemm": round(ms_serial, 3),
+                   "ms_decode_overlapped": round(ms_overlap, 3),
+                   "overlap_overhead_pct": round(100.0 * (ms_overlap / ms_gemm - 1.0), 2),
+                   "gemm": "torch.matmul (cuBLAS), BF16, weights (out, in) used transposed"},
+        "clocks": clk.summary(), "gpu_launches": args.steps * len(layers),
+    }
+
+
 def run_workload(args):
     """One JSON line per tensor of a single-tensor workload. A step is one ep_decompress_into of the
     tensor. Each timed step is bracketed by its own CUDA events, with a 256 MB write between steps that
@@ -676,6 +782,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         lines = [run_reference(args)]
+    elif args.workload == "dit276_gemm_overhead":
+        lines = [run_gemm_overhead(args)]
     elif args.workload == "dit276_bf16_4bpp":
         lines = [run_ours(args)]
     else:
