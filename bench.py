@@ -258,12 +258,17 @@ def run_ours(args):
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         torch.cuda.synchronize(device)
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps - 1)]
         start.record(stream)
-        for _ in range(args.steps):
+        for k in range(args.steps):
             step()
+            if k < args.steps - 1:
+                marks[k].record(stream)  # step boundaries, for the median and best step
         stop.record(stream)
         torch.cuda.synchronize(device)
     ms_total = start.elapsed_time(stop)
+    bounds = [start] + marks + [stop]
+    per_step = sorted(bounds[k].elapsed_time(bounds[k + 1]) for k in range(args.steps))
     status = ep.device_status(stream)
     if status:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -313,7 +318,8 @@ def run_ours(args):
                    "rel_l2_pooled": None if rel_l2 is None else round(rel_l2, 5),
                    "rel_l2_layer_mean": None if rel_l2_mean is None else round(rel_l2_mean, 5),
                    "encode_wall_s": round(enc_wall, 2), "encode_cpu_s": round(enc_cpu, 2),
-                   "encode_threads": workers, "encode_cuda": gpu_enc},
+                   "encode_threads": workers, "encode_cuda": gpu_enc,
+                   "step_ms_median": round(statistics.median(per_step), 4), "step_ms_best": round(per_step[0], 4)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_kind} copy bandwidth",
