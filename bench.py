@@ -335,7 +335,7 @@ def run_ours(args):
     return line
 
 
-def time_cuda_encoder(blobs, layers, target_bpp, device, workers=4):
+def time_cuda_encoder(blobs, layers, target_bpp, device, workers=8):
     """Encodes every layer again with the CUDA encoder (ep_compress_cuda), the inputs already in device
     memory, and checks each blob against the host encoder's bytes. `workers` host threads encode
     layers concurrently, each on its own CUDA stream. Returns the wall time of the whole set."""

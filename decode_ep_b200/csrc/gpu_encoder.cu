@@ -68,21 +68,38 @@ __device__ __forceinline__ uint16_t bf16_rne(float f) {
 
 // Row scales: s_row = bf16(fl32(sqrt(Σ w² / N))), the sum in double and index order, then the largest
 // |w| / s over rows with s != 0. A correctly rounded division is monotonic, so the largest quotient is
-// the quotient of the largest |w|: one division per row. One thread per row.
-__global__ void row_scales_kernel(Src src, int64_t M, uint16_t* sbits, float* s_out, unsigned long long* amax_bits,
-                                  int* nonfinite) {
+// the quotient of the largest |w|: one division per row. One thread per row, reading it in index
+// order. The chain of N dependent double additions per row sets the kernel's time; a row's values are
+// reused from L1, so staging them through shared memory does not help.
+constexpr int kScaleWarps = 4;
+
+template <int DT>
+__device__ __forceinline__ float load_as(const uint8_t* base, int64_t k) {
+    if constexpr (DT == EP_BF16) return __uint_as_float(uint32_t(reinterpret_cast<const uint16_t*>(base)[k]) << 16);
+    else if constexpr (DT == EP_FP16) return __half2float(__ushort_as_half(reinterpret_cast<const unsigned short*>(base)[k]));
+    else if constexpr (DT == EP_FP32) return reinterpret_cast<const float*>(base)[k];
+    else if constexpr (DT == EP_FP8_E4M3) return e4m3_to_float(base[k]);
+    else return float(reinterpret_cast<const int8_t*>(base)[k]);
+}
+
+template <int DT>
+__global__ void __launch_bounds__(32 * kScaleWarps) row_scales_kernel(Src src, int64_t M, uint16_t* sbits, float* s_out,
+                                                                     unsigned long long* amax_bits, int* nonfinite) {
     const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= M) return;
+    const uint8_t* row = src.base + i * src.stride * int64_t(DT == EP_FP32 ? 4 : (DT == EP_BF16 || DT == EP_FP16 ? 2 : 1));
     double acc = 0.0;
     float wmax = 0.f;
+    bool finite = true;
     for (int64_t j = 0; j < src.N; ++j) {
-        const float w = load_w(src, i, j);
-        if (!isfinite(w)) {
-            atomicOr(nonfinite, 1);
-            return;
-        }
+        const float w = load_as<DT>(row, j);
+        finite = finite && isfinite(w);
         acc = __dadd_rn(acc, __dmul_rn(double(w), double(w)));
         wmax = fmaxf(wmax, fabsf(w));
+    }
+    if (!finite) {
+        atomicOr(nonfinite, 1);
+        return;
     }
     const float rms = __double2float_rn(__dsqrt_rn(__ddiv_rn(acc, double(src.N))));
     const uint16_t sb = bf16_rne(rms);
@@ -91,6 +108,20 @@ __global__ void row_scales_kernel(Src src, int64_t M, uint16_t* sbits, float* s_
     s_out[i] = s;
     const double m = s != 0.f ? __ddiv_rn(double(wmax), double(s)) : 0.0;
     atomicMax(amax_bits, static_cast<unsigned long long>(__double_as_longlong(m)));  // m >= 0: bits order as values
+}
+
+// Launches row_scales_kernel for the source's dtype.
+inline cudaError_t launch_row_scales(const Src& src, int64_t M, uint16_t* sbits, float* s_out,
+                                     unsigned long long* amax_bits, int* nonfinite, cudaStream_t st) {
+    const unsigned blocks = unsigned((M + 32 * kScaleWarps - 1) / (32 * kScaleWarps));
+    switch (src.dtype) {
+        case EP_BF16: row_scales_kernel<EP_BF16><<<blocks, 32 * kScaleWarps, 0, st>>>(src, M, sbits, s_out, amax_bits, nonfinite); break;
+        case EP_FP16: row_scales_kernel<EP_FP16><<<blocks, 32 * kScaleWarps, 0, st>>>(src, M, sbits, s_out, amax_bits, nonfinite); break;
+        case EP_FP32: row_scales_kernel<EP_FP32><<<blocks, 32 * kScaleWarps, 0, st>>>(src, M, sbits, s_out, amax_bits, nonfinite); break;
+        case EP_FP8_E4M3: row_scales_kernel<EP_FP8_E4M3><<<blocks, 32 * kScaleWarps, 0, st>>>(src, M, sbits, s_out, amax_bits, nonfinite); break;
+        default: row_scales_kernel<EP_INT8><<<blocks, 32 * kScaleWarps, 0, st>>>(src, M, sbits, s_out, amax_bits, nonfinite); break;
+    }
+    return cudaGetLastError();
 }
 
 // Quantises group q of row i at alpha: x_k = (alpha w_k) / s in double, then the nearest E8 point.
@@ -303,12 +334,43 @@ namespace {
 using namespace enc;
 
 // Stream-ordered device scratch, released on the stream when it goes out of scope.
+// The encoder's stream-ordered scratch pool on the current device, created on first use. Freed scratch
+// up to 1 GiB stays mapped in the pool for the next call; above that it goes back at the next
+// synchronisation.
+cudaError_t scratch_pool(cudaMemPool_t* out) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64];
+    static bool made[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!made[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        e = cudaMemPoolCreate(&pools[dev], &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = uint64_t(1) << 30;
+        e = cudaMemPoolSetAttribute(pools[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) return e;
+        made[dev] = true;
+    }
+    *out = pools[dev];
+    return cudaSuccess;
+}
+
 struct DevBuf {
     void* p = nullptr;
     cudaStream_t s = nullptr;
     cudaError_t alloc(size_t bytes, cudaStream_t st) {
         s = st;
-        return cudaMallocAsync(&p, bytes ? bytes : 16, st);
+        cudaMemPool_t pool;
+        cudaError_t e = scratch_pool(&pool);
+        if (e != cudaSuccess) return e;
+        return cudaMallocFromPoolAsync(&p, bytes ? bytes : 16, pool, st);
     }
     ~DevBuf() {
         if (p) cudaFreeAsync(p, s);
@@ -370,9 +432,8 @@ extern "C" ep_status ep_compress_cuda(const void* dev_data, ep_dtype dt, int64_t
         EPK_CUDA(d_counts.alloc(sizeof(unsigned long long) * genc::kHistBins, st));
         unsigned long long* small = d_small.as<unsigned long long>();
         EPK_CUDA(cudaMemsetAsync(small, 0, 64, st));
-        genc::row_scales_kernel<<<blocks_for(M, 128), 128, 0, st>>>(src, M, d_sbits.as<uint16_t>(), d_s.as<float>(), small,
-                                                                    reinterpret_cast<int*>(small + 3));
-        EPK_CUDA(cudaGetLastError());
+        EPK_CUDA(genc::launch_row_scales(src, M, d_sbits.as<uint16_t>(), d_s.as<float>(), small,
+                                         reinterpret_cast<int*>(small + 3), st));
         std::vector<uint16_t> sbits(static_cast<size_t>(M));
         unsigned long long hsmall[4];
         EPK_CUDA(cudaMemcpyAsync(sbits.data(), d_sbits.p, size_t(M) * 2, cudaMemcpyDeviceToHost, st));
@@ -644,9 +705,7 @@ extern "C" ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt,
     const genc::Src src{static_cast<const uint8_t*>(dev_data), int(dt), N, row_stride};
     try {
         EPK_CUDA(cudaMemsetAsync(small, 0, 64, st));
-        genc::row_scales_kernel<<<blocks_for(M, 128), 128, 0, st>>>(src, M, d_sbits, d_s, small,
-                                                                    reinterpret_cast<int*>(small + 3));
-        EPK_CUDA(cudaGetLastError());
+        EPK_CUDA(genc::launch_row_scales(src, M, d_sbits, d_s, small, reinterpret_cast<int*>(small + 3), st));
         std::vector<uint16_t> sbits(static_cast<size_t>(M));
         unsigned long long hsmall[4];
         EPK_CUDA(cudaMemcpyAsync(sbits.data(), d_sbits, size_t(M) * 2, cudaMemcpyDeviceToHost, st));

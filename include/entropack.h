@@ -111,8 +111,9 @@ ep_status ep_compress(const void* data, int is_device, ep_dtype dt, int64_t rows
  *             synchronises this stream several times and returns when the blob is complete.
  * opt         NULL means the defaults; opt->threads is ignored.
  * Other arguments and the ownership of *blob as for ep_compress (release with ep_blob_free).
- * Device scratch (about 10 bytes per parameter) comes from cudaMallocAsync on the stream and is
- * released before the call returns.
+ * Device scratch (about 10 bytes per parameter) comes stream-ordered from a memory pool that the
+ * library creates per device. Each call frees its scratch before it returns. The pool keeps up to
+ * 1 GiB of freed scratch mapped for the next call, and releases the rest.
  * Errors: as ep_compress; EP_ERR_ARG also when dev_data is not device memory; EP_ERR_CUDA for a failed
  *         allocation, launch or copy.
  */
