@@ -99,6 +99,10 @@ struct Params {
     uint32_t k2, k4, kneg4096, k128;
     uint32_t off_scales, off_tables, off_offsets, off_payload, tables_len;
     uint64_t payload_bytes;
+    // The next blob of a sequence (ep_decompress_many), or null: its tables, tile offsets and scales
+    // are pulled into L2 while this one decodes.
+    const uint8_t* next_blob;
+    uint32_t next_meta_off, next_meta_bytes;  // [off_scales, off_payload) of the next blob
 };
 
 __device__ int g_status;
@@ -171,6 +175,18 @@ __device__ __forceinline__ uint32_t entry_template(int c, int sym, uint32_t f) {
 //      each symbol with f > 0 drops D[s] at slot cum[s] (the marker);
 //   3. each thread takes 36 consecutive entries of the 9 x 4096, starts from the marker in force at its
 //      first slot (a 7-step binary search over cum) and carries markers forward: entry = D + (slot << 20).
+// Starts the copy of the serialised tables (the first kScratchTableCap bytes of the section, zero past
+// its end) into scratch, as one copy group. The section start is 16-byte aligned (header check).
+__device__ __forceinline__ void stage_tables_async(const Params& p, uint8_t* scratch) {
+    const uint32_t tlen = p.tables_len < kScratchTableCap ? p.tables_len : kScratchTableCap;
+    const uint32_t off = 16 * threadIdx.x;
+    if (off < kScratchTableCap) {
+        const uint32_t n = off < tlen ? min(16u, tlen - off) : 0u;
+        cp_async16(smem_addr(scratch + kScratchBytes + off), n ? p.blob + p.off_tables + off : p.blob, n);
+    }
+    cp_async_commit();
+}
+
 __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch) {
     uint32_t* cum = reinterpret_cast<uint32_t*>(scratch + kScratchCum);    // [9][129]
     uint8_t* tbytes = scratch + kScratchBytes;
@@ -178,14 +194,14 @@ __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch)
     uint32_t* t32 = reinterpret_cast<uint32_t*>(tables);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // Pass 1.
+    // Pass 1. The serialised bytes were staged by stage_tables_async (the older of this thread's two
+    // copy groups).
     {
         uint4* t4 = reinterpret_cast<uint4*>(tables);
         for (uint32_t i = tid; i < kTablesBytes / 16; i += kThreads) t4[i] = make_uint4(0u, 0u, 0u, 0u);
     }
     const uint32_t tlen = p.tables_len < kScratchTableCap ? p.tables_len : kScratchTableCap;
-    const uint8_t* tb = p.blob + p.off_tables;
-    for (uint32_t i = tid; i < kScratchTableCap; i += kThreads) tbytes[i] = i < tlen ? __ldg(tb + i) : 0;
+    cp_async_wait<1>();
     __syncthreads();
 
     // Pass 2: one thread per symbol. Threads 0-127 hold START, then 64 threads (two warps) per context
@@ -680,10 +696,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
                                                        : rings_after + (warp - rings_before) * kRingBytes)};
 
     grid_dependents_launch();  // lets the next launch of a sequence start its prologue early
+    stage_tables_async(p, scratch);
+
+    // The next layer's metadata (tables, tile offsets, scales) goes to L2 now, so its prologue reads L2.
+    if (p.next_blob) {
+        const uint32_t lines = (p.next_meta_bytes + 127) / 128;
+        for (uint32_t l = blockIdx.x + gridDim.x * threadIdx.x; l < lines; l += gridDim.x * kThreads)
+            prefetch_l2(p.next_blob + p.next_meta_off + 128ull * l);
+    }
 
     // Tiles are dealt round-robin over the CTAs first, so that consecutive tiles land on different SMs
     // and a partial last wave is spread over the whole GPU: tile = (k * kWarps + warp) * grid + block.
-    // The copies of the warp's first tile are issued before the table build, which hides them.
+    // The copies of the warp's first tile are issued before the table build, which hides them. Every
+    // thread commits exactly one group here (empty without a first tile), behind the tables' group.
     uint32_t slot = warp;
     bool first_issued = false;
     {
@@ -693,10 +718,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
             if (tile_geometry(p, toff, tile, per_tile, tg)) {
                 const uint32_t first = min(tg.chunks, kRingChunks);
                 for (uint32_t c = 0; c < first; ++c) issue_chunk(payload, tg, c, ring.base, lane);
-                cp_async_commit();
                 first_issued = true;
             }
         }
+        cp_async_commit();
     }
     build_tables(p, tables, scratch);
     grid_dependency_wait();  // stores below may overwrite what the previous launch of a sequence wrote
@@ -846,8 +871,10 @@ ep_status launch_mode(const dev::Params& p, cudaStream_t stream, int device, boo
     return EP_OK;
 }
 
+// next_hdr / next_dev: the following blob of a sequence (its metadata is prefetched to L2), or null.
 ep_status launch_decode(const uint8_t* host_hdr, const void* dev_blob, size_t blob_bytes, void* dst, size_t dst_bytes,
-                        int mode, void* stream_ptr, bool chained) {
+                        int mode, void* stream_ptr, bool chained, const uint8_t* next_hdr = nullptr,
+                        const void* next_dev = nullptr) {
     if (!host_hdr || !dev_blob || !dst) return fail(EP_ERR_ARG, "decode: NULL argument");
     Header h;
     if (!parse_header(host_hdr, h)) return fail(EP_ERR_CORRUPT, "decode: malformed EPK1 header");
@@ -890,6 +917,14 @@ ep_status launch_decode(const uint8_t* host_hdr, const void* dev_blob, size_t bl
     p.off_payload = h.off_payload;
     p.tables_len = h.off_offsets - h.off_tables;
     p.payload_bytes = h.total - h.off_payload;
+    p.next_blob = nullptr;
+    p.next_meta_off = p.next_meta_bytes = 0;
+    Header hn;
+    if (next_hdr && next_dev && parse_header(next_hdr, hn)) {  // headers of a sequence are checked up front
+        p.next_blob = static_cast<const uint8_t*>(next_dev);
+        p.next_meta_off = hn.off_scales;
+        p.next_meta_bytes = hn.off_payload - hn.off_scales;
+    }
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
     switch (mode) {
         case dev::kBF16: return launch_mode<dev::kBF16>(p, stream, device, chained);
@@ -933,7 +968,8 @@ extern "C" ep_status ep_decompress_many(int count, const uint8_t* const* host_hd
         Header h;
         parse_header(host_hdrs[i], h);
         ep_status st = launch_decode(host_hdrs[i], dev_blobs[i], blob_bytes[i], dsts[i], dst_bytes[i], h.dtype,
-                                     cuda_stream, i > 0);
+                                     cuda_stream, i > 0, i + 1 < count ? host_hdrs[i + 1] : nullptr,
+                                     i + 1 < count ? dev_blobs[i + 1] : nullptr);
         if (st != EP_OK) return st;
     }
     return EP_OK;
