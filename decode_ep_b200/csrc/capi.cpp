@@ -2,7 +2,10 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <string>
+
+#include <cuda_runtime.h>
 
 #include "capi_internal.h"
 #include "entropack.h"
@@ -42,6 +45,31 @@ uint32_t crc32(const uint8_t* p, uint64_t n) {
     uint32_t c = 0xFFFFFFFFu;
     for (uint64_t i = 0; i < n; ++i) c = kCrc.t[(c ^ p[i]) & 0xFFu] ^ (c >> 8);
     return c ^ 0xFFFFFFFFu;
+}
+
+cudaError_t scratch_pool(cudaMemPool_t* out) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64];
+    static bool made[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!made[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        e = cudaMemPoolCreate(&pools[dev], &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = uint64_t(1) << 30;
+        e = cudaMemPoolSetAttribute(pools[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) return e;
+        made[dev] = true;
+    }
+    *out = pools[dev];
+    return cudaSuccess;
 }
 
 ep_status validate_blob(const uint8_t* p, uint64_t bytes) {

@@ -3,6 +3,8 @@
 
 #include <cstdint>
 
+#include <cuda_runtime.h>
+
 #include "entropack.h"
 
 namespace epk {
@@ -18,5 +20,10 @@ uint32_t crc32(const uint8_t* p, uint64_t n);
 
 // Full host validation of a blob (header, sections, tables, offsets, CRC).
 ep_status validate_blob(const uint8_t* blob, uint64_t bytes);
+
+// The library's stream-ordered scratch pool on the current device, created on first use. Freed
+// scratch up to 1 GiB stays mapped for the next call; above that it goes back at the next
+// synchronisation.
+cudaError_t scratch_pool(cudaMemPool_t* out);
 
 }  // namespace epk

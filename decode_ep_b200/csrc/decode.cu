@@ -103,6 +103,9 @@ struct Params {
     // are pulled into L2 while this one decodes.
     const uint8_t* next_blob;
     uint32_t next_meta_off, next_meta_bytes;  // [off_scales, off_payload) of the next blob
+    // The fused entries of this blob, 9 x 4096 in shared-memory block order, built once for the whole
+    // sequence by expand_tables_kernel; null means each CTA builds them (build_tables).
+    const uint32_t* pre_tables;
 };
 
 __device__ int g_status;
@@ -175,6 +178,14 @@ __device__ __forceinline__ uint32_t entry_template(int c, int sym, uint32_t f) {
 //      each symbol with f > 0 drops D[s] at slot cum[s] (the marker);
 //   3. each thread takes 36 consecutive entries of the 9 x 4096, starts from the marker in force at its
 //      first slot (a 7-step binary search over cum) and carries markers forward: entry = D + (slot << 20).
+// Starts the copy of pre-built fused entries (9 x 4096 words, 144 KB) into the table region, as one
+// copy group: nine 16-byte copies per thread.
+__device__ __forceinline__ void load_tables_async(const Params& p, uint8_t* tables) {
+    const uint32_t dst = smem_addr(tables);
+    for (uint32_t i = threadIdx.x; i < kTablesBytes / 16; i += kThreads) cp_async16(dst + 16 * i, p.pre_tables + 4 * i, 16);
+    cp_async_commit();
+}
+
 // Starts the copy of the serialised tables (the first kScratchTableCap bytes of the section, zero past
 // its end) into scratch, as one copy group. The section start is 16-byte aligned (header check).
 __device__ __forceinline__ void stage_tables_async(const Params& p, uint8_t* scratch) {
@@ -672,6 +683,65 @@ __device__ __forceinline__ uint32_t fast_rounds(const Params& p, uint32_t t0, co
 
 // ---------------------------------------------------------------------------------- kernel
 
+// Fused entries of a sequence of blobs, built once per (blob, context) instead of once per CTA. Block
+// (layer, c) unpacks context c's frequencies, accumulates cum, checks the table and writes the 4096
+// entries of its block: entry(t) = template[s] + ((t - cum[s]) << 20) for the symbol s owning slot t,
+// the same words as build_tables.
+constexpr int kMaxExpandJobs = 512;
+struct ExpandArgs {
+    const uint8_t* tables[kMaxExpandJobs];  // tables section of each blob (16-byte aligned)
+    uint32_t tables_len[kMaxExpandJobs];
+    uint32_t* out;                          // count x 9 x 4096 words
+    int count;
+};
+
+__global__ void __launch_bounds__(256) expand_tables_kernel(const ExpandArgs a) {
+    __shared__ uint8_t bytes[kScratchTableCap];
+    __shared__ uint32_t cum[129], tmpl[128];
+    const int layer = blockIdx.x / kNumCtx, c = blockIdx.x % kNumCtx, tid = threadIdx.x;
+    if (layer >= a.count) return;
+    const uint32_t tlen = a.tables_len[layer] < kScratchTableCap ? a.tables_len[layer] : kScratchTableCap;
+    for (uint32_t i = tid; i < kScratchTableCap; i += blockDim.x) bytes[i] = i < tlen ? __ldg(a.tables[layer] + i) : 0;
+    __syncthreads();
+    const int A = c == 0 ? 128 : 64;
+    const uint32_t lo = bytes[c], cnt = bytes[kNumCtx + c];
+    if (tid < 128) {
+        uint32_t bit0 = 0;
+        for (int k = 0; k < c; ++k) bit0 += 12u * bytes[kNumCtx + k];
+        const uint32_t bits_len = tlen > 2 * kNumCtx ? tlen - 2 * kNumCtx : 0;
+        uint32_t f = 0;
+        if (tid < A && uint32_t(tid) >= lo && uint32_t(tid) < lo + cnt) {
+            const uint32_t bit = bit0 + 12 * (uint32_t(tid) - lo), byte = bit >> 3;
+            uint32_t w = 0;
+            for (int k = 0; k < 3; ++k)
+                if (byte + k < bits_len) w |= uint32_t(bytes[2 * kNumCtx + byte + k]) << (8 * k);
+            f = (w >> (bit & 7)) & 0xFFFu;
+        }
+        tmpl[tid] = f;  // the frequency for now; the template once cum is known
+    }
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t acc = 0;
+        for (int s = 0; s < A; ++s) { cum[s] = acc; acc += tmpl[s]; }
+        cum[A] = acc;
+        const bool ok = cnt == 0 ? acc == 0 : (acc == kProbScale && cnt >= 2);
+        if (!ok) atomicOr(&g_status, int(EP_DEV_BAD_TABLES));
+    }
+    __syncthreads();
+    if (tid < A) tmpl[tid] = entry_template(c, tid, tmpl[tid]);
+    __syncthreads();
+    // 16 consecutive slots per thread: a binary search for the owner of the first, then a walk.
+    uint32_t* out = a.out + size_t(layer) * (kTablesBytes / 4) + block_of(c) / 4;
+    const uint32_t first = 16 * uint32_t(tid);
+    int s = 0;
+    for (int step = 64; step >= 1; step >>= 1)
+        if (s + step < A && cum[s + step] <= first) s += step;
+    for (uint32_t t = first; t < first + 16; ++t) {
+        while (s + 1 < A && t >= cum[s + 1]) ++s;
+        out[t] = tmpl[s] + ((t - cum[s]) << 20);
+    }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -696,7 +766,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
                                                        : rings_after + (warp - rings_before) * kRingBytes)};
 
     grid_dependents_launch();  // lets the next launch of a sequence start its prologue early
-    stage_tables_async(p, scratch);
+    if (p.pre_tables)
+        load_tables_async(p, tables);
+    else
+        stage_tables_async(p, scratch);
 
     // The next layer's metadata (tables, tile offsets, scales) goes to L2 now, so its prologue reads L2.
     if (p.next_blob) {
@@ -723,7 +796,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
         }
         cp_async_commit();
     }
-    build_tables(p, tables, scratch);
+    if (p.pre_tables) {
+        cp_async_wait<1>();  // the tables' group; the first tile's copies may still be in flight
+        __syncthreads();
+    } else {
+        build_tables(p, tables, scratch);
+    }
     grid_dependency_wait();  // stores below may overwrite what the previous launch of a sequence wrote
 
     for (;; slot += kWarps) {
@@ -874,7 +952,7 @@ ep_status launch_mode(const dev::Params& p, cudaStream_t stream, int device, boo
 // next_hdr / next_dev: the following blob of a sequence (its metadata is prefetched to L2), or null.
 ep_status launch_decode(const uint8_t* host_hdr, const void* dev_blob, size_t blob_bytes, void* dst, size_t dst_bytes,
                         int mode, void* stream_ptr, bool chained, const uint8_t* next_hdr = nullptr,
-                        const void* next_dev = nullptr) {
+                        const void* next_dev = nullptr, const uint32_t* pre_tables = nullptr) {
     if (!host_hdr || !dev_blob || !dst) return fail(EP_ERR_ARG, "decode: NULL argument");
     Header h;
     if (!parse_header(host_hdr, h)) return fail(EP_ERR_CORRUPT, "decode: malformed EPK1 header");
@@ -919,6 +997,7 @@ ep_status launch_decode(const uint8_t* host_hdr, const void* dev_blob, size_t bl
     p.payload_bytes = h.total - h.off_payload;
     p.next_blob = nullptr;
     p.next_meta_off = p.next_meta_bytes = 0;
+    p.pre_tables = pre_tables;
     Header hn;
     if (next_hdr && next_dev && parse_header(next_hdr, hn)) {  // headers of a sequence are checked up front
         p.next_blob = static_cast<const uint8_t*>(next_dev);
@@ -964,14 +1043,50 @@ extern "C" ep_status ep_decompress_many(int count, const uint8_t* const* host_hd
             return fail(EP_ERR_CORRUPT, "ep_decompress_many: blob %d has a malformed header", i);
         if (h.total != blob_bytes[i]) return fail(EP_ERR_BUFFER, "ep_decompress_many: blob %d size mismatch", i);
     }
+    // The fused entries of every blob, built once for the sequence into stream-ordered scratch (144 KB per
+    // blob). The first decode launches in plain stream order behind the expand kernel, and every later
+    // one starts after it, so all of them read finished tables. Without the scratch, each CTA builds
+    // its own tables.
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    constexpr size_t kWords = dev::kTablesBytes / 4;
+    uint32_t* pre = nullptr;
+    if (count >= 2) {
+        cudaMemPool_t pool;
+        if (scratch_pool(&pool) != cudaSuccess ||
+            cudaMallocFromPoolAsync(reinterpret_cast<void**>(&pre), size_t(count) * dev::kTablesBytes, pool, stream) !=
+                cudaSuccess) {
+            cudaGetLastError();
+            pre = nullptr;
+        }
+        for (int b = 0; pre && b < count; b += dev::kMaxExpandJobs) {
+            dev::ExpandArgs a;
+            a.count = count - b < dev::kMaxExpandJobs ? count - b : dev::kMaxExpandJobs;
+            a.out = pre + size_t(b) * kWords;
+            for (int j = 0; j < a.count; ++j) {
+                Header h;
+                parse_header(host_hdrs[b + j], h);
+                a.tables[j] = static_cast<const uint8_t*>(dev_blobs[b + j]) + h.off_tables;
+                a.tables_len[j] = h.off_offsets - h.off_tables;
+            }
+            dev::expand_tables_kernel<<<unsigned(a.count) * kNumCtx, 256, 0, stream>>>(a);
+            if (cudaGetLastError() != cudaSuccess) {
+                cudaFreeAsync(pre, stream);
+                pre = nullptr;
+            }
+        }
+    }
     for (int i = 0; i < count; ++i) {
         Header h;
         parse_header(host_hdrs[i], h);
         ep_status st = launch_decode(host_hdrs[i], dev_blobs[i], blob_bytes[i], dsts[i], dst_bytes[i], h.dtype,
                                      cuda_stream, i > 0, i + 1 < count ? host_hdrs[i + 1] : nullptr,
-                                     i + 1 < count ? dev_blobs[i + 1] : nullptr);
-        if (st != EP_OK) return st;
+                                     i + 1 < count ? dev_blobs[i + 1] : nullptr, pre ? pre + size_t(i) * kWords : nullptr);
+        if (st != EP_OK) {
+            if (pre) cudaFreeAsync(pre, stream);
+            return st;
+        }
     }
+    if (pre) cudaFreeAsync(pre, stream);
     return EP_OK;
 }
 

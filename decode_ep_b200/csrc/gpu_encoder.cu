@@ -334,34 +334,6 @@ namespace {
 using namespace enc;
 
 // Stream-ordered device scratch, released on the stream when it goes out of scope.
-// The encoder's stream-ordered scratch pool on the current device, created on first use. Freed scratch
-// up to 1 GiB stays mapped in the pool for the next call; above that it goes back at the next
-// synchronisation.
-cudaError_t scratch_pool(cudaMemPool_t* out) {
-    static std::mutex mu;
-    static cudaMemPool_t pools[64];
-    static bool made[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lk(mu);
-    if (!made[dev]) {
-        cudaMemPoolProps props = {};
-        props.allocType = cudaMemAllocationTypePinned;
-        props.location.type = cudaMemLocationTypeDevice;
-        props.location.id = dev;
-        e = cudaMemPoolCreate(&pools[dev], &props);
-        if (e != cudaSuccess) return e;
-        uint64_t keep = uint64_t(1) << 30;
-        e = cudaMemPoolSetAttribute(pools[dev], cudaMemPoolAttrReleaseThreshold, &keep);
-        if (e != cudaSuccess) return e;
-        made[dev] = true;
-    }
-    *out = pools[dev];
-    return cudaSuccess;
-}
-
 struct DevBuf {
     void* p = nullptr;
     cudaStream_t s = nullptr;
