@@ -182,11 +182,18 @@ ep_status ep_decompress_into(const uint8_t* host_hdr, const void* dev_blob, size
  * argument rules of ep_decompress_into for each one. This is the layer-sequence form of the hot
  * path, for example all linear layers of a model before a forward pass.
  *
- * The first launch is ordered after earlier work on the stream as usual. Each later launch is a
- * programmatic dependent launch of the one before it: it may expand its frequency tables and
- * prefetch its first tiles while the previous decode drains, and it stores nothing until that
- * decode has finished. Overlapping dsts are therefore written in order. One requirement follows
- * from the early reads: no blob in the list may be written by the decodes listed before it.
+ * With two or more blobs, one expand kernel first builds every blob's fused decode tables (144 KB per
+ * blob) into device scratch, taken stream-ordered from a memory pool that the library keeps per
+ * device and released stream-ordered after the last decode. Each decode CTA then copies its
+ * tables instead of rebuilding them. If the scratch cannot be had, each CTA builds its own tables,
+ * as ep_decompress_into does.
+ *
+ * The first decode is ordered after earlier work on the stream, the expand kernel included, as
+ * usual. Each later decode is a programmatic dependent launch of the one before it: it may load
+ * its tables, prefetch its first tiles and pull the next blob's metadata into L2 while the
+ * previous decode drains, and it stores nothing until that decode has finished. Overlapping dsts
+ * are therefore written in order. One requirement follows from the early reads: no blob in the
+ * list may be written by the decodes listed before it.
  * Every header is validated before anything launches, so an error launches nothing.
  * Errors: as ep_decompress_into, for the first failing blob.
  */
