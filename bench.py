@@ -278,8 +278,14 @@ def run_ours(args):
     ms_per_step = ms_max / args.steps
     value = weak_scaling_value(world, n_params, ms_per_step)
 
-    # Roofline of the decode kernel: algorithmic bytes (blob read once + container written once)
-    # over the summed per-launch event durations of one pass.
+    # Roofline of the decode kernel over the timed region: algorithmic bytes per launch (blob read once
+    # + container written once) over the average launch duration of the timed steps, i.e. the step's
+    # device time / its 276 decode launches (the step's one table-expansion launch counts in the time).
+    alg_bytes = blob_bytes + 2 * n_params
+    per_launch_ms = ms_per_step / len(layers)
+    achieved = (alg_bytes / len(layers)) / (per_launch_ms * 1e-3) / 1e9
+    # For comparison, the same kernel launched alone, one layer at a time, after the timed region: no
+    # chaining, and each CTA builds its own tables.
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in layers]
     for (a, b), h, p, n in zip(evs, hdrs, ptrs, sizes):
         a.record(stream)
@@ -287,8 +293,6 @@ def run_ours(args):
         b.record(stream)
     torch.cuda.synchronize(device)
     kernel_ms = sum(a.elapsed_time(b) for a, b in evs)
-    alg_bytes = blob_bytes + 2 * n_params
-    achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
     peak, peak_kind = measured_hbm_peak()
     tr = committed_traffic()
     traffic = None
@@ -324,13 +328,15 @@ def run_ours(args):
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_kind} copy bandwidth",
                      "per_launch_algorithmic_bytes": alg_bytes / len(layers),
-                     "per_launch_us": round(1e3 * kernel_ms / len(layers), 3),
-                     "kernel_ms_per_pass": round(kernel_ms, 4),
+                     "per_launch_us": round(1e3 * per_launch_ms, 3),
+                     "duration_source": "timed region: ms_per_step / decode launches per step",
+                     "isolated_launches_ms_per_pass": round(kernel_ms, 4),
+                     "isolated_launches_frac": round(alg_bytes / (kernel_ms * 1e-3) / 1e9 / peak, 4),
                      "frac_of_nominal_8TBs": round(achieved / 8000.0, 4)},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clk.summary(),
-        "gpu_launches": len(layers) * args.steps,
+        "gpu_launches": (len(layers) + (1 if len(layers) >= 2 else 0)) * args.steps,  # decodes + table expansion
     }
     return line
 
