@@ -62,7 +62,8 @@ def parse_args():
     ap.add_argument("--json-out", default="", help="appends each printed JSON line to this file")
     ap.add_argument("--workload", default="dit276_bf16_4bpp",
                     choices=["dit276_bf16_4bpp", "quickstart256_bf16_3.5bpp", "lognormal3072_bf16_4bpp", "sweep4096",
-                             "fp8_8192x28672_5bpp", "int8_8192x28672_3bpp", "dit276_gemm_overhead"],
+                             "fp8_8192x28672_5bpp", "int8_8192x28672_3bpp", "dit276_gemm_overhead",
+                             "dit276_fp8_gemm_overhead"],
                     help="the default is the headline line; the others print one line per tensor")
     return ap.parse_args()
 
@@ -579,25 +580,39 @@ def oracle_rate(blob, shape, seconds, workers):
     return done / (time.perf_counter() - t0)
 
 
-def run_gemm_overhead(args, tokens=4096):
+def to_e4m3_rows(w):
+    """FP8 e4m3 weight codes of w: each row scaled so its largest magnitude is 448, then cast."""
+    f = w.float()
+    f = f * (448.0 / f.abs().amax(dim=1, keepdim=True).clamp_min(1e-30))
+    return f.clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+
+
+def run_gemm_overhead(args, tokens=4096, fp8=False):
     """Decode overhead against the layer GEMMs of a prefill-sized forward pass (the pages measure it as
     the denoising-step time with compressed vs BF16 weights; that needs the real model, so this times
     the proxy: the 276 layer GEMMs y = x W^T on `tokens` synthetic activations, in layer order).
       gemm:      BF16 weights resident, GEMMs only (cuBLAS through torch.matmul);
       serial:    each layer decoded into one reused buffer, then its GEMM;
       overlap:   layer i+1 decodes on a second stream into the other of two buffers while GEMM i runs.
-    value = serial / gemm - 1 (the overhead); the overlap figure is reported beside it."""
+    value = serial / gemm - 1 (the overhead); the overlap figure is reported beside it.
+    fp8: the weights are per-row-scaled FP8 e4m3 codes of the same layers, compressed at 5 bpp and
+    decoded into e4m3; activations are e4m3 too, and the GEMMs are torch._scaled_mm with unit scales
+    and BF16 output (cuBLASLt FP8)."""
     import decode_ep_b200 as ep
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     layers = layer_list(args.layers)
+    target = 5.0 if fp8 else args.target_bpp
+    wdt = torch.float8_e4m3fn if fp8 else torch.bfloat16
     ws = [synth.dit_layer(i, shape=(M, N)).to(device) for i, _, M, N in layers]
+    if fp8:
+        ws = [to_e4m3_rows(w) for w in ws]
     streams_enc = [torch.cuda.Stream(device) for _ in range(4)]
 
     def enc(k):
         with torch.cuda.stream(streams_enc[k % 4]):
-            return ep.compress(ws[k], ep.EntroPackLossyConfig(args.target_bpp, encoder="cuda"))
+            return ep.compress(ws[k], ep.EntroPackLossyConfig(target, encoder="cuda"))
 
     with cf.ThreadPoolExecutor(max_workers=4) as ex:
         blobs = list(ex.map(enc, range(len(layers))))
@@ -606,15 +621,22 @@ def run_gemm_overhead(args, tokens=4096):
     del ws
     g = torch.Generator(device=device).manual_seed(7)
     xs = {N: torch.randn(tokens, N, generator=g, device=device, dtype=torch.bfloat16) for _, _, _, N in layers}
+    if fp8:
+        xs = {N: x.clamp(-448.0, 448.0).to(torch.float8_e4m3fn) for N, x in xs.items()}
+        one = torch.ones((), device=device, dtype=torch.float32)
     max_numel = max(M * N for _, _, M, N in layers)
     y = torch.empty(tokens * max(M for _, _, M, _ in layers), dtype=torch.bfloat16, device=device)
-    wbuf = [torch.empty(max_numel, dtype=torch.bfloat16, device=device) for _ in range(2)]
+    wbuf = [torch.empty(max_numel, dtype=wdt, device=device) for _ in range(2)]
     main = torch.cuda.current_stream(device)
     side = torch.cuda.Stream(device)
 
     def gemm(k, w):
         _, _, M, N = layers[k]
-        torch.matmul(xs[N], w.reshape(-1)[: M * N].view(M, N).t(), out=y[: tokens * M].view(tokens, M))
+        wk = w.reshape(-1)[: M * N].view(M, N).t()
+        if fp8:
+            torch._scaled_mm(xs[N], wk, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        else:
+            torch.matmul(xs[N], wk, out=y[: tokens * M].view(tokens, M))
 
     def step_gemm():
         for k in range(len(layers)):
@@ -670,17 +692,20 @@ def run_gemm_overhead(args, tokens=4096):
     if ep.device_status(main):
         raise RuntimeError("device status set")
     flops = 2.0 * tokens * sum(M * N for _, _, M, N in layers)
+    kind = "FP8 e4m3 at 5 bpp, FP8 GEMMs" if fp8 else "BF16 at 4 bpp, BF16 GEMMs"
     return {
-        "metric": "decode overhead on the 276 layer GEMMs of a 4096-token prefill (serial decode+GEMM / GEMM - 1)",
+        "metric": f"decode overhead on the 276 layer GEMMs of a 4096-token prefill ({kind}; serial decode+GEMM / GEMM - 1)",
         "value": round(100.0 * (ms_serial / ms_gemm - 1.0), 2), "unit": "%", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_serial, 3), "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16 GEMM; u32+f32 decode", "data": "synthetic",
-        "config": {"workload": "dit276_gemm_overhead", "tokens": tokens, "layers": len(layers),
-                   "target_bpp": args.target_bpp, "gemm_tflops": round(flops / (ms_gemm * 1e-3) / 1e12, 1),
+        "vs_baseline": None, "dtype": ("fp8" if fp8 else "bf16") + " GEMM; u32+f32 decode", "data": "synthetic",
+        "config": {"workload": "dit276_fp8_gemm_overhead" if fp8 else "dit276_gemm_overhead", "tokens": tokens,
+                   "layers": len(layers), "target_bpp": target, "gemm_tflops": round(flops / (ms_gemm * 1e-3) / 1e12, 1),
                    "ms_gemm_only": round(ms_gemm, 3), "ms_decode_then_gemm": round(ms_serial, 3),
                    "ms_decode_overlapped": round(ms_overlap, 3),
                    "overlap_overhead_pct": round(100.0 * (ms_overlap / ms_gemm - 1.0), 2),
-                   "gemm": "torch.matmul (cuBLAS), BF16, weights (out, in) used transposed"},
+                   "gemm": ("torch._scaled_mm (cuBLASLt), FP8 e4m3 x e4m3 -> BF16, unit scales" if fp8 else
+                            "torch.matmul (cuBLAS), BF16") + ", weights (out, in) used transposed",
+                   "actual_bpp": round(8 * sum(len(c.blob) for c in blobs) / sum(M * N for _, _, M, N in layers), 4)},
         "clocks": clk.summary(), "gpu_launches": args.steps * len(layers),
     }
 
@@ -796,6 +821,8 @@ def main():
         lines = [run_reference(args)]
     elif args.workload == "dit276_gemm_overhead":
         lines = [run_gemm_overhead(args)]
+    elif args.workload == "dit276_fp8_gemm_overhead":
+        lines = [run_gemm_overhead(args, fp8=True)]
     elif args.workload == "dit276_bf16_4bpp":
         lines = [run_ours(args)]
     else:
