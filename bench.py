@@ -490,9 +490,12 @@ def cpu_baseline(blobs, layers, seconds):
     workers = os.cpu_count() or 1
     plan = cpu_sample_plan(blobs, layers)
     n, dt = oracle_decode_for(seconds, blobs, layers, plan, workers)
+    n1, dt1 = oracle_decode_for(max(1.0, seconds / 4), blobs, layers, plan, 1)
     return {"value": round(n / dt / 1e9, 5), "unit": "Gparams/s", "cores": workers, "kind": "oracle",
+            "single_thread_value": round(n1 / dt1 / 1e9, 5),
             "sample": f"{n} parameters: runs of 16 tiles taken round-robin across all {len(layers)} layers, "
-                      f"decoded by the C oracle on {workers} threads for {dt:.1f} s"}
+                      f"decoded by the C oracle on {workers} threads for {dt:.1f} s; single thread: {n1} "
+                      f"parameters in {dt1:.1f} s"}
 
 
 # ------------------------------------------------------------------------ reference arm
