@@ -89,3 +89,20 @@ def test_cuda_encoder_errors(ep):
     with pytest.raises(ep.EntroPackError) as e:
         ep.compress(w.cpu(), ep.EntroPackLossyConfig(3.0, encoder="cuda"))
     assert e.value.status == -1
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_cuda_encoder_matches_host_bytes_fuzz(ep, seed):
+    import random
+    rnd = random.Random(2000 + seed)
+    M, N = rnd.randint(1, 200), 8 * rnd.randint(1, 64)
+    kind = rnd.choice(["bf16", "fp16", "fp32", "fp8", "int8"])
+    if kind == "fp8":
+        w = synth.fp8_codes(M, N, seed=seed)
+    elif kind == "int8":
+        w = synth.int8_codes(M, N, seed=seed)
+    else:
+        w = synth.gaussian(M, N, seed=seed, std=rnd.choice([0.02, 1.0, 300.0]), container=kind)
+    cfg = dict(target_bpp=round(rnd.uniform(0.3, 11.0), 3), rounds_per_tile=rnd.choice([0, 1, 3, 16, 33]))
+    host, dev = both(ep, w, cfg)
+    assert dev.blob == host.blob

@@ -135,3 +135,30 @@ def test_decode_rejects_bad_arguments_without_launching(ep):
     assert L.ep_decompress_into(hdr, fake_dev, len(c.blob), fake_dev, 1000, None) == -9         # dst too small
     assert L.ep_decompress_into(b"EPK2" + hdr[4:], fake_dev, len(c.blob), fake_dev, 1 << 20, None) == -6
     assert L.ep_decompress_into(None, fake_dev, len(c.blob), fake_dev, 1 << 20, None) == -1
+
+
+def _fuzz_case(seed):
+    """A seeded random tensor, target and tile size: shapes from one row to a few hundred, every container."""
+    import random
+    rnd = random.Random(seed)
+    M, N = rnd.randint(1, 160), 8 * rnd.randint(1, 48)
+    kind = rnd.choice(["bf16", "fp16", "fp32", "fp8", "int8", "outliers"])
+    if kind == "fp8":
+        w = synth.fp8_codes(M, N, seed=seed)
+    elif kind == "int8":
+        w = synth.int8_codes(M, N, seed=seed)
+    elif kind == "outliers":
+        w = synth.gaussian(M, N, seed=seed, container="fp32")
+        w.view(-1)[:: max(1, (M * N) // 7)] *= 300.0  # a few escapes
+        w = w.to(torch.bfloat16)
+    else:
+        w = synth.gaussian(M, N, seed=seed, std=rnd.choice([0.02, 1.0, 300.0]), container=kind)
+    return w, round(rnd.uniform(0.3, 11.0), 3), rnd.choice([0, 1, 2, 5, 16, 40])
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_host_encoder_matches_oracle_bytes_fuzz(ep, orc, seed):
+    w, target, G = _fuzz_case(1000 + seed)
+    ob, _ = orc.compress(synth.container_bits(w), synth.dtype_code(w), target, G if G else 16)
+    c = ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G if G else 16))
+    assert c.blob == ob
