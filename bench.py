@@ -63,7 +63,7 @@ def parse_args():
     ap.add_argument("--workload", default="dit276_bf16_4bpp",
                     choices=["dit276_bf16_4bpp", "quickstart256_bf16_3.5bpp", "lognormal3072_bf16_4bpp", "sweep4096",
                              "fp8_8192x28672_5bpp", "int8_8192x28672_3bpp", "dit276_gemm_overhead",
-                             "dit276_fp8_gemm_overhead"],
+                             "dit276_fp8_gemm_overhead", "dit276_mixed_2.3bpp"],
                     help="the default is the headline line; the others print one line per tensor")
     return ap.parse_args()
 
@@ -123,6 +123,11 @@ class ClockSampler:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
                                           "-lms", "50", "-i", str(self.index)], stdout=self.f,
                                          stderr=subprocess.DEVNULL)
+            # nvidia-smi takes a moment to start: wait (at most 3 s) for its first sample, so that a
+            # short timed region is still covered.
+            t0 = time.perf_counter()
+            while time.perf_counter() - t0 < 3.0 and self.proc.poll() is None and os.fstat(self.f.fileno()).st_size == 0:
+                time.sleep(0.02)
         except Exception:
             self.proc = None
         return self
@@ -739,6 +744,118 @@ def run_gemm_overhead(args, tokens=4096, fp8=False):
     }
 
 
+def run_mixed(args, mean_bpp=2.3):
+    """The 276-layer set at a mean of 2.3 bpp with a bitrate per layer (the README's "extreme mixed
+    bitrate" packs reach 2.3 bpp on Z-Image-Turbo by allocating bits per layer by sensitivity). Each
+    layer's target comes from ep_plan_bitrates with weight = synthetic sensitivity x mean square weight;
+    the same layers at one uniform 2.3 bpp target are the comparison. Both sets are encoded by the CUDA
+    encoder. A step is one ep_decompress_many over the 276 blobs, as in the headline line; value is the
+    mixed set's decode rate. config carries the uniform set's rate and both sets' storage and
+    sensitivity-weighted squared error."""
+    import decode_ep_b200 as ep
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    layers = layer_list(args.layers)
+    sens = synth.layer_sensitivity(len(layers))
+    shapes = [(M, N) for _, _, M, N in layers]
+    n_params = sum(M * N for M, N in shapes)
+
+    torch_threads = torch.get_num_threads()
+    torch.set_num_threads(1)
+    with cf.ThreadPoolExecutor(max_workers=max(1, min(os.cpu_count() or 1, 32))) as ex:
+        ws = list(ex.map(lambda it: synth.dit_layer(it[0], shape=(it[2], it[3])).to(device), layers))
+    torch.set_num_threads(torch_threads)
+    msq = [float(w.float().square().mean()) for w in ws]
+    weights = [s * m for s, m in zip(sens, msq)]
+    t0 = time.perf_counter()
+    targets = ep.plan_bitrates(shapes, weights, mean_bpp)
+    plan_s = time.perf_counter() - t0
+
+    streams = [torch.cuda.Stream(device) for _ in range(4)]
+
+    def encode(tlist):
+        def job(k):
+            with torch.cuda.stream(streams[k % 4]):
+                return ep.compress(ws[k], ep.EntroPackLossyConfig(tlist[k], encoder="cuda"))
+        with cf.ThreadPoolExecutor(max_workers=4) as ex:
+            out = list(ex.map(job, range(len(layers))))
+        torch.cuda.synchronize(device)
+        return out
+
+    sets = {"mixed": encode(targets), "uniform": encode([mean_bpp] * len(layers))}
+    max_numel = max(M * N for M, N in shapes)
+    out = torch.empty(max_numel, dtype=torch.bfloat16, device=device)
+    views = [out[: M * N].view(M, N) for M, N in shapes]
+    stream = torch.cuda.current_stream(device)
+    res = {}
+    for name, blobs in sets.items():
+        cost = num = den = 0.0
+        for k, c in enumerate(blobs):
+            ep.decompress_into(c, views[k], stream)
+            d = views[k].double() - ws[k].double()
+            sse = float(d.square().sum())
+            cost += sens[k] * sse
+            num, den = num + sse, den + float(ws[k].double().square().sum())
+        batch = ep.LayerBatch(list(zip(blobs, views)), stream)
+        for _ in range(args.warmup):
+            batch.run()
+        torch.cuda.synchronize(device)
+        if world > 1:
+            torch.distributed.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local) as clk:
+            torch.cuda.synchronize(device)
+            a.record(stream)
+            for _ in range(args.steps):
+                batch.run()
+            b.record(stream)
+            torch.cuda.synchronize(device)
+        if ep.device_status(stream):
+            raise RuntimeError(f"{name}: device status set")
+        (ms,) = max_over_ranks([a.elapsed_time(b)], device)
+        blob_bytes = sum(len(c.blob) for c in blobs)
+        res[name] = {"ms_per_step": ms / args.steps, "blob_bytes": blob_bytes, "cost": cost,
+                     "rel_l2": (num / den) ** 0.5, "clocks": clk.summary()}
+    del ws
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return None
+    m, u = res["mixed"], res["uniform"]
+    alg = m["blob_bytes"] + 2 * n_params
+    per_launch_ms = m["ms_per_step"] / len(layers)
+    achieved = (alg / len(layers)) / (per_launch_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    return {
+        "metric": "decode Gparams/s and % of HBM roofline (276-layer DiT set, per-layer bitrate, mean 2.3 bpp) on 1 B200",
+        "value": round(weak_scaling_value(world, n_params, m["ms_per_step"]), 2), "unit": "Gparams/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(m["ms_per_step"], 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32+f32", "data": "synthetic",
+        "config": {"workload": "dit276_mixed_2.3bpp", "layers": len(layers), "params": n_params,
+                   "mean_target_bpp": mean_bpp, "sensitivity": "synth.layer_sensitivity: lognormal, sigma 1, seed 20000",
+                   "plan_weight": "sensitivity x mean square weight", "plan_ms": round(1e3 * plan_s, 3),
+                   "target_bpp_min": round(min(targets), 3), "target_bpp_max": round(max(targets), 3),
+                   "actual_bpp_mixed": round(8 * m["blob_bytes"] / n_params, 4),
+                   "actual_bpp_uniform": round(8 * u["blob_bytes"] / n_params, 4),
+                   "weighted_sq_error_mixed_over_uniform": round(m["cost"] / u["cost"], 4),
+                   "rel_l2_pooled_mixed": round(m["rel_l2"], 5), "rel_l2_pooled_uniform": round(u["rel_l2"], 5),
+                   "uniform_gparams_s": round(weak_scaling_value(world, n_params, u["ms_per_step"]), 2),
+                   "uniform_ms_per_step": round(u["ms_per_step"], 4),
+                   "l2": "inputs larger than L2 (blobs %.2f GB read per step)" % (m["blob_bytes"] / 1e9),
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None, "peak_source": f"{peak_kind} copy bandwidth",
+                     "per_launch_algorithmic_bytes": alg / len(layers),
+                     "duration_source": "timed region: ms_per_step / decode launches per step"},
+        "cpu_baseline": None, "e2e": None, "clocks": m["clocks"],
+        "gpu_launches": (len(layers) + (1 if len(layers) >= 2 else 0)) * args.steps,
+    }
+
+
 def run_workload(args):
     """One JSON line per tensor of a single-tensor workload. A step is one ep_decompress_into of the
     tensor. Each timed step is bracketed by its own CUDA events, with a 256 MB write between steps that
@@ -852,6 +969,8 @@ def main():
         lines = [run_gemm_overhead(args)]
     elif args.workload == "dit276_fp8_gemm_overhead":
         lines = [run_gemm_overhead(args, fp8=True)]
+    elif args.workload == "dit276_mixed_2.3bpp":
+        lines = [run_mixed(args)]
     elif args.workload == "dit276_bf16_4bpp":
         lines = [run_ours(args)]
     else:

@@ -24,7 +24,7 @@ import torch
 from . import build as _build
 
 __all__ = ["EntroPackLossyConfig", "CompressedTensor", "EntroPackError", "LayerBatch", "compress", "decompress",
-           "decompress_into", "decompress_many", "decode_coords", "device_status", "blob_info", "lib"]
+           "decompress_into", "decompress_many", "decode_coords", "device_status", "blob_info", "plan_bitrates", "lib"]
 
 EP_BF16, EP_FP16, EP_FP32, EP_FP8_E4M3, EP_INT8 = 1, 2, 3, 4, 5
 _TORCH_TO_EP = {torch.bfloat16: EP_BF16, torch.float16: EP_FP16, torch.float32: EP_FP32,
@@ -77,11 +77,13 @@ def lib() -> ctypes.CDLL:
                                          c.POINTER(c.c_size_t), c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
                                          c.c_void_p]
         L.ep_get_device_status.argtypes = [c.c_void_p, c.POINTER(c.c_int32)]
+        L.ep_plan_bitrates.argtypes = [c.c_int64, c.POINTER(c.c_int64), c.POINTER(c.c_int64), c.POINTER(c.c_double),
+                                       c.c_double, c.c_double, c.c_double, c.POINTER(_Options), c.POINTER(c.c_double)]
         L.ep_status_string.restype = c.c_char_p
         L.ep_status_string.argtypes = [c.c_int]
         L.ep_last_error.restype = c.c_char_p
         for name in ("ep_compress", "ep_compress_cuda", "ep_blob_info", "ep_decompress_into", "ep_decode_coords_into", "ep_decompress",
-                     "ep_get_device_status", "ep_decompress_many"):
+                     "ep_get_device_status", "ep_decompress_many", "ep_plan_bitrates"):
             getattr(L, name).restype = c.c_int
         _lib = L
     return _lib
@@ -223,6 +225,26 @@ def compress_cuda_noalloc(tensor: torch.Tensor, config: EntroPackLossyConfig | f
                                             ctypes.byref(actual))
     _check(st, "compress_cuda_noalloc")
     return CompressedTensor(ctypes.string_at(buf, nbytes.value), (rows, cols), tensor.dtype, actual.value)
+
+
+def plan_bitrates(shapes, weights, mean_bpp: float, min_bpp: float = 0.001, max_bpp: float = 11.0,
+                  rounds_per_tile: int = 0) -> list[float]:
+    """ep_plan_bitrates: per-layer target bitrates that spend ``mean_bpp`` bits per parameter over the
+    layers ``shapes`` [(rows, cols), ...], weighting layer i's squared error by ``weights[i]`` (the
+    README's mixed-bitrate packs, which allocate bits by per-layer sensitivity). Each result is a
+    target for ``compress``."""
+    n = len(shapes)
+    if n != len(weights) or n == 0:
+        raise EntroPackError(-1, "plan_bitrates: need one weight per shape, and at least one layer")
+    I64, F64 = ctypes.c_int64 * n, ctypes.c_double * n
+    rows, cols = I64(*[int(r) for r, _ in shapes]), I64(*[int(c) for _, c in shapes])
+    w, out = F64(*[float(x) for x in weights]), F64()
+    opt = _Options()
+    lib().ep_options_default(ctypes.byref(opt))
+    opt.rounds_per_tile = int(rounds_per_tile)
+    _check(lib().ep_plan_bitrates(n, rows, cols, w, float(mean_bpp), float(min_bpp), float(max_bpp),
+                                  ctypes.byref(opt), out), "plan_bitrates")
+    return list(out)
 
 
 def _stream_ptr(stream) -> int | None:

@@ -144,6 +144,39 @@ ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt, int64_t ro
                                    double target_bpp, const ep_options* opt, void* cuda_stream, uint8_t* blob,
                                    size_t blob_capacity, size_t* blob_bytes, double* actual_bpp);
 
+/*
+ * ep_plan_bitrates: per-layer targets for a set of tensors that share one storage budget.
+ *
+ * The EntroPack README ("Pre-quantised models") describes packs whose bitrate is allocated layer by
+ * layer by sensitivity, at 2.3 to 3.0 bits per parameter on average; it does not give the rule. This
+ * function implements the high-rate allocation: layer i, coded at a data rate of R bits per
+ * parameter, is taken to have a squared weight error proportional to weight[i] * 2^(-2R). It returns
+ * the bpp_out[i] (whole-blob bits per parameter, as ep_compress takes them) that minimise
+ *     sum_i rows[i]*cols[i] * weight[i] * 2^(-2 (bpp_out[i] - meta_i))
+ * subject to sum_i rows[i]*cols[i]*bpp_out[i] = mean_bpp * sum_i rows[i]*cols[i] and
+ * max(min_bpp, meta_i) <= bpp_out[i] <= max_bpp. meta_i is layer i's metadata in bits per parameter
+ * (header, row scales, the largest possible tables section, tile offsets and the per-tile state cost
+ * of the encoders' storage estimate, at the tile size opt gives or the encoders' automatic one).
+ * The solution has one water level theta: bpp_out[i] = clamp(meta_i + log2(weight[i])/2 + theta).
+ *
+ * n           number of layers, >= 1. rows, cols, weight: host arrays of n entries; bpp_out receives n.
+ * weight      > 0 and finite: the cost of a unit of mean squared error in layer i, in the units the
+ *             caller cares about. For an error in the weights' own units use sensitivity times the
+ *             layer's mean square weight (the encoders normalise each row, so the error of a layer
+ *             scales with its mean square).
+ * opt         may be NULL; only rounds_per_tile is read (0 = the encoders' automatic choice).
+ *
+ * Budgets below every layer's floor give each layer its floor (the blobs then overshoot, as
+ * ep_compress does for a target below the metadata); budgets above every ceiling give each max_bpp.
+ * Pure host arithmetic: no device, no allocation visible to the caller.
+ * Errors: EP_ERR_ARG (NULL, n < 1, a weight not finite and > 0, rounds_per_tile > 1024),
+ * EP_ERR_SHAPE (a layer that ep_compress would reject), EP_ERR_TARGET (a bound outside [0.001, 11],
+ * min_bpp > max_bpp or mean_bpp > max_bpp). bpp_out is written only on EP_OK.
+ */
+ep_status ep_plan_bitrates(int64_t n, const int64_t* rows, const int64_t* cols, const double* weight,
+                           double mean_bpp, double min_bpp, double max_bpp, const ep_options* opt,
+                           double* bpp_out);
+
 /* Releases a blob returned by ep_compress or ep_compress_cuda. NULL is accepted. */
 void ep_blob_free(uint8_t* blob);
 

@@ -89,6 +89,17 @@ def dit_layer(i: int, shape: tuple[int, int] | None = None, sigma: float = 0.3) 
     return w.to(torch.bfloat16)
 
 
+def layer_sensitivity(n: int, seed: int = 20000, sigma: float = 1.0) -> list[float]:
+    """A synthetic per-layer sensitivity: n draws of exp(sigma * z), z ~ N(0, 1), in layer order.
+
+    The pages' mixed-bitrate packs rank layers by a sensitivity measured on the real model, which is
+    not available; this stands in for it with a lognormal spread (sigma = 1: the middle two thirds of
+    layers within a factor e of the median).
+    """
+    z = torch.randn(n, generator=_gen(seed), dtype=torch.float64)
+    return [float(v) for v in torch.exp(sigma * z)]
+
+
 def gaussian(M: int, N: int, seed: int, std: float = 0.02, container: str = "fp32") -> torch.Tensor:
     """M x N with entries N(0, std^2). Drawn in float32, then cast to the container."""
     w = torch.randn(M, N, generator=_gen(seed)) * std

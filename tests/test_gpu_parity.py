@@ -288,3 +288,28 @@ def test_decompress_many_matches_single_decodes(orc):
     status_clean()
     last = bf[-1]
     assert np.array_equal(gpu_bits(views[-1]), orc.decompress(last.blob))
+
+
+def test_planned_mixed_bitrate_sequence(orc):
+    """Layers given per-layer targets by ep_plan_bitrates (a spread of rates, r > 0 on the top ones),
+    encoded by the CUDA encoder, decoded as one sequence: every output equals the oracle's decode of
+    the same blob, and the set's storage lands on the planned mean."""
+    import math
+    import random
+    shapes = [(512, 256), (256, 1024), (64, 3840), (1024, 512), (384, 384), (3840, 64)]
+    rnd = random.Random(3)
+    sens = [math.exp(rnd.gauss(0.0, 2.0)) for _ in shapes]
+    ws = [synth.dit_layer(40 + i, shape=s).cuda() for i, s in enumerate(shapes)]
+    weights = [s * float(w.float().square().mean()) for s, w in zip(sens, ws)]
+    mean = 3.0
+    targets = ep.plan_bitrates(shapes, weights, mean)
+    assert max(targets) - min(targets) > 2.0
+    comps = [ep.compress(w, ep.EntroPackLossyConfig(t, encoder="cuda")) for w, t in zip(ws, targets)]
+    outs = [torch.empty(c.shape, dtype=c.dtype, device="cuda") for c in comps]
+    ep.LayerBatch(list(zip(comps, outs))).run()
+    torch.cuda.synchronize()
+    status_clean()
+    for c, o in zip(comps, outs):
+        assert np.array_equal(gpu_bits(o), orc.decompress(c.blob))
+    n = sum(r * k for r, k in shapes)
+    assert 8 * sum(len(c.blob) for c in comps) / n <= mean + 0.05
