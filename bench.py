@@ -930,9 +930,18 @@ def run_workload(args):
             e2e = {"value": round(world * n_params / (ms * 1e-3) / 1e9, 3), "unit": "Gparams/s",
                    "h2d_bytes_per_step": len(c.blob), "d2h_bytes_per_step": out_bytes, "ms_per_step": round(ms, 4)}
         cpu = None
+        orc_enc = None
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             import oracle
             oracle.build()
+            if n_params <= (1 << 24):
+                # The oracle encoder on the same tensor (single thread), for the encoder comparison; the
+                # 235M-parameter code matrices are skipped to keep the run within minutes.
+                t_o = time.perf_counter()
+                ob, _ = oracle.compress(synth.container_bits(w), synth.dtype_code(w), target,
+                                       int.from_bytes(c.header[20:22], "little"))
+                orc_enc = {"seconds": round(time.perf_counter() - t_o, 3), "threads": 1,
+                           "bytes_identical_to_host_encoder": ob == c.blob}
             cores = os.cpu_count() or 1
             many = oracle_rate(c.blob, (M, N), args.cpu_seconds / 4, cores)
             one = oracle_rate(c.blob, (M, N), args.cpu_seconds / 8, 1)
@@ -948,7 +957,7 @@ def run_workload(args):
             "config": {"workload": label, "shape": [M, N], "params": n_params, "container": str(c.dtype).replace("torch.", ""),
                        "target_bpp": target, "actual_bpp": round(c.actual_bpp, 4),
                        "rounds_per_tile": int.from_bytes(c.header[20:22], "little"),
-                       "rel_l2": round(rel, 6), "encode_s": round(t_enc, 3),
+                       "rel_l2": round(rel, 6), "encode_s": round(t_enc, 3), "oracle_encode": orc_enc,
                        "l2": "256 MB write between timed steps (L2 flushed)", "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": None, "peak_source": f"{peak_kind} copy bandwidth",
