@@ -144,6 +144,35 @@ __device__ __forceinline__ void sub_mul_f32x2(float a0, float a1, float k0, floa
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(r), "l"(cc));
     asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(r));
 }
+// Bulk copies (TMA, no multicast) completed on a shared-memory mbarrier.
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// dst and src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+// Polls phase `parity` of the barrier at most `tries` times; true once it has completed.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t tries) {
+    for (uint32_t i = 0; i < tries; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+constexpr uint32_t kTableWaitTries = 1u << 14;
+
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
 
@@ -180,10 +209,15 @@ __device__ __forceinline__ uint32_t entry_template(int c, int sym, uint32_t f) {
 //      first slot (a 7-step binary search over cum) and carries markers forward: entry = D + (slot << 20).
 // Starts the copy of pre-built fused entries (9 x 4096 words, 144 KB) into the table region, as one
 // copy group: nine 16-byte copies per thread.
-__device__ __forceinline__ void load_tables_async(const Params& p, uint8_t* tables) {
-    const uint32_t dst = smem_addr(tables);
-    for (uint32_t i = threadIdx.x; i < kTablesBytes / 16; i += kThreads) cp_async16(dst + 16 * i, p.pre_tables + 4 * i, 16);
-    cp_async_commit();
+// A sequence's prepared entries (144 KB) arrive by nine bulk copies, issued by thread 0 and completed on
+// the mbarrier `bar` (phase 0). The barrier must have been initialised, and the initialisation seen by
+// every thread, before the call.
+__device__ __forceinline__ void load_tables_bulk(const Params& p, uint8_t* tables, uint32_t bar) {
+    if (threadIdx.x == 0) {
+        mbar_expect_tx(bar, kTablesBytes);
+        for (uint32_t c = 0; c < kTablesBytes / kCtxBytes; ++c)
+            bulk_copy_g2s(smem_addr(tables) + c * kCtxBytes, p.pre_tables + c * (kCtxBytes / 4), kCtxBytes, bar);
+    }
 }
 
 // Starts the copy of the serialised tables (the first kScratchTableCap bytes of the section, zero past
@@ -766,10 +800,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
                                                        : rings_after + (warp - rings_before) * kRingBytes)};
 
     grid_dependents_launch();  // lets the next launch of a sequence start its prologue early
-    if (p.pre_tables)
-        load_tables_async(p, tables);
-    else
+    const uint32_t bar = smem_addr(scratch);  // the build scratch is unused when the tables are prepared
+    if (p.pre_tables) {
+        if (threadIdx.x == 0) mbar_init(bar, 1);
+        __syncthreads();
+        load_tables_bulk(p, tables, bar);
+    } else {
         stage_tables_async(p, scratch);
+    }
 
     // The next layer's metadata (tables, tile offsets, scales) goes to L2 now, so its prologue reads L2.
     if (p.next_blob) {
@@ -781,7 +819,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
     // Tiles are dealt round-robin over the CTAs first, so that consecutive tiles land on different SMs
     // and a partial last wave is spread over the whole GPU: tile = (k * kWarps + warp) * grid + block.
     // The copies of the warp's first tile are issued before the table build, which hides them. Every
-    // thread commits exactly one group here (empty without a first tile), behind the tables' group.
+    // thread commits exactly one group here (empty without a first tile), behind the tables' group when
+    // the tables are built here.
     uint32_t slot = warp;
     bool first_issued = false;
     {
@@ -796,15 +835,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
         }
         cp_async_commit();
     }
+    bool tables_ok = true;
     if (p.pre_tables) {
-        cp_async_wait<1>();  // the tables' group; the first tile's copies may still be in flight
-        __syncthreads();
+        // The first tile's copies may still be in flight. A copy that has not landed after the bounded
+        // wait flags the launch, and the CTA decodes nothing (after a second bounded wait, so that no
+        // copy still writes into its shared memory when it exits).
+        const bool ok = mbar_wait(bar, 0, kTableWaitTries);
+        if (__syncthreads_or(!ok)) {
+            if (threadIdx.x == 0) atomicOr(&g_status, int(EP_DEV_TABLE_COPY));
+            mbar_wait(bar, 0, kTableWaitTries);
+            tables_ok = false;
+        }
     } else {
         build_tables(p, tables, scratch);
     }
     grid_dependency_wait();  // stores below may overwrite what the previous launch of a sequence wrote
 
-    for (;; slot += kWarps) {
+    for (; tables_ok; slot += kWarps) {
         const uint32_t tile = slot * gridDim.x + blockIdx.x;
         if (tile >= p.T) break;
         TileGeom tg;

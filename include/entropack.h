@@ -63,6 +63,7 @@ typedef enum {
 #define EP_DEV_CORRUPT_TILE 1u  /* a tile's final rANS states or its word count did not check out */
 #define EP_DEV_BAD_OFFSETS 2u   /* a tile offset points outside the payload */
 #define EP_DEV_BAD_TABLES 4u    /* a frequency table does not sum to 4096 */
+#define EP_DEV_TABLE_COPY 8u    /* a sequence's prepared tables did not reach a CTA in time; it decoded nothing */
 
 /* Encoder options. Start from ep_options_default(). */
 typedef struct {
