@@ -501,8 +501,8 @@ struct RawWindow {
 // Fast round: every lane holds a group, the tile has no escapes, and the round's words are in the ring.
 // Values come from the entries' value fields. RAW: the tile carries r >= 1 raw low bits per coordinate,
 // taken from `raw` (loaded a round ahead); then t = hi 2^r + lo and the parity of u_0..u_6 is that of
-// the lo's.
-template <int MODE, bool WRAP, bool RAW = false>
+// the lo's. WAIT: the warp's first stores of the launch; they wait for the previous launch of a sequence.
+template <int MODE, bool WRAP, bool RAW = false, bool WAIT = false>
 __device__ __forceinline__ void round_fast(const Params& p, uint32_t t0, uint32_t& x, uint32_t& pa, uint32_t ring_base,
                                            uint32_t g, uint32_t lt_mask, const RowCursor& rc,
                                            const RawWindow* raw = nullptr) {
@@ -562,6 +562,7 @@ __device__ __forceinline__ void round_fast(const Params& p, uint32_t t0, uint32_
 #pragma unroll
         for (int i = 0; i < 8; ++i) z[i] = __float2int_rn((m[i] - (i < 7 ? K : K7)) * 2.0f);
     }
+    if constexpr (WAIT) grid_dependency_wait();
     store_group<MODE>(p.dst, g, y, z);
 }
 
@@ -678,17 +679,29 @@ __device__ __forceinline__ void issue_chunk(const uint8_t* payload, const TileGe
 // end: reads stay within 512 bytes of it, still inside the CTA's shared memory (the scratch region
 // follows the last ring). A longer stream runs here while a round cannot reach the ring's end, and its
 // next chunk is copied into the slot the rounds have left behind. The raw window of the next round is
-// loaded while the current one decodes. Returns the number of rounds done.
+// loaded while the current one decodes. Returns the number of rounds done. If `waited` is false, the
+// first round waits for the previous launch of a sequence before its stores, and sets it.
 template <int MODE, bool RAW>
 __device__ __forceinline__ uint32_t fast_rounds(const Params& p, uint32_t t0, const TileGeom& tg, const uint8_t* payload,
                                                 uint32_t ring_base, uint32_t lane, uint32_t lt_mask,
                                                 const uint16_t* scales, RowCursor& rc, TileState& st, uint32_t& issued,
-                                                const uint8_t* rawsec, uint32_t raw_avail) {
+                                                const uint8_t* rawsec, uint32_t raw_avail, bool& waited) {
     const uint32_t Rf = tg.ng / 32, r = uint32_t(p.r);
     const uint32_t pa_lim = ring_base + (tg.chunks <= kRingChunks ? kRingBytes : kRingBytes - 2 * kRoundWords);
     uint32_t k = 0, g = tg.g0 + lane, x = st.x, pa = ring_base + st.pb;
     RawWindow cur, nxt;
     if (RAW) cur.load(rawsec, raw_avail, lane, r);
+    if (!waited && Rf > 0 && pa <= pa_lim) {
+        // Round 0 decodes while the previous launch may still be running; only its stores wait. No chunk
+        // is due yet: the first kRingChunks chunks were issued with the tile.
+        if (RAW) nxt.load(rawsec, raw_avail, 32 + lane, r);
+        round_fast<MODE, false, RAW, true>(p, t0, x, pa, 0, g, lt_mask, rc, &cur);
+        rc.advance(p, scales);
+        if (RAW) cur = nxt;
+        waited = true;
+        k = 1;
+        g += 32;
+    }
     if (tg.chunks <= kRingChunks) {
         for (; k < Rf && pa <= pa_lim; ++k, g += 32) {
             if (RAW) nxt.load(rawsec, raw_avail, 32 * (k + 1) + lane, r);
@@ -849,7 +862,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
     } else {
         build_tables(p, tables, scratch);
     }
-    grid_dependency_wait();  // stores below may overwrite what the previous launch of a sequence wrote
+    // Stores may overwrite what the previous launch of a sequence wrote, so each warp waits for it
+    // before its first store: after decoding its first round, when that round is a fast one.
+    bool waited = false;
 
     for (; tables_ok; slot += kWarps) {
         const uint32_t tile = slot * gridDim.x + blockIdx.x;
@@ -894,12 +909,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
 
         if (!tg.esc) {
             k = tg.raw ? fast_rounds<MODE, true>(p, t0, tg, payload, ring.base, lane, lt_mask, scales, rc, st, issued,
-                                                 rawsec, raw_avail)
+                                                 rawsec, raw_avail, waited)
                        : fast_rounds<MODE, false>(p, t0, tg, payload, ring.base, lane, lt_mask, scales, rc, st, issued,
-                                                  rawsec, raw_avail);
+                                                  rawsec, raw_avail, waited);
         }
 
         if (k < R) {
+            if (!waited) {
+                grid_dependency_wait();
+                waited = true;
+            }
             // Rolling ring: tiles with escapes or raw bits, the last rounds of a stream longer than the
             // ring, and the ragged last round. Up to three chunks in flight; one more per round while the
             // chunk it replaces lies wholly behind pb.
@@ -949,6 +968,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
         if (!ok && lane == 0) atomicOr(&g_status, int(EP_DEV_CORRUPT_TILE));
     }
     if (first_issued) cp_async_wait<0>();
+    // A launch of a sequence ends after the one before it, whether or not this warp stored anything.
+    if (!waited) grid_dependency_wait();
 }
 
 
