@@ -32,6 +32,7 @@
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "capi_internal.h"
@@ -103,6 +104,7 @@ struct Params {
     // are pulled into L2 while this one decodes.
     const uint8_t* next_blob;
     uint32_t next_meta_off, next_meta_bytes;  // [off_scales, off_payload) of the next blob
+    uint32_t test_no_table_copy;              // test hook: leave the prepared-table copies unissued
     // The fused entries of this blob, 9 x 4096 in shared-memory block order, built once for the whole
     // sequence by expand_tables_kernel; null means each CTA builds them (build_tables).
     const uint32_t* pre_tables;
@@ -158,12 +160,13 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
                  "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
 }
-// Polls phase `parity` of the barrier at most `tries` times; true once it has completed.
+// Polls phase `parity` of the barrier at most `tries` times, each poll suspending the thread for at most
+// about 1 us; true once the phase has completed.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t tries) {
     for (uint32_t i = 0; i < tries; ++i) {
         uint32_t done;
         asm volatile(
-            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 1000;\n selp.u32 %0, 1, 0, p;\n}"
             : "=r"(done)
             : "r"(bar), "r"(parity)
             : "memory");
@@ -215,7 +218,7 @@ __device__ __forceinline__ uint32_t entry_template(int c, int sym, uint32_t f) {
 __device__ __forceinline__ void load_tables_bulk(const Params& p, uint8_t* tables, uint32_t bar) {
     if (threadIdx.x == 0) {
         mbar_expect_tx(bar, kTablesBytes);
-        for (uint32_t c = 0; c < kTablesBytes / kCtxBytes; ++c)
+        for (uint32_t c = 0; c < (p.test_no_table_copy ? 0u : kTablesBytes / kCtxBytes); ++c)
             bulk_copy_g2s(smem_addr(tables) + c * kCtxBytes, p.pre_tables + c * (kCtxBytes / 4), kCtxBytes, bar);
     }
 }
@@ -1020,7 +1023,8 @@ ep_status launch_mode(const dev::Params& p, cudaStream_t stream, int device, boo
 // next_hdr / next_dev: the following blob of a sequence (its metadata is prefetched to L2), or null.
 ep_status launch_decode(const uint8_t* host_hdr, const void* dev_blob, size_t blob_bytes, void* dst, size_t dst_bytes,
                         int mode, void* stream_ptr, bool chained, const uint8_t* next_hdr = nullptr,
-                        const void* next_dev = nullptr, const uint32_t* pre_tables = nullptr) {
+                        const void* next_dev = nullptr, const uint32_t* pre_tables = nullptr,
+                        bool test_no_table_copy = false) {
     if (!host_hdr || !dev_blob || !dst) return fail(EP_ERR_ARG, "decode: NULL argument");
     Header h;
     if (!parse_header(host_hdr, h)) return fail(EP_ERR_CORRUPT, "decode: malformed EPK1 header");
@@ -1066,6 +1070,7 @@ ep_status launch_decode(const uint8_t* host_hdr, const void* dev_blob, size_t bl
     p.next_blob = nullptr;
     p.next_meta_off = p.next_meta_bytes = 0;
     p.pre_tables = pre_tables;
+    p.test_no_table_copy = test_no_table_copy ? 1u : 0u;
     Header hn;
     if (next_hdr && next_dev && parse_header(next_hdr, hn)) {  // headers of a sequence are checked up front
         p.next_blob = static_cast<const uint8_t*>(next_dev);
@@ -1143,12 +1148,17 @@ extern "C" ep_status ep_decompress_many(int count, const uint8_t* const* host_hd
             }
         }
     }
+    // Test hook (see the header): the prepared-table copies are left unissued, so that every CTA's
+    // bounded wait for them runs out.
+    const char* hook = std::getenv("EPK_TEST_TABLE_COPY_TIMEOUT");
+    const bool no_copy = hook && hook[0] == '1';
     for (int i = 0; i < count; ++i) {
         Header h;
         parse_header(host_hdrs[i], h);
         ep_status st = launch_decode(host_hdrs[i], dev_blobs[i], blob_bytes[i], dsts[i], dst_bytes[i], h.dtype,
                                      cuda_stream, i > 0, i + 1 < count ? host_hdrs[i + 1] : nullptr,
-                                     i + 1 < count ? dev_blobs[i + 1] : nullptr, pre ? pre + size_t(i) * kWords : nullptr);
+                                     i + 1 < count ? dev_blobs[i + 1] : nullptr, pre ? pre + size_t(i) * kWords : nullptr,
+                                     no_copy);
         if (st != EP_OK) {
             if (pre) cudaFreeAsync(pre, stream);
             return st;

@@ -218,18 +218,22 @@ ep_status ep_decompress_into(const uint8_t* host_hdr, const void* dev_blob, size
  *
  * With two or more blobs, one expand kernel first builds every blob's fused decode tables (144 KB per
  * blob) into device scratch, taken stream-ordered from a memory pool that the library keeps per
- * device and released stream-ordered after the last decode. Each decode CTA then copies its
- * tables instead of rebuilding them. If the scratch cannot be had, each CTA builds its own tables,
- * as ep_decompress_into does.
+ * device and released stream-ordered after the last decode. Each decode CTA then takes its tables
+ * by bulk copies (TMA, completed on a shared-memory barrier) instead of rebuilding them. Its wait for
+ * them is bounded; a copy that has not landed in time sets EP_DEV_TABLE_COPY, and that CTA decodes
+ * nothing. If the scratch cannot be had, each CTA builds its own tables, as ep_decompress_into does.
  *
  * The first decode is ordered after earlier work on the stream, the expand kernel included, as
  * usual. Each later decode is a programmatic dependent launch of the one before it: it may load
- * its tables, prefetch its first tiles and pull the next blob's metadata into L2 while the
- * previous decode drains, and it stores nothing until that decode has finished. Overlapping dsts
- * are therefore written in order. One requirement follows from the early reads: no blob in the
- * list may be written by the decodes listed before it.
+ * its tables, prefetch its first tiles, pull the next blob's metadata into L2 and decode each
+ * warp's first round while the previous decode drains, and it stores nothing until that decode has
+ * finished. Overlapping dsts are therefore written in order. One requirement follows from the early
+ * reads: no blob in the list may be written by the decodes listed before it.
  * Every header is validated before anything launches, so an error launches nothing.
  * Errors: as ep_decompress_into, for the first failing blob.
+ * Test hook: with the environment variable EPK_TEST_TABLE_COPY_TIMEOUT set to 1 when the call is made,
+ * the table copies are not issued, so every CTA's bounded wait runs out (each poll suspends about
+ * 1 us, 2^14 polls twice) and EP_DEV_TABLE_COPY is set. The test suite uses it to check that path.
  */
 ep_status ep_decompress_many(int count, const uint8_t* const* host_hdrs, const void* const* dev_blobs,
                              const size_t* blob_bytes, void* const* dsts, const size_t* dst_bytes,

@@ -313,3 +313,21 @@ def test_planned_mixed_bitrate_sequence(orc):
         assert np.array_equal(gpu_bits(o), orc.decompress(c.blob))
     n = sum(r * k for r, k in shapes)
     assert 8 * sum(len(c.blob) for c in comps) / n <= mean + 0.05
+
+
+def test_table_copy_wait_runs_out_into_status(orc, monkeypatch):
+    """The bounded wait for a sequence's table copies: with the copies left unissued (test hook), every
+    CTA gives up, sets EP_DEV_TABLE_COPY and decodes nothing; the context stays usable."""
+    comps = [ep.compress(synth.gaussian(64, 256, seed=s, container="bf16"), 4.0) for s in (21, 22)]
+    outs = [torch.zeros(c.shape, dtype=c.dtype, device="cuda") for c in comps]
+    status_clean()
+    monkeypatch.setenv("EPK_TEST_TABLE_COPY_TIMEOUT", "1")
+    ep.decompress_many(list(zip(comps, outs)))
+    st = ep.device_status()
+    monkeypatch.delenv("EPK_TEST_TABLE_COPY_TIMEOUT")
+    assert st & 8
+    assert all(int(o.view(torch.int16).abs().sum()) == 0 for o in outs)  # nothing was stored
+    ep.decompress_many(list(zip(comps, outs)))
+    status_clean()
+    for c, o in zip(comps, outs):
+        assert np.array_equal(gpu_bits(o), orc.decompress(c.blob))
