@@ -41,7 +41,7 @@ def _rank_main(rank, world, port, results):
 
 def test_max_over_ranks_and_weak_scaling_two_gloo_ranks():
     world = 2
-    results = mp.Manager().dict()
+    results = mp.get_context("spawn").Manager().dict()  # no fork of this (threaded) process
     mp.spawn(_rank_main, args=(world, _free_port(), results), nprocs=world, join=True)
     for r in range(world):
         ms, best, value = results[r]
