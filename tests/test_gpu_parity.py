@@ -331,3 +331,32 @@ def test_table_copy_wait_runs_out_into_status(orc, monkeypatch):
     status_clean()
     for c, o in zip(comps, outs):
         assert np.array_equal(gpu_bits(o), orc.decompress(c.blob))
+
+
+def test_decompress_many_edge_counts(orc):
+    """Sequences of 0 and 1 blobs, and one longer than an expand launch takes (512 blobs): the tables are
+    then prepared by two expand launches. Small mixed shapes and containers, each checked against the
+    oracle."""
+    ep.decompress_many([])
+    status_clean()
+    one = ep.compress(synth.gaussian(40, 64, seed=31, container="fp16"), 5.0)
+    out1 = torch.empty(one.shape, dtype=one.dtype, device="cuda")
+    ep.decompress_many([(one, out1)])
+    status_clean()
+    assert np.array_equal(gpu_bits(out1), orc.decompress(one.blob))
+    comps = []
+    for i in range(530):
+        M, N = 1 + (i * 7) % 23, 8 * (1 + (i * 5) % 9)
+        kind = ("bf16", "fp16", "fp32")[i % 3]
+        comps.append(ep.compress(synth.gaussian(M, N, seed=1000 + i, container=kind), 1.0 + (i % 9)))
+    outs = [torch.empty(c.shape, dtype=c.dtype, device="cuda") for c in comps]
+    ep.decompress_many(list(zip(comps, outs)))
+    torch.cuda.synchronize()
+    status_clean()
+    for c, o in zip(comps, outs):
+        want = orc.decompress(c.blob)
+        got = gpu_bits(o)
+        if got.dtype == np.float32:
+            assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+        else:
+            assert np.array_equal(got, want)
