@@ -642,7 +642,10 @@ def run_gemm_overhead(args, tokens=4096, fp8=False):
     the proxy: the 276 layer GEMMs y = x W^T on `tokens` synthetic activations, in layer order).
       gemm:      BF16 weights resident, GEMMs only (cuBLAS through torch.matmul);
       serial:    each layer decoded into one reused buffer, then its GEMM;
-      overlap:   layer i+1 decodes on a second stream into the other of two buffers while GEMM i runs.
+      overlap:   layer i+1 decodes on a second stream into the other of two buffers while GEMM i runs;
+      blocks:    each transformer block's layers (8 per block, then the 4 projections) decode as one
+                 sequence (ep_decompress_many: tables prepared once, launches chained) into their own
+                 buffers, then the block's GEMMs run.
     value = serial / gemm - 1 (the overhead); the overlap figure is reported beside it.
     fp8: the weights are per-row-scaled FP8 e4m3 codes of the same layers, compressed at 5 bpp and
     decoded into e4m3; activations are e4m3 too, and the GEMMs are torch._scaled_mm with unit scales
@@ -691,6 +694,28 @@ def run_gemm_overhead(args, tokens=4096, fp8=False):
         for k in range(len(layers)):
             gemm(k, resident[k])
 
+    # Blocks of consecutive layers decoded as one sequence each, into per-layer views of one buffer.
+    block_of_layer = [min(i // 8, 34) for i in range(len(layers))]
+    blocks = {}
+    for k, bi in enumerate(block_of_layer):
+        blocks.setdefault(bi, []).append(k)
+    block_elems = max(sum(layers[k][2] * layers[k][3] for k in ks) for ks in blocks.values())
+    bbuf = torch.empty(block_elems, dtype=wdt, device=device)
+    block_runs = []
+    for ks in blocks.values():
+        views, off = [], 0
+        for k in ks:
+            _, _, M, N = layers[k]
+            views.append(bbuf[off: off + M * N].view(M, N))
+            off += M * N
+        block_runs.append((ks, views, ep.LayerBatch([(blobs[k], v) for k, v in zip(ks, views)], main)))
+
+    def step_blocks():
+        for ks, views, batch in block_runs:
+            batch.run()
+            for k, v in zip(ks, views):
+                gemm(k, v)
+
     def step_serial():
         for k, c in enumerate(blobs):
             out = wbuf[0][: c.shape[0] * c.shape[1]].view(c.shape)
@@ -738,6 +763,7 @@ def run_gemm_overhead(args, tokens=4096, fp8=False):
         ms_gemm = timed(step_gemm)
         ms_serial = timed(step_serial)
         ms_overlap = timed(step_overlap)
+        ms_blocks = timed(step_blocks)
     if ep.device_status(main):
         raise RuntimeError("device status set")
     flops = 2.0 * tokens * sum(M * N for _, _, M, N in layers)
@@ -752,10 +778,12 @@ def run_gemm_overhead(args, tokens=4096, fp8=False):
                    "ms_gemm_only": round(ms_gemm, 3), "ms_decode_then_gemm": round(ms_serial, 3),
                    "ms_decode_overlapped": round(ms_overlap, 3),
                    "overlap_overhead_pct": round(100.0 * (ms_overlap / ms_gemm - 1.0), 2),
+                   "ms_block_sequences": round(ms_blocks, 3),
+                   "block_sequences_overhead_pct": round(100.0 * (ms_blocks / ms_gemm - 1.0), 2),
                    "gemm": ("torch._scaled_mm (cuBLASLt), FP8 e4m3 x e4m3 -> BF16, unit scales" if fp8 else
                             "torch.matmul (cuBLAS), BF16") + ", weights (out, in) used transposed",
                    "actual_bpp": round(8 * sum(len(c.blob) for c in blobs) / sum(M * N for _, _, M, N in layers), 4)},
-        "clocks": clk.summary(), "gpu_launches": args.steps * len(layers),
+        "clocks": clk.summary(), "gpu_launches": args.steps * len(layers),  # the serial pass's decodes
     }
 
 
