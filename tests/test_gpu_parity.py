@@ -360,3 +360,39 @@ def test_decompress_many_edge_counts(orc):
             assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
         else:
             assert np.array_equal(got, want)
+
+
+@pytest.mark.slow
+def test_full_276_layer_sequence_sampled(orc):
+    """The benchmark's launch configuration at full size: all 276 DiT-like layers (6.17 G parameters at
+    4 bpp, CUDA encoder) decoded by one ep_decompress_many (tables prepared once, chained launches), each
+    layer into its own buffer. Eight sampled tiles (the first and the last among them) of every 17th layer
+    and of the last layer are compared with the oracle's decode of the same tiles."""
+    import concurrent.futures as cf
+    shapes = synth.dit_layer_shapes()
+    with cf.ThreadPoolExecutor(max_workers=8) as ex:
+        futs = [ex.submit(synth.dit_layer, i, (M, N)) for i, (_, M, N) in enumerate(shapes)]
+        comps = []
+        for f in futs:
+            w = f.result().cuda()
+            comps.append(ep.compress(w, ep.EntroPackLossyConfig(4.0, encoder="cuda")))
+            del w
+    outs = [torch.empty(c.shape, dtype=c.dtype, device="cuda") for c in comps]
+    ep.decompress_many(list(zip(comps, outs)))
+    torch.cuda.synchronize()
+    status_clean()
+    n = sum(M * N for _, M, N in shapes)
+    assert 8 * sum(len(c.blob) for c in comps) / n <= 4.05
+    rng = np.random.default_rng(7)
+    for i in sorted(set(list(range(0, len(shapes), 17)) + [len(shapes) - 1])):
+        c = comps[i]
+        info = orc.blob_info(c.blob)
+        T, per_tile = info["num_tiles"], 32 * info["G"] * 8
+        tiles = sorted(set([0, T - 1] + [int(t) for t in rng.integers(0, T, size=6)]))
+        want = np.zeros(c.shape, np.uint16)
+        mask = np.zeros(c.shape, bool)
+        for j in tiles:
+            orc.decode_tiles(c.blob, j, j + 1, want)
+            mask.reshape(-1)[j * per_tile: (j + 1) * per_tile] = True
+        got = gpu_bits(outs[i])
+        assert np.array_equal(got[mask], want[mask]), f"layer {i}"
