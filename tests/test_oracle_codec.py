@@ -346,3 +346,68 @@ def test_corruption_is_detected(orc):
     hdr = bytearray(blob); hdr[70] ^= 1   # a scale byte: caught by the CRC
     with pytest.raises(orc.OracleError):
         orc.blob_info(bytes(hdr))
+
+
+# ------------------------------------------------- the rescale against its plain definition
+
+def _ordered(bits: np.ndarray, nbits: int) -> np.ndarray:
+    """Sign-magnitude bit patterns mapped to integers in value order, so that adjacent representable
+    values differ by 1 (both zeros map to 0)."""
+    b = bits.astype(np.int64)
+    sign = 1 << (nbits - 1)
+    return np.where(b & sign, -(b & (sign - 1)), b)
+
+
+RESCALE_CASES = [
+    ("fp32_2.3", lambda: synth.gaussian(256, 512, seed=2, container="fp32"), 2.3),
+    ("fp32_5", lambda: synth.gaussian(256, 512, seed=2, container="fp32"), 5.0),
+    ("fp32_11", lambda: synth.gaussian(256, 512, seed=2, container="fp32"), 11.0),
+    ("fp32_11_outliers", lambda: synth.lognormal_rows_with_outliers(n=512, seed=5, outlier_frac=1e-3).float(), 11.0),
+    ("bf16_4", lambda: synth.dit_layer(7, shape=(512, 512)), 4.0),
+    ("fp16_8", lambda: synth.gaussian(256, 512, seed=2, container="fp16"), 8.0),
+    ("fp8_5", lambda: synth.fp8_codes(128, 512, seed=3), 5.0),
+    ("int8_3", lambda: synth.int8_codes(128, 512, seed=4), 3.0),
+]
+
+
+@pytest.mark.parametrize("name,maker,target", RESCALE_CASES, ids=[c[0] for c in RESCALE_CASES])
+def test_rescale_within_one_container_ulp_of_its_definition(orc, name, maker, target):
+    """The per-row rescale (modelscope paper page, summary: 行重缩放) has a plain definition: the decoded
+    value is s_row·v/α in binary32, rounded to the container. Written out literally that is
+    fl32(fl32(s_row·v)/α). The oracle computes fl32(v·fl32(s_row/α)), one correctly rounded factor per row
+    and one multiply. Here the two are compared element by element on oracle-decoded blobs in all five
+    containers, the definition evaluated independently in numpy: s_row (a bf16) times v = z/2 in float64
+    is exact, one rounding to float32, one IEEE float32 division.
+
+    Bound: RN(s/α) = (s/α)(1 + d) with |d| <= 2^-24, so v·RN(s/α) lies less than one binary32 ulp from
+    s·v/α before its rounding, and less than 1.5 ulp after it; the definition lies within 0.5 ulp. Two
+    binary32 values less than 2 ulp apart are at most 1 ulp apart, and a monotone container rounding
+    keeps them at most one container step apart."""
+    w = maker()
+    a, dt = bits(w)
+    blob, _ = orc.compress(a, dt, target, 16)
+    info = orc.blob_info(blob)
+    out, z = orc.decompress(blob, with_coords=True)
+    off = int.from_bytes(blob[28:32], "little")
+    sbits = np.frombuffer(blob[off: off + 2 * info["rows"]], np.uint16)
+    s = (sbits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    sv = (s[:, None] * (z.astype(np.float64) * 0.5)).astype(np.float32)
+    y_def = (sv / np.float32(info["alpha"])).astype(np.float32)
+    ref = orc.to_container(y_def, dt).reshape(out.shape)
+    if dt in (1, 2):
+        d = np.abs(_ordered(out.view(np.uint16), 16) - _ordered(ref.view(np.uint16), 16))
+    elif dt == 3:
+        d = np.abs(_ordered(out.view(np.uint32), 32) - _ordered(ref.view(np.uint32), 32))
+    elif dt == 4:
+        d = np.abs(_ordered(out.view(np.uint8), 8) - _ordered(ref.view(np.uint8), 8))
+    else:
+        d = np.abs(out.astype(np.int64) - ref.astype(np.int64))
+    assert d.max() <= 1, f"{name}: {int(d.max())} container ulps from fl32(fl32(s*v)/alpha)"
+    frac = float((d > 0).mean())
+    print(f"{name}: {frac:.4%} of values one container ulp from the literal definition")
+    if dt == 3:
+        assert frac > 0.0  # the two orders are distinct readings in binary32 (3 to 26 % of values here)
+    # a planted mistake must fail the pin: the rescale applied with alpha in place of 1/alpha
+    wrong = orc.to_container((sv * np.float32(info["alpha"])).astype(np.float32), dt).reshape(out.shape)
+    if np.any(z != 0):
+        assert not np.array_equal(wrong, out)
