@@ -64,7 +64,7 @@ def parse_args():
     ap.add_argument("--workload", default="dit276_bf16_4bpp",
                     choices=["dit276_bf16_4bpp", "quickstart256_bf16_3.5bpp", "lognormal3072_bf16_4bpp", "sweep4096",
                              "fp8_8192x28672_5bpp", "int8_8192x28672_3bpp", "dit276_gemm_overhead",
-                             "dit276_fp8_gemm_overhead", "dit276_mixed_2.3bpp"],
+                             "dit276_fp8_gemm_overhead", "dit276_mixed_2.3bpp", "cuda_encode_gate_10240x3840"],
                     help="the default is the headline line; the others print one line per tensor")
     return ap.parse_args()
 
@@ -387,15 +387,17 @@ def time_cuda_encoder(blobs, layers, target_bpp, device, workers=8):
             g = ep.compress(inputs[k], ep.EntroPackLossyConfig(target_bpp, encoder="cuda"))
         return g.blob == blobs[k].blob
 
-    torch.cuda.synchronize(device)
-    t0 = time.perf_counter()
-    with cf.ThreadPoolExecutor(max_workers=workers) as ex:
-        same = all(ex.map(job, range(len(layers))))
-    torch.cuda.synchronize(device)
-    wall = time.perf_counter() - t0
+    walls, same = [], True
+    for _ in range(2):  # the first pass also pays module loading and the scratch pool's growth
+        torch.cuda.synchronize(device)
+        t0 = time.perf_counter()
+        with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+            same = all(ex.map(job, range(len(layers)))) and same
+        torch.cuda.synchronize(device)
+        walls.append(time.perf_counter() - t0)
     del inputs
-    return {"seconds": round(wall, 3), "layers": len(layers), "host_threads": workers,
-            "inputs": "resident in device memory", "bytes_identical_to_host_encoder": same}
+    return {"seconds": round(walls[1], 3), "seconds_first_pass": round(walls[0], 3), "layers": len(layers),
+            "host_threads": workers, "inputs": "resident in device memory", "bytes_identical_to_host_encoder": same}
 
 
 def run_e2e(args, L, blobs, layers, device, stream):
@@ -1013,6 +1015,28 @@ def run_workload(args):
     return lines if rank == 0 else None
 
 
+def run_cuda_encode_gate(args):
+    """The CUDA encoder (ep_compress_cuda) on one 10240x3840 BF16 layer of the DiT-like set (layer 4) at the
+    target bitrate, input in device memory: one untimed call (module load, scratch pool), then `--steps`
+    timed calls. The profile of its kernels is taken on this command."""
+    import decode_ep_b200 as ep
+    torch.cuda.set_device(0)
+    w = synth.dit_layer(4).cuda()
+    cfg = ep.EntroPackLossyConfig(args.target_bpp, encoder="cuda")
+    ref = ep.compress(w, cfg)
+    times = []
+    for _ in range(max(1, args.steps)):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        c = ep.compress(w, cfg)
+        torch.cuda.synchronize()
+        times.append(time.perf_counter() - t0)
+        assert c.blob == ref.blob
+    return {"workload": "cuda_encode_gate_10240x3840", "metric": "CUDA encoder wall time per tensor", "unit": "s",
+            "value": round(statistics.median(times), 4), "best": round(min(times), 4), "steps": len(times),
+            "params": w.numel(), "actual_bpp": round(ref.actual_bpp, 4), "higher_is_better": False}
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -1025,6 +1049,8 @@ def main():
         lines = [run_mixed(args)]
     elif args.workload == "dit276_bf16_4bpp":
         lines = [run_ours(args)]
+    elif args.workload == "cuda_encode_gate_10240x3840":
+        lines = [run_cuda_encode_gate(args)]
     else:
         lines = run_workload(args)
     for line in lines or []:

@@ -201,17 +201,6 @@ __device__ __forceinline__ uint32_t entry_template(int c, int sym, uint32_t f) {
     return ((f & 0xFFFu) << 8) | (c <= 4 ? (cls << 7) | field : field);
 }
 
-// Expands the serialised tables into the fused entries. The entry of slot t in a context is
-// D[s] + (t << 20), where s is the symbol owning the slot (cum[s] <= t < cum[s] + f[s]) and
-// D[s] = template[s] - (cum[s] << 20); D is never 0, since f >= 1 sits in bits 8-19. Three passes, no
-// branching per slot:
-//   1. zero the 144 KB and stage the serialised bytes;
-//   2. one thread per symbol unpacks its 12-bit frequency; warp scans prefix-sum them into cum, and
-//      each symbol with f > 0 drops D[s] at slot cum[s] (the marker);
-//   3. each thread takes 36 consecutive entries of the 9 x 4096, starts from the marker in force at its
-//      first slot (a 7-step binary search over cum) and carries markers forward: entry = D + (slot << 20).
-// Starts the copy of pre-built fused entries (9 x 4096 words, 144 KB) into the table region, as one
-// copy group: nine 16-byte copies per thread.
 // A sequence's prepared entries (144 KB) arrive by nine bulk copies, issued by thread 0 and completed on
 // the mbarrier `bar` (phase 0). The barrier must have been initialised, and the initialisation seen by
 // every thread, before the call.
@@ -235,6 +224,15 @@ __device__ __forceinline__ void stage_tables_async(const Params& p, uint8_t* scr
     cp_async_commit();
 }
 
+// Expands the serialised tables into the fused entries. The entry of slot t in a context is
+// D[s] + (t << 20), where s is the symbol owning the slot (cum[s] <= t < cum[s] + f[s]) and
+// D[s] = template[s] - (cum[s] << 20); D is never 0, since f >= 1 sits in bits 8-19. Three passes, no
+// branching per slot:
+//   1. zero the 144 KB (the serialised bytes were staged by stage_tables_async);
+//   2. one thread per symbol unpacks its 12-bit frequency; warp scans prefix-sum them into cum, and
+//      each symbol with f > 0 drops D[s] at slot cum[s] (the marker);
+//   3. each thread takes 36 consecutive entries of the 9 x 4096, starts from the marker in force at its
+//      first slot (a 7-step binary search over cum) and carries markers forward: entry = D + (slot << 20).
 __device__ void build_tables(const Params& p, uint8_t* tables, uint8_t* scratch) {
     uint32_t* cum = reinterpret_cast<uint32_t*>(scratch + kScratchCum);    // [9][129]
     uint8_t* tbytes = scratch + kScratchBytes;

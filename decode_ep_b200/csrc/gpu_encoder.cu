@@ -351,11 +351,12 @@ struct DevBuf {
     T* as() const { return static_cast<T*>(p); }
 };
 
-#define EPK_CUDA(call)                                                                              \
+#define EPK_CUDA_IN(fn, call)                                                                       \
     do {                                                                                             \
         cudaError_t e_ = (call);                                                                     \
-        if (e_ != cudaSuccess) return fail(EP_ERR_CUDA, "ep_compress_cuda: %s: %s", #call, cudaGetErrorString(e_)); \
+        if (e_ != cudaSuccess) return fail(EP_ERR_CUDA, fn ": %s: %s", #call, cudaGetErrorString(e_)); \
     } while (0)
+#define EPK_CUDA(call) EPK_CUDA_IN("ep_compress_cuda", call)
 
 unsigned blocks_for(int64_t n, int per) { return unsigned((n + per - 1) / per); }
 
@@ -593,6 +594,8 @@ struct Carve {
 }  // namespace
 }  // namespace epk
 
+#define EPK_CUDA_NA(call) EPK_CUDA_IN("ep_compress_cuda_noalloc", call)
+
 extern "C" ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt, int64_t rows, int64_t cols,
                                               int64_t row_stride, double target_bpp, const ep_options* opt_in,
                                               void* cuda_stream, uint8_t* blob, size_t blob_capacity,
@@ -660,29 +663,43 @@ extern "C" ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt,
     }
 
     int device = 0;
-    EPK_CUDA(cudaGetDevice(&device));
+    EPK_CUDA_NA(cudaGetDevice(&device));
     if (device < 0 || device >= 64) return fail(EP_ERR_CUDA, "ep_compress_cuda_noalloc: device %d out of range", device);
+    // The static area used is the current device's, so the input must live there too.
+    if (pa.device != device)
+        return fail(EP_ERR_ARG, "ep_compress_cuda_noalloc: the input is on device %d, the current device is %d",
+                    pa.device, device);
     StaticScratch& ss = g_static[device];
     std::lock_guard<std::mutex> lock(ss.mu);
     if (!ss.resolved) {  // once per device, with that device current
-        EPK_CUDA(cudaGetSymbolAddress(&ss.addr, genc::g_static_scratch));
+        EPK_CUDA_NA(cudaGetSymbolAddress(&ss.addr, genc::g_static_scratch));
         ss.resolved = true;
     }
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    // Every exit from here on, error paths included, first drains the stream: no kernel or copy of this
+    // call may still use the static area once the lock is released. Declared after the lock, so it runs
+    // before the unlock.
+    struct DrainOnExit {
+        cudaStream_t s;
+        ~DrainOnExit() {
+            cudaStreamSynchronize(s);
+            cudaGetLastError();
+        }
+    } drain{st};
     Carve carve{static_cast<unsigned char*>(ss.addr)};
     plan(carve, &d_sbits, &d_s, &small, &d_counts, &pcounts, &d_tq, &d_bq, &d_tabs, &d_words, &d_states, &d_nwords,
          &d_esc, &d_start, &d_payload);
     unsigned long long* pesc = pcounts + size_t(genc::kHistBins) * genc::kMaxProbes;
 
-    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const genc::Src src{static_cast<const uint8_t*>(dev_data), int(dt), N, row_stride};
     try {
-        EPK_CUDA(cudaMemsetAsync(small, 0, 64, st));
-        EPK_CUDA(genc::launch_row_scales(src, M, d_sbits, d_s, small, reinterpret_cast<int*>(small + 3), st));
+        EPK_CUDA_NA(cudaMemsetAsync(small, 0, 64, st));
+        EPK_CUDA_NA(genc::launch_row_scales(src, M, d_sbits, d_s, small, reinterpret_cast<int*>(small + 3), st));
         std::vector<uint16_t> sbits(static_cast<size_t>(M));
         unsigned long long hsmall[4];
-        EPK_CUDA(cudaMemcpyAsync(sbits.data(), d_sbits, size_t(M) * 2, cudaMemcpyDeviceToHost, st));
-        EPK_CUDA(cudaMemcpyAsync(hsmall, small, sizeof(hsmall), cudaMemcpyDeviceToHost, st));
-        EPK_CUDA(cudaStreamSynchronize(st));
+        EPK_CUDA_NA(cudaMemcpyAsync(sbits.data(), d_sbits, size_t(M) * 2, cudaMemcpyDeviceToHost, st));
+        EPK_CUDA_NA(cudaMemcpyAsync(hsmall, small, sizeof(hsmall), cudaMemcpyDeviceToHost, st));
+        EPK_CUDA_NA(cudaStreamSynchronize(st));
         if (int(hsmall[3])) return fail(EP_ERR_NONFINITE, "ep_compress_cuda_noalloc: NaN or Inf in the input");
         double amax;
         std::memcpy(&amax, &hsmall[0], 8);
@@ -711,16 +728,16 @@ extern "C" ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt,
                     nlo[2 * n + 2] = nlo[n], nhi[2 * n + 2] = nmid[n];
                 }
             }
-            EPK_CUDA(cudaMemsetAsync(pcounts, 0, sizeof(unsigned long long) * genc::kHistBins * nodes, st));
-            EPK_CUDA(cudaMemsetAsync(pesc, 0, sizeof(unsigned long long) * genc::kMaxProbes, st));
+            EPK_CUDA_NA(cudaMemsetAsync(pcounts, 0, sizeof(unsigned long long) * genc::kHistBins * nodes, st));
+            EPK_CUDA_NA(cudaMemsetAsync(pesc, 0, sizeof(unsigned long long) * genc::kMaxProbes, st));
             genc::sample_counts_kernel<<<dim3(blocks_for(Rs * gpr, 256), unsigned(nodes)), 256, 0, st>>>(
                 src, M, gpr, Rs, d_s, pr, pcounts, pesc);
-            EPK_CUDA(cudaGetLastError());
-            EPK_CUDA(cudaMemcpyAsync(hcounts.data(), pcounts, sizeof(unsigned long long) * genc::kHistBins * nodes,
+            EPK_CUDA_NA(cudaGetLastError());
+            EPK_CUDA_NA(cudaMemcpyAsync(hcounts.data(), pcounts, sizeof(unsigned long long) * genc::kHistBins * nodes,
                                      cudaMemcpyDeviceToHost, st));
-            EPK_CUDA(cudaMemcpyAsync(hcounts.data() + size_t(genc::kHistBins) * genc::kMaxProbes, pesc,
+            EPK_CUDA_NA(cudaMemcpyAsync(hcounts.data() + size_t(genc::kHistBins) * genc::kMaxProbes, pesc,
                                      sizeof(unsigned long long) * nodes, cudaMemcpyDeviceToHost, st));
-            EPK_CUDA(cudaStreamSynchronize(st));
+            EPK_CUDA_NA(cudaStreamSynchronize(st));
             for (int n = 0, step = 0; step < depth; ++step) {
                 std::copy(hcounts.begin() + size_t(n) * genc::kHistBins, hcounts.begin() + size_t(n + 1) * genc::kHistBins,
                           counts.begin());
@@ -734,39 +751,39 @@ extern "C" ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt,
         const float alpha = float(std::exp2(lo));
 
         // Quantisation, raw bits, tables.
-        EPK_CUDA(cudaMemsetAsync(small + 2, 0, 8, st));
+        EPK_CUDA_NA(cudaMemsetAsync(small + 2, 0, 8, st));
         genc::quantize_kernel<<<blocks_for(NG, 256), 256, 0, st>>>(src, NG, gpr, d_s, alpha, d_tq, d_bq, small + 2);
-        EPK_CUDA(cudaGetLastError());
+        EPK_CUDA_NA(cudaGetLastError());
         unsigned long long tmax_u = 0;
-        EPK_CUDA(cudaMemcpyAsync(&tmax_u, small + 2, 8, cudaMemcpyDeviceToHost, st));
-        EPK_CUDA(cudaStreamSynchronize(st));
+        EPK_CUDA_NA(cudaMemcpyAsync(&tmax_u, small + 2, 8, cudaMemcpyDeviceToHost, st));
+        EPK_CUDA_NA(cudaStreamSynchronize(st));
         const int64_t tmax = int64_t(tmax_u);
         int r = raw_bits_for(alpha);
         while (r < 12 && tmax >= (int64_t(1) << (15 + r))) ++r;
         if (tmax >= (int64_t(1) << (15 + r))) return fail(EP_ERR_ARG, "ep_compress_cuda_noalloc: value range too wide to code");
-        EPK_CUDA(cudaMemsetAsync(d_counts, 0, sizeof(unsigned long long) * genc::kHistBins, st));
+        EPK_CUDA_NA(cudaMemsetAsync(d_counts, 0, sizeof(unsigned long long) * genc::kHistBins, st));
         genc::full_counts_kernel<<<std::min<unsigned>(blocks_for(NG, 256), 148u * 8u), 256, 0, st>>>(d_tq, d_bq, NG, r,
                                                                                                    d_counts);
-        EPK_CUDA(cudaGetLastError());
-        EPK_CUDA(cudaMemcpyAsync(counts.data(), d_counts, sizeof(unsigned long long) * genc::kHistBins,
+        EPK_CUDA_NA(cudaGetLastError());
+        EPK_CUDA_NA(cudaMemcpyAsync(counts.data(), d_counts, sizeof(unsigned long long) * genc::kHistBins,
                                  cudaMemcpyDeviceToHost, st));
-        EPK_CUDA(cudaStreamSynchronize(st));
+        EPK_CUDA_NA(cudaStreamSynchronize(st));
         Tables tab;
         tab.build(counts);
 
         // Tiles.
-        EPK_CUDA(cudaMemcpyAsync(d_tabs, tab.f, sizeof(uint32_t) * genc::kHistBins, cudaMemcpyHostToDevice, st));
-        EPK_CUDA(cudaMemcpyAsync(d_tabs + genc::kHistBins, tab.cum, sizeof(uint32_t) * genc::kHistBins,
+        EPK_CUDA_NA(cudaMemcpyAsync(d_tabs, tab.f, sizeof(uint32_t) * genc::kHistBins, cudaMemcpyHostToDevice, st));
+        EPK_CUDA_NA(cudaMemcpyAsync(d_tabs + genc::kHistBins, tab.cum, sizeof(uint32_t) * genc::kHistBins,
                                  cudaMemcpyHostToDevice, st));
         genc::encode_tiles_kernel<<<blocks_for(T, 8), 256, 0, st>>>(d_tq, d_bq, NG, T, G, r, d_tabs,
                                                                    d_tabs + genc::kHistBins, d_words, d_states,
                                                                    d_nwords, d_esc);
-        EPK_CUDA(cudaGetLastError());
+        EPK_CUDA_NA(cudaGetLastError());
         std::vector<uint32_t> nwords(T);
         std::vector<uint8_t> esc(T);
-        EPK_CUDA(cudaMemcpyAsync(nwords.data(), d_nwords, size_t(T) * 4, cudaMemcpyDeviceToHost, st));
-        EPK_CUDA(cudaMemcpyAsync(esc.data(), d_esc, size_t(T), cudaMemcpyDeviceToHost, st));
-        EPK_CUDA(cudaStreamSynchronize(st));
+        EPK_CUDA_NA(cudaMemcpyAsync(nwords.data(), d_nwords, size_t(T) * 4, cudaMemcpyDeviceToHost, st));
+        EPK_CUDA_NA(cudaMemcpyAsync(esc.data(), d_esc, size_t(T), cudaMemcpyDeviceToHost, st));
+        EPK_CUDA_NA(cudaStreamSynchronize(st));
         std::vector<uint64_t> start(size_t(T) + 1, 0);
         for (uint32_t j = 0; j < T; ++j) {
             const int64_t ng = std::min(per_tile, NG - int64_t(j) * per_tile);
@@ -779,14 +796,14 @@ extern "C" ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt,
                         (unsigned long long)L.total, (unsigned long long)blob_capacity);
 
         // Payload in the static area (zeroed first: padding bytes stay zero), then into the caller's buffer.
-        EPK_CUDA(cudaMemcpyAsync(d_start, start.data(), sizeof(uint64_t) * (size_t(T) + 1), cudaMemcpyHostToDevice, st));
-        EPK_CUDA(cudaMemsetAsync(d_payload, 0, size_t(start[T]), st));
+        EPK_CUDA_NA(cudaMemcpyAsync(d_start, start.data(), sizeof(uint64_t) * (size_t(T) + 1), cudaMemcpyHostToDevice, st));
+        EPK_CUDA_NA(cudaMemsetAsync(d_payload, 0, size_t(start[T]), st));
         genc::assemble_kernel<<<blocks_for(T, 8), 256, 0, st>>>(d_payload, d_start, d_states, d_words, d_nwords, d_tq,
                                                               NG, T, G, r);
-        EPK_CUDA(cudaGetLastError());
+        EPK_CUDA_NA(cudaGetLastError());
         std::memset(blob, 0, size_t(L.off_payload));
-        EPK_CUDA(cudaMemcpyAsync(blob + L.off_payload, d_payload, size_t(start[T]), cudaMemcpyDeviceToHost, st));
-        EPK_CUDA(cudaStreamSynchronize(st));
+        EPK_CUDA_NA(cudaMemcpyAsync(blob + L.off_payload, d_payload, size_t(start[T]), cudaMemcpyDeviceToHost, st));
+        EPK_CUDA_NA(cudaStreamSynchronize(st));
         write_metadata(blob, L, dt, r, rows, cols, alpha, uint32_t(G), T, sbits.data(), tab, start.data(), esc.data());
         finish_crc(blob, L);
         *blob_bytes = size_t(L.total);

@@ -136,9 +136,14 @@ ep_status ep_compress_cuda(const void* dev_data, ep_dtype dt, int64_t rows, int6
  * blob        caller-owned host buffer of blob_capacity bytes; the blob is written there and *blob_bytes
  *             receives its size. 8*rows*cols + 2*rows + 4096 bytes always suffice; a smaller buffer that
  *             cannot hold the blob gives EP_ERR_BUFFER.
- * Races       the array is shared by every call on a device in the process. Calls on one device are
- *             serialised by a lock held for the whole call, and each call synchronises cuda_stream before
- *             it returns, so no two calls use the array at once. Other processes have their own array.
+ * Set-up      the first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *             that device current, and keeps it for later calls. Make that first call before any stream
+ *             capture. A cudaDeviceReset discards the array with the context; calls after one are not
+ *             supported. dev_data must be on the current device (EP_ERR_ARG otherwise).
+ * Races       the array is shared by every call on a device in the process, and keeps the last call's
+ *             contents. Calls on one device are serialised by a lock held for the whole call, and once
+ *             a call has queued work it synchronises cuda_stream before it returns, on error paths too,
+ *             so no two calls of this library use the array at once. Other processes have their own array.
  * Other arguments and errors as ep_compress_cuda.
  */
 ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt, int64_t rows, int64_t cols, int64_t row_stride,

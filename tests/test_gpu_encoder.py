@@ -1,8 +1,11 @@
-"""CUDA encoder parity: ep_compress_cuda must write the same blob bytes as the host encoder.
+"""CUDA encoder parity: ep_compress_cuda must write the same blob bytes as the oracle encoder and the host
+encoder.
 
-The host encoder is itself byte-identical to the oracle on these cases (test_lib_cpu), so equal bytes
-here tie the GPU encoder to the oracle too. Integer and byte work is held to bit-exactness: every
-scale, every bisection decision, every lattice point and every rANS word must agree.
+The CUDA encoder and the host encoder compile the same lattice and table code, so agreement between those
+two alone would not check that code. Every case is therefore also compared, byte for byte, with the
+oracle's encoder (oracle/, which shares no code with either) on the same input, the oracle taking the
+tile size G from the product blob's header. Integer and byte work is held to bit-exactness: every scale,
+every bisection decision, every lattice point and every rANS word must agree.
 """
 import pytest
 import torch
@@ -44,11 +47,29 @@ def both(ep, w, cfg_kwargs):
     return host, dev
 
 
+def oracle_bytes(orc, w, target, blob):
+    """The oracle encoder's blob for the same input and target, at the tile size G the product chose."""
+    G = int.from_bytes(blob[20:22], "little")
+    ob, _ = orc.compress(synth.container_bits(w.cpu()), synth.dtype_code(w), target, G)
+    return ob
+
+
 @pytest.mark.parametrize("name,maker,target,G", CASES, ids=[c[0] for c in CASES])
-def test_cuda_encoder_matches_host_bytes(ep, name, maker, target, G):
-    host, dev = both(ep, maker(), dict(target_bpp=target, rounds_per_tile=G))
+def test_cuda_encoder_matches_oracle_and_host_bytes(ep, orc, name, maker, target, G):
+    w = maker()
+    host, dev = both(ep, w, dict(target_bpp=target, rounds_per_tile=G))
+    assert dev.blob == oracle_bytes(orc, w, target, dev.blob), "CUDA encoder differs from the oracle encoder"
     assert dev.blob == host.blob
     assert dev.actual_bpp == host.actual_bpp
+
+
+@pytest.mark.parametrize("workload", ["lognormal3072", "dit_q_3840"])
+def test_cuda_encoder_matches_oracle_full_size(ep, orc, workload):
+    """Full-size tensors against the oracle encoder directly: the 3072x3072 lognormal-rows matrix with
+    outliers and one 3840x3840 layer of the DiT-like set, both at 4 bpp."""
+    w = synth.lognormal_rows_with_outliers() if workload == "lognormal3072" else synth.dit_layer(0)
+    dev = ep.compress(w.cuda(), ep.EntroPackLossyConfig(4.0, encoder="cuda"))
+    assert dev.blob == oracle_bytes(orc, w, 4.0, dev.blob)
 
 
 @pytest.mark.parametrize("workload", ["lognormal3072", "dit_gate", "fp8_rows", "sweep_6bpp"])
@@ -92,7 +113,7 @@ def test_cuda_encoder_errors(ep):
 
 
 @pytest.mark.parametrize("seed", range(16))
-def test_cuda_encoder_matches_host_bytes_fuzz(ep, seed):
+def test_cuda_encoder_matches_oracle_and_host_bytes_fuzz(ep, orc, seed):
     import random
     rnd = random.Random(2000 + seed)
     M, N = rnd.randint(1, 200), 8 * rnd.randint(1, 64)
@@ -106,3 +127,4 @@ def test_cuda_encoder_matches_host_bytes_fuzz(ep, seed):
     cfg = dict(target_bpp=round(rnd.uniform(0.3, 11.0), 3), rounds_per_tile=rnd.choice([0, 1, 3, 16, 33]))
     host, dev = both(ep, w, cfg)
     assert dev.blob == host.blob
+    assert dev.blob == oracle_bytes(orc, w, cfg["target_bpp"], dev.blob)

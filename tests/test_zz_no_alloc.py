@@ -41,6 +41,45 @@ def test_two_calls_in_a_row_match_the_allocating_entry_point(ep):
     assert y.shape == w2.shape
 
 
+def test_calls_allocate_no_device_memory(ep):
+    """The property the entry point exists for: after a first call (which resolves the static area), further
+    calls leave the device's free memory (cudaMemGetInfo) and the reserved size of the device's current
+    memory pool unchanged."""
+    from cuda.bindings import runtime as rt
+    w = synth.gaussian(1024, 1024, seed=23, container="bf16").cuda()
+    torch.cuda.synchronize()
+    ep.compress_cuda_noalloc(w, 4.0)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    err, pool = rt.cudaDeviceGetMemPool(torch.cuda.current_device())
+    assert err == rt.cudaError_t.cudaSuccess
+
+    def pool_bytes():
+        e, v = rt.cudaMemPoolGetAttribute(pool, rt.cudaMemPoolAttr.cudaMemPoolAttrReservedMemCurrent)
+        assert e == rt.cudaError_t.cudaSuccess
+        return int(v)
+
+    reserved0 = pool_bytes()
+    for _ in range(2):
+        ep.compress_cuda_noalloc(w, 4.0)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert pool_bytes() == reserved0
+
+
+def test_input_on_another_device_is_rejected(ep):
+    if torch.cuda.device_count() < 2:
+        pytest.skip("needs two devices")
+    w = synth.quickstart_256().to("cuda:1")
+    buf = (ctypes.c_uint8 * (1 << 20))()
+    nbytes, bpp = ctypes.c_size_t(), ctypes.c_double()
+    opt = ep.EntroPackLossyConfig(3.5)._options()
+    with torch.cuda.device(0):
+        st = ep.lib().ep_compress_cuda_noalloc(w.data_ptr(), 1, 256, 256, 256, 3.5, ctypes.byref(opt), None, buf,
+                                               1 << 20, ctypes.byref(nbytes), ctypes.byref(bpp))
+    assert st == -1
+
+
 def test_oversize_request_is_rejected_and_the_next_call_works(ep):
     big = synth.gaussian(4096, 4096, seed=2, container="bf16").cuda()  # needs far more than the static area
     with pytest.raises(ep.EntroPackError) as e:
