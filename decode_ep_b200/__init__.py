@@ -41,7 +41,8 @@ class EntroPackError(RuntimeError):
 
 class _Options(ctypes.Structure):
     _fields_ = [("rounds_per_tile", ctypes.c_uint32), ("sample_coords", ctypes.c_uint32),
-                ("bisection_iters", ctypes.c_uint32), ("threads", ctypes.c_int32)]
+                ("bisection_iters", ctypes.c_uint32), ("threads", ctypes.c_int32),
+                ("format_version", ctypes.c_uint32)]
 
 
 _lib = None
@@ -107,6 +108,8 @@ class EntroPackLossyConfig:
     encoder: "host" runs the multithreaded host encoder (ep_compress; CUDA inputs are copied to the host
     once). "cuda" runs the GPU encoder (ep_compress_cuda) on a CUDA input, on the current stream. Both
     write the same blob bytes.
+    format_version: 2 (the default) writes 8-bit frequency tables with one rANS renormalisation per pair
+    of symbols, the faster decode on B200; 1 writes 12-bit tables with one renormalisation per symbol.
     """
     target_bpp: float
     rounds_per_tile: int = 0
@@ -114,9 +117,11 @@ class EntroPackLossyConfig:
     bisection_iters: int = 40
     threads: int = 0
     encoder: str = "host"
+    format_version: int = 2
 
     def _options(self) -> _Options:
-        return _Options(self.rounds_per_tile, self.sample_coords, self.bisection_iters, self.threads)
+        return _Options(self.rounds_per_tile, self.sample_coords, self.bisection_iters, self.threads,
+                        self.format_version)
 
 
 @dataclass
@@ -228,7 +233,7 @@ def compress_cuda_noalloc(tensor: torch.Tensor, config: EntroPackLossyConfig | f
 
 
 def plan_bitrates(shapes, weights, mean_bpp: float, min_bpp: float = 0.001, max_bpp: float = 11.0,
-                  rounds_per_tile: int = 0) -> list[float]:
+                  rounds_per_tile: int = 0, format_version: int = 2) -> list[float]:
     """ep_plan_bitrates: per-layer target bitrates that spend ``mean_bpp`` bits per parameter over the
     layers ``shapes`` [(rows, cols), ...], weighting layer i's squared error by ``weights[i]`` (the
     README's mixed-bitrate packs, which allocate bits by per-layer sensitivity). Each result is a
@@ -242,6 +247,7 @@ def plan_bitrates(shapes, weights, mean_bpp: float, min_bpp: float = 0.001, max_
     opt = _Options()
     lib().ep_options_default(ctypes.byref(opt))
     opt.rounds_per_tile = int(rounds_per_tile)
+    opt.format_version = int(format_version)
     _check(lib().ep_plan_bitrates(n, rows, cols, w, float(mean_bpp), float(min_bpp), float(max_bpp),
                                   ctypes.byref(opt), out), "plan_bitrates")
     return list(out)

@@ -79,7 +79,9 @@ ep_status validate_blob(const uint8_t* p, uint64_t bytes) {
     if (!parse_header(p, h)) return fail(EP_ERR_CORRUPT, "malformed EPK1 header");
     if (h.total != bytes) return fail(EP_ERR_CORRUPT, "header says %llu bytes, have %llu", (unsigned long long)h.total,
                                       (unsigned long long)bytes);
-    // Tables: lo/cnt bounds, then the 12-bit frequencies.
+    // Tables: lo/cnt bounds, then the frequencies (12-bit in version 1, 8-bit in version 2).
+    const int fbits = prob_bits_of_version(h.version);
+    const uint32_t scale = 1u << fbits;
     const uint8_t* tb = p + h.off_tables;
     uint64_t avail = h.off_offsets - h.off_tables, nsym = 0;
     if (avail < 2 * kNumCtx) return fail(EP_ERR_CORRUPT, "tables section too short");
@@ -88,22 +90,22 @@ ep_status validate_blob(const uint8_t* p, uint64_t bytes) {
         if ((cnt == 0 && lo != 0) || lo + cnt > (c == 0 ? 128 : 64)) return fail(EP_ERR_CORRUPT, "context %d out of range", c);
         nsym += uint64_t(cnt);
     }
-    uint64_t used = 2 * kNumCtx + (12 * nsym + 7) / 8;
+    uint64_t used = 2 * kNumCtx + (uint64_t(fbits) * nsym + 7) / 8;
     if (pad16(used) != avail) return fail(EP_ERR_CORRUPT, "tables section size mismatch");
     const uint8_t* bits = tb + 2 * kNumCtx;
     uint64_t pos = 0;
     for (int c = 0; c < kNumCtx; ++c) {
         int cnt = tb[kNumCtx + c];
         uint32_t sum = 0, fmax = 0;
-        for (int k = 0; k < cnt; ++k, pos += 12) {
+        for (int k = 0; k < cnt; ++k, pos += uint64_t(fbits)) {
             uint32_t v = 0;
-            for (int b = 0; b < 12; ++b) v |= uint32_t((bits[(pos + b) >> 3] >> ((pos + b) & 7)) & 1u) << b;
+            for (int b = 0; b < fbits; ++b) v |= uint32_t((bits[(pos + b) >> 3] >> ((pos + b) & 7)) & 1u) << b;
             sum += v;
             fmax = v > fmax ? v : fmax;
         }
-        if (cnt == 1) return fail(EP_ERR_CORRUPT, "context %d: a single symbol must be stored as 4095 + 1", c);
-        if (cnt >= 2 && (sum != kProbScale || fmax > kProbScale - 1))
-            return fail(EP_ERR_CORRUPT, "context %d: frequencies do not sum to 4096", c);
+        if (cnt == 1) return fail(EP_ERR_CORRUPT, "context %d: a single symbol must be stored as %u + 1", c, scale - 1);
+        if (cnt >= 2 && (sum != scale || fmax > scale - 1))
+            return fail(EP_ERR_CORRUPT, "context %d: frequencies do not sum to %u", c, scale);
     }
     // Tile offsets: start at 0, non-decreasing, last one ends the blob.
     uint64_t prev = 0;

@@ -1,6 +1,6 @@
 // Host-side pieces shared by the two EPK1 encoders (the multithreaded host encoder and the CUDA
-// encoder): 12-bit table fitting, the sampled storage estimate, the raw-bit and tile-size choices and
-// the blob's metadata sections. Both encoders call these, so every decision that fixes the blob's
+// encoder): table fitting (12-bit for format version 1, 8-bit with rare symbols escaped for version 2),
+// the sampled storage estimate, the raw-bit and tile-size choices and the blob's metadata sections. Both encoders call these, so every decision that fixes the blob's
 // bytes is taken by the same code.
 #pragma once
 
@@ -53,28 +53,28 @@ inline uint32_t auto_rounds_per_tile(int64_t NG) {
 
 using Counts = std::vector<uint64_t>;  // [kNumCtx][128]
 
-// 12-bit normalisation: f = max(1, floor(4096 n_s / n)) for present symbols. The rounding gap is
-// closed at the largest frequency, or in steps of whole units when there is too much. No f exceeds
-// 4095: a single present symbol gets 4095, and its neighbour (s + 1, or s - 1 at the alphabet's
-// end) gets 1.
-inline void normalize(const uint64_t* cnt, int A, uint32_t* f) {
+// Normalisation to a total of `scale` (4096 or 256): f = max(1, floor(scale n_s / n)) for present
+// symbols. The rounding gap is closed at the largest frequency, or in steps of whole units when there is
+// too much. No f exceeds scale - 1: a single present symbol gets scale - 1, and its neighbour (s + 1, or
+// s - 1 at the alphabet's end) gets 1.
+inline void normalize(const uint64_t* cnt, int A, uint32_t scale, uint32_t* f) {
     uint64_t total = 0;
     int present = 0;
     for (int s = 0; s < A; ++s) { total += cnt[s]; present += cnt[s] != 0; f[s] = 0; }
     if (!present) return;
     if (present == 1) {
         for (int s = 0; s < A; ++s)
-            if (cnt[s]) { f[s] = kProbScale - 1; f[s + 1 < A ? s + 1 : s - 1] = 1; }
+            if (cnt[s]) { f[s] = scale - 1; f[s + 1 < A ? s + 1 : s - 1] = 1; }
         return;
     }
     int64_t sum = 0;
     for (int s = 0; s < A; ++s) {
         if (!cnt[s]) continue;
-        uint64_t q = cnt[s] * uint64_t(kProbScale) / total;
+        uint64_t q = cnt[s] * uint64_t(scale) / total;
         f[s] = q ? uint32_t(q) : 1u;
         sum += f[s];
     }
-    int64_t d = int64_t(kProbScale) - sum;
+    int64_t d = int64_t(scale) - sum;
     while (d) {
         int best = -1;
         for (int s = 0; s < A; ++s) if (f[s] && (best < 0 || f[s] > f[best])) best = s;
@@ -87,17 +87,48 @@ inline void normalize(const uint64_t* cnt, int A, uint32_t* f) {
     }
 }
 
+// Version 2: the counts of rare symbols move onto their escape symbol (index 63 of the symbol's coset
+// half in START, 63 elsewhere). Rare: seen in fewer than 1/2^kEscShift of the context's coordinates; hi in
+// [-2, 2] (idx 29..33) is never escaped, so an escaped coordinate always has magnitude class 1.
+inline void escape_rare(Counts& c) {
+    for (int k = 0; k < kNumCtx; ++k) {
+        const int A = k == 0 ? 128 : 64;
+        uint64_t* n = &c[size_t(k) * 128];
+        uint64_t total = 0;
+        for (int s = 0; s < A; ++s) total += n[s];
+        for (int s = 0; s < A; ++s) {
+            const int idx = s & 63;
+            if (idx == kEscIdx || (idx >= 29 && idx <= 33) || n[s] == 0) continue;
+            if ((n[s] << kEscShift) < total) {
+                n[(s & 64) | kEscIdx] += n[s];
+                n[s] = 0;
+            }
+        }
+    }
+}
+
+// The counts the tables of format `version` are fitted to.
+inline Counts prepared_counts(const Counts& raw, int version) {
+    Counts c = raw;
+    if (version == 2) escape_rare(c);
+    return c;
+}
+
 struct Tables {
+    int version = 1, bits = kProbBits;
     uint32_t f[kNumCtx][128];
     uint32_t cum[kNumCtx][128];
     int lo[kNumCtx], cnt[kNumCtx];
     uint64_t nsym = 0;
 
-    void build(const Counts& c) {
+    // c: prepared counts (prepared_counts).
+    void build(const Counts& c, int ver) {
+        version = ver;
+        bits = prob_bits_of_version(ver);
         nsym = 0;
         for (int k = 0; k < kNumCtx; ++k) {
             int A = k == 0 ? 128 : 64;
-            normalize(&c[size_t(k) * 128], A, f[k]);
+            normalize(&c[size_t(k) * 128], A, 1u << bits, f[k]);
             for (int s = A; s < 128; ++s) f[k][s] = 0;
             int first = -1, last = -1;
             for (int s = 0; s < A; ++s) if (f[k][s]) { if (first < 0) first = s; last = s; }
@@ -108,34 +139,40 @@ struct Tables {
             for (int s = 0; s < 128; ++s) { cum[k][s] = acc; acc += f[k][s]; }
         }
     }
-    uint64_t serialized_bytes() const { return 2 * kNumCtx + (12 * nsym + 7) / 8; }
+    uint64_t serialized_bytes() const { return 2 * kNumCtx + (uint64_t(bits) * nsym + 7) / 8; }
     void serialize(uint8_t* out) const {
         for (int k = 0; k < kNumCtx; ++k) { out[k] = uint8_t(lo[k]); out[kNumCtx + k] = uint8_t(cnt[k]); }
-        uint8_t* bits = out + 2 * kNumCtx;
+        uint8_t* bytes = out + 2 * kNumCtx;
         uint64_t pos = 0;
         for (int k = 0; k < kNumCtx; ++k)
-            for (int s = lo[k]; s < lo[k] + cnt[k]; ++s, pos += 12) {
+            for (int s = lo[k]; s < lo[k] + cnt[k]; ++s, pos += uint64_t(bits)) {
                 uint32_t v = f[k][s];
                 uint32_t word = v << (pos & 7);  // 12 + 7 bits fit in three bytes
-                bits[pos >> 3] |= uint8_t(word);
-                bits[(pos >> 3) + 1] |= uint8_t(word >> 8);
-                if (word >> 16) bits[(pos >> 3) + 2] |= uint8_t(word >> 16);
+                bytes[pos >> 3] |= uint8_t(word);
+                if (word >> 8) bytes[(pos >> 3) + 1] |= uint8_t(word >> 8);
+                if (word >> 16) bytes[(pos >> 3) + 2] |= uint8_t(word >> 16);
             }
     }
+    // The table symbol coded for `sym` of context k: itself, or its escape when the tables give it no
+    // frequency (a rare symbol of version 2).
+    int coded(int k, int sym) const { return f[k][sym] ? sym : ((sym & 64) | kEscIdx); }
 };
 
 // Storage estimate in bytes from the symbol counts of a row sample: the ideal code length under the
 // tables fitted to the sample, plus escapes and raw bits, scaled to the whole tensor, plus the exact
 // metadata and 104 bytes per tile for the final states (their low half carries payload).
-inline double estimate_from_counts(const Counts& total, uint64_t n_esc, int r, int64_t Rs, int64_t gpr, int64_t NG,
+inline double estimate_from_counts(const Counts& raw, int version, int r, int64_t Rs, int64_t gpr, int64_t NG,
                                    int64_t M, uint32_t T) {
+    const Counts total = prepared_counts(raw, version);
     Tables tab;
-    tab.build(total);
+    tab.build(total, version);
+    uint64_t n_esc = 0;
+    for (int k = 0; k < kNumCtx; ++k) n_esc += total[size_t(k) * 128 + kEscIdx] + (k == 0 ? total[64 + kEscIdx] : 0);
     double bits = 0.0;
     for (int k = 0; k < kNumCtx; ++k)
         for (int sy = tab.lo[k]; sy < tab.lo[k] + tab.cnt[k]; ++sy) {
             uint64_t n = total[size_t(k) * 128 + sy];
-            if (n) bits += double(n) * (12.0 - std::log2(double(tab.f[k][sy])));
+            if (n) bits += double(n) * (double(tab.bits) - std::log2(double(tab.f[k][sy])));
         }
     double ng_s = double(Rs * gpr);
     bits += 16.0 * double(n_esc) + 8.0 * double(r) * ng_s;
@@ -167,7 +204,7 @@ inline void write_metadata(uint8_t* blob, const BlobLayout& L, ep_dtype dt, int 
                            float alpha, uint32_t G, uint32_t T, const uint16_t* sbits, const Tables& tab,
                            const uint64_t* start, const uint8_t* esc) {
     std::memcpy(blob, "EPK1", 4);
-    wr16(blob + 4, 1);
+    wr16(blob + 4, uint32_t(tab.version));
     blob[6] = uint8_t(dt);
     blob[7] = uint8_t(r);
     wr32(blob + 8, uint32_t(rows));

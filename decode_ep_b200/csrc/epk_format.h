@@ -1,6 +1,7 @@
 // Internal constants and the host-side header reader of the EPK1 blob, used by the host encoder,
 // the C ABI and the decode launcher. The byte layout:
-//   header (64 B) | scales M x bf16 | tables: lo[9], cnt[9], 12-bit frequencies packed LSB-first |
+//   header (64 B) | scales M x bf16 | tables: lo[9], cnt[9], frequencies packed LSB-first (12-bit in
+//   format version 1, 8-bit in version 2) |
 //   tile offsets (T+1) x u32 (start/16 | has_esc<<31) | payload: per tile 32 x u32 states,
 //   raw low bits (groups*r bytes, padded to 4), u16 word stream, zero padding to 16.
 // Every section starts 16-byte aligned; all fields are little-endian.
@@ -15,11 +16,20 @@ namespace epk {
 constexpr uint32_t kHeaderBytes = 64;
 constexpr int kLanes = 32;
 constexpr int kNumCtx = 9;
+// Format version 1: 12-bit tables, the state renormalised after every symbol.
 constexpr int kProbBits = 12;
 constexpr uint32_t kProbScale = 1u << kProbBits;  // 4096
+// Format version 2: 8-bit tables, the state renormalised after every pair of symbols; rare symbols are
+// sent as escapes (a symbol seen in fewer than 1/2^kEscShift of its context's coordinates, other than
+// hi in [-2, 2]), and a round's escape words follow its last pair.
+constexpr int kProbBitsV2 = 8;
+constexpr uint32_t kProbScaleV2 = 1u << kProbBitsV2;  // 256
+constexpr int kEscShift = 12;
 constexpr uint32_t kRansL = 1u << 16;             // state lower bound; 16-bit refills
 constexpr int kEscIdx = 63;
 constexpr int kMaxG = 1024;
+
+inline int prob_bits_of_version(int version) { return version == 1 ? kProbBits : kProbBitsV2; }
 
 inline uint64_t pad16(uint64_t n) { return (n + 15) & ~uint64_t(15); }
 inline uint64_t pad4(uint64_t n) { return (n + 3) & ~uint64_t(3); }
@@ -46,7 +56,7 @@ inline int elem_bytes(int dtype) {
 
 // Header fields as the decoder needs them.
 struct Header {
-    int dtype = 0, r = 0, G = 0;
+    int version = 0, dtype = 0, r = 0, G = 0;
     uint32_t M = 0, N = 0, T = 0;
     float alpha = 0.f;
     uint32_t off_scales = 0, off_tables = 0, off_offsets = 0, off_payload = 0;
@@ -56,7 +66,9 @@ struct Header {
 
 // Parses and checks the 64-byte header alone (no sections). Returns false if malformed.
 inline bool parse_header(const uint8_t* p, Header& h) {
-    if (std::memcmp(p, "EPK1", 4) != 0 || rd16(p + 4) != 1) return false;
+    if (std::memcmp(p, "EPK1", 4) != 0) return false;
+    h.version = int(rd16(p + 4));
+    if (h.version != 1 && h.version != 2) return false;
     h.dtype = p[6];
     h.r = p[7];
     h.M = rd32(p + 8);

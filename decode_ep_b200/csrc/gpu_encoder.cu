@@ -5,10 +5,10 @@
 // The method's steps (arXiv 2609.34185, abstract; modelscope summary) map onto kernels:
 //   - row scales s_row = bf16(RMS) and max |w|/s: one thread per row, summing in index order;
 //   - rate control: bisection on log2(alpha). Each probe quantises the row sample on the GPU and counts
-//     (context, symbol) pairs there; the host fits the 12-bit tables to the counts and takes the storage
+//     (context, symbol) pairs there; the host fits the frequency tables to the counts and takes the storage
 //     estimate with the same code as the host encoder;
 //   - quantisation of every group to E8 at the final alpha, then the counts of the whole tensor;
-//   - rANS coding: one warp per tile, in the exact reverse of the decode order. The lanes that emit a
+//   - rANS coding: one warp per tile, in the exact reverse of the decode order of the blob's format version. The lanes that emit a
 //     word at a step place it with a ballot and a popcount, from the end of the tile's word buffer, so
 //     the buffer reads forward in decode order;
 //   - assembly: one warp per tile copies states, raw low bits and words to the tile's offset.
@@ -136,15 +136,12 @@ __device__ __forceinline__ int quantize_group(const Src& src, const float* s, in
 }
 
 // Adds a thread's 8 (context, symbol) pairs to the block's shared histogram.
-__device__ __forceinline__ void count_group(unsigned int* h, int b, const int32_t* t, int r, unsigned int& n_esc) {
+__device__ __forceinline__ void count_group(unsigned int* h, int b, const int32_t* t, int r) {
     uint8_t ctx[8], sym[8];
     int32_t hi[8];
     group_syms(b, t, r, ctx, sym, hi);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        atomicAdd(&h[ctx[k] * 128 + sym[k]], 1u);
-        n_esc += idx_of(hi[k]) == kEscIdx;
-    }
+    for (int k = 0; k < 8; ++k) atomicAdd(&h[ctx[k] * 128 + sym[k]], 1u);
 }
 
 __device__ __forceinline__ void flush_hist(const unsigned int* h, unsigned long long* counts) {
@@ -161,25 +158,22 @@ struct Probes {
 };
 
 // Counts of the row sample at probe blockIdx.y's alpha: rows floor(k M / Rs), k < Rs, every group of
-// each. counts and n_esc_out hold one histogram and one escape count per probe.
+// each. counts holds one histogram per probe.
 __global__ void sample_counts_kernel(Src src, int64_t M, int64_t gpr, int64_t Rs, const float* s, Probes pr,
-                                     unsigned long long* counts, unsigned long long* n_esc_out) {
+                                     unsigned long long* counts) {
     const float alpha = pr.alpha[blockIdx.y];
     const int r = pr.r[blockIdx.y];
     counts += size_t(blockIdx.y) * kHistBins;
-    n_esc_out += blockIdx.y;
     __shared__ unsigned int h[kHistBins];
     for (int k = threadIdx.x; k < kHistBins; k += blockDim.x) h[k] = 0;
     __syncthreads();
     const int64_t gi = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-    unsigned int n_esc = 0;
     if (gi < Rs * gpr) {
         const int64_t k = gi / gpr, q = gi - k * gpr, row = (k * M) / Rs;
         int32_t t[8];
         const int b = quantize_group(src, s, row, q, alpha, t);
-        count_group(h, b, t, r, n_esc);
+        count_group(h, b, t, r);
     }
-    if (n_esc) atomicAdd(n_esc_out, static_cast<unsigned long long>(n_esc));
     __syncthreads();
     flush_hist(h, counts);
 }
@@ -213,12 +207,11 @@ __global__ void full_counts_kernel(const int32_t* tq, const uint8_t* bq, int64_t
     __shared__ unsigned int h[kHistBins];
     for (int k = threadIdx.x; k < kHistBins; k += blockDim.x) h[k] = 0;
     __syncthreads();
-    unsigned int n_esc = 0;
     for (int64_t g = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; g < NG; g += int64_t(gridDim.x) * blockDim.x) {
         int32_t t[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) t[k] = tq[g * 8 + k];
-        count_group(h, bq[g], t, r, n_esc);
+        count_group(h, bq[g], t, r);
     }
     __syncthreads();
     flush_hist(h, counts);
@@ -279,6 +272,82 @@ __global__ void encode_tiles_kernel(const int32_t* tq, const uint8_t* bq, int64_
             }
             cur -= __popc(mw);
             if (active) x = (x / f) * kProbScale + (x % f) + c;
+        }
+    }
+    states[int64_t(tile) * 32 + lane] = x;
+    if (lane == 0) {
+        nwords[tile] = uint32_t(cap - cur);
+        esc_flag[tile] = any_esc ? 1 : 0;
+    }
+}
+
+// Format version 2: rANS coding of one tile per warp, in the exact reverse of its decode order. The words
+// are placed from the end of the tile's buffer backwards, as in encode_tiles_kernel. Per round, from the
+// last: the round's escape words (positions descending; within a position the highest lane takes the
+// highest slot), then each pair of positions from the last: lanes with x >= f1 f2 2^16 place x & 0xFFFF
+// and shift x right by 16, then x <- C(s2, x), x <- C(s1, x) in base 256. A symbol the tables give no
+// frequency is coded as its escape (ftab is indexed by context * 128 + symbol).
+__global__ void encode_tiles_v2_kernel(const int32_t* tq, const uint8_t* bq, int64_t NG, uint32_t T, int G, int r,
+                                       const uint32_t* ftab, const uint32_t* ctab, uint16_t* words, uint32_t* states,
+                                       uint32_t* nwords, uint8_t* esc_flag) {
+    __shared__ uint32_t F[kHistBins], C[kHistBins];
+    for (int k = threadIdx.x; k < kHistBins; k += blockDim.x) {
+        F[k] = ftab[k];
+        C[k] = ctab[k];
+    }
+    __syncthreads();
+    const uint32_t lane = threadIdx.x & 31, tile = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (tile >= T) return;
+    const int64_t per = 32 * int64_t(G), g0 = int64_t(tile) * per, ng = min(per, NG - g0), cap = 16 * per;
+    uint16_t* wbuf = words + int64_t(tile) * cap;
+    const uint32_t gt = ~((2u << lane) - 1u);  // lanes above this one
+    uint32_t x = kRansL;
+    int64_t cur = cap;
+    bool any_esc = false;
+    for (int64_t k = (ng + 31) / 32 - 1; k >= 0; --k) {
+        const int64_t gl = 32 * k + lane;
+        const bool active = gl < ng;
+        uint8_t ctx[8] = {0}, sym[8] = {0};
+        int32_t hi[8] = {0};
+        if (active) {
+            int32_t t[8];
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) t[kk] = tq[(g0 + gl) * 8 + kk];
+            group_syms(bq[g0 + gl], t, r, ctx, sym, hi);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (F[ctx[i] * 128 + sym[i]] == 0) sym[i] = uint8_t((sym[i] & 64) | kEscIdx);
+        }
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+            const bool e = active && (sym[i] & 63) == kEscIdx;
+            const uint32_t me = __ballot_sync(0xFFFFFFFFu, e);
+            if (me) {
+                if (e) wbuf[cur - 1 - __popc(me & gt)] = uint16_t(int16_t(hi[i]));
+                cur -= __popc(me);
+                any_esc = true;
+            }
+        }
+#pragma unroll
+        for (int p = 3; p >= 0; --p) {
+            uint32_t f1 = 1, c1 = 0, f2 = 1, c2 = 0;
+            if (active) {
+                f1 = F[ctx[2 * p] * 128 + sym[2 * p]];
+                c1 = C[ctx[2 * p] * 128 + sym[2 * p]];
+                f2 = F[ctx[2 * p + 1] * 128 + sym[2 * p + 1]];
+                c2 = C[ctx[2 * p + 1] * 128 + sym[2 * p + 1]];
+            }
+            const bool emit = active && x >= ((f1 * f2) << 16);  // f1 f2 <= 255^2: the product fits 32 bits
+            const uint32_t mw = __ballot_sync(0xFFFFFFFFu, emit);
+            if (emit) {
+                wbuf[cur - 1 - __popc(mw & gt)] = uint16_t(x);
+                x >>= 16;
+            }
+            cur -= __popc(mw);
+            if (active) {
+                x = (x / f2) * kProbScaleV2 + (x % f2) + c2;
+                x = (x / f1) * kProbScaleV2 + (x % f1) + c1;
+            }
         }
     }
     states[int64_t(tile) * 32 + lane] = x;
@@ -382,9 +451,11 @@ extern "C" ep_status ep_compress_cuda(const void* dev_data, ep_dtype dt, int64_t
     ep_options_default(&opt);
     if (opt_in) opt = *opt_in;
     if (opt.rounds_per_tile == 0) opt.rounds_per_tile = auto_rounds_per_tile(rows * cols / 8);
+    if (opt.format_version == 0) opt.format_version = 2;
     if (opt.rounds_per_tile < 1 || opt.rounds_per_tile > uint32_t(kMaxG) || opt.sample_coords < 1 ||
-        opt.bisection_iters > 200)
+        opt.bisection_iters > 200 || opt.format_version > 2)
         return fail(EP_ERR_ARG, "ep_compress_cuda: bad options");
+    const int version = int(opt.format_version);
     cudaPointerAttributes pa;
     if (cudaPointerGetAttributes(&pa, dev_data) != cudaSuccess || pa.type != cudaMemoryTypeDevice) {
         cudaGetLastError();
@@ -401,7 +472,7 @@ extern "C" ep_status ep_compress_cuda(const void* dev_data, ep_dtype dt, int64_t
         DevBuf d_sbits, d_s, d_small, d_counts;
         EPK_CUDA(d_sbits.alloc(size_t(M) * 2, st));
         EPK_CUDA(d_s.alloc(size_t(M) * 4, st));
-        EPK_CUDA(d_small.alloc(64, st));  // [0] amax bits, [1] n_esc, [2] tmax, [3] nonfinite flag
+        EPK_CUDA(d_small.alloc(64, st));  // [0] amax bits, [2] tmax, [3] nonfinite flag
         EPK_CUDA(d_counts.alloc(sizeof(unsigned long long) * genc::kHistBins, st));
         unsigned long long* small = d_small.as<unsigned long long>();
         EPK_CUDA(cudaMemsetAsync(small, 0, 64, st));
@@ -423,10 +494,9 @@ extern "C" ep_status ep_compress_cuda(const void* dev_data, ep_dtype dt, int64_t
         // follow the exact sequence of the one-probe-per-step bisection.
         const int64_t Rs = std::min<int64_t>(M, (int64_t(opt.sample_coords) + N - 1) / N);
         DevBuf d_pcounts;
-        EPK_CUDA(d_pcounts.alloc(sizeof(unsigned long long) * (genc::kHistBins + 1) * genc::kMaxProbes, st));
+        EPK_CUDA(d_pcounts.alloc(sizeof(unsigned long long) * genc::kHistBins * genc::kMaxProbes, st));
         unsigned long long* pcounts = d_pcounts.as<unsigned long long>();
-        unsigned long long* pesc = pcounts + size_t(genc::kHistBins) * genc::kMaxProbes;
-        std::vector<unsigned long long> hcounts(size_t(genc::kHistBins + 1) * genc::kMaxProbes);
+        std::vector<unsigned long long> hcounts(size_t(genc::kHistBins) * genc::kMaxProbes);
         Counts counts(size_t(genc::kHistBins));
         double lo = -12.0, hi = 15.0;
         if (amax > 0.0) hi = std::min(hi, 22.0 - std::log2(amax));
@@ -449,20 +519,16 @@ extern "C" ep_status ep_compress_cuda(const void* dev_data, ep_dtype dt, int64_t
                 }
             }
             EPK_CUDA(cudaMemsetAsync(pcounts, 0, sizeof(unsigned long long) * genc::kHistBins * nodes, st));
-            EPK_CUDA(cudaMemsetAsync(pesc, 0, sizeof(unsigned long long) * genc::kMaxProbes, st));
             genc::sample_counts_kernel<<<dim3(blocks_for(Rs * gpr, 256), unsigned(nodes)), 256, 0, st>>>(
-                src, M, gpr, Rs, d_s.as<float>(), pr, pcounts, pesc);
+                src, M, gpr, Rs, d_s.as<float>(), pr, pcounts);
             EPK_CUDA(cudaGetLastError());
             EPK_CUDA(cudaMemcpyAsync(hcounts.data(), pcounts, sizeof(unsigned long long) * genc::kHistBins * nodes,
                                      cudaMemcpyDeviceToHost, st));
-            EPK_CUDA(cudaMemcpyAsync(hcounts.data() + size_t(genc::kHistBins) * genc::kMaxProbes, pesc,
-                                     sizeof(unsigned long long) * nodes, cudaMemcpyDeviceToHost, st));
             EPK_CUDA(cudaStreamSynchronize(st));
             for (int n = 0, step = 0; step < depth; ++step) {
                 std::copy(hcounts.begin() + size_t(n) * genc::kHistBins, hcounts.begin() + size_t(n + 1) * genc::kHistBins,
                           counts.begin());
-                const double est = estimate_from_counts(counts, hcounts[size_t(genc::kHistBins) * genc::kMaxProbes + n],
-                                                        pr.r[n], Rs, gpr, NG, M, T);
+                const double est = estimate_from_counts(counts, version, pr.r[n], Rs, gpr, NG, M, T);
                 if (8.0 * est <= budget) { lo = nmid[n]; n = 2 * n + 1; }
                 else { hi = nmid[n]; n = 2 * n + 2; }
             }
@@ -496,7 +562,7 @@ extern "C" ep_status ep_compress_cuda(const void* dev_data, ep_dtype dt, int64_t
                                  cudaMemcpyDeviceToHost, st));
         EPK_CUDA(cudaStreamSynchronize(st));
         Tables tab;
-        tab.build(counts);
+        tab.build(prepared_counts(counts, version), version);
 
         // Tiles: rANS words per tile, then sizes, offsets and the payload.
         DevBuf d_tabs, d_words, d_states, d_nwords, d_esc;
@@ -508,7 +574,7 @@ extern "C" ep_status ep_compress_cuda(const void* dev_data, ep_dtype dt, int64_t
         EPK_CUDA(d_states.alloc(size_t(T) * 32 * 4, st));
         EPK_CUDA(d_nwords.alloc(size_t(T) * 4, st));
         EPK_CUDA(d_esc.alloc(size_t(T), st));
-        genc::encode_tiles_kernel<<<blocks_for(T, 8), 256, 0, st>>>(
+        (version == 1 ? genc::encode_tiles_kernel : genc::encode_tiles_v2_kernel)<<<blocks_for(T, 8), 256, 0, st>>>(
             d_tq.as<int32_t>(), d_bq.as<uint8_t>(), NG, T, G, r, d_tabs.as<uint32_t>(),
             d_tabs.as<uint32_t>() + genc::kHistBins, d_words.as<uint16_t>(), d_states.as<uint32_t>(),
             d_nwords.as<uint32_t>(), d_esc.as<uint8_t>());
@@ -613,9 +679,11 @@ extern "C" ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt,
     ep_options_default(&opt);
     if (opt_in) opt = *opt_in;
     if (opt.rounds_per_tile == 0) opt.rounds_per_tile = auto_rounds_per_tile(rows * cols / 8);
+    if (opt.format_version == 0) opt.format_version = 2;
     if (opt.rounds_per_tile < 1 || opt.rounds_per_tile > uint32_t(kMaxG) || opt.sample_coords < 1 ||
-        opt.bisection_iters > 200)
+        opt.bisection_iters > 200 || opt.format_version > 2)
         return fail(EP_ERR_ARG, "ep_compress_cuda_noalloc: bad options");
+    const int version = int(opt.format_version);
     cudaPointerAttributes pa;
     if (cudaPointerGetAttributes(&pa, dev_data) != cudaSuccess || pa.type != cudaMemoryTypeDevice) {
         cudaGetLastError();
@@ -639,7 +707,7 @@ extern "C" ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt,
         *s = c.take<float>(size_t(M) * 4);
         *small = c.take<unsigned long long>(64);
         *counts = c.take<unsigned long long>(sizeof(unsigned long long) * genc::kHistBins);
-        *pcounts = c.take<unsigned long long>(sizeof(unsigned long long) * (genc::kHistBins + 1) * genc::kMaxProbes);
+        *pcounts = c.take<unsigned long long>(sizeof(unsigned long long) * genc::kHistBins * genc::kMaxProbes);
         *tq = c.take<int32_t>(size_t(NG) * 32);
         *bq = c.take<uint8_t>(size_t(NG));
         *tabs = c.take<uint32_t>(2 * sizeof(uint32_t) * genc::kHistBins);
@@ -689,7 +757,6 @@ extern "C" ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt,
     Carve carve{static_cast<unsigned char*>(ss.addr)};
     plan(carve, &d_sbits, &d_s, &small, &d_counts, &pcounts, &d_tq, &d_bq, &d_tabs, &d_words, &d_states, &d_nwords,
          &d_esc, &d_start, &d_payload);
-    unsigned long long* pesc = pcounts + size_t(genc::kHistBins) * genc::kMaxProbes;
 
     const genc::Src src{static_cast<const uint8_t*>(dev_data), int(dt), N, row_stride};
     try {
@@ -706,7 +773,7 @@ extern "C" ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt,
 
         // Rate control, four bisection steps per launch, exactly as ep_compress_cuda.
         const int64_t Rs = std::min<int64_t>(M, (int64_t(opt.sample_coords) + N - 1) / N);
-        std::vector<unsigned long long> hcounts(size_t(genc::kHistBins + 1) * genc::kMaxProbes);
+        std::vector<unsigned long long> hcounts(size_t(genc::kHistBins) * genc::kMaxProbes);
         Counts counts(size_t(genc::kHistBins));
         double lo = -12.0, hi = 15.0;
         if (amax > 0.0) hi = std::min(hi, 22.0 - std::log2(amax));
@@ -729,20 +796,16 @@ extern "C" ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt,
                 }
             }
             EPK_CUDA_NA(cudaMemsetAsync(pcounts, 0, sizeof(unsigned long long) * genc::kHistBins * nodes, st));
-            EPK_CUDA_NA(cudaMemsetAsync(pesc, 0, sizeof(unsigned long long) * genc::kMaxProbes, st));
             genc::sample_counts_kernel<<<dim3(blocks_for(Rs * gpr, 256), unsigned(nodes)), 256, 0, st>>>(
-                src, M, gpr, Rs, d_s, pr, pcounts, pesc);
+                src, M, gpr, Rs, d_s, pr, pcounts);
             EPK_CUDA_NA(cudaGetLastError());
             EPK_CUDA_NA(cudaMemcpyAsync(hcounts.data(), pcounts, sizeof(unsigned long long) * genc::kHistBins * nodes,
                                      cudaMemcpyDeviceToHost, st));
-            EPK_CUDA_NA(cudaMemcpyAsync(hcounts.data() + size_t(genc::kHistBins) * genc::kMaxProbes, pesc,
-                                     sizeof(unsigned long long) * nodes, cudaMemcpyDeviceToHost, st));
             EPK_CUDA_NA(cudaStreamSynchronize(st));
             for (int n = 0, step = 0; step < depth; ++step) {
                 std::copy(hcounts.begin() + size_t(n) * genc::kHistBins, hcounts.begin() + size_t(n + 1) * genc::kHistBins,
                           counts.begin());
-                const double est = estimate_from_counts(counts, hcounts[size_t(genc::kHistBins) * genc::kMaxProbes + n],
-                                                        pr.r[n], Rs, gpr, NG, M, T);
+                const double est = estimate_from_counts(counts, version, pr.r[n], Rs, gpr, NG, M, T);
                 if (8.0 * est <= budget) { lo = nmid[n]; n = 2 * n + 1; }
                 else { hi = nmid[n]; n = 2 * n + 2; }
             }
@@ -769,13 +832,13 @@ extern "C" ep_status ep_compress_cuda_noalloc(const void* dev_data, ep_dtype dt,
                                  cudaMemcpyDeviceToHost, st));
         EPK_CUDA_NA(cudaStreamSynchronize(st));
         Tables tab;
-        tab.build(counts);
+        tab.build(prepared_counts(counts, version), version);
 
         // Tiles.
         EPK_CUDA_NA(cudaMemcpyAsync(d_tabs, tab.f, sizeof(uint32_t) * genc::kHistBins, cudaMemcpyHostToDevice, st));
         EPK_CUDA_NA(cudaMemcpyAsync(d_tabs + genc::kHistBins, tab.cum, sizeof(uint32_t) * genc::kHistBins,
                                  cudaMemcpyHostToDevice, st));
-        genc::encode_tiles_kernel<<<blocks_for(T, 8), 256, 0, st>>>(d_tq, d_bq, NG, T, G, r, d_tabs,
+        (version == 1 ? genc::encode_tiles_kernel : genc::encode_tiles_v2_kernel)<<<blocks_for(T, 8), 256, 0, st>>>(d_tq, d_bq, NG, T, G, r, d_tabs,
                                                                    d_tabs + genc::kHistBins, d_words, d_states,
                                                                    d_nwords, d_esc);
         EPK_CUDA_NA(cudaGetLastError());

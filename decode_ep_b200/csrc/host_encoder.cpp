@@ -5,8 +5,8 @@
 //   - Each 8-wide group is quantised to the nearest E8 point at one global resolution alpha.
 //   - Alpha comes from bisection on log2(alpha) against a storage estimate taken on a sample of
 //     rows, so the full stream is never re-encoded (paper page abstract; techmoon article).
-//   - The coordinates are rANS-coded under 9 conditional 12-bit tables, in independent tiles of
-//     32 interleaved lanes (abstract; modelscope summary).
+//   - The coordinates are rANS-coded under 9 conditional tables (8-bit in format version 2, 12-bit in
+//     version 1), in independent tiles of 32 interleaved lanes (abstract; modelscope summary).
 // All floating point is IEEE double/binary32, round-to-nearest, with no FMA contraction. The
 // build passes -ffp-contract=off, so every estimate and every quantisation decision is a fixed
 // function of the input, whatever the thread count.
@@ -147,12 +147,11 @@ struct Encoder {
     }
 
     // Storage estimate in bytes from the row sample (same definition the format fixes).
-    double estimate(float alpha, uint32_t sample_coords) const {
+    double estimate(float alpha, uint32_t sample_coords, int version) const {
         int64_t Rs = std::min<int64_t>(M, (int64_t(sample_coords) + N - 1) / N);
         int r = raw_bits_for(alpha);
         int nt = std::max(1, threads);
         std::vector<Counts> counts(size_t(nt), Counts(size_t(kNumCtx) * 128, 0));
-        std::vector<uint64_t> esc(size_t(nt), 0);
         parallel_for(Rs, threads, [&](int64_t b, int64_t e, int th) {
             std::vector<float> w(static_cast<size_t>(N));
             std::vector<int32_t> t(static_cast<size_t>(N));
@@ -166,20 +165,14 @@ struct Encoder {
                     uint8_t ctx[8], sym[8];
                     int32_t hi[8];
                     group_syms(cb[size_t(q)], &t[size_t(q * 8)], r, ctx, sym, hi);
-                    for (int i = 0; i < 8; ++i) {
-                        c[size_t(ctx[i]) * 128 + sym[i]]++;
-                        esc[size_t(th)] += idx_of(hi[i]) == kEscIdx;
-                    }
+                    for (int i = 0; i < 8; ++i) c[size_t(ctx[i]) * 128 + sym[i]]++;
                 }
             }
         });
         Counts total(size_t(kNumCtx) * 128, 0);
-        uint64_t n_esc = 0;
-        for (int th = 0; th < nt; ++th) {
+        for (int th = 0; th < nt; ++th)
             for (size_t k = 0; k < total.size(); ++k) total[k] += counts[size_t(th)][k];
-            n_esc += esc[size_t(th)];
-        }
-        return estimate_from_counts(total, n_esc, r, Rs, gpr, NG, M, T);
+        return estimate_from_counts(total, version, r, Rs, gpr, NG, M, T);
     }
 };
 
@@ -189,6 +182,10 @@ struct TileBytes {
     bool has_esc = false;
 };
 
+void write_tile(const std::vector<int32_t>& tq, int64_t g0, int64_t ng, int r, const uint32_t* x,
+                const std::vector<uint16_t>& words, bool has_esc, TileBytes& out);
+
+// Version 1 tile: the decode order of the format document, run backwards.
 void encode_tile(const std::vector<int32_t>& tq, const std::vector<uint8_t>& bq, int64_t g0, int64_t ng, int r,
                  const Tables& tab, TileBytes& out) {
     uint32_t x[kLanes];
@@ -219,6 +216,13 @@ void encode_tile(const std::vector<int32_t>& tq, const std::vector<uint8_t>& bq,
             }
         }
     }
+    write_tile(tq, g0, ng, r, x, words, has_esc, out);
+}
+
+// One tile's bytes from its final states and pushed words: states, the raw section (8 fields of r bits per
+// group, LSB-first), the words in reverse push order, zero padding to 16 bytes.
+void write_tile(const std::vector<int32_t>& tq, int64_t g0, int64_t ng, int r, const uint32_t* x,
+                const std::vector<uint16_t>& words, bool has_esc, TileBytes& out) {
     uint64_t raw = pad4(uint64_t(ng) * uint64_t(r));
     uint64_t size = pad16(128 + raw + 2 * uint64_t(words.size()));
     out.bytes.assign(size_t(size), 0);
@@ -251,6 +255,47 @@ void encode_tile(const std::vector<int32_t>& tq, const std::vector<uint8_t>& bq,
     out.has_esc = has_esc;
 }
 
+// Version 2 tile: pairs of positions (2p, 2p + 1) share one renormalisation, and a round's escape words
+// follow its last pair, positions ascending, lanes ascending. Run backwards: the round's escape words
+// (positions and lanes descending), then each pair from the last: if x >= f1 f2 2^16 the lane pushes
+// x & 0xFFFF and sets x >>= 16, then x <- C(s2, x) and x <- C(s1, x) in base 256.
+void encode_tile_v2(const std::vector<int32_t>& tq, const std::vector<uint8_t>& bq, int64_t g0, int64_t ng, int r,
+                    const Tables& tab, TileBytes& out) {
+    uint32_t x[kLanes];
+    for (auto& v : x) v = kRansL;
+    std::vector<uint16_t> words;
+    words.reserve(size_t(ng) * 4);
+    int64_t R = (ng + 31) / 32;
+    bool has_esc = false;
+    uint8_t ctx[kLanes][8], sym[kLanes][8];
+    int32_t hi[kLanes][8];
+    for (int64_t k = R - 1; k >= 0; --k) {
+        int nl = int(std::min<int64_t>(32, ng - 32 * k));
+        for (int L = 0; L < nl; ++L) {
+            int64_t g = g0 + 32 * k + L;
+            group_syms(bq[size_t(g)], &tq[size_t(g * 8)], r, ctx[L], sym[L], hi[L]);
+            for (int i = 0; i < 8; ++i) sym[L][i] = uint8_t(tab.coded(ctx[L][i], sym[L][i]));
+        }
+        for (int i = 7; i >= 0; --i)
+            for (int L = nl - 1; L >= 0; --L)
+                if ((sym[L][i] & 63) == kEscIdx) {
+                    words.push_back(uint16_t(int16_t(hi[L][i])));
+                    has_esc = true;
+                }
+        for (int pr = 3; pr >= 0; --pr)
+            for (int L = nl - 1; L >= 0; --L) {
+                const int i1 = 2 * pr, i2 = 2 * pr + 1;
+                const uint32_t f1 = tab.f[ctx[L][i1]][sym[L][i1]], c1 = tab.cum[ctx[L][i1]][sym[L][i1]];
+                const uint32_t f2 = tab.f[ctx[L][i2]][sym[L][i2]], c2 = tab.cum[ctx[L][i2]][sym[L][i2]];
+                uint32_t xv = x[L];
+                if (uint64_t(xv) >= (uint64_t(f1 * f2) << 16)) { words.push_back(uint16_t(xv)); xv >>= 16; }
+                xv = (xv / f2) * kProbScaleV2 + (xv % f2) + c2;
+                x[L] = (xv / f1) * kProbScaleV2 + (xv % f1) + c1;
+            }
+    }
+    write_tile(tq, g0, ng, r, x, words, has_esc, out);
+}
+
 }  // namespace
 }  // namespace epk
 
@@ -262,6 +307,7 @@ extern "C" void ep_options_default(ep_options* opt) {
     opt->sample_coords = 1u << 18;
     opt->bisection_iters = 40;
     opt->threads = 0;
+    opt->format_version = 2;
 }
 
 extern "C" ep_status ep_compress(const void* data, int is_device, ep_dtype dt, int64_t rows, int64_t cols,
@@ -281,9 +327,11 @@ extern "C" ep_status ep_compress(const void* data, int is_device, ep_dtype dt, i
     ep_options_default(&opt);
     if (opt_in) opt = *opt_in;
     if (opt.rounds_per_tile == 0) opt.rounds_per_tile = auto_rounds_per_tile(rows * cols / 8);
+    if (opt.format_version == 0) opt.format_version = 2;
     if (opt.rounds_per_tile < 1 || opt.rounds_per_tile > uint32_t(kMaxG) || opt.sample_coords < 1 ||
-        opt.bisection_iters > 200)
+        opt.bisection_iters > 200 || opt.format_version > 2)
         return fail(EP_ERR_ARG, "ep_compress: bad options");
+    const int version = int(opt.format_version);
     int threads = opt.threads > 0 ? opt.threads : int(std::max(1u, std::thread::hardware_concurrency()));
 
     // Device input: one copy to the host, rows packed.
@@ -314,7 +362,7 @@ extern "C" ep_status ep_compress(const void* data, int is_device, ep_dtype dt, i
         for (uint32_t it = 0; it < opt.bisection_iters; ++it) {
             double mid = 0.5 * (lo + hi);
             float a = float(std::exp2(mid));
-            if (8.0 * enc.estimate(a, opt.sample_coords) <= budget) lo = mid; else hi = mid;
+            if (8.0 * enc.estimate(a, opt.sample_coords, version) <= budget) lo = mid; else hi = mid;
         }
         float alpha = float(std::exp2(lo));
 
@@ -354,7 +402,7 @@ extern "C" ep_status ep_compress(const void* data, int is_device, ep_dtype dt, i
         Counts total(size_t(kNumCtx) * 128, 0);
         for (auto& c : counts) for (size_t k = 0; k < total.size(); ++k) total[k] += c[k];
         Tables tab;
-        tab.build(total);
+        tab.build(prepared_counts(total, version), version);
 
         // Tiles, in parallel.
         uint32_t T = enc.T;
@@ -363,7 +411,8 @@ extern "C" ep_status ep_compress(const void* data, int is_device, ep_dtype dt, i
         parallel_for(T, threads, [&](int64_t b, int64_t e, int) {
             for (int64_t j = b; j < e; ++j) {
                 int64_t g0 = j * per_tile, ng = std::min(per_tile, NG - g0);
-                encode_tile(tq, bq, g0, ng, r, tab, tiles[size_t(j)]);
+                if (version == 1) encode_tile(tq, bq, g0, ng, r, tab, tiles[size_t(j)]);
+                else encode_tile_v2(tq, bq, g0, ng, r, tab, tiles[size_t(j)]);
             }
         });
         std::vector<uint64_t> start(size_t(T) + 1, 0);

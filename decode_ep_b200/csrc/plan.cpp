@@ -25,17 +25,20 @@
 namespace epk {
 namespace {
 
-// Largest tables section: 9 contexts of lo and count bytes, then 12 bits for each of 128 + 8 x 64 symbols.
-constexpr uint64_t kMaxTablesBytes = 2 * kNumCtx + (12 * (128 + 8 * 64) + 7) / 8;
+// Largest tables section of format `version`: 9 contexts of lo and count bytes, then one frequency for each
+// of 128 + 8 x 64 symbols (12 bits in version 1, 8 in version 2).
+uint64_t max_tables_bytes(int version) {
+    return 2 * kNumCtx + (uint64_t(prob_bits_of_version(version)) * (128 + 8 * 64) + 7) / 8;
+}
 
 // Metadata bytes of an rows x cols blob with G rounds per tile: header, row scales, the largest tables
 // section (the only part that depends on the data), tile offsets, and 104 bytes per tile for the final
 // rANS states: 128 bytes of states, less the 32 bytes of payload they carry on average, plus 8 of padding.
 // These are the charges the encoders' own storage estimate makes.
-double metadata_bytes(int64_t rows, int64_t cols, uint32_t G) {
+double metadata_bytes(int64_t rows, int64_t cols, uint32_t G, int version) {
     const uint64_t NG = uint64_t(rows) * uint64_t(cols) / 8;
     const uint64_t T = (NG + 32ull * G - 1) / (32ull * G);
-    return double(kHeaderBytes + pad16(2 * uint64_t(rows)) + pad16(kMaxTablesBytes) + pad16(4 * (T + 1)) +
+    return double(kHeaderBytes + pad16(2 * uint64_t(rows)) + pad16(max_tables_bytes(version)) + pad16(4 * (T + 1)) +
                   T * (128 - 32 + 8));
 }
 
@@ -54,7 +57,9 @@ extern "C" ep_status ep_plan_bitrates(int64_t n, const int64_t* rows, const int6
     ep_options opt;
     ep_options_default(&opt);
     if (opt_in) opt = *opt_in;
-    if (opt.rounds_per_tile > uint32_t(kMaxG)) return fail(EP_ERR_ARG, "ep_plan_bitrates: bad rounds_per_tile");
+    if (opt.format_version == 0) opt.format_version = 2;
+    if (opt.rounds_per_tile > uint32_t(kMaxG) || opt.format_version > 2)
+        return fail(EP_ERR_ARG, "ep_plan_bitrates: bad rounds_per_tile or format_version");
 
     const size_t count = static_cast<size_t>(n);
     std::vector<double> c(count), lo(count), hi(count), np(count);
@@ -68,7 +73,7 @@ extern "C" ep_status ep_plan_bitrates(int64_t n, const int64_t* rows, const int6
             return fail(EP_ERR_ARG, "ep_plan_bitrates: layer %lld: weight must be finite and > 0", (long long)i);
         const uint32_t G = opt.rounds_per_tile ? opt.rounds_per_tile : enc::auto_rounds_per_tile(M * N / 8);
         np[i] = double(M) * double(N);
-        const double meta = 8.0 * metadata_bytes(M, N, G) / np[i];
+        const double meta = 8.0 * metadata_bytes(M, N, G, int(opt.format_version)) / np[i];
         c[i] = meta + 0.5 * std::log2(weight[i]);
         hi[i] = max_bpp;
         lo[i] = std::min(std::max(min_bpp, meta), max_bpp);

@@ -75,6 +75,11 @@ typedef struct {
     uint32_t sample_coords;   /* rate-control sample: about this many coordinates of whole rows. Default 2^18 */
     uint32_t bisection_iters; /* bisection steps on log2(alpha). Default 40 */
     int32_t threads;          /* encoder threads; 0 = all hardware threads */
+    uint32_t format_version;  /* 2 (the default; 0 also means 2): 8-bit frequency tables, the rANS state
+                                 renormalised once per pair of symbols, rare symbols sent as escapes. 1:
+                                 12-bit frequency tables, the state renormalised after every symbol. Both
+                                 decode with the same calls; version 2 decodes faster on B200 at a
+                                 slightly higher error for the same storage. */
 } ep_options;
 
 void ep_options_default(ep_options* opt);

@@ -48,17 +48,18 @@ def lib():
         L.orc_crc32.argtypes = [c.c_void_p, c.c_size_t]
         L.orc_e8_nearest.argtypes = [c.c_void_p, c.c_void_p, c.c_void_p]
         L.orc_normalize.argtypes = [c.c_void_p, c.c_int, c.c_void_p]
+        L.orc_normalize_bits.argtypes = [c.c_void_p, c.c_int, c.c_int, c.c_void_p]
         L.orc_to_container.argtypes = [c.c_void_p, c.c_int64, c.c_int, c.c_void_p]
         L.orc_from_container.argtypes = [c.c_void_p, c.c_int64, c.c_int, c.c_void_p]
         L.orc_compress.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_double, c.c_int,
-                                   c.c_double, c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
+                                   c.c_double, c.c_int, c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
                                    c.POINTER(c.c_double)]
         L.orc_free.argtypes = [c.c_void_p]
         L.orc_estimate_bytes.restype = c.c_double
-        L.orc_estimate_bytes.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int, c.c_float]
+        L.orc_estimate_bytes.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int, c.c_float, c.c_int]
         L.orc_blob_info.argtypes = [c.c_void_p, c.c_size_t, c.POINTER(c.c_int), c.POINTER(c.c_int64),
                                     c.POINTER(c.c_int64), c.POINTER(c.c_float), c.POINTER(c.c_int),
-                                    c.POINTER(c.c_int), c.POINTER(c.c_uint32)]
+                                    c.POINTER(c.c_int), c.POINTER(c.c_uint32), c.POINTER(c.c_int)]
         L.orc_decode_tiles.argtypes = [c.c_void_p, c.c_size_t, c.c_uint32, c.c_uint32, c.c_void_p,
                                        c.c_void_p]
         L.orc_decompress.argtypes = [c.c_void_p, c.c_size_t, c.c_void_p, c.c_void_p]
@@ -97,10 +98,11 @@ def e8_nearest(x) -> tuple[int, np.ndarray]:
     return int(b[0]), u
 
 
-def normalize(counts) -> np.ndarray:
+def normalize(counts, bits: int = 12) -> np.ndarray:
+    """Frequencies of `bits` bits (12: format version 1, 8: version 2) for the symbol counts."""
     c = np.ascontiguousarray(counts, dtype=np.uint64)
     f = np.zeros(c.size, np.uint32)
-    _check(lib().orc_normalize(_ptr(c), int(c.size), _ptr(f)), "normalize")
+    _check(lib().orc_normalize_bits(_ptr(c), int(c.size), int(bits), _ptr(f)), "normalize")
     return f
 
 
@@ -119,15 +121,16 @@ def from_container(a: np.ndarray, dtype: int) -> np.ndarray:
 
 
 def compress(data: np.ndarray, dtype: int, target_bpp: float, rounds_per_tile: int = 16,
-             force_alpha: float = 0.0) -> tuple[bytes, float]:
-    """Compress a row-major 2-D container array (the raw container bit patterns)."""
+             force_alpha: float = 0.0, prob_bits: int = 8) -> tuple[bytes, float]:
+    """Compress a row-major 2-D container array (the raw container bit patterns). prob_bits 8 writes
+    format version 2 (8-bit tables, pairs of symbols per renormalisation), 12 writes version 1."""
     a = np.ascontiguousarray(data)
     assert a.ndim == 2 and a.dtype.itemsize == ELEM.get(dtype, a.dtype.itemsize)
     blob = ctypes.c_void_p()
     nbytes = ctypes.c_size_t()
     actual = ctypes.c_double()
     st = lib().orc_compress(_ptr(a), dtype, a.shape[0], a.shape[1], float(target_bpp),
-                            int(rounds_per_tile), float(force_alpha), ctypes.byref(blob),
+                            int(rounds_per_tile), float(force_alpha), int(prob_bits), ctypes.byref(blob),
                             ctypes.byref(nbytes), ctypes.byref(actual))
     _check(st, "compress")
     try:
@@ -137,20 +140,22 @@ def compress(data: np.ndarray, dtype: int, target_bpp: float, rounds_per_tile: i
     return out, actual.value
 
 
-def estimate_bytes(data: np.ndarray, dtype: int, alpha: float, rounds_per_tile: int = 16) -> float:
+def estimate_bytes(data: np.ndarray, dtype: int, alpha: float, rounds_per_tile: int = 16,
+                   prob_bits: int = 8) -> float:
     a = np.ascontiguousarray(data)
     return float(lib().orc_estimate_bytes(_ptr(a), dtype, a.shape[0], a.shape[1], rounds_per_tile,
-                                          float(alpha)))
+                                          float(alpha), int(prob_bits)))
 
 
 def blob_info(blob: bytes) -> dict:
     c = ctypes
     dt, M, N, al, r, G, T = c.c_int(), c.c_int64(), c.c_int64(), c.c_float(), c.c_int(), c.c_int(), c.c_uint32()
+    ver = c.c_int()
     st = lib().orc_blob_info(blob, len(blob), c.byref(dt), c.byref(M), c.byref(N), c.byref(al),
-                             c.byref(r), c.byref(G), c.byref(T))
+                             c.byref(r), c.byref(G), c.byref(T), c.byref(ver))
     _check(st, "blob_info")
     return {"dtype": dt.value, "rows": M.value, "cols": N.value, "alpha": al.value, "r": r.value,
-            "G": G.value, "num_tiles": T.value}
+            "G": G.value, "num_tiles": T.value, "version": ver.value}
 
 
 def decompress(blob: bytes, with_coords: bool = False):

@@ -16,8 +16,13 @@
  *  - decode = symbol decode, arithmetic inverse of the lattice map, per-row
  *    rescale, with no symbol tensor or codebook — modelscope summary.
  * Every detail the pages leave open is read as the format document states
- * (E8 = D8 ∪ D8+½, 9 contexts of 12-bit tables conditioned on the coset bit
- * and the previous coordinate's magnitude class, 32-lane interleaved rANS).
+ * (E8 = D8 ∪ D8+½, 9 contexts of frequency tables conditioned on the coset
+ * bit and the previous coordinate's magnitude class, 32-lane interleaved
+ * rANS). The format has two versions, and this file follows both:
+ *  - version 1: 12-bit tables, the state renormalised after every symbol;
+ *  - version 2: 8-bit tables, the state renormalised after every pair of
+ *    symbols, rare symbols sent as escapes, and a round's escape words read
+ *    after its last pair.
  */
 #include "entropack_oracle.h"
 
@@ -30,11 +35,16 @@ enum { OK = 0, E_ARG = -1, E_DTYPE = -2, E_SHAPE = -3, E_TARGET = -4, E_NONFINIT
 
 #define LANES 32
 #define NCTX 9
-#define PROB_BITS 12
+#define PROB_BITS 12      /* version 1 */
 #define PROB_SCALE 4096u
+#define PROB_BITS_V2 8    /* version 2 */
+#define PROB_SCALE_V2 256u
 #define RANS_L 65536u
 #define ESC_IDX 63
 #define HEADER_BYTES 64
+/* Version 2: a symbol (other than hi in [-2, 2]) seen in fewer than 1/2^ESC_SHIFT of its
+ * context's coordinates is sent as an escape. */
+#define ESC_SHIFT 12
 
 /* ---------------------------------------------------------------- helpers */
 
@@ -254,10 +264,20 @@ static int context_of(int i, int64_t hi_prev, int b) {
 
 /* --------------------------------------------------- frequency normalisation */
 
-/* n is the alphabet size. Every present symbol gets f >= 1 and no f exceeds 4095: a context with
- * a single present symbol s gives it 4095 and its neighbour (s + 1, or s - 1 at the end of the
- * alphabet) the remaining 1. */
-int orc_normalize(const uint64_t* counts, int n, uint32_t* f) {
+/* n is the alphabet size, scale = 2^bits the table total (4096 in version 1, 256 in version 2).
+ * Every present symbol gets f >= 1 and no f exceeds scale - 1: a context with a single present
+ * symbol s gives it scale - 1 and its neighbour (s + 1, or s - 1 at the end of the alphabet) the
+ * remaining 1. */
+static int normalize_scale(const uint64_t* counts, int n, uint32_t scale, uint32_t* f);
+
+int orc_normalize(const uint64_t* counts, int n, uint32_t* f) { return normalize_scale(counts, n, PROB_SCALE, f); }
+
+int orc_normalize_bits(const uint64_t* counts, int n, int bits, uint32_t* f) {
+    if (bits != PROB_BITS && bits != PROB_BITS_V2) return E_ARG;
+    return normalize_scale(counts, n, 1u << bits, f);
+}
+
+static int normalize_scale(const uint64_t* counts, int n, uint32_t scale, uint32_t* f) {
     uint64_t total = 0;
     int present = 0;
     for (int s = 0; s < n; s++) { total += counts[s]; if (counts[s]) present++; }
@@ -266,7 +286,7 @@ int orc_normalize(const uint64_t* counts, int n, uint32_t* f) {
     if (present == 1) {
         for (int s = 0; s < n; s++)
             if (counts[s]) {
-                f[s] = PROB_SCALE - 1;
+                f[s] = scale - 1;
                 f[s + 1 < n ? s + 1 : s - 1] = 1;
             }
         return OK;
@@ -274,11 +294,11 @@ int orc_normalize(const uint64_t* counts, int n, uint32_t* f) {
     int64_t sum = 0;
     for (int s = 0; s < n; s++) {
         if (!counts[s]) continue;
-        uint64_t q = (counts[s] * (uint64_t)PROB_SCALE) / total;
+        uint64_t q = (counts[s] * (uint64_t)scale) / total;
         f[s] = q < 1 ? 1 : (uint32_t)q;
         sum += f[s];
     }
-    int64_t d = (int64_t)PROB_SCALE - sum;
+    int64_t d = (int64_t)scale - sum;
     while (d != 0) {
         int best = -1;
         for (int s = 0; s < n; s++)
@@ -296,6 +316,7 @@ int orc_normalize(const uint64_t* counts, int n, uint32_t* f) {
 /* ------------------------------------------------------- model (17 tables) */
 
 typedef struct {
+    int bits;                /* table precision: 12 (version 1) or 8 (version 2) */
     int lo[NCTX], cnt[NCTX];
     uint32_t f[NCTX][128];   /* indexed by symbol */
     uint32_t cum[NCTX][129]; /* cumulative, indexed by symbol */
@@ -303,11 +324,41 @@ typedef struct {
 
 static int ctx_alphabet(int c) { return c == 0 ? 128 : 64; }
 
-static void model_from_counts(uint64_t counts[NCTX][128], Model* m) {
+/* The escape symbol of a context symbol s: index 63 of s's coset half (START codes 64 b + idx). */
+static int esc_symbol_of(int s) { return (s & 64) | ESC_IDX; }
+
+/* Version 2: moves the counts of rare symbols onto their escape symbol. A symbol is rare when it is
+ * seen in fewer than 1/2^ESC_SHIFT of its context's coordinates. hi in [-2, 2] (idx 29..33) is never
+ * escaped, so an escaped coordinate always has magnitude class 1. */
+static void escape_rare(uint64_t counts[NCTX][128]) {
+    for (int c = 0; c < NCTX; c++) {
+        int A = ctx_alphabet(c);
+        uint64_t n = 0;
+        for (int s = 0; s < A; s++) n += counts[c][s];
+        for (int s = 0; s < A; s++) {
+            int idx = s & 63;
+            if (idx == ESC_IDX || (idx >= 29 && idx <= 33) || counts[c][s] == 0) continue;
+            if ((counts[c][s] << ESC_SHIFT) < n) {
+                counts[c][esc_symbol_of(s)] += counts[c][s];
+                counts[c][s] = 0;
+            }
+        }
+    }
+}
+
+/* The counts a table of precision `bits` is fitted to: version 2 first moves rare symbols onto the
+ * escapes. */
+static void prepare_counts(uint64_t counts[NCTX][128], int bits) {
+    if (bits == PROB_BITS_V2) escape_rare(counts);
+}
+
+/* Fits the tables to prepared counts. */
+static void model_from_counts(uint64_t counts[NCTX][128], int bits, Model* m) {
     memset(m, 0, sizeof(*m));
+    m->bits = bits;
     for (int c = 0; c < NCTX; c++) {
         int A = ctx_alphabet(c), lo = -1, hi = -1;
-        orc_normalize(counts[c], A, m->f[c]);
+        normalize_scale(counts[c], A, 1u << bits, m->f[c]);
         for (int s = 0; s < A; s++) if (m->f[c][s]) { if (lo < 0) lo = s; hi = s; }
         m->lo[c] = lo < 0 ? 0 : lo;
         m->cnt[c] = lo < 0 ? 0 : hi - lo + 1;
@@ -317,10 +368,12 @@ static void model_from_counts(uint64_t counts[NCTX][128], Model* m) {
     }
 }
 
+/* Frequencies are stored as m->bits-bit fields, packed LSB-first (12 bits in version 1, one byte each
+ * in version 2). */
 static uint64_t tables_bytes(const Model* m) {
     uint64_t nsym = 0;
     for (int c = 0; c < NCTX; c++) nsym += (uint64_t)m->cnt[c];
-    return 2 * NCTX + (12 * nsym + 7) / 8;
+    return 2 * NCTX + ((uint64_t)m->bits * nsym + 7) / 8;
 }
 
 static void write_tables(const Model* m, uint8_t* out) {
@@ -330,15 +383,18 @@ static void write_tables(const Model* m, uint8_t* out) {
     for (int c = 0; c < NCTX; c++) {
         for (int s = m->lo[c]; s < m->lo[c] + m->cnt[c]; s++) {
             uint32_t v = m->f[c][s];
-            for (int k = 0; k < 12; k++, bit++)
+            for (int k = 0; k < m->bits; k++, bit++)
                 if ((v >> k) & 1) bits[bit >> 3] |= (uint8_t)(1u << (bit & 7));
         }
     }
 }
 
-/* Returns 0 or E_CORRUPT. avail = bytes available for the tables section. */
-static int read_tables(const uint8_t* in, uint64_t avail, Model* m, uint64_t* used) {
+/* Returns 0 or E_CORRUPT. avail = bytes available for the tables section; bits = the precision the
+ * header's version fixes. */
+static int read_tables(const uint8_t* in, uint64_t avail, int bits_per_f, Model* m, uint64_t* used) {
     memset(m, 0, sizeof(*m));
+    m->bits = bits_per_f;
+    const uint32_t scale = 1u << bits_per_f;
     if (avail < 2 * NCTX) return E_CORRUPT;
     uint64_t nsym = 0;
     for (int c = 0; c < NCTX; c++) {
@@ -348,7 +404,7 @@ static int read_tables(const uint8_t* in, uint64_t avail, Model* m, uint64_t* us
         if (m->lo[c] + m->cnt[c] > ctx_alphabet(c)) return E_CORRUPT;
         nsym += (uint64_t)m->cnt[c];
     }
-    *used = 2 * NCTX + (12 * nsym + 7) / 8;
+    *used = 2 * NCTX + ((uint64_t)bits_per_f * nsym + 7) / 8;
     if (*used > avail) return E_CORRUPT;
     const uint8_t* bits = in + 2 * NCTX;
     uint64_t bit = 0;
@@ -356,16 +412,16 @@ static int read_tables(const uint8_t* in, uint64_t avail, Model* m, uint64_t* us
         uint32_t total = 0;
         for (int s = m->lo[c]; s < m->lo[c] + m->cnt[c]; s++) {
             uint32_t v = 0;
-            for (int k = 0; k < 12; k++, bit++) v |= (uint32_t)((bits[bit >> 3] >> (bit & 7)) & 1) << k;
+            for (int k = 0; k < bits_per_f; k++, bit++) v |= (uint32_t)((bits[bit >> 3] >> (bit & 7)) & 1) << k;
             m->f[c][s] = v;
             total += v;
         }
         if (m->cnt[c] == 1) {
-            return E_CORRUPT; /* a lone symbol is stored as 4095 + 1 */
+            return E_CORRUPT; /* a lone symbol is stored as (scale - 1) + 1 */
         } else if (m->cnt[c] >= 2) {
-            if (total != PROB_SCALE) return E_CORRUPT;
+            if (total != scale) return E_CORRUPT;
             for (int s = m->lo[c]; s < m->lo[c] + m->cnt[c]; s++)
-                if (m->f[c][s] > PROB_SCALE - 1) return E_CORRUPT;
+                if (m->f[c][s] > scale - 1) return E_CORRUPT;
         }
         uint32_t acc = 0;
         for (int s = 0; s < 128; s++) { m->cum[c][s] = acc; acc += m->f[c][s]; }
@@ -420,14 +476,24 @@ static void quantize_group(const Tensor* t, int64_t g, float alpha, Group* out) 
     group_from_point(b, u, out);
 }
 
-/* The symbols of one group at raw-bit count r: ctx, sym (table index) and hi per position. */
-static void group_symbols(const Group* g, int r, int ctx[8], int sym[8], int64_t hi[8]) {
+/* The symbols of one group at raw-bit count r: ctx, sym (table index) and hi per position. With a
+ * model m (NULL while counting), a symbol the tables give no frequency (a rare symbol of version 2) is
+ * replaced by its escape; esc[i] (if not NULL) tells whether position i is sent as an escape. The
+ * context comes from the previous coordinate's true hi: an escaped coordinate has |hi| >= 3, so its
+ * class is 1 either way. */
+static void group_symbols_m(const Group* g, int r, const Model* m, int ctx[8], int sym[8], int64_t hi[8], int esc[8]) {
     for (int i = 0; i < 8; i++) {
         hi[i] = floor_shift(g->t[i], r);
         int idx = sym_index(hi[i]);
         ctx[i] = context_of(i, i ? hi[i - 1] : 0, g->b);
         sym[i] = (i == 0) ? 64 * g->b + idx : idx;
+        if (m && m->f[ctx[i]][sym[i]] == 0) sym[i] = esc_symbol_of(sym[i]);
+        if (esc) esc[i] = (sym[i] & 63) == ESC_IDX;
     }
+}
+
+static void group_symbols(const Group* g, int r, int ctx[8], int sym[8], int64_t hi[8]) {
+    group_symbols_m(g, r, NULL, ctx, sym, hi, NULL);
 }
 
 /* Smallest r with 8·2^r >= alpha, at most 12. */
@@ -448,7 +514,7 @@ static double metadata_bytes(int64_t M, uint64_t T, const Model* m) {
 }
 
 /* Sampled storage estimate (format document, encoder choices, item 5). */
-static double estimate_bytes(const Tensor* t, int G, float alpha) {
+static double estimate_bytes(const Tensor* t, int G, float alpha, int pbits) {
     int64_t M = t->M, N = t->N, gpr = N / 8;
     int64_t Rs = (262144 + N - 1) / N;
     if (Rs > M) Rs = M;
@@ -464,19 +530,21 @@ static double estimate_bytes(const Tensor* t, int G, float alpha) {
             int64_t hi[8];
             quantize_group(t, row * gpr + q, alpha, &g);
             group_symbols(&g, r, ctx, sym, hi);
-            for (int i = 0; i < 8; i++) {
-                counts[ctx[i]][sym[i]]++;
-                if (sym_index(hi[i]) == ESC_IDX) n_esc++;
-            }
+            for (int i = 0; i < 8; i++) counts[ctx[i]][sym[i]]++;
             ng_s++;
         }
     }
+    prepare_counts(counts, pbits);
+    for (int c = 0; c < NCTX; c++) {
+        n_esc += counts[c][ESC_IDX];
+        if (c == 0) n_esc += counts[c][64 | ESC_IDX];
+    }
     Model m;
-    model_from_counts(counts, &m);
+    model_from_counts(counts, pbits, &m);
     double bits = 0.0;
     for (int c = 0; c < NCTX; c++)
         for (int s = m.lo[c]; s < m.lo[c] + m.cnt[c]; s++)
-            if (counts[c][s]) bits += (double)counts[c][s] * (12.0 - log2((double)m.f[c][s]));
+            if (counts[c][s]) bits += (double)counts[c][s] * ((double)pbits - log2((double)m.f[c][s]));
     bits += 16.0 * (double)n_esc + 8.0 * (double)r * (double)ng_s;
     double bits_full = bits * (double)t->NG / (double)ng_s;
     return metadata_bytes(M, num_tiles(t->NG, G), &m) + ceil(bits_full / 8.0);
@@ -489,10 +557,11 @@ static int check_shape(int dtype, int64_t M, int64_t N) {
     return OK;
 }
 
-double orc_estimate_bytes(const void* data, int dtype, int64_t M, int64_t N, int G, float alpha) {
+double orc_estimate_bytes(const void* data, int dtype, int64_t M, int64_t N, int G, float alpha, int prob_bits) {
     Tensor t;
+    if (prob_bits != PROB_BITS && prob_bits != PROB_BITS_V2) return -1.0;
     if (check_shape(dtype, M, N) || tensor_load(data, dtype, M, N, &t)) return -1.0;
-    double e = estimate_bytes(&t, G, alpha);
+    double e = estimate_bytes(&t, G, alpha, prob_bits);
     tensor_free(&t);
     return e;
 }
@@ -533,6 +602,32 @@ static int push_word(Words* ws, uint32_t v) {
 
 typedef struct { uint8_t* bytes; uint64_t size; int has_esc; } TileOut;
 
+/* Lays out one tile: the 32 final states, the raw low bits (8 fields of r bits per group, LSB-first),
+ * the pushed words in reverse push order, zero padding to 16 bytes. Frees the word list. */
+static int finish_tile(const Group* groups, int64_t g0, int64_t ng, int r, const uint32_t x[LANES], Words* ws,
+                       int has_esc, TileOut* out) {
+    uint64_t raw = pad4((uint64_t)ng * (uint64_t)r);
+    uint64_t size = pad16(128 + raw + 2 * (uint64_t)ws->n);
+    uint8_t* p = (uint8_t*)calloc((size_t)size, 1);
+    if (!p) { free(ws->w); return E_NOMEM; }
+    for (int L = 0; L < LANES; L++) put_u32(p + 4 * L, x[L]);
+    uint8_t* rawp = p + 128;
+    for (int64_t q = 0; q < ng && r > 0; q++) {
+        for (int i = 0; i < 8; i++) {
+            int64_t t = groups[g0 + q].t[i];
+            int64_t lo = t - floor_shift(t, r) * ((int64_t)1 << r);
+            uint64_t bit = 8 * (uint64_t)r * (uint64_t)q + (uint64_t)(i * r);
+            for (int k = 0; k < r; k++, bit++)
+                if ((lo >> k) & 1) rawp[bit >> 3] |= (uint8_t)(1u << (bit & 7));
+        }
+    }
+    uint8_t* sp = p + 128 + raw;
+    for (size_t n = 0; n < ws->n; n++) put_u16(sp + 2 * n, ws->w[ws->n - 1 - n]); /* reversed */
+    out->bytes = p; out->size = size; out->has_esc = has_esc;
+    free(ws->w);
+    return OK;
+}
+
 /* Encode one tile: the decode order of the format document, run backwards. */
 static int encode_tile(const Group* groups, int64_t g0, int64_t ng, int r, const Model* m, TileOut* out) {
     uint32_t x[LANES];
@@ -570,39 +665,63 @@ static int encode_tile(const Group* groups, int64_t g0, int64_t ng, int r, const
             }
         }
     }
-    {
-        uint64_t raw = pad4((uint64_t)ng * (uint64_t)r);
-        uint64_t size = pad16(128 + raw + 2 * (uint64_t)ws.n);
-        uint8_t* p = (uint8_t*)calloc((size_t)size, 1);
-        if (!p) goto nomem;
-        for (int L = 0; L < LANES; L++) put_u32(p + 4 * L, x[L]);
-        uint8_t* rawp = p + 128;
-        for (int64_t q = 0; q < ng && r > 0; q++) {
-            for (int i = 0; i < 8; i++) {
-                int64_t t = groups[g0 + q].t[i];
-                int64_t lo = t - floor_shift(t, r) * ((int64_t)1 << r);
-                uint64_t bit = 8 * (uint64_t)r * (uint64_t)q + (uint64_t)(i * r);
-                for (int k = 0; k < r; k++, bit++)
-                    if ((lo >> k) & 1) rawp[bit >> 3] |= (uint8_t)(1u << (bit & 7));
+    return finish_tile(groups, g0, ng, r, x, &ws, has_esc, out);
+nomem:
+    free(ws.w);
+    return E_NOMEM;
+}
+
+/* Version 2 tile: the decode order of the format document (pairs of positions share one
+ * renormalisation; a round's escape words follow its last pair), run backwards. Every coordinate
+ * before its pair is encoded: if x >= f1 f2 2^16 the lane first pushes x & 0xFFFF and sets x >>= 16,
+ * then x <- C(s2, x), then x <- C(s1, x), with C(s, x) = floor(x/f) 2^8 + (x mod f) + cum. */
+static int encode_tile_v2(const Group* groups, int64_t g0, int64_t ng, int r, const Model* m, TileOut* out) {
+    uint32_t x[LANES];
+    Words ws = {0, 0, 0};
+    int64_t R = (ng + 31) / 32;
+    int has_esc = 0;
+    for (int L = 0; L < LANES; L++) x[L] = RANS_L;
+    for (int64_t k = R - 1; k >= 0; k--) {
+        int ctx[LANES][8], sym[LANES][8], esc[LANES][8];
+        int64_t hi[LANES][8];
+        for (int L = 0; L < LANES; L++)
+            if (32 * k + L < ng) group_symbols_m(&groups[g0 + 32 * k + L], r, m, ctx[L], sym[L], hi[L], esc[L]);
+        /* Escape words of the round, reversed: positions descending, lanes descending. */
+        for (int i = 7; i >= 0; i--)
+            for (int L = LANES - 1; L >= 0; L--) {
+                if (32 * k + L >= ng || !esc[L][i]) continue;
+                if (push_word(&ws, (uint32_t)(uint16_t)(int16_t)hi[L][i])) goto nomem;
+                has_esc = 1;
+            }
+        /* Pairs, reversed: renormalise, then C(s2, x), then C(s1, x). */
+        for (int p = 3; p >= 0; p--) {
+            for (int L = LANES - 1; L >= 0; L--) {
+                if (32 * k + L >= ng) continue;
+                int i1 = 2 * p, i2 = 2 * p + 1;
+                uint32_t f1 = m->f[ctx[L][i1]][sym[L][i1]], c1 = m->cum[ctx[L][i1]][sym[L][i1]];
+                uint32_t f2 = m->f[ctx[L][i2]][sym[L][i2]], c2 = m->cum[ctx[L][i2]][sym[L][i2]];
+                if ((uint64_t)x[L] >= (((uint64_t)f1 * f2) << 16)) {
+                    if (push_word(&ws, x[L] & 0xFFFFu)) goto nomem;
+                    x[L] >>= 16;
+                }
+                x[L] = (x[L] / f2) * PROB_SCALE_V2 + (x[L] % f2) + c2;
+                x[L] = (x[L] / f1) * PROB_SCALE_V2 + (x[L] % f1) + c1;
             }
         }
-        uint8_t* sp = p + 128 + raw;
-        for (size_t n = 0; n < ws.n; n++) put_u16(sp + 2 * n, ws.w[ws.n - 1 - n]); /* reversed */
-        out->bytes = p; out->size = size; out->has_esc = has_esc;
     }
-    free(ws.w);
-    return OK;
+    return finish_tile(groups, g0, ng, r, x, &ws, has_esc, out);
 nomem:
     free(ws.w);
     return E_NOMEM;
 }
 
 int orc_compress(const void* data, int dtype, int64_t M, int64_t N, double target_bpp, int G,
-                 double force_alpha, uint8_t** blob_out, size_t* bytes_out, double* actual_bpp) {
+                 double force_alpha, int prob_bits, uint8_t** blob_out, size_t* bytes_out, double* actual_bpp) {
     int st = check_shape(dtype, M, N);
     if (st) return st;
     if (!(target_bpp >= 0.001 && target_bpp <= 11.0)) return E_TARGET; /* also rejects NaN */
     if (G < 1 || G > 1024 || !blob_out || !bytes_out) return E_ARG;
+    if (prob_bits != PROB_BITS && prob_bits != PROB_BITS_V2) return E_ARG;
     Tensor t;
     if ((st = tensor_load(data, dtype, M, N, &t))) return st;
 
@@ -624,7 +743,7 @@ int orc_compress(const void* data, int dtype, int64_t M, int64_t N, double targe
         for (int it = 0; it < 40; it++) {
             double mid = 0.5 * (lo + hi);
             float a = (float)exp2(mid);
-            if (8.0 * estimate_bytes(&t, G, a) <= budget) lo = mid; else hi = mid;
+            if (8.0 * estimate_bytes(&t, G, a, prob_bits) <= budget) lo = mid; else hi = mid;
         }
         alpha = (float)exp2(lo);
     }
@@ -653,8 +772,9 @@ int orc_compress(const void* data, int dtype, int64_t M, int64_t N, double targe
         group_symbols(&groups[g], r, ctx, sym, hi);
         for (int i = 0; i < 8; i++) counts[ctx[i]][sym[i]]++;
     }
+    prepare_counts(counts, prob_bits);
     Model m;
-    model_from_counts(counts, &m);
+    model_from_counts(counts, prob_bits, &m);
 
     uint64_t T = num_tiles(t.NG, G);
     TileOut* tiles = (TileOut*)calloc((size_t)T, sizeof(TileOut));
@@ -662,7 +782,9 @@ int orc_compress(const void* data, int dtype, int64_t M, int64_t N, double targe
     uint64_t payload = 0;
     for (uint64_t j = 0; j < T; j++) {
         int64_t g0 = (int64_t)j * 32 * G, ng = t.NG - g0 < 32LL * G ? t.NG - g0 : 32LL * G;
-        if ((st = encode_tile(groups, g0, ng, r, &m, &tiles[j]))) break;
+        st = prob_bits == PROB_BITS ? encode_tile(groups, g0, ng, r, &m, &tiles[j])
+                                    : encode_tile_v2(groups, g0, ng, r, &m, &tiles[j]);
+        if (st) break;
         payload += tiles[j].size;
     }
     uint8_t* blob = NULL;
@@ -678,7 +800,7 @@ int orc_compress(const void* data, int dtype, int64_t M, int64_t N, double targe
         else if (!(blob = (uint8_t*)calloc((size_t)total, 1))) st = E_NOMEM;
         if (!st) {
             memcpy(blob, "EPK1", 4);
-            put_u16(blob + 4, 1);
+            put_u16(blob + 4, prob_bits == PROB_BITS ? 1 : 2);
             blob[6] = (uint8_t)dtype;
             blob[7] = (uint8_t)r;
             put_u32(blob + 8, (uint32_t)M);
@@ -720,7 +842,7 @@ void orc_free(void* p) { free(p); }
 /* ----------------------------------------------------------------- decoder */
 
 typedef struct {
-    int dtype, r, G;
+    int version, dtype, r, G;
     int64_t M, N, NG;
     float alpha;
     uint64_t T, off_scales, off_tables, off_offsets, off_payload, total;
@@ -730,7 +852,9 @@ typedef struct {
 static int parse_blob(const uint8_t* p, size_t bytes, Blob* b, int check_crc) {
     memset(b, 0, sizeof(*b));
     if (!p || bytes < HEADER_BYTES) return E_CORRUPT;
-    if (memcmp(p, "EPK1", 4) != 0 || get_u16(p + 4) != 1) return E_CORRUPT;
+    if (memcmp(p, "EPK1", 4) != 0) return E_CORRUPT;
+    b->version = (int)get_u16(p + 4);
+    if (b->version != 1 && b->version != 2) return E_CORRUPT;
     b->dtype = p[6];
     b->r = p[7];
     b->M = get_u32(p + 8);
@@ -753,7 +877,8 @@ static int parse_blob(const uint8_t* p, size_t bytes, Blob* b, int check_crc) {
         return E_CORRUPT;
     if (b->off_tables >= bytes) return E_CORRUPT;
     uint64_t used;
-    if (read_tables(p + b->off_tables, bytes - b->off_tables, &b->m, &used)) return E_CORRUPT;
+    if (read_tables(p + b->off_tables, bytes - b->off_tables, b->version == 1 ? PROB_BITS : PROB_BITS_V2, &b->m, &used))
+        return E_CORRUPT;
     if (b->off_offsets != b->off_tables + pad16(used)) return E_CORRUPT;
     if (b->off_payload != b->off_offsets + pad16(4 * (b->T + 1)) || b->off_payload > bytes) return E_CORRUPT;
     uint64_t prev = 0;
@@ -777,10 +902,11 @@ static int parse_blob(const uint8_t* p, size_t bytes, Blob* b, int check_crc) {
 }
 
 int orc_blob_info(const uint8_t* blob, size_t bytes, int* dtype, int64_t* M, int64_t* N, float* alpha,
-                  int* r, int* G, uint32_t* T) {
+                  int* r, int* G, uint32_t* T, int* version) {
     Blob b;
     int st = parse_blob(blob, bytes, &b, 1);
     if (st) return st;
+    if (version) *version = b.version;
     if (dtype) *dtype = b.dtype;
     if (M) *M = b.M;
     if (N) *N = b.N;
@@ -882,13 +1008,100 @@ static int decode_tile(const uint8_t* p, const Blob* b, uint64_t j, void* dst, i
     return OK;
 }
 
+/* Version 2 tile. Per round k, for each pair of positions (2p, 2p + 1): every lane decodes the two
+ * symbols, the second in the context the first one's class gives (an escape has class 1), with
+ * slot = x & 255 and x <- f (x >> 8) + slot - cum; then, in ascending lane order, every lane with
+ * x < 2^16 reads one word: x <- (x << 16) | w. After the fourth pair come the round's escape words:
+ * positions ascending, lanes ascending, one int16 hi each. The raw low bits, the inverse lattice map and
+ * the rescale are those of version 1. */
+static int decode_tile_v2(const uint8_t* p, const Blob* b, uint64_t j, void* dst, int32_t* zout) {
+    const Model* m = &b->m;
+    uint64_t start = (uint64_t)(get_u32(p + b->off_offsets + 4 * j) & 0x7FFFFFFFu) * 16;
+    uint64_t end = (uint64_t)(get_u32(p + b->off_offsets + 4 * (j + 1)) & 0x7FFFFFFFu) * 16;
+    const uint8_t* tile = p + b->off_payload + start;
+    uint64_t tile_bytes = end - start;
+    int64_t g0 = (int64_t)j * 32 * b->G;
+    int64_t ng = b->NG - g0 < 32LL * b->G ? b->NG - g0 : 32LL * b->G;
+    int r = b->r;
+    uint64_t raw = pad4((uint64_t)ng * (uint64_t)r);
+    if (tile_bytes < 128 + raw) return E_CORRUPT;
+    const uint8_t* rawp = tile + 128;
+    const uint8_t* wp = tile + 128 + raw;
+    uint64_t cap = (tile_bytes - 128 - raw) / 2, pos = 0;
+    uint32_t x[LANES];
+    for (int L = 0; L < LANES; L++) x[L] = get_u32(tile + 4 * L);
+    int64_t gpr = b->N / 8, R = (ng + 31) / 32;
+
+    for (int64_t k = 0; k < R; k++) {
+        int b_of[LANES] = {0}, idx[LANES][8], cls_prev[LANES] = {0};
+        for (int pp = 0; pp < 4; pp++) {
+            for (int i = 2 * pp; i <= 2 * pp + 1; i++) {
+                for (int L = 0; L < LANES; L++) {
+                    if (32 * k + L >= ng) continue;
+                    int c = (i == 0) ? 0 : (i < 7 ? 1 : 5) + 2 * b_of[L] + cls_prev[L];
+                    uint32_t slot = x[L] & (PROB_SCALE_V2 - 1);
+                    int s = find_symbol(m, c, slot);
+                    if (s < 0) return E_CORRUPT;
+                    x[L] = m->f[c][s] * (x[L] >> PROB_BITS_V2) + slot - m->cum[c][s];
+                    if (i == 0) b_of[L] = s >> 6;
+                    idx[L][i] = s & 63;
+                    cls_prev[L] = idx[L][i] == ESC_IDX ? 1 : mag_class(idx[L][i] - 31, b_of[L]);
+                }
+            }
+            for (int L = 0; L < LANES; L++) {
+                if (32 * k + L >= ng || x[L] >= RANS_L) continue;
+                if (pos >= cap) return E_CORRUPT;
+                x[L] = (x[L] << 16) | get_u16(wp + 2 * pos++);
+            }
+        }
+        int64_t hi[LANES][8];
+        for (int i = 0; i < 8; i++)
+            for (int L = 0; L < LANES; L++) {
+                if (32 * k + L >= ng) continue;
+                if (idx[L][i] == ESC_IDX) {
+                    if (pos >= cap) return E_CORRUPT;
+                    hi[L][i] = (int16_t)get_u16(wp + 2 * pos++);
+                } else {
+                    hi[L][i] = idx[L][i] - 31;
+                }
+            }
+        for (int L = 0; L < LANES; L++) {
+            int64_t q = 32 * k + L;
+            if (q >= ng) continue;
+            int64_t t[8];
+            for (int i = 0; i < 8; i++) {
+                int64_t lo = 0;
+                uint64_t bit = 8 * (uint64_t)r * (uint64_t)q + (uint64_t)(i * r);
+                for (int kb = 0; kb < r; kb++, bit++) lo |= (int64_t)((rawp[bit >> 3] >> (bit & 7)) & 1) << kb;
+                t[i] = hi[L][i] * ((int64_t)1 << r) + lo;
+            }
+            /* Algebraic inverse of the lattice map, then the per-row rescale. */
+            int64_t g = g0 + q, row = g / gpr, col = (g % gpr) * 8;
+            int64_t u[8], sum = 0;
+            for (int i = 0; i < 7; i++) { u[i] = t[i]; sum += u[i]; }
+            u[7] = 2 * t[7] + (sum & 1);
+            float c_row = bf16_to_f32((uint16_t)get_u16(p + b->off_scales + 2 * row)) / b->alpha;
+            for (int i = 0; i < 8; i++) {
+                int64_t z = 2 * u[i] + b_of[L];
+                float v = (float)z * 0.5f;
+                float y = v * c_row;
+                store_value(dst, b->dtype, row * b->N + col + i, y);
+                if (zout) zout[row * b->N + col + i] = (int32_t)z;
+            }
+        }
+    }
+    for (int L = 0; L < LANES; L++) if (x[L] != RANS_L) return E_CORRUPT;
+    if (pos > cap || cap - pos > 7) return E_CORRUPT;
+    return OK;
+}
+
 int orc_decode_tiles(const uint8_t* blob, size_t bytes, uint32_t t0, uint32_t t1, void* dst, int32_t* zout) {
     Blob b;
     int st = parse_blob(blob, bytes, &b, 0);
     if (st) return st;
     if (t0 > t1 || t1 > b.T || !dst) return E_ARG;
     for (uint64_t j = t0; j < t1; j++)
-        if ((st = decode_tile(blob, &b, j, dst, zout))) return st;
+        if ((st = (b.version == 1 ? decode_tile : decode_tile_v2)(blob, &b, j, dst, zout))) return st;
     return OK;
 }
 

@@ -29,24 +29,27 @@ void orc_e8_nearest(const double* x, int32_t* b, int64_t* u);
 
 /* 12-bit normalisation of n <= 128 symbol counts into f[n]; returns 0. */
 int orc_normalize(const uint64_t* counts, int n, uint32_t* f);
+/* The same at `bits` = 12 (version 1) or 8 (version 2); -1 for any other precision. */
+int orc_normalize_bits(const uint64_t* counts, int n, int bits, uint32_t* f);
 
 /* Container conversions (n elements). from_container returns -5 on NaN/Inf. */
 void orc_to_container(const float* y, int64_t n, int dtype, void* out);
 int orc_from_container(const void* in, int64_t n, int dtype, float* out);
 
 /* Lossy compression of a row-major M x N container tensor. G = rounds per
- * tile. force_alpha > 0 skips rate control and uses that resolution. The blob
- * is malloc'd; release it with orc_free. */
+ * tile. force_alpha > 0 skips rate control and uses that resolution.
+ * prob_bits = 12 writes format version 1, 8 writes version 2. The blob is
+ * malloc'd; release it with orc_free. */
 int orc_compress(const void* data, int dtype, int64_t M, int64_t N, double target_bpp, int G,
-                 double force_alpha, uint8_t** blob, size_t* bytes, double* actual_bpp);
+                 double force_alpha, int prob_bits, uint8_t** blob, size_t* bytes, double* actual_bpp);
 void orc_free(void* p);
 
 /* Sampled storage estimate, in bytes, of coding the tensor at resolution alpha. */
-double orc_estimate_bytes(const void* data, int dtype, int64_t M, int64_t N, int G, float alpha);
+double orc_estimate_bytes(const void* data, int dtype, int64_t M, int64_t N, int G, float alpha, int prob_bits);
 
 /* Full validation (header, sections, tables, CRC) and header fields. */
 int orc_blob_info(const uint8_t* blob, size_t bytes, int* dtype, int64_t* M, int64_t* N,
-                  float* alpha, int* r, int* G, uint32_t* T);
+                  float* alpha, int* r, int* G, uint32_t* T, int* version);
 
 /* Decode tiles [t0, t1) into dst (the full M x N container buffer; only the
  * tiles' groups are written). zout, if not NULL, receives z = 2v (int32) for

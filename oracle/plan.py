@@ -19,9 +19,10 @@ with one theta for every layer; bound layers sit at their bound. The oracle find
 bisection on the budget (which rises with theta), 200 halvings in double precision.
 
 meta_i is written out from the EPK1 format description: a 64-byte header, bf16 row scales padded to
-16 bytes, the largest tables section (18 bytes of context ranges and 12 bits for each of the 640
-symbols, padded), the (T+1) u32 tile offsets padded, and the storage estimate's 104 bytes per tile
-for the final rANS states. T = ceil(groups / (32 G)), with the format's automatic tile size G.
+16 bytes, the largest tables section (18 bytes of context ranges and one frequency for each of the 640
+symbols, 8 bits in format version 2 and 12 in version 1, padded), the (T+1) u32 tile offsets padded, and
+the storage estimate's 104 bytes per tile for the final rANS states. T = ceil(groups / (32 G)), with the
+format's automatic tile size G.
 
 Parity pins: ``tests/test_plan.py`` checks this against a general constrained solver
 (scipy's SLSQP) on the same objective, the closed form of the unbounded case, and the section sizes
@@ -51,19 +52,20 @@ def auto_rounds(groups: int) -> int:
     return int(min(24, max(12, math.ceil(groups / (32 * slots * waves)))))
 
 
-def metadata_bits_per_param(rows: int, cols: int, rounds: int = 0) -> float:
+def metadata_bits_per_param(rows: int, cols: int, rounds: int = 0, version: int = 2) -> float:
     groups = rows * cols // 8
     G = rounds if rounds else auto_rounds(groups)
     tiles = -(-groups // (32 * G))
-    tables = 2 * 9 + -(-12 * MAX_TABLE_SYMBOLS // 8)
+    fbits = 12 if version == 1 else 8
+    tables = 2 * 9 + -(-fbits * MAX_TABLE_SYMBOLS // 8)
     meta = HEADER_BYTES + pad16(2 * rows) + pad16(tables) + pad16(4 * (tiles + 1)) + 104 * tiles
     return 8.0 * meta / (rows * cols)
 
 
-def plan(shapes, weights, mean_bpp, min_bpp=0.001, max_bpp=11.0, rounds=0):
+def plan(shapes, weights, mean_bpp, min_bpp=0.001, max_bpp=11.0, rounds=0, version=2):
     """Per-layer targets b_i (list of floats) for layers of the given (rows, cols) shapes."""
     n = [r * c for r, c in shapes]
-    meta = [metadata_bits_per_param(r, c, rounds) for r, c in shapes]
+    meta = [metadata_bits_per_param(r, c, rounds, version) for r, c in shapes]
     lo = [min(max(min_bpp, m), max_bpp) for m in meta]
     hi = [max_bpp] * len(shapes)
     free = [m + 0.5 * math.log2(w) for m, w in zip(meta, weights)]
@@ -90,7 +92,7 @@ def plan(shapes, weights, mean_bpp, min_bpp=0.001, max_bpp=11.0, rounds=0):
     return rates(0.5 * (a + b))
 
 
-def objective(shapes, weights, bpp, rounds=0):
+def objective(shapes, weights, bpp, rounds=0, version=2):
     """The quantity the plan minimises, for any assignment of targets."""
-    return sum(r * c * w * 2.0 ** (-2.0 * (b - metadata_bits_per_param(r, c, rounds)))
+    return sum(r * c * w * 2.0 ** (-2.0 * (b - metadata_bits_per_param(r, c, rounds, version)))
                for (r, c), w, b in zip(shapes, weights, bpp))

@@ -3,7 +3,7 @@
 Covered here:
 - libentropack.so loads and exports every function that include/entropack.h declares;
 - the host encoder (product) and the oracle encoder are independent implementations of the same
-  format, and they produce byte-identical blobs;
+  format, and they produce byte-identical blobs in both format versions;
 - the host validator accepts every good blob and rejects corrupted ones;
 - the C ABI returns the documented status codes for bad input (README, Config table: the target
   range; 2-D only).
@@ -63,12 +63,17 @@ CASES = [
 ]
 
 
+PBITS = {1: 12, 2: 8}  # format version -> frequency precision
+
+
+@pytest.mark.parametrize("version", [2, 1])
 @pytest.mark.parametrize("name,maker,target,G", CASES, ids=[c[0] for c in CASES])
-def test_host_encoder_matches_oracle_bytes(ep, orc, name, maker, target, G):
+def test_host_encoder_matches_oracle_bytes(ep, orc, name, maker, target, G, version):
     w = maker()
-    ob, obpp = orc.compress(synth.container_bits(w), synth.dtype_code(w), target, G)
-    c = ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G))
+    ob, obpp = orc.compress(synth.container_bits(w), synth.dtype_code(w), target, G, prob_bits=PBITS[version])
+    c = ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G, format_version=version))
     assert c.blob == ob
+    assert orc.blob_info(c.blob)["version"] == version
     assert c.actual_bpp == pytest.approx(obpp)
     info = ep.blob_info(c.blob)
     assert (info["rows"], info["cols"]) == tuple(w.shape)
@@ -156,9 +161,11 @@ def _fuzz_case(seed):
     return w, round(rnd.uniform(0.3, 11.0), 3), rnd.choice([0, 1, 2, 5, 16, 40])
 
 
+@pytest.mark.parametrize("version", [2, 1])
 @pytest.mark.parametrize("seed", range(12))
-def test_host_encoder_matches_oracle_bytes_fuzz(ep, orc, seed):
+def test_host_encoder_matches_oracle_bytes_fuzz(ep, orc, seed, version):
     w, target, G = _fuzz_case(1000 + seed)
-    ob, _ = orc.compress(synth.container_bits(w), synth.dtype_code(w), target, G if G else 16)
-    c = ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G if G else 16))
+    ob, _ = orc.compress(synth.container_bits(w), synth.dtype_code(w), target, G if G else 16,
+                         prob_bits=PBITS[version])
+    c = ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G if G else 16, format_version=version))
     assert c.blob == ob

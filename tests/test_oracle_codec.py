@@ -57,6 +57,38 @@ def test_crc32_matches_zlib(orc):
         assert orc.crc32(data) == zlib.crc32(data)
 
 
+def test_normalize_8bit_cases(orc):
+    """Version 2's 8-bit tables follow the same rule at a total of 256."""
+    assert list(orc.normalize([1, 1], bits=8)) == [128, 128]
+    assert list(orc.normalize([3, 1], bits=8)) == [192, 64]
+    assert list(orc.normalize([0, 5, 0], bits=8)) == [0, 255, 1]
+    assert list(orc.normalize([1, 0, 1000000], bits=8)) == [1, 0, 255]
+    assert list(orc.normalize([1, 1, 1, 997], bits=8)) == [1, 1, 1, 253]
+    rng = np.random.default_rng(6)
+    for _ in range(300):
+        n = int(rng.integers(2, 129))
+        counts = rng.integers(0, 5, size=n) * rng.integers(0, 10 ** int(rng.integers(0, 7)), size=n)
+        f = orc.normalize(counts, bits=8)
+        present = counts > 0
+        if present.sum() >= 2:
+            assert f.sum() == 256 and f.max() <= 255 and np.all(f[present] >= 1) and np.all(f[~present] == 0)
+
+
+def test_version2_escapes_rare_symbols(orc):
+    """Version 2 sends rare symbols as escapes: a Gaussian matrix with a sparse set of moderate outliers
+    (|hi| up to about 30, inside the 12-bit alphabet) codes them as escapes at 8 bits but not at 12, and both
+    round-trip exactly."""
+    w = synth.gaussian(256, 512, seed=30, container="fp32")
+    w.view(-1)[::997] *= 3.0
+    w = w.to(torch.bfloat16)
+    offs = {}
+    for pbits in PBITS:
+        blob, _, info, _ = roundtrip_case(orc, w, 4.0, pbits=pbits)
+        o = np.frombuffer(blob, dtype="<u4", offset=int.from_bytes(blob[36:40], "little"), count=info["num_tiles"] + 1)
+        offs[pbits] = (o[:-1] >> 31).mean()
+    assert offs[12] == 0.0 and offs[8] > 0.5
+
+
 def test_normalize_invariants(orc):
     assert list(orc.normalize([1, 1])) == [2048, 2048]
     assert list(orc.normalize([3, 1])) == [3072, 1024]
@@ -86,9 +118,10 @@ def test_normalize_invariants(orc):
 
 # -------------------------------------------------------------- round trip
 
-def roundtrip_case(orc, w, target=4.0, G=16, force_alpha=0.0):
+def roundtrip_case(orc, w, target=4.0, G=16, force_alpha=0.0, pbits=8):
     a, dt = bits(w)
-    blob, bpp = orc.compress(a, dt, target, G, force_alpha)
+    blob, bpp = orc.compress(a, dt, target, G, force_alpha, prob_bits=pbits)
+    assert orc.blob_info(blob)["version"] == (1 if pbits == 12 else 2)
     info = orc.blob_info(blob)
     out, z = orc.decompress(blob, with_coords=True)
     zq, s = orc.quantize(a, dt, info["alpha"])
@@ -101,24 +134,31 @@ def roundtrip_case(orc, w, target=4.0, G=16, force_alpha=0.0):
     return blob, bpp, info, out
 
 
-def test_roundtrip_quickstart(orc):
+PBITS = [8, 12]  # format version 2 and version 1
+
+
+@pytest.mark.parametrize("pbits", PBITS)
+def test_roundtrip_quickstart(orc, pbits):
     w = synth.quickstart_256()
-    blob, bpp, info, _ = roundtrip_case(orc, w, 3.5)
+    blob, bpp, info, _ = roundtrip_case(orc, w, 3.5, pbits=pbits)
     assert info["num_tiles"] == 16 and info["r"] == 0
 
 
-def test_roundtrip_all_zero_is_exact_metadata(orc):
-    """All-zero input: every used context holds one symbol (stored as 4095 + 1), which costs
-    log2(4096/4095) bits a coordinate. That stays inside the 32 states (no word is emitted), so each
-    tile is 128 bytes and the blob size is metadata only."""
-    M, N, G = 96, 64, 2
+@pytest.mark.parametrize("pbits,G,target", [(8, 2, 2.0), (12, 2, 2.0), (8, 16, 0.5)])
+def test_roundtrip_all_zero_is_exact_metadata(orc, pbits, G, target):
+    """All-zero input: every used context holds one symbol (stored as 2^bits - 1, plus 1 on a neighbour),
+    which costs log2(2^bits / (2^bits - 1)) bits a coordinate: 0.00035 at 12 bits, 0.0056 at 8. Over a
+    lane's 16 or 128 coordinates that stays inside its state (no word is emitted), so each tile is 128
+    bytes and the blob size is metadata only."""
+    M, N = 96, 64
     w = torch.zeros(M, N, dtype=torch.bfloat16)
-    blob, bpp, info, out = roundtrip_case(orc, w, 2.0, G)
+    blob, bpp, info, out = roundtrip_case(orc, w, target, G, pbits=pbits)
+    assert info["r"] == 0  # targets low enough that no raw bits fit the budget
     T = math.ceil(M * N / 8 / (32 * G))
     pad = lambda n: (n + 15) // 16 * 16
     # contexts reached: START, ctx 1 (b=0, class 0) and ctx 5 (position 7, b=0, class 0); each stores
     # its one symbol and the neighbour that takes f = 1
-    tables = 18 + math.ceil(12 * 6 / 8)
+    tables = 18 + math.ceil(pbits * 6 / 8)
     assert len(blob) == 64 + pad(2 * M) + pad(tables) + pad(4 * (T + 1)) + T * 128
     payload = blob[-T * 128:]
     states = np.frombuffer(payload, dtype="<u4")
@@ -126,15 +166,17 @@ def test_roundtrip_all_zero_is_exact_metadata(orc):
     assert np.all(out == 0)
 
 
-def test_roundtrip_outliers_and_escapes(orc):
+@pytest.mark.parametrize("pbits", PBITS)
+def test_roundtrip_outliers_and_escapes(orc, pbits):
     w = synth.lognormal_rows_with_outliers(n=256, seed=11, outlier_frac=2e-3, outlier_mult=40.0)
-    blob, bpp, info, _ = roundtrip_case(orc, w, 4.0)
+    blob, bpp, info, _ = roundtrip_case(orc, w, 4.0, pbits=pbits)
     offs = np.frombuffer(blob, dtype="<u4", offset=int.from_bytes(blob[36:40], "little"),
                          count=info["num_tiles"] + 1)
     assert (offs >> 31).any(), "outliers this large must produce ESC symbols"
 
 
-def test_roundtrip_extreme_escape_values(orc):
+@pytest.mark.parametrize("pbits", PBITS)
+def test_roundtrip_extreme_escape_values(orc, pbits):
     """int16 extremes of hi: one huge entry per row forces |hi| near 2^15 at r = 0."""
     M, N = 64, 4096
     g = torch.Generator().manual_seed(5)
@@ -142,40 +184,46 @@ def test_roundtrip_extreme_escape_values(orc):
     w[:, 7] = 1.0
     w[::2, 9] = -1.0
     w = w.to(torch.float32)
-    roundtrip_case(orc, w, 3.0, force_alpha=450.0)
+    roundtrip_case(orc, w, 3.0, force_alpha=450.0, pbits=pbits)
 
 
-def test_roundtrip_r12_and_raw_bits(orc):
+@pytest.mark.parametrize("pbits", PBITS)
+def test_roundtrip_r12_and_raw_bits(orc, pbits):
     g = torch.Generator().manual_seed(6)
     w = torch.randn(40, 8, generator=g).to(torch.float32)
-    _, _, info, _ = roundtrip_case(orc, w, 11.0, G=1, force_alpha=32768.0)
+    _, _, info, _ = roundtrip_case(orc, w, 11.0, G=1, force_alpha=32768.0, pbits=pbits)
     assert info["r"] == 12
     w2 = synth.gaussian(128, 128, seed=8, container="fp16")
-    _, _, info2, _ = roundtrip_case(orc, w2, 9.0)
+    _, _, info2, _ = roundtrip_case(orc, w2, 9.0, pbits=pbits)
     assert 0 < info2["r"] < 12
 
 
+@pytest.mark.parametrize("pbits", PBITS)
 @pytest.mark.parametrize("M,N,G", [(129, 8, 2), (1, 8, 1), (3, 40, 1), (33, 64, 3), (200, 96, 1024)])
-def test_roundtrip_ragged_tiles(orc, M, N, G):
+def test_roundtrip_ragged_tiles(orc, M, N, G, pbits):
     """Partial last rounds and tiles: e.g. 129x8 with G=2 is 64 + 64 + 1 groups (a 1-group tile)."""
     w = synth.gaussian(M, N, seed=M * 7 + N, container="bf16")
-    _, _, info, _ = roundtrip_case(orc, w, 3.0, G)
+    _, _, info, _ = roundtrip_case(orc, w, 3.0, G, pbits=pbits)
     assert info["num_tiles"] == math.ceil(M * N / 8 / (32 * G))
 
 
+@pytest.mark.parametrize("pbits", PBITS)
 @pytest.mark.parametrize("maker,target", [(lambda: synth.fp8_codes(64, 512, seed=3), 5.0),
                                           (lambda: synth.int8_codes(64, 512, seed=4), 3.0)])
-def test_roundtrip_low_precision_containers(orc, maker, target):
+def test_roundtrip_low_precision_containers(orc, maker, target, pbits):
     w = maker()
-    _, bpp, _, out = roundtrip_case(orc, w, target)
+    _, bpp, _, out = roundtrip_case(orc, w, target, pbits=pbits)
     assert abs(bpp - target) <= 0.05 or bpp < target
 
 
 # ------------------------------------------------------------- code length
 
-def ideal_bits_from_coords(orc, z, r):
-    """Ideal code length Σ -log2(f/4096) of the symbols, under 12-bit tables fitted to them,
-    with the coordinate-to-symbol map restated from the format (independent of the oracle)."""
+def ideal_bits_from_coords(orc, z, r, pbits=12):
+    """Ideal code length Σ -log2(f/2^bits) of the symbols, under tables fitted to them, with the
+    coordinate-to-symbol map restated from the format (independent of the oracle). At 8 bits (format
+    version 2) the rare-symbol rule is restated too: in each context, a symbol other than hi in [-2, 2]
+    seen in fewer than 1/4096 of the context's coordinates is sent as its escape (index 63 of its coset
+    half), 16 raw bits more."""
     M, N = z.shape
     u = (z - (z & 1)) // 2   # z = 2u + b
     b = (z[:, 0::8] & 1).reshape(-1)
@@ -192,25 +240,37 @@ def ideal_bits_from_coords(orc, z, r):
     for i in range(1, 8):
         ctx = (1 if i < 7 else 5) + 2 * b + cls[:, i - 1]
         np.add.at(counts, (ctx, idx[:, i]), 1)
+    if pbits == 8:
+        for c in range(9):
+            A = 128 if c == 0 else 64
+            n = int(counts[c][:A].sum())
+            for sym in range(A):
+                k = sym & 63
+                if k == 63 or 29 <= k <= 33 or counts[c][sym] == 0:
+                    continue
+                if int(counts[c][sym]) * 4096 < n:
+                    counts[c][(sym & 64) | 63] += counts[c][sym]
+                    counts[c][sym] = 0
     total = 0.0
     for c in range(9):
-        f = orc.normalize(counts[c][:128 if c == 0 else 64])
+        f = orc.normalize(counts[c][:128 if c == 0 else 64], bits=pbits)
         nz = counts[c][:f.size] > 0
-        total += float((counts[c][:f.size][nz] * (12.0 - np.log2(f[nz].astype(np.float64)))).sum())
-    n_esc = int((idx == 63).sum())
+        total += float((counts[c][:f.size][nz] * (pbits - np.log2(f[nz].astype(np.float64)))).sum())
+    n_esc = int(counts[:, 63].sum() + counts[0, 127])
     return total + 16 * n_esc + 8 * r * u.shape[0]
 
 
+@pytest.mark.parametrize("pbits", PBITS)
 @pytest.mark.parametrize("target", [2.0, 3.5, 7.0])
-def test_coded_size_close_to_ideal(orc, target):
+def test_coded_size_close_to_ideal(orc, target, pbits):
     """The rANS payload (stream words plus raw bytes, with the states counted at ~24 bits each) is within
-    1% + 64 bytes of the ideal code length of the coded symbols."""
+    1% + 64 bytes of the ideal code length of the coded symbols, under the version's tables."""
     w = synth.gaussian(512, 512, seed=21, container="bf16")
     a, dt = bits(w)
-    blob, _ = orc.compress(a, dt, target)
+    blob, _ = orc.compress(a, dt, target, prob_bits=pbits)
     info = orc.blob_info(blob)
     _, z = orc.decompress(blob, with_coords=True)
-    ideal = ideal_bits_from_coords(orc, z, info["r"]) / 8
+    ideal = ideal_bits_from_coords(orc, z, info["r"], pbits) / 8
     off_payload = int.from_bytes(blob[40:44], "little")
     T = info["num_tiles"]
     payload = len(blob) - off_payload
