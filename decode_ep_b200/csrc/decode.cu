@@ -34,6 +34,7 @@
 
 #include <cstdlib>
 #include <mutex>
+#include <vector>
 
 #include "capi_internal.h"
 #include "entropack.h"
@@ -97,7 +98,7 @@ struct Params {
     float alpha, inv_alpha;  // inv_alpha = RN(1 / alpha), computed on the host
     // Multipliers kept out of the compiler's sight (2, 4, -4096, 128), so that the products below are
     // issued as integer multiply-adds instead of ALU shifts: the loop saturates the ALU pipe first.
-    uint32_t k2, k4, kneg4096, k128;
+    uint32_t k2, k4, kneg4096, k128, kneg256;
     uint32_t off_scales, off_tables, off_offsets, off_payload, tables_len;
     uint64_t payload_bytes;
     // The next blob of a sequence (ep_decompress_many), or null: its tables, tile offsets and scales
@@ -974,6 +975,561 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Params p) {
 }
 
 
+// ===================================================================== format version 2
+//
+// Version 2 codes the same coordinates with 8-bit frequencies, so one renormalisation serves a pair of
+// symbols (positions 0-1, 2-3, 4-5, 6-7): from a state in [2^16, 2^32), two symbols take at most 16 bits,
+// and one 16-bit word restores the range. The tables are 9 contexts x 256 slots of 4-byte fused entries,
+// 9 KB, which each CTA builds in about a microsecond. Rare symbols are escapes; their words follow the
+// round's fourth pair and are read only when some lane of the warp met one.
+namespace v2 {
+
+// Fused entry of one slot: value field (bits 0-7: 2 idx + b at positions 0..6, 4 idx + b at position 7),
+// escape flag (bit 9), magnitude class of the coordinate (bit 10, picks the next context's 1 KB block),
+// coset bit b (bit 11, START only: picks the b half), f (bits 16-23) and slot - cum (bits 24-31).
+constexpr uint32_t kEscBit = 1u << 9;
+constexpr uint32_t kClassBit = 1u << 10;
+constexpr uint32_t kCosetBit = 1u << 11;
+constexpr uint32_t kPos7Bit = 1u << 12;
+// Blocks: contexts 1..8 at (c - 1) KB, so (b, class) select bits 11 and 10 and position 7 adds bit 12;
+// START at 8 KB. The region sits on a 16 KB boundary of the shared window, so the bits combine by OR.
+constexpr uint32_t kCtxBytes = 256 * 4;
+constexpr uint32_t kStartOffset = 8 * kCtxBytes;
+constexpr uint32_t kTablesBytes = 9 * kCtxBytes;
+constexpr uint32_t kTableAlign = 16 * 1024;
+__host__ __device__ constexpr uint32_t block_of(int c) { return c == 0 ? kStartOffset : uint32_t(c - 1) * kCtxBytes; }
+
+// Warps per CTA: one CTA per SM.
+constexpr int kWarpsV2 = 32;
+constexpr int kThreadsV2 = kWarpsV2 * 32;
+
+// Per-warp stream rings: 4 KB, enough for the whole word stream of a tile up to about 7 bits per
+// coordinate at 16 rounds; longer streams are read from global memory by the general rounds.
+constexpr uint32_t kRingBytes = 4096;
+constexpr uint32_t kChunkBytes = 512;
+constexpr uint32_t kRingChunks = kRingBytes / kChunkBytes;
+constexpr uint32_t kRingsBytes = kWarpsV2 * kRingBytes;
+// Scratch of the table build: f and cum per context and symbol (u16), and the staged table bytes.
+constexpr uint32_t kScratchF = 0;                               // u16 [9][128]
+constexpr uint32_t kScratchCum = kScratchF + kNumCtx * 128 * 2; // u16 [9][129]
+constexpr uint32_t kScratchBytesOff = (kScratchCum + kNumCtx * 129 * 2 + 15) & ~15u;
+constexpr uint32_t kScratchTableCap = 1024;                     // a valid blob's tables take 658 bytes at most
+constexpr uint32_t kScratchSize = kScratchBytesOff + kScratchTableCap;
+// [pad to 4 KB][rings][pad to 16 KB][tables][scratch][slack]. At least kOverrunBytes follow the last ring.
+constexpr uint32_t kSlackBytes = 6 * 1024;
+constexpr uint32_t kSmemBytes = kRingBytes + kRingsBytes + kTableAlign + kTablesBytes + kScratchSize + kSlackBytes;
+static_assert(kSmemBytes <= 227 * 1024, "exceeds the per-block shared memory of sm_100");
+// Words one round can take: one refill per pair and lane, plus one escape word per coordinate.
+constexpr uint32_t kRoundWords = 4 * 32 + 8 * 32;
+// Fast rounds run without checking the stream position; they are capped so that a corrupt stream stays in
+// the shared allocation: at most kMaxFastRounds * 2 * kRoundWords bytes past a ring's end.
+constexpr uint32_t kMaxFastRounds = 24;
+constexpr uint32_t kOverrunBytes = kMaxFastRounds * 2 * kRoundWords + 64;
+
+// Words of a stream that sits wholly in the warp's ring, at ring coordinate pb (callers keep a round's reads
+// inside the ring).
+struct RingWords {
+    uint32_t base;
+    __device__ __forceinline__ uint32_t at(uint32_t pb) const { return ld_shared_u16(base + pb); }
+};
+
+// The fused entry of symbol `sym` of context c without its slot - cum field.
+__device__ __forceinline__ uint32_t entry_template_v2(int c, int sym, uint32_t f) {
+    const int b = c == 0 ? (sym >> 6) : (c <= 4 ? (c - 1) >> 1 : (c - 5) >> 1);
+    const int idx = sym & 63, hi = idx - 31;
+    const bool esc = idx == kEscIdx;
+    uint32_t e = (f & 0xFFu) << 16;
+    if (esc) e |= kEscBit;
+    if (c <= 4) {  // START and positions 1..6: v = hi + b/2; the class picks the next context
+        e |= uint32_t(2 * idx + b);
+        if (esc || mag_class(hi, b)) e |= kClassBit;  // an escape always has |hi| >= 3
+        if (c == 0 && b) e |= kCosetBit;
+    } else {       // position 7 codes h: 2h + b/2 (the parity is added later)
+        e |= uint32_t(4 * idx + b);
+    }
+    return e;
+}
+
+// Builds the 9 x 256 fused entries of the blob's tables in shared memory. Pass 1: one warp per context
+// reads its 8-bit frequencies (4 symbols a lane) and prefix-sums them into cum, checking that a used
+// context sums to 256. Pass 2: each thread fills slots, finding the symbol that owns each by binary search.
+__device__ void build_tables_v2(const Params& p, uint8_t* tables, uint8_t* scratch) {
+    uint16_t* F = reinterpret_cast<uint16_t*>(scratch + kScratchF);
+    uint16_t* cum = reinterpret_cast<uint16_t*>(scratch + kScratchCum);
+    uint8_t* tb = scratch + kScratchBytesOff;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t tlen = p.tables_len < kScratchTableCap ? p.tables_len : kScratchTableCap;
+    for (uint32_t i = tid; i < kScratchTableCap; i += kThreadsV2) tb[i] = i < tlen ? __ldg(p.blob + p.off_tables + i) : 0;
+    __syncthreads();
+    if (warp < kNumCtx) {
+        const int c = warp, A = c == 0 ? 128 : 64;
+        const uint32_t lo = tb[c], cnt = tb[kNumCtx + c];
+        uint32_t off = 2 * kNumCtx;
+        for (int k = 0; k < c; ++k) off += tb[kNumCtx + k];
+        uint32_t f[4], part = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t s = 4 * lane + j;
+            f[j] = (s < uint32_t(A) && s >= lo && s < lo + cnt && off + s - lo < kScratchTableCap) ? tb[off + s - lo] : 0u;
+            part += f[j];
+        }
+        uint32_t incl = part;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t v = __shfl_up_sync(kFullMask, incl, d);
+            if (lane >= d) incl += v;
+        }
+        uint32_t acc = incl - part;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t s = 4 * lane + j;
+            if (s < 128) {
+                F[c * 128 + s] = uint16_t(f[j]);
+                cum[c * 129 + s] = uint16_t(acc);
+            }
+            acc += f[j];
+        }
+        const uint32_t total = __shfl_sync(kFullMask, incl, 31);
+        if (lane == 0) {
+            cum[c * 129 + 128] = uint16_t(total);
+            const bool ok = cnt == 0 ? total == 0 : (total == kProbScaleV2 && cnt >= 2);
+            if (!ok && blockIdx.x == 0) atomicOr(&g_status, int(EP_DEV_BAD_TABLES));
+        }
+    }
+    __syncthreads();
+    uint32_t* t32 = reinterpret_cast<uint32_t*>(tables);
+    for (uint32_t k = tid; k < kNumCtx * 256; k += kThreadsV2) {
+        const int c = int(k >> 8), A = c == 0 ? 128 : 64;
+        const uint32_t t = k & 255;
+        const uint16_t* cc = cum + c * 129;
+        int s = 0;
+#pragma unroll
+        for (int step = 64; step >= 1; step >>= 1)  // largest s < A with cum[s] <= t
+            if (s + step < A && cc[s + step] <= t) s += step;
+        const uint32_t f = F[c * 128 + s];
+        // A slot past the table's end (a corrupt table) gets f = 0: the tile check flags it.
+        const uint32_t e = (t >= cc[s] && t < cc[s] + f) ? entry_template_v2(c, s, f) | ((t - cc[s]) << 24) : 0u;
+        t32[block_of(c) / 4 + t] = e;
+    }
+    __syncthreads();
+}
+
+// One symbol step: the fused entry of the context block B at slot x & 255, then x <- f (x >> 8) + slot - cum.
+__device__ __forceinline__ uint32_t symbol(const Params& p, uint32_t B, uint32_t& x) {
+    const uint32_t q = x >> 8;
+    const uint32_t e = ld_shared_u32((x + q * p.kneg256) * p.k4 + B);  // B + 4 (x mod 256)
+    x = __byte_perm(e, 0u, 0x4442u) * q + (e >> 24);
+    return e;
+}
+
+// The pair's refill from the warp's ring: lanes with x < 2^16 take the next words in lane order. pa is
+// the shared address of the next word; k2 = 2 (a multiplier kept in a register so the address arithmetic
+// runs as multiply-adds). Every lane loads (the address stays in the ring), and only the lanes that need
+// the word merge it, by a predicated byte permute: no branch.
+__device__ __forceinline__ void refill(uint32_t& x, uint32_t& pa, uint32_t lt_mask, uint32_t k2) {
+    asm volatile(
+        "{\n"
+        " .reg .pred p;\n"
+        " .reg .b32 m, t, c, a, w;\n"
+        " setp.lt.u32 p, %0, 65536;\n"
+        " vote.sync.ballot.b32 m, p, 0xffffffff;\n"
+        " and.b32 t, m, %2;\n"
+        " popc.b32 c, t;\n"
+        " mad.lo.u32 a, c, %3, %1;\n"
+        " ld.shared.u16 w, [a];\n"
+        " @p prmt.b32 %0, %0, w, 0x1054;\n"
+        " popc.b32 c, m;\n"
+        " mad.lo.u32 %1, c, %3, %1;\n"
+        "}"
+        : "+r"(x), "+r"(pa)
+        : "r"(lt_mask), "r"(k2));
+}
+
+// Values of one group from the value bits mb[i]: 1.5 * 2^22 + F/2 with F = 2 idx + b at positions 0..6 and
+// 4 idx + b at position 7 (before pi is added), built by ORing the entries' value fields into the mantissa
+// (see round_fast of version 1). two_pi = 2 pi comes from the XOR of the idx parities.
+template <int MODE, bool WAIT>
+__device__ __forceinline__ void store_fast(const Params& p, const uint32_t* mb, uint32_t two_pi, uint32_t g, float c) {
+    float m[8], y[8];
+    int32_t z[8];
+#pragma unroll
+    for (int i = 0; i < 7; ++i) m[i] = __uint_as_float(mb[i]);
+    m[7] = __uint_as_float(mb[7] + two_pi);
+    const float K = kHalfMagicF + 31.0f, K7 = kHalfMagicF + 62.0f;
+#pragma unroll
+    for (int i = 0; i < 6; i += 2) sub_mul_f32x2(m[i], m[i + 1], K, K, c, y[i], y[i + 1]);
+    sub_mul_f32x2(m[6], m[7], K, K7, c, y[6], y[7]);
+    if constexpr (MODE == kCoords) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) z[i] = __float2int_rn((m[i] - (i < 7 ? K : K7)) * 2.0f);
+    }
+    if constexpr (WAIT) grid_dependency_wait();
+    store_group<MODE>(p.dst, g, y, z);
+}
+
+// Values of one group in general: hi from the entries or the escape words, lo from the raw section, then
+// t = hi 2^r + lo, u_7 = 2 t_7 + pi, z = 2u + b and y = RN(z/2 * c).
+template <int MODE>
+__device__ __forceinline__ void store_general(const Params& p, const uint32_t* e, const int32_t* hesc, uint32_t escm,
+                                              const uint32_t* win, uint32_t g, float c) {
+    const int r = p.r;
+    int32_t t[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t idx = i < 7 ? (e[i] >> 1) & 63u : (e[i] >> 2) & 63u;
+        const int32_t hi = (escm >> i) & 1u ? hesc[i] : int32_t(idx) - 31;
+        int32_t lo = 0;
+        if (r > 0) {
+            const uint32_t bp = uint32_t(i) * uint32_t(r), sel = bp >> 5, sh = bp & 31;
+            const uint32_t wa = sel == 0 ? win[0] : (sel == 1 ? win[1] : win[2]);
+            const uint32_t wb = sel == 0 ? win[1] : win[2];
+            lo = int32_t(__funnelshift_r(wa, wb, sh) & ((1u << r) - 1u));
+        }
+        t[i] = hi * (1 << r) + lo;
+    }
+    const int32_t b = int32_t(e[0] & 1u);
+    int32_t s7 = 0;
+#pragma unroll
+    for (int i = 0; i < 7; ++i) s7 += t[i];
+    float y[8];
+    int32_t z[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int32_t u = i < 7 ? t[i] : 2 * t[7] + (s7 & 1);
+        z[i] = 2 * u + b;
+        y[i] = __fmul_rn(__int2float_rn(z[i]) * 0.5f, c);
+    }
+    store_group<MODE>(p.dst, g, y, z);
+}
+
+// The 96-bit window of raw bits of group q (8r bits at byte q r of the tile's raw section).
+__device__ __forceinline__ void raw_window(const uint8_t* rawsec, uint32_t raw_avail, uint32_t q, int r, uint32_t* win) {
+    win[0] = win[1] = win[2] = 0;
+    if (r <= 0) return;
+    const uint32_t o = q * uint32_t(r), a = o & ~3u, sh = (o & 3u) * 8;
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        w[j] = (a + 4 * j + 4 <= raw_avail) ? __ldg(reinterpret_cast<const uint32_t*>(rawsec + a) + j) : 0u;
+    win[0] = __funnelshift_r(w[0], w[1], sh);
+    win[1] = __funnelshift_r(w[1], w[2], sh);
+    win[2] = __funnelshift_r(w[2], w[3], sh);
+}
+
+// Three-input logic in one instruction: (a & b) | c, a ^ b ^ c and a | b | c.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t xor3(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0x96;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t or3(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xFE;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// Fast round: every lane holds a group, r = 0, and the whole stream sits in the warp's ring (pa is the
+// shared address of the next word). Each entry is turned into its value bits at once; the XOR of the entries
+// of positions 0..6 carries the idx parities (bit 1) and their OR the escape flag. ESC: the tile holds an
+// escape (its offset entry says so). Then, when some lane of the warp met one in this round, its words are
+// read after the fourth pair, and each escaped position's value bits and parity are rebuilt from the word's
+// hi (an escape's field, 2 * 63 + b or 4 * 63 + b, marks it).
+template <int MODE, bool WAIT, bool ESC>
+__device__ __forceinline__ void round_fast_v2(const Params& p, uint32_t t0, uint32_t& x, uint32_t& pa, uint32_t g,
+                                              uint32_t lt_mask, float c, uint32_t k2) {
+    uint32_t mb[8], e, e2, par, escs;
+    e = symbol(p, t0 | kStartOffset, x);
+    mb[0] = and_or(e, 0x7Fu, kHalfMagic);
+    const uint32_t gbase = and_or(e, kCosetBit, t0);
+    e2 = symbol(p, and_or(e, kClassBit, gbase), x);
+    mb[1] = and_or(e2, 0x7Fu, kHalfMagic);
+    par = e ^ e2;
+    escs = e | e2;
+    refill(x, pa, lt_mask, k2);
+#pragma unroll
+    for (int i = 2; i < 6; i += 2) {
+        e = symbol(p, and_or(e2, kClassBit, gbase), x);
+        mb[i] = and_or(e, 0x7Fu, kHalfMagic);
+        e2 = symbol(p, and_or(e, kClassBit, gbase), x);
+        mb[i + 1] = and_or(e2, 0x7Fu, kHalfMagic);
+        par = xor3(par, e, e2);
+        escs = or3(escs, e, e2);
+        refill(x, pa, lt_mask, k2);
+    }
+    e = symbol(p, and_or(e2, kClassBit, gbase), x);
+    mb[6] = and_or(e, 0x7Fu, kHalfMagic);
+    e2 = symbol(p, and_or(e, kClassBit, gbase | kPos7Bit), x);
+    mb[7] = and_or(e2, 0xFFu, kHalfMagic);
+    par ^= e;
+    escs = or3(escs, e, e2);
+    refill(x, pa, lt_mask, k2);
+    if (ESC && __any_sync(kFullMask, escs & kEscBit)) {
+        const uint32_t b = mb[0] & 1u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const bool esc = i < 7 ? (mb[i] & 0x7Eu) == 0x7Eu : (mb[7] & 0xFCu) == 0xFCu;
+            const uint32_t me = __ballot_sync(kFullMask, esc);
+            if (me) {
+                const uint32_t w = ld_shared_u16(pa + __popc(me & lt_mask) * k2);
+                pa += __popc(me) * k2;
+                if (esc) {
+                    const int32_t idx = int32_t(int16_t(w)) + 31;  // hi + 31, any int16 hi
+                    if (i < 7) {
+                        mb[i] = kHalfMagic + uint32_t(2 * idx) + b;
+                        par ^= (uint32_t(idx) & 1u) << 1 ^ 2u;      // replace idx 63's parity by idx's
+                    } else {
+                        mb[7] = kHalfMagic + uint32_t(4 * idx) + b;
+                    }
+                }
+            }
+        }
+    }
+    store_fast<MODE, WAIT>(p, mb, ~par & 2u, g, c);
+}
+
+// General round: ragged rounds (PARTIAL: some lanes hold no group), raw low bits, and streams read from
+// global memory with bounds checks (Words = GlobalWords) or from the ring (RingWords).
+template <int MODE, bool PARTIAL, class Words>
+__device__ __forceinline__ void round_general_v2(const Params& p, uint32_t t0, const Words& words, const uint8_t* rawsec,
+                                              uint32_t raw_avail, TileState& st, uint32_t q, bool active, uint32_t g,
+                                              uint32_t lt_mask, float c) {
+    const bool on = !PARTIAL || active;
+    uint32_t win[3];
+    raw_window(rawsec, raw_avail, q, on ? p.r : 0, win);
+    uint32_t x = st.x, pb = st.pb;
+    uint32_t e[8];
+    uint32_t gbase = t0, B = t0 | kStartOffset;
+#pragma unroll
+    for (int pr = 0; pr < 4; ++pr) {
+#pragma unroll
+        for (int i = 2 * pr; i <= 2 * pr + 1; ++i) {
+            e[i] = 0;
+            if (on) {
+                const uint32_t qq = x >> 8;
+                e[i] = ld_shared_u32(B + ((x & 255u) << 2));
+                x = ((e[i] >> 16) & 0xFFu) * qq + (e[i] >> 24);
+            }
+            if (i == 0) gbase = t0 | (e[0] & kCosetBit);
+            B = (i == 6 ? (gbase | kPos7Bit) : gbase) | (e[i] & kClassBit);
+        }
+        const bool need = on && x < kRansL;
+        const uint32_t m = __ballot_sync(kFullMask, need);
+        const uint32_t w = words.at(pb + 2 * __popc(m & lt_mask));
+        x = __byte_perm(x, w, need ? 0x1054u : 0x3210u);
+        pb += 2 * __popc(m);
+    }
+    int32_t hesc[8];
+    uint32_t escm = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const bool esc = on && (e[i] & kEscBit);
+        const uint32_t me = __ballot_sync(kFullMask, esc);
+        hesc[i] = 0;
+        if (me) {
+            const uint32_t w = words.at(pb + 2 * __popc(me & lt_mask));
+            if (esc) hesc[i] = int32_t(int16_t(w));
+            pb += 2 * __popc(me);
+        }
+        escm |= esc ? 1u << i : 0u;
+    }
+    st.x = x;
+    st.pb = pb;
+    if (on) store_general<MODE>(p, e, hesc, escm, win, g, c);
+}
+
+static_assert(kTablesBytes + kScratchSize + kSlackBytes >= kOverrunBytes, "a corrupt stream could read past the allocation");
+
+// Rounds [0, Rf) of a tile from the ring, Rf <= kMaxFastRounds. A valid stream ends inside the ring; a corrupt
+// one may run past it, by at most 768 bytes a round, into the shared memory that follows (kSmemBytes keeps
+// kOverrunBytes after the last ring), and the tile check flags it. kr0: the round's column in its row, in
+// rounds, when rows hold whole rounds. If `waited` is false, the first round waits for the previous launch of a
+// sequence before its stores, and sets it. Returns the number of rounds done.
+template <int MODE, bool ESC>
+__device__ __forceinline__ uint32_t fast_rounds_v2(const Params& p, uint32_t t0, TileState& st, uint32_t ring_base,
+                                                   uint32_t g, uint32_t lt_mask, uint32_t Rf, uint32_t kr,
+                                                   const uint16_t* scales, RowCursor& rc, bool& waited) {
+    uint32_t k = 0, x = st.x, pa = ring_base + st.pb;
+    if (p.gpr % 32 == 0) {
+        // Rows hold whole rounds: every lane of a round is in the same row, and the row changes for all lanes
+        // at once, every gpr / 32 rounds.
+        const uint32_t rpr = p.gpr / 32;
+        float c = rc.scale();
+        if (!waited && Rf > 0) {
+            round_fast_v2<MODE, true, ESC>(p, t0, x, pa, g, lt_mask, c, p.k2);
+            waited = true;
+            k = 1;
+            g += 32;
+            if (++kr == rpr) {
+                kr = 0;
+                rc.row += 1;
+                rc.load_scale(p, scales);
+                c = rc.scale();
+            }
+        }
+        for (; k < Rf; ++k, g += 32) {
+            round_fast_v2<MODE, false, ESC>(p, t0, x, pa, g, lt_mask, c, p.k2);
+            if (++kr == rpr) {
+                kr = 0;
+                rc.row += 1;
+                rc.load_scale(p, scales);
+                c = rc.scale();
+            }
+        }
+    } else {
+        if (!waited && Rf > 0) {
+            round_fast_v2<MODE, true, ESC>(p, t0, x, pa, g, lt_mask, rc.scale(), p.k2);
+            rc.advance(p, scales);
+            waited = true;
+            k = 1;
+            g += 32;
+        }
+        for (; k < Rf; ++k, g += 32) {
+            round_fast_v2<MODE, false, ESC>(p, t0, x, pa, g, lt_mask, rc.scale(), p.k2);
+            rc.advance(p, scales);
+        }
+    }
+    st.x = x;
+    st.pb = pa - ring_base;
+    return k;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreadsV2, 1) decode_kernel(const Params p) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    const uint32_t raw_base = smem_addr(smem_raw);
+    const uint32_t ring_pad = (kRingBytes - (raw_base & (kRingBytes - 1))) & (kRingBytes - 1);
+    uint8_t* rings = smem_raw + ring_pad;
+    const uint32_t after_rings = raw_base + ring_pad + kRingsBytes;
+    const uint32_t tbl_pad = (kTableAlign - (after_rings & (kTableAlign - 1))) & (kTableAlign - 1);
+    uint8_t* tables = rings + kRingsBytes + tbl_pad;
+    uint8_t* scratch = tables + kTablesBytes;
+    const uint32_t t0 = smem_addr(tables);
+
+    const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const uint16_t* scales = reinterpret_cast<const uint16_t*>(p.blob + p.off_scales);
+    const uint32_t* toff = reinterpret_cast<const uint32_t*>(p.blob + p.off_offsets);
+    const uint8_t* payload = p.blob + p.off_payload;
+    const uint32_t per_tile = 32 * p.G;
+    const uint32_t ring_base = smem_addr(rings + warp * kRingBytes);
+
+    grid_dependents_launch();
+
+    if (p.next_blob) {
+        const uint32_t lines = (p.next_meta_bytes + 127) / 128;
+        for (uint32_t l = blockIdx.x + gridDim.x * threadIdx.x; l < lines; l += gridDim.x * kThreadsV2)
+            prefetch_l2(p.next_blob + p.next_meta_off + 128ull * l);
+    }
+
+    // The first tile's stream copies are issued before the table build, which hides them.
+    uint32_t slot = warp;
+    bool first_issued = false;
+    {
+        const uint32_t tile = slot * gridDim.x + blockIdx.x;
+        if (tile < p.T) {
+            TileGeom tg;
+            if (tile_geometry(p, toff, tile, per_tile, tg)) {
+                const uint32_t n = min(tg.chunks, kRingChunks);
+                for (uint32_t ch = 0; ch < n; ++ch) {
+                    const uint32_t off = ch * kChunkBytes + 16 * lane;
+                    const uint32_t nb = off < tg.span ? min(16u, tg.span - off) : 0u;
+                    cp_async16(ring_base + off, nb ? payload + tg.start + tg.a0 + off : payload, nb);
+                }
+                first_issued = true;
+            }
+        }
+        cp_async_commit();
+    }
+    build_tables_v2(p, tables, scratch);
+    bool waited = false;
+
+    // Every decision below is taken for the whole warp (a vote, or values of the tile index and the kernel
+    // parameters only), so that the compiler sees warp-uniform control flow in the round loops.
+    for (;; slot += kWarpsV2) {
+        const uint32_t tile = slot * gridDim.x + blockIdx.x;
+        if (tile >= p.T) break;
+        const uint32_t ng = min(per_tile, p.NG - tile * per_tile);
+        TileGeom tg;
+        if (!__all_sync(kFullMask, tile_geometry(p, toff, tile, per_tile, tg))) {
+            if (lane == 0) atomicOr(&g_status, int(EP_DEV_BAD_OFFSETS));
+            first_issued = false;
+            continue;
+        }
+        const uint8_t* tp = payload + tg.start;
+        TileState st;
+        st.x = __ldg(reinterpret_cast<const uint32_t*>(tp) + lane);
+        st.pb = tg.lead;
+        const GlobalWords gwords{tp + tg.a0, tg.lead, tg.span};
+        {
+            const uint32_t next = tile + kWarpsV2 * gridDim.x;
+            if (next < p.T) {
+                const uint64_t ns = uint64_t(__ldg(toff + next) & 0x7FFFFFFFu) * 16 + 128ull * lane;
+                if (ns < p.payload_bytes) prefetch_l2(payload + ns);
+            }
+        }
+        RowCursor rc;
+        rc.start(p, scales, tg.g0 + lane);
+        const uint8_t* rawsec = tp + 128;
+        const uint32_t raw_avail = tg.tile_bytes - 128;
+        const uint32_t R = (ng + 31) / 32;
+        const bool in_ring = __all_sync(kFullMask, tg.chunks <= kRingChunks);
+        if (!first_issued && in_ring) {
+            for (uint32_t ch = 0; ch < tg.chunks; ++ch) {
+                const uint32_t off = ch * kChunkBytes + 16 * lane;
+                const uint32_t nb = off < tg.span ? min(16u, tg.span - off) : 0u;
+                cp_async16(ring_base + off, nb ? tp + tg.a0 + off : tp, nb);
+            }
+            cp_async_commit();
+        }
+        first_issued = false;
+        cp_async_wait<0>();
+        __syncwarp();
+
+        uint32_t k = 0;
+        if (in_ring && p.r == 0) {
+            const uint32_t Rf = min(ng / 32, kMaxFastRounds);
+            const uint32_t kr0 = ((tile * per_tile) % p.gpr) / 32;
+            if (__any_sync(kFullMask, tg.esc))
+                k = fast_rounds_v2<MODE, true>(p, t0, st, ring_base, tg.g0 + lane, lt_mask, Rf, kr0, scales, rc, waited);
+            else
+                k = fast_rounds_v2<MODE, false>(p, t0, st, ring_base, tg.g0 + lane, lt_mask, Rf, kr0, scales, rc, waited);
+            if (k < R) rc.start(p, scales, tg.g0 + 32 * k + lane);
+        }
+        if (k < R) {
+            if (!waited) {
+                grid_dependency_wait();
+                waited = true;
+            }
+            const RingWords ring{ring_base};
+            for (; k < R; ++k) {
+                const uint32_t q = 32 * k + lane, g = tg.g0 + q;
+                const bool full = 32 * k + 32 <= ng;
+                if (in_ring && full && __all_sync(kFullMask, st.pb + 2 * kRoundWords <= kRingBytes)) {
+                    round_general_v2<MODE, false>(p, t0, ring, rawsec, raw_avail, st, q, true, g, lt_mask, rc.scale());
+                } else {
+                    round_general_v2<MODE, true>(p, t0, gwords, rawsec, raw_avail, st, q, q < ng, g, lt_mask,
+                                              rc.scale());
+                }
+                rc.advance(p, scales);
+            }
+        }
+        __syncwarp();
+        const uint32_t used = st.pb - tg.lead, cap = tg.span - tg.lead;
+        const bool ok = __all_sync(kFullMask, st.x == kRansL) && used <= cap && cap - used <= 14;
+        if (!ok && lane == 0) atomicOr(&g_status, int(EP_DEV_CORRUPT_TILE));
+    }
+    if (first_issued) cp_async_wait<0>();
+    if (!waited) grid_dependency_wait();
+}
+
+}  // namespace v2
+
+
 }  // namespace dev
 
 // ------------------------------------------------------------------------------- launcher
@@ -982,21 +1538,25 @@ namespace {
 
 struct DeviceInfo {
     int sms = 0;
-    bool configured[8] = {false};
+    bool configured[8] = {false};     // version 1 kernels, by mode
+    bool configured_v2[8] = {false};  // version 2 kernels, by mode
 };
 std::mutex g_dev_mu;
 DeviceInfo g_dev[64];
 
 template <int MODE>
-ep_status launch_mode(const dev::Params& p, cudaStream_t stream, int device, bool chained) {
+ep_status launch_mode(const dev::Params& p, cudaStream_t stream, int device, bool chained, int version) {
+    const void* fn = version == 1 ? reinterpret_cast<const void*>(dev::decode_kernel<MODE>)
+                                  : reinterpret_cast<const void*>(dev::v2::decode_kernel<MODE>);
+    const uint32_t smem = version == 1 ? dev::kSmemBytes : dev::v2::kSmemBytes;
     {
         std::lock_guard<std::mutex> lk(g_dev_mu);
         DeviceInfo& d = g_dev[device];
-        if (!d.configured[MODE]) {
-            cudaError_t e = cudaFuncSetAttribute(dev::decode_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 int(dev::kSmemBytes));
+        bool& configured = version == 1 ? d.configured[MODE] : d.configured_v2[MODE];
+        if (!configured) {
+            cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
             if (e != cudaSuccess) return fail(EP_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-            d.configured[MODE] = true;
+            configured = true;
         }
     }
     // One CTA per SM, or one per tile when there are fewer tiles than SMs.
@@ -1004,15 +1564,16 @@ ep_status launch_mode(const dev::Params& p, cudaStream_t stream, int device, boo
     if (grid == 0) grid = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(dev::kThreads);
-    cfg.dynamicSmemBytes = dev::kSmemBytes;
+    cfg.blockDim = dim3(version == 1 ? dev::kThreads : dev::v2::kThreadsV2);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = chained ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, dev::decode_kernel<MODE>, p);
+    cudaError_t e = version == 1 ? cudaLaunchKernelEx(&cfg, dev::decode_kernel<MODE>, p)
+                                 : cudaLaunchKernelEx(&cfg, dev::v2::decode_kernel<MODE>, p);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(EP_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
     return EP_OK;
@@ -1059,6 +1620,7 @@ ep_status launch_decode(const uint8_t* host_hdr, const void* dev_blob, size_t bl
     p.k4 = 4;
     p.kneg4096 = 0xFFFFF000u;
     p.k128 = 128;
+    p.kneg256 = 0xFFFFFF00u;
     p.off_scales = h.off_scales;
     p.off_tables = h.off_tables;
     p.off_offsets = h.off_offsets;
@@ -1076,13 +1638,14 @@ ep_status launch_decode(const uint8_t* host_hdr, const void* dev_blob, size_t bl
         p.next_meta_bytes = hn.off_payload - hn.off_scales;
     }
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    const int v = h.version;
     switch (mode) {
-        case dev::kBF16: return launch_mode<dev::kBF16>(p, stream, device, chained);
-        case dev::kFP16: return launch_mode<dev::kFP16>(p, stream, device, chained);
-        case dev::kFP32: return launch_mode<dev::kFP32>(p, stream, device, chained);
-        case dev::kFP8: return launch_mode<dev::kFP8>(p, stream, device, chained);
-        case dev::kINT8: return launch_mode<dev::kINT8>(p, stream, device, chained);
-        case dev::kCoords: return launch_mode<dev::kCoords>(p, stream, device, chained);
+        case dev::kBF16: return launch_mode<dev::kBF16>(p, stream, device, chained, v);
+        case dev::kFP16: return launch_mode<dev::kFP16>(p, stream, device, chained, v);
+        case dev::kFP32: return launch_mode<dev::kFP32>(p, stream, device, chained, v);
+        case dev::kFP8: return launch_mode<dev::kFP8>(p, stream, device, chained, v);
+        case dev::kINT8: return launch_mode<dev::kINT8>(p, stream, device, chained, v);
+        case dev::kCoords: return launch_mode<dev::kCoords>(p, stream, device, chained, v);
     }
     return fail(EP_ERR_DTYPE, "decode: unknown dtype %d", mode);
 }
@@ -1114,29 +1677,41 @@ extern "C" ep_status ep_decompress_many(int count, const uint8_t* const* host_hd
             return fail(EP_ERR_CORRUPT, "ep_decompress_many: blob %d has a malformed header", i);
         if (h.total != blob_bytes[i]) return fail(EP_ERR_BUFFER, "ep_decompress_many: blob %d size mismatch", i);
     }
-    // The fused entries of every blob, built once for the sequence into stream-ordered scratch (144 KB per
-    // blob). The first decode launches in plain stream order behind the expand kernel, and every later
-    // one starts after it, so all of them read finished tables. Without the scratch, each CTA builds
-    // its own tables.
+    // The fused entries of every version-1 blob, built once for the sequence into stream-ordered scratch
+    // (144 KB per blob). The first decode launches in plain stream order behind the expand kernel, and every
+    // later one starts after it, so all of them read finished tables. Without the scratch, each CTA builds
+    // its own tables. Version-2 tables (9 KB) are always built by each CTA: that takes about a microsecond.
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     constexpr size_t kWords = dev::kTablesBytes / 4;
+    std::vector<int> v1;  // indices of the version-1 blobs, in order; blob v1[j] takes prepared slot j
+    std::vector<int> slot_of(size_t(count), -1);
+    for (int i = 0; i < count; ++i) {
+        Header h;
+        parse_header(host_hdrs[i], h);
+        if (h.version == 1) {
+            slot_of[size_t(i)] = int(v1.size());
+            v1.push_back(i);
+        }
+    }
+    const int n1 = int(v1.size());
     uint32_t* pre = nullptr;
-    if (count >= 2) {
+    if (count >= 2 && n1 >= 1) {
         cudaMemPool_t pool;
         if (scratch_pool(&pool) != cudaSuccess ||
-            cudaMallocFromPoolAsync(reinterpret_cast<void**>(&pre), size_t(count) * dev::kTablesBytes, pool, stream) !=
+            cudaMallocFromPoolAsync(reinterpret_cast<void**>(&pre), size_t(n1) * dev::kTablesBytes, pool, stream) !=
                 cudaSuccess) {
             cudaGetLastError();
             pre = nullptr;
         }
-        for (int b = 0; pre && b < count; b += dev::kMaxExpandJobs) {
+        for (int b = 0; pre && b < n1; b += dev::kMaxExpandJobs) {
             dev::ExpandArgs a;
-            a.count = count - b < dev::kMaxExpandJobs ? count - b : dev::kMaxExpandJobs;
+            a.count = n1 - b < dev::kMaxExpandJobs ? n1 - b : dev::kMaxExpandJobs;
             a.out = pre + size_t(b) * kWords;
             for (int j = 0; j < a.count; ++j) {
                 Header h;
-                parse_header(host_hdrs[b + j], h);
-                a.tables[j] = static_cast<const uint8_t*>(dev_blobs[b + j]) + h.off_tables;
+                const int i = v1[size_t(b + j)];
+                parse_header(host_hdrs[i], h);
+                a.tables[j] = static_cast<const uint8_t*>(dev_blobs[i]) + h.off_tables;
                 a.tables_len[j] = h.off_offsets - h.off_tables;
             }
             dev::expand_tables_kernel<<<unsigned(a.count) * kNumCtx, 256, 0, stream>>>(a);
@@ -1153,10 +1728,11 @@ extern "C" ep_status ep_decompress_many(int count, const uint8_t* const* host_hd
     for (int i = 0; i < count; ++i) {
         Header h;
         parse_header(host_hdrs[i], h);
+        const int slot = slot_of[size_t(i)];
         ep_status st = launch_decode(host_hdrs[i], dev_blobs[i], blob_bytes[i], dsts[i], dst_bytes[i], h.dtype,
                                      cuda_stream, i > 0, i + 1 < count ? host_hdrs[i + 1] : nullptr,
-                                     i + 1 < count ? dev_blobs[i + 1] : nullptr, pre ? pre + size_t(i) * kWords : nullptr,
-                                     no_copy);
+                                     i + 1 < count ? dev_blobs[i + 1] : nullptr,
+                                     (pre && slot >= 0) ? pre + size_t(slot) * kWords : nullptr, no_copy);
         if (st != EP_OK) {
             if (pre) cudaFreeAsync(pre, stream);
             return st;

@@ -41,6 +41,9 @@ CASES = [
 ]
 
 
+VERSIONS = [2, 1]
+
+
 def both(ep, w, cfg_kwargs):
     host = ep.compress(w, ep.EntroPackLossyConfig(**cfg_kwargs))
     dev = ep.compress(w.cuda(), ep.EntroPackLossyConfig(encoder="cuda", **cfg_kwargs))
@@ -48,27 +51,32 @@ def both(ep, w, cfg_kwargs):
 
 
 def oracle_bytes(orc, w, target, blob):
-    """The oracle encoder's blob for the same input and target, at the tile size G the product chose."""
+    """The oracle encoder's blob for the same input and target, at the tile size G and format version the
+    product chose."""
     G = int.from_bytes(blob[20:22], "little")
-    ob, _ = orc.compress(synth.container_bits(w.cpu()), synth.dtype_code(w), target, G)
+    version = int.from_bytes(blob[4:6], "little")
+    ob, _ = orc.compress(synth.container_bits(w.cpu()), synth.dtype_code(w), target, G,
+                         prob_bits=12 if version == 1 else 8)
     return ob
 
 
+@pytest.mark.parametrize("version", VERSIONS)
 @pytest.mark.parametrize("name,maker,target,G", CASES, ids=[c[0] for c in CASES])
-def test_cuda_encoder_matches_oracle_and_host_bytes(ep, orc, name, maker, target, G):
+def test_cuda_encoder_matches_oracle_and_host_bytes(ep, orc, name, maker, target, G, version):
     w = maker()
-    host, dev = both(ep, w, dict(target_bpp=target, rounds_per_tile=G))
+    host, dev = both(ep, w, dict(target_bpp=target, rounds_per_tile=G, format_version=version))
     assert dev.blob == oracle_bytes(orc, w, target, dev.blob), "CUDA encoder differs from the oracle encoder"
     assert dev.blob == host.blob
     assert dev.actual_bpp == host.actual_bpp
 
 
+@pytest.mark.parametrize("version", VERSIONS)
 @pytest.mark.parametrize("workload", ["lognormal3072", "dit_q_3840"])
-def test_cuda_encoder_matches_oracle_full_size(ep, orc, workload):
+def test_cuda_encoder_matches_oracle_full_size(ep, orc, workload, version):
     """Full-size tensors against the oracle encoder directly: the 3072x3072 lognormal-rows matrix with
     outliers and one 3840x3840 layer of the DiT-like set, both at 4 bpp."""
     w = synth.lognormal_rows_with_outliers() if workload == "lognormal3072" else synth.dit_layer(0)
-    dev = ep.compress(w.cuda(), ep.EntroPackLossyConfig(4.0, encoder="cuda"))
+    dev = ep.compress(w.cuda(), ep.EntroPackLossyConfig(4.0, encoder="cuda", format_version=version))
     assert dev.blob == oracle_bytes(orc, w, 4.0, dev.blob)
 
 
@@ -112,8 +120,9 @@ def test_cuda_encoder_errors(ep):
     assert e.value.status == -1
 
 
+@pytest.mark.parametrize("version", VERSIONS)
 @pytest.mark.parametrize("seed", range(16))
-def test_cuda_encoder_matches_oracle_and_host_bytes_fuzz(ep, orc, seed):
+def test_cuda_encoder_matches_oracle_and_host_bytes_fuzz(ep, orc, seed, version):
     import random
     rnd = random.Random(2000 + seed)
     M, N = rnd.randint(1, 200), 8 * rnd.randint(1, 64)
@@ -124,7 +133,8 @@ def test_cuda_encoder_matches_oracle_and_host_bytes_fuzz(ep, orc, seed):
         w = synth.int8_codes(M, N, seed=seed)
     else:
         w = synth.gaussian(M, N, seed=seed, std=rnd.choice([0.02, 1.0, 300.0]), container=kind)
-    cfg = dict(target_bpp=round(rnd.uniform(0.3, 11.0), 3), rounds_per_tile=rnd.choice([0, 1, 3, 16, 33]))
+    cfg = dict(target_bpp=round(rnd.uniform(0.3, 11.0), 3), rounds_per_tile=rnd.choice([0, 1, 3, 16, 33]),
+               format_version=version)
     host, dev = both(ep, w, cfg)
     assert dev.blob == host.blob
     assert dev.blob == oracle_bytes(orc, w, cfg["target_bpp"], dev.blob)

@@ -113,26 +113,32 @@ EDGE = [
 ]
 
 
+VERSIONS = [2, 1]  # format version 2 (8-bit tables, the default) and version 1 (12-bit tables)
+
+
+@pytest.mark.parametrize("version", VERSIONS)
 @pytest.mark.parametrize("name,maker,target,G", EDGE, ids=[e[0] for e in EDGE])
-def test_parity_edge_cases(orc, name, maker, target, G):
-    c = ep.compress(maker(), ep.EntroPackLossyConfig(target, rounds_per_tile=G))
+def test_parity_edge_cases(orc, name, maker, target, G, version):
+    c = ep.compress(maker(), ep.EntroPackLossyConfig(target, rounds_per_tile=G, format_version=version))
     check_full(orc, c)
 
 
-def test_parity_r12_extremes(orc):
+@pytest.mark.parametrize("version", VERSIONS)
+def test_parity_r12_extremes(orc, version):
     g = torch.Generator().manual_seed(6)
     w = torch.randn(40, 8, generator=g)
-    c = ep.compress(w, ep.EntroPackLossyConfig(11.0, rounds_per_tile=1))
+    c = ep.compress(w, ep.EntroPackLossyConfig(11.0, rounds_per_tile=1, format_version=version))
     check_full(orc, c)
     # int16-range escapes at r = 0 come from the oracle encoder with a forced alpha
     w2 = torch.randn(64, 4096, generator=g) * 1e-3
     w2[:, 7] = 1.0
     w2[::2, 9] = -1.0
-    blob, _ = orc.compress(w2.numpy(), 3, 3.0, 16, 450.0)
+    blob, _ = orc.compress(w2.numpy(), 3, 3.0, 16, 450.0, prob_bits=12 if version == 1 else 8)
     check_full(orc, ep.CompressedTensor.from_blob(blob))
 
 
-def test_parity_random_fuzz(orc):
+@pytest.mark.parametrize("version", VERSIONS)
+def test_parity_random_fuzz(orc, version):
     rng = np.random.default_rng(2024)
     for it in range(30):
         M = int(rng.integers(1, 300)); N = 8 * int(rng.integers(1, 80))
@@ -140,41 +146,45 @@ def test_parity_random_fuzz(orc):
         w = synth.gaussian(M, N, seed=1000 + it, container=cont, std=float(rng.uniform(0.001, 3)))
         target = float(rng.uniform(0.3, 11.0))
         G = int(rng.choice([1, 2, 3, 16, 40]))
-        check_full(orc, ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G)))
+        check_full(orc, ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G, format_version=version)))
 
 
 # ------------------------------------------------------------------ full-size workloads
 
-def test_parity_quickstart_256(orc):
-    c = ep.compress(synth.quickstart_256(), 3.5)
+@pytest.mark.parametrize("version", VERSIONS)
+def test_parity_quickstart_256(orc, version):
+    c = ep.compress(synth.quickstart_256(), ep.EntroPackLossyConfig(3.5, format_version=version))
     assert abs(c.actual_bpp - 3.5) <= 0.05
     out = ep.decompress(c)
     assert out.shape == (256, 256) and out.dtype == torch.bfloat16
     check_full(orc, c)
 
 
-def test_parity_3072_lognormal_outliers(orc):
-    c = ep.compress(synth.lognormal_rows_with_outliers(), 4.0)
+@pytest.mark.parametrize("version", VERSIONS)
+def test_parity_3072_lognormal_outliers(orc, version):
+    c = ep.compress(synth.lognormal_rows_with_outliers(), ep.EntroPackLossyConfig(4.0, format_version=version))
     assert c.actual_bpp <= 4.05
     check_every_tile(orc, c)
 
 
+@pytest.mark.parametrize("version", VERSIONS)
 @pytest.mark.parametrize("i", [0, 4, 6, 7, 272, 273, 274])
-def test_parity_dit_layer_shapes(orc, i):
+def test_parity_dit_layer_shapes(orc, i, version):
     """One layer of every distinct shape of the 276-layer DiT-like set, at 4 bpp."""
     w = synth.dit_layer(i)
-    c = ep.compress(w, 4.0)
+    c = ep.compress(w, ep.EntroPackLossyConfig(4.0, format_version=version))
     assert c.actual_bpp <= 4.05
     check_every_tile(orc, c)
 
 
-def test_parity_bitrate_sweep_4096(orc):
+@pytest.mark.parametrize("version", VERSIONS)
+def test_parity_bitrate_sweep_4096(orc, version):
     base = synth.gaussian(4096, 4096, seed=2, container="fp32")
     for cont in ("bf16", "fp16", "fp32"):
         w = base.to(synth.CONTAINERS[cont])
         prev = None
         for target in (0.5, 1.0, 2.3, 3.0, 5.0, 6.0, 8.0, 11.0):
-            c = ep.compress(w, target)
+            c = ep.compress(w, ep.EntroPackLossyConfig(target, format_version=version))
             assert abs(c.actual_bpp - target) <= 0.05
             check_every_tile(orc, c)
             y = ep.decompress(c).float()
@@ -184,21 +194,23 @@ def test_parity_bitrate_sweep_4096(orc):
             prev = err
 
 
+@pytest.mark.parametrize("version", VERSIONS)
 @pytest.mark.parametrize("kind", ["fp8", "int8"])
-def test_parity_llm_prefill_containers(orc, kind):
+def test_parity_llm_prefill_containers(orc, kind, version):
     if kind == "fp8":
         w, target = synth.fp8_codes(), 5.0
     else:
         w, target = synth.int8_codes(), 3.0
-    c = ep.compress(w, target)
+    c = ep.compress(w, ep.EntroPackLossyConfig(target, format_version=version))
     assert abs(c.actual_bpp - target) <= 0.05
     check_every_tile(orc, c)
 
 
 # -------------------------------------------------------------------- faults, made on the host
 
-def test_corrupt_payload_sets_status_not_fault(orc):
-    c = ep.compress(synth.gaussian(512, 512, seed=3, container="bf16"), 4.0)
+@pytest.mark.parametrize("version", VERSIONS)
+def test_corrupt_payload_sets_status_not_fault(orc, version):
+    c = ep.compress(synth.gaussian(512, 512, seed=3, container="bf16"), ep.EntroPackLossyConfig(4.0, format_version=version))
     off_payload = int.from_bytes(c.blob[40:44], "little")
     rng = np.random.default_rng(1)
     hits = 0
@@ -216,8 +228,9 @@ def test_corrupt_payload_sets_status_not_fault(orc):
     check_full(orc, c)
 
 
-def test_corrupt_offsets_and_tables_flags(orc):
-    c = ep.compress(synth.gaussian(512, 512, seed=4, container="bf16"), 4.0)
+@pytest.mark.parametrize("version", VERSIONS)
+def test_corrupt_offsets_and_tables_flags(orc, version):
+    c = ep.compress(synth.gaussian(512, 512, seed=4, container="bf16"), ep.EntroPackLossyConfig(4.0, format_version=version))
     hdr = c.blob[:64]
     off_tables = int.from_bytes(hdr[32:36], "little")
     off_offsets = int.from_bytes(hdr[36:40], "little")
@@ -273,6 +286,9 @@ def test_decompress_many_matches_single_decodes(orc):
              for i, shp in enumerate([(384, 256), (1024, 512), (64, 3840), (3840, 64), (1536, 256)])]
     comps.append(ep.compress(synth.fp8_codes(256, 512, seed=5), 5.0))
     comps.append(ep.compress(synth.gaussian(300, 200, seed=6, container="fp32"), 7.0))
+    # version-1 blobs in the same sequence: their tables are prepared once, the others' built per CTA
+    comps.append(ep.compress(synth.dit_layer(12, shape=(512, 512)), ep.EntroPackLossyConfig(4.0, format_version=1)))
+    comps.append(ep.compress(synth.gaussian(96, 512, seed=7, container="bf16"), ep.EntroPackLossyConfig(6.0, format_version=1)))
     outs = [torch.empty(c.shape, dtype=c.dtype, device="cuda") for c in comps]
     batch = ep.LayerBatch(list(zip(comps, outs)))
     for _ in range(3):
@@ -324,7 +340,9 @@ def test_planned_mixed_bitrate_sequence(orc):
 def test_table_copy_wait_runs_out_into_status(orc, monkeypatch):
     """The bounded wait for a sequence's table copies: with the copies left unissued (test hook), every
     CTA gives up, sets EP_DEV_TABLE_COPY and decodes nothing; the context stays usable."""
-    comps = [ep.compress(synth.gaussian(64, 256, seed=s, container="bf16"), 4.0) for s in (21, 22)]
+    # The prepared-table copies serve version-1 blobs (version-2 tables are built in each CTA).
+    comps = [ep.compress(synth.gaussian(64, 256, seed=s, container="bf16"), ep.EntroPackLossyConfig(4.0, format_version=1))
+             for s in (21, 22)]
     outs = [torch.zeros(c.shape, dtype=c.dtype, device="cuda") for c in comps]
     status_clean()
     monkeypatch.setenv("EPK_TEST_TABLE_COPY_TIMEOUT", "1")
@@ -354,7 +372,8 @@ def test_decompress_many_edge_counts(orc):
     for i in range(530):
         M, N = 1 + (i * 7) % 23, 8 * (1 + (i * 5) % 9)
         kind = ("bf16", "fp16", "fp32")[i % 3]
-        comps.append(ep.compress(synth.gaussian(M, N, seed=1000 + i, container=kind), 1.0 + (i % 9)))
+        comps.append(ep.compress(synth.gaussian(M, N, seed=1000 + i, container=kind),
+                                 ep.EntroPackLossyConfig(1.0 + (i % 9), format_version=1 + i % 2)))
     outs = [torch.empty(c.shape, dtype=c.dtype, device="cuda") for c in comps]
     ep.decompress_many(list(zip(comps, outs)))
     torch.cuda.synchronize()
