@@ -395,12 +395,15 @@ struct RowCursor {
     // s - alpha * q0 (Markstein). This matches IEEE division for every bf16 s >= 2^-96 with a quotient
     // in [2^-96, 2^96] (checked exhaustively over all such s for thousands of alphas). Anything else,
     // zero rows included, takes the IEEE division.
-    __device__ __forceinline__ void load_scale(const Params& p, const uint16_t* scales) {
-        if (row >= p.M) return;  // lanes past the last group
-        const float s = __uint_as_float(uint32_t(__ldg(scales + row)) << 16);
+    static __device__ __forceinline__ float scale_of(const Params& p, const uint16_t* scales, uint32_t r) {
+        const float s = __uint_as_float(uint32_t(__ldg(scales + r)) << 16);
         const float q0 = __fmul_rn(s, p.inv_alpha);
         const float q = __fmaf_rn(__fmaf_rn(-p.alpha, q0, s), p.inv_alpha, q0);
-        c_row = (s >= 0x1p-96f && q >= 0x1p-96f && q <= 0x1p96f) ? q : __fdiv_rn(s, p.alpha);
+        return (s >= 0x1p-96f && q >= 0x1p-96f && q <= 0x1p96f) ? q : __fdiv_rn(s, p.alpha);
+    }
+    __device__ __forceinline__ void load_scale(const Params& p, const uint16_t* scales) {
+        if (row >= p.M) return;  // lanes past the last group
+        c_row = scale_of(p, scales, row);
     }
     __device__ __forceinline__ void start(const Params& p, const uint16_t* scales, uint32_t g) {
         row = g / p.gpr;
@@ -1003,11 +1006,11 @@ __host__ __device__ constexpr uint32_t block_of(int c) { return c == 0 ? kStartO
 constexpr int kWarpsV2 = 32;
 constexpr int kThreadsV2 = kWarpsV2 * 32;
 
-// Per-warp stream rings: 4 KB, enough for the whole word stream of a tile up to about 7 bits per
-// coordinate at 16 rounds; longer streams are read from global memory by the general rounds.
-constexpr uint32_t kRingBytes = 4096;
-constexpr uint32_t kChunkBytes = 512;
-constexpr uint32_t kRingChunks = kRingBytes / kChunkBytes;
+// Per-warp tile buffers: 5 KB. A tile is copied whole (states, raw bits, word stream) into its warp's buffer,
+// at the bottom or the top. While a warp decodes one tile, the copy of its next tile lands at the other end
+// when the two fit together (about 4.4 KB at 4 bits per coordinate), so the next tile's data is there when
+// the warp gets to it. Tiles larger than the buffer are read from global memory by the general rounds.
+constexpr uint32_t kRingBytes = 5 * 1024;
 constexpr uint32_t kRingsBytes = kWarpsV2 * kRingBytes;
 // Scratch of the table build: f and cum per context and symbol (u16), and the staged table bytes.
 constexpr uint32_t kScratchF = 0;                               // u16 [9][128]
@@ -1015,9 +1018,9 @@ constexpr uint32_t kScratchCum = kScratchF + kNumCtx * 128 * 2; // u16 [9][129]
 constexpr uint32_t kScratchBytesOff = (kScratchCum + kNumCtx * 129 * 2 + 15) & ~15u;
 constexpr uint32_t kScratchTableCap = 1024;                     // a valid blob's tables take 658 bytes at most
 constexpr uint32_t kScratchSize = kScratchBytesOff + kScratchTableCap;
-// [pad to 4 KB][rings][pad to 16 KB][tables][scratch][slack]. At least kOverrunBytes follow the last ring.
+// [pad to 16 B][rings][pad to 16 KB][tables][scratch][slack]. At least kOverrunBytes follow the last ring.
 constexpr uint32_t kSlackBytes = 6 * 1024;
-constexpr uint32_t kSmemBytes = kRingBytes + kRingsBytes + kTableAlign + kTablesBytes + kScratchSize + kSlackBytes;
+constexpr uint32_t kSmemBytes = 16 + kRingsBytes + kTableAlign + kTablesBytes + kScratchSize + kSlackBytes;
 static_assert(kSmemBytes <= 227 * 1024, "exceeds the per-block shared memory of sm_100");
 // Words one round can take: one refill per pair and lane, plus one escape word per coordinate.
 constexpr uint32_t kRoundWords = 4 * 32 + 8 * 32;
@@ -1053,13 +1056,20 @@ __device__ __forceinline__ uint32_t entry_template_v2(int c, int sym, uint32_t f
 // Builds the 9 x 256 fused entries of the blob's tables in shared memory. Pass 1: one warp per context
 // reads its 8-bit frequencies (4 symbols a lane) and prefix-sums them into cum, checking that a used
 // context sums to 256. Pass 2: each thread fills slots, finding the symbol that owns each by binary search.
-__device__ void build_tables_v2(const Params& p, uint8_t* tables, uint8_t* scratch) {
+// Byte `threadIdx.x` of the serialised tables (zero past their end): loaded first thing in the kernel, so
+// that it does not queue behind the tiles' copies.
+__device__ __forceinline__ uint32_t table_byte(const Params& p) {
+    const uint32_t tlen = p.tables_len < kScratchTableCap ? p.tables_len : kScratchTableCap;
+    return threadIdx.x < tlen ? uint32_t(__ldg(p.blob + p.off_tables + threadIdx.x)) : 0u;
+}
+
+__device__ void build_tables_v2(const Params& p, uint8_t* tables, uint8_t* scratch, uint32_t tbyte) {
     uint16_t* F = reinterpret_cast<uint16_t*>(scratch + kScratchF);
     uint16_t* cum = reinterpret_cast<uint16_t*>(scratch + kScratchCum);
     uint8_t* tb = scratch + kScratchBytesOff;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const uint32_t tlen = p.tables_len < kScratchTableCap ? p.tables_len : kScratchTableCap;
-    for (uint32_t i = tid; i < kScratchTableCap; i += kThreadsV2) tb[i] = i < tlen ? __ldg(p.blob + p.off_tables + i) : 0;
+    static_assert(kScratchTableCap == kThreadsV2, "one table byte per thread");
+    tb[tid] = uint8_t(tbyte);
     __syncthreads();
     if (warp < kNumCtx) {
         const int c = warp, A = c == 0 ? 128 : 64;
@@ -1346,38 +1356,38 @@ static_assert(kTablesBytes + kScratchSize + kSlackBytes >= kOverrunBytes, "a cor
 
 // Rounds [0, Rf) of a tile from the ring, Rf <= kMaxFastRounds. A valid stream ends inside the ring; a corrupt
 // one may run past it, by at most 768 bytes a round, into the shared memory that follows (kSmemBytes keeps
-// kOverrunBytes after the last ring), and the tile check flags it. kr0: the round's column in its row, in
-// rounds, when rows hold whole rounds. If `waited` is false, the first round waits for the previous launch of a
-// sequence before its stores, and sets it. Returns the number of rounds done.
-template <int MODE, bool ESC>
+// kOverrunBytes after the last ring), and the tile check flags it. If `waited` is false, the first round waits
+// for the previous launch of a sequence before its stores, and sets it. Returns the number of rounds done.
+//
+// UNIFORM: rows hold whole rounds (gpr % 32 == 0), so every lane of a round is in the same row and the row
+// changes for all lanes at once, every gpr / 32 rounds. The tile spans at most kMaxFastRounds rows from row0:
+// lane i computes the factor of row row0 + i once, and each round takes its row's factor by a shuffle, with
+// no load on the round's path. kr: the first round's column in its row, in rounds. Otherwise the lanes'
+// rows move on their own (RowCursor).
+template <int MODE, bool ESC, bool UNIFORM>
 __device__ __forceinline__ uint32_t fast_rounds_v2(const Params& p, uint32_t t0, TileState& st, uint32_t ring_base,
-                                                   uint32_t g, uint32_t lt_mask, uint32_t Rf, uint32_t kr,
+                                                   uint32_t g, uint32_t lt_mask, uint32_t Rf, uint32_t row0, uint32_t kr,
                                                    const uint16_t* scales, RowCursor& rc, bool& waited) {
     uint32_t k = 0, x = st.x, pa = ring_base + st.pb;
-    if (p.gpr % 32 == 0) {
-        // Rows hold whole rounds: every lane of a round is in the same row, and the row changes for all lanes
-        // at once, every gpr / 32 rounds.
-        const uint32_t rpr = p.gpr / 32;
-        float c = rc.scale();
+    if constexpr (UNIFORM) {
+        const uint32_t rpr = p.gpr / 32, lane = threadIdx.x & 31;
+        const float cvec = row0 + lane < p.M ? RowCursor::scale_of(p, scales, row0 + lane) : 0.f;
+        uint32_t ri = 0;
         if (!waited && Rf > 0) {
-            round_fast_v2<MODE, true, ESC>(p, t0, x, pa, g, lt_mask, c, p.k2);
+            round_fast_v2<MODE, true, ESC>(p, t0, x, pa, g, lt_mask, __shfl_sync(kFullMask, cvec, 0), p.k2);
             waited = true;
             k = 1;
             g += 32;
             if (++kr == rpr) {
                 kr = 0;
-                rc.row += 1;
-                rc.load_scale(p, scales);
-                c = rc.scale();
+                ++ri;
             }
         }
         for (; k < Rf; ++k, g += 32) {
-            round_fast_v2<MODE, false, ESC>(p, t0, x, pa, g, lt_mask, c, p.k2);
+            round_fast_v2<MODE, false, ESC>(p, t0, x, pa, g, lt_mask, __shfl_sync(kFullMask, cvec, ri), p.k2);
             if (++kr == rpr) {
                 kr = 0;
-                rc.row += 1;
-                rc.load_scale(p, scales);
-                c = rc.scale();
+                ++ri;
             }
         }
     } else {
@@ -1398,13 +1408,35 @@ __device__ __forceinline__ uint32_t fast_rounds_v2(const Params& p, uint32_t t0,
     return k;
 }
 
+// Offset entries of a tile (start / 16 with the escape flag, end / 16), or zeros past the last tile.
+struct TileOffs {
+    uint32_t e0, e1;
+};
+__device__ __forceinline__ TileOffs load_offs(const Params& p, const uint32_t* toff, uint32_t tile) {
+    TileOffs o{0u, 0u};
+    if (tile < p.T) {
+        o.e0 = __ldg(toff + tile);
+        o.e1 = __ldg(toff + tile + 1);
+    }
+    return o;
+}
+// Byte size of a tile whose offsets are sane (start <= end <= payload, at least its 128 bytes of states), else 0.
+__device__ __forceinline__ uint32_t tile_size(const Params& p, const TileOffs& o) {
+    const uint64_t start = uint64_t(o.e0 & 0x7FFFFFFFu) * 16, end = uint64_t(o.e1 & 0x7FFFFFFFu) * 16;
+    return (end >= start + 128 && end <= p.payload_bytes && end - start <= 0x7FFFFFF0ull) ? uint32_t(end - start) : 0u;
+}
+// Copies a whole tile (sz bytes, a multiple of 16) from global memory to shared address dst: 16 bytes a lane.
+__device__ __forceinline__ void copy_tile(uint32_t dst, const uint8_t* src, uint32_t sz, uint32_t lane) {
+    for (uint32_t o = 16 * lane; o < sz; o += 512) cp_async16(dst + o, src + o, 16);
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreadsV2, 1) decode_kernel(const Params p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
+    const uint32_t tbyte = table_byte(p);
     const uint32_t raw_base = smem_addr(smem_raw);
-    const uint32_t ring_pad = (kRingBytes - (raw_base & (kRingBytes - 1))) & (kRingBytes - 1);
-    uint8_t* rings = smem_raw + ring_pad;
-    const uint32_t after_rings = raw_base + ring_pad + kRingsBytes;
+    uint8_t* rings = smem_raw;
+    const uint32_t after_rings = raw_base + kRingsBytes;
     const uint32_t tbl_pad = (kTableAlign - (after_rings & (kTableAlign - 1))) & (kTableAlign - 1);
     uint8_t* tables = rings + kRingsBytes + tbl_pad;
     uint8_t* scratch = tables + kTablesBytes;
@@ -1417,6 +1449,7 @@ __global__ void __launch_bounds__(kThreadsV2, 1) decode_kernel(const Params p) {
     const uint8_t* payload = p.blob + p.off_payload;
     const uint32_t per_tile = 32 * p.G;
     const uint32_t ring_base = smem_addr(rings + warp * kRingBytes);
+    const uint32_t stride = kWarpsV2 * gridDim.x;  // tiles are dealt round-robin over the CTAs first
 
     grid_dependents_launch();
 
@@ -1426,104 +1459,116 @@ __global__ void __launch_bounds__(kThreadsV2, 1) decode_kernel(const Params p) {
             prefetch_l2(p.next_blob + p.next_meta_off + 128ull * l);
     }
 
-    // The first tile's stream copies are issued before the table build, which hides them.
-    uint32_t slot = warp;
-    bool first_issued = false;
+    // The first tile's copy is issued before the table build, which hides it. `pending`: whether a copy group
+    // is committed and not yet waited for.
+    uint32_t tile = warp * gridDim.x + blockIdx.x;
+    TileOffs cur = load_offs(p, toff, tile), nxt = load_offs(p, toff, tile + stride);
+    uint32_t place = 0;  // where the current tile sits in the warp's buffer
+    uint32_t pending = 0;
     {
-        const uint32_t tile = slot * gridDim.x + blockIdx.x;
-        if (tile < p.T) {
-            TileGeom tg;
-            if (tile_geometry(p, toff, tile, per_tile, tg)) {
-                const uint32_t n = min(tg.chunks, kRingChunks);
-                for (uint32_t ch = 0; ch < n; ++ch) {
-                    const uint32_t off = ch * kChunkBytes + 16 * lane;
-                    const uint32_t nb = off < tg.span ? min(16u, tg.span - off) : 0u;
-                    cp_async16(ring_base + off, nb ? payload + tg.start + tg.a0 + off : payload, nb);
-                }
-                first_issued = true;
-            }
+        const uint32_t sz = tile_size(p, cur);
+        if (tile < p.T && sz && sz <= kRingBytes) {
+            copy_tile(ring_base, payload + uint64_t(cur.e0 & 0x7FFFFFFFu) * 16, sz, lane);
+            cp_async_commit();
+            pending = 1;
         }
-        cp_async_commit();
     }
-    build_tables_v2(p, tables, scratch);
+    build_tables_v2(p, tables, scratch, tbyte);
     bool waited = false;
 
     // Every decision below is taken for the whole warp (a vote, or values of the tile index and the kernel
     // parameters only), so that the compiler sees warp-uniform control flow in the round loops.
-    for (;; slot += kWarpsV2) {
-        const uint32_t tile = slot * gridDim.x + blockIdx.x;
-        if (tile >= p.T) break;
+    for (; tile < p.T; tile += stride) {
         const uint32_t ng = min(per_tile, p.NG - tile * per_tile);
-        TileGeom tg;
-        if (!__all_sync(kFullMask, tile_geometry(p, toff, tile, per_tile, tg))) {
-            if (lane == 0) atomicOr(&g_status, int(EP_DEV_BAD_OFFSETS));
-            first_issued = false;
-            continue;
-        }
-        const uint8_t* tp = payload + tg.start;
-        TileState st;
-        st.x = __ldg(reinterpret_cast<const uint32_t*>(tp) + lane);
-        st.pb = tg.lead;
-        const GlobalWords gwords{tp + tg.a0, tg.lead, tg.span};
-        {
-            const uint32_t next = tile + kWarpsV2 * gridDim.x;
-            if (next < p.T) {
-                const uint64_t ns = uint64_t(__ldg(toff + next) & 0x7FFFFFFFu) * 16 + 128ull * lane;
-                if (ns < p.payload_bytes) prefetch_l2(payload + ns);
-            }
-        }
-        RowCursor rc;
-        rc.start(p, scales, tg.g0 + lane);
-        const uint8_t* rawsec = tp + 128;
-        const uint32_t raw_avail = tg.tile_bytes - 128;
-        const uint32_t R = (ng + 31) / 32;
-        const bool in_ring = __all_sync(kFullMask, tg.chunks <= kRingChunks);
-        if (!first_issued && in_ring) {
-            for (uint32_t ch = 0; ch < tg.chunks; ++ch) {
-                const uint32_t off = ch * kChunkBytes + 16 * lane;
-                const uint32_t nb = off < tg.span ? min(16u, tg.span - off) : 0u;
-                cp_async16(ring_base + off, nb ? tp + tg.a0 + off : tp, nb);
-            }
-            cp_async_commit();
-        }
-        first_issued = false;
+        const uint32_t raw = (ng * uint32_t(p.r) + 3u) & ~3u, s0 = 128 + raw;
+        const uint32_t sz = __shfl_sync(kFullMask, tile_size(p, cur), 0);
+        const bool ok = sz >= s0;
+        const bool in_ring = ok && sz <= kRingBytes;
+        // The next tile's copy goes to the other end of the buffer now, if both fit.
+        const uint32_t ntile = tile + stride;
+        const uint32_t nsz = __shfl_sync(kFullMask, tile_size(p, nxt), 0);
+        const bool early = ntile < p.T && nsz && (in_ring ? sz + nsz <= kRingBytes : nsz <= kRingBytes);
+        const uint32_t nplace = early && in_ring && place == 0 ? kRingBytes - nsz : 0u;
+        const TileOffs after = load_offs(p, toff, ntile + stride);
+        // Wait for this tile's copy (if any), then start the next tile's: it lands while this one decodes.
         cp_async_wait<0>();
         __syncwarp();
+        pending = 0;
+        if (early) {
+            copy_tile(ring_base + nplace, payload + uint64_t(nxt.e0 & 0x7FFFFFFFu) * 16, nsz, lane);
+            cp_async_commit();
+            pending = 1;
+        }
+        if (!ok) {
+            if (lane == 0) atomicOr(&g_status, int(EP_DEV_BAD_OFFSETS));
+        } else {
+            const uint32_t rb = ring_base + place;
+            const uint8_t* tp = payload + uint64_t(cur.e0 & 0x7FFFFFFFu) * 16;
+            TileState st;
+            st.x = in_ring ? ld_shared_u32(rb + 4 * lane) : __ldg(reinterpret_cast<const uint32_t*>(tp) + lane);
+            st.pb = s0;
+            const GlobalWords gwords{tp, s0, sz};
+            if (!early && ntile < p.T) {  // the next tile's copy comes after this one: pull it toward L2
+                const uint64_t ns = uint64_t(nxt.e0 & 0x7FFFFFFFu) * 16 + 128ull * lane;
+                if (ns < p.payload_bytes) prefetch_l2(payload + ns);
+            }
+            RowCursor rc;
+            const uint8_t* rawsec = tp + 128;
+            const uint32_t raw_avail = sz - 128;
+            const uint32_t R = (ng + 31) / 32;
+            const uint32_t gt0 = tile * per_tile;
 
-        uint32_t k = 0;
-        if (in_ring && p.r == 0) {
-            const uint32_t Rf = min(ng / 32, kMaxFastRounds);
-            const uint32_t kr0 = ((tile * per_tile) % p.gpr) / 32;
-            if (__any_sync(kFullMask, tg.esc))
-                k = fast_rounds_v2<MODE, true>(p, t0, st, ring_base, tg.g0 + lane, lt_mask, Rf, kr0, scales, rc, waited);
-            else
-                k = fast_rounds_v2<MODE, false>(p, t0, st, ring_base, tg.g0 + lane, lt_mask, Rf, kr0, scales, rc, waited);
-            if (k < R) rc.start(p, scales, tg.g0 + 32 * k + lane);
-        }
-        if (k < R) {
-            if (!waited) {
-                grid_dependency_wait();
-                waited = true;
-            }
-            const RingWords ring{ring_base};
-            for (; k < R; ++k) {
-                const uint32_t q = 32 * k + lane, g = tg.g0 + q;
-                const bool full = 32 * k + 32 <= ng;
-                if (in_ring && full && __all_sync(kFullMask, st.pb + 2 * kRoundWords <= kRingBytes)) {
-                    round_general_v2<MODE, false>(p, t0, ring, rawsec, raw_avail, st, q, true, g, lt_mask, rc.scale());
+            uint32_t k = 0;
+            if (in_ring && p.r == 0) {
+                const uint32_t Rf = min(ng / 32, kMaxFastRounds);
+                const uint32_t row0 = gt0 / p.gpr, kr0 = (gt0 - row0 * p.gpr) / 32;
+                const bool esc = __any_sync(kFullMask, cur.e0 >> 31);
+                if (p.gpr % 32 == 0) {
+                    k = esc ? fast_rounds_v2<MODE, true, true>(p, t0, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited)
+                            : fast_rounds_v2<MODE, false, true>(p, t0, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited);
                 } else {
-                    round_general_v2<MODE, true>(p, t0, gwords, rawsec, raw_avail, st, q, q < ng, g, lt_mask,
-                                              rc.scale());
+                    rc.start(p, scales, gt0 + lane);
+                    k = esc ? fast_rounds_v2<MODE, true, false>(p, t0, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited)
+                            : fast_rounds_v2<MODE, false, false>(p, t0, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited);
                 }
-                rc.advance(p, scales);
             }
+            if (k < R) {
+                rc.start(p, scales, gt0 + 32 * k + lane);
+                if (!waited) {
+                    grid_dependency_wait();
+                    waited = true;
+                }
+                const RingWords ring{rb};
+                for (; k < R; ++k) {
+                    const uint32_t q = 32 * k + lane, g = gt0 + q;
+                    const bool full = 32 * k + 32 <= ng;
+                    // Ring reads of a round stay within the tile's own bytes (a round takes at most 768).
+                    if (in_ring && full && __all_sync(kFullMask, st.pb + 2 * kRoundWords <= sz)) {
+                        round_general_v2<MODE, false>(p, t0, ring, rawsec, raw_avail, st, q, true, g, lt_mask, rc.scale());
+                    } else {
+                        round_general_v2<MODE, true>(p, t0, gwords, rawsec, raw_avail, st, q, q < ng, g, lt_mask,
+                                                      rc.scale());
+                    }
+                    rc.advance(p, scales);
+                }
+            }
+            __syncwarp();
+            const uint32_t used = st.pb - s0, cap = sz - s0;  // bytes of stream read / present
+            const bool good = __all_sync(kFullMask, st.x == kRansL) && used <= cap && cap - used <= 14;
+            if (!good && lane == 0) atomicOr(&g_status, int(EP_DEV_CORRUPT_TILE));
         }
-        __syncwarp();
-        const uint32_t used = st.pb - tg.lead, cap = tg.span - tg.lead;
-        const bool ok = __all_sync(kFullMask, st.x == kRansL) && used <= cap && cap - used <= 14;
-        if (!ok && lane == 0) atomicOr(&g_status, int(EP_DEV_CORRUPT_TILE));
+        // The buffer is free now: a next tile that did not fit beside this one is copied to the bottom.
+        if (!early && ntile < p.T && nsz && nsz <= kRingBytes) {
+            __syncwarp();
+            copy_tile(ring_base, payload + uint64_t(nxt.e0 & 0x7FFFFFFFu) * 16, nsz, lane);
+            cp_async_commit();
+            pending = 1;
+        }
+        place = early ? nplace : 0u;
+        cur = nxt;
+        nxt = after;
     }
-    if (first_issued) cp_async_wait<0>();
+    if (pending) cp_async_wait<0>();
     if (!waited) grid_dependency_wait();
 }
 
