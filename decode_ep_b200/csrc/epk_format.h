@@ -24,7 +24,7 @@ constexpr uint32_t kProbScale = 1u << kProbBits;  // 4096
 // hi in [-2, 2]), and a round's escape words follow its last pair.
 constexpr int kProbBitsV2 = 8;
 constexpr uint32_t kProbScaleV2 = 1u << kProbBitsV2;  // 256
-constexpr int kEscShift = 12;
+constexpr int kEscShift = 14;
 constexpr uint32_t kRansL = 1u << 16;             // state lower bound; 16-bit refills
 constexpr int kEscIdx = 63;
 constexpr int kMaxG = 1024;

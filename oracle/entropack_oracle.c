@@ -44,7 +44,7 @@ enum { OK = 0, E_ARG = -1, E_DTYPE = -2, E_SHAPE = -3, E_TARGET = -4, E_NONFINIT
 #define HEADER_BYTES 64
 /* Version 2: a symbol (other than hi in [-2, 2]) seen in fewer than 1/2^ESC_SHIFT of its
  * context's coordinates is sent as an escape. */
-#define ESC_SHIFT 12
+#define ESC_SHIFT 14
 
 /* ---------------------------------------------------------------- helpers */
 
