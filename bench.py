@@ -631,70 +631,64 @@ def oracle_rate(blob, shape, seconds, workers):
     return done / (time.perf_counter() - t0)
 
 
-def to_e4m3_rows(w):
-    """FP8 e4m3 weight codes of w: each row scaled so its largest magnitude is 448, then cast."""
-    f = w.float()
-    f = f * (448.0 / f.abs().amax(dim=1, keepdim=True).clamp_min(1e-30))
-    return f.clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
-
-
 def run_gemm_overhead(args, tokens=4096, fp8=False):
-    """Decode overhead against the layer GEMMs of a prefill-sized forward pass (the pages measure it as
-    the denoising-step time with compressed vs BF16 weights; that needs the real model, so this times
-    the proxy: the 276 layer GEMMs y = x W^T on `tokens` synthetic activations, in layer order).
-      gemm:      BF16 weights resident, GEMMs only (cuBLAS through torch.matmul);
-      serial:    each layer decoded into one reused buffer, then its GEMM;
-      overlap:   layer i+1 decodes on a second stream into the other of two buffers while GEMM i runs;
+    """Decode overhead against the layer GEMMs of a prefill-sized forward pass, through the library's
+    CompressedLinear layers (the pages measure it as the denoising-step time with compressed vs BF16 weights;
+    that needs the real model, so this times the proxy: the 276 layer GEMMs y = x W^T + b on `tokens`
+    synthetic activations, in layer order).
+      gemm:      each layer's GEMM on its decoded weight kept resident (CompressedLinear.forward_with);
+      serial:    each CompressedLinear decodes its weight into the library's workspace, then its GEMM;
+      overlap:   the layers linked by link_prefetch: layer i+1 decodes on the workspace's decode stream into
+                 the other buffer while GEMM i runs;
       blocks:    each transformer block's layers (8 per block, then the 4 projections) decode as one
-                 sequence (ep_decompress_many: tables prepared once, launches chained) into their own
-                 buffers, then the block's GEMMs run.
-    value = serial / gemm - 1 (the overhead); the overlap figure is reported beside it.
-    fp8: the weights are per-row-scaled FP8 e4m3 codes of the same layers, compressed at 5 bpp and
-    decoded into e4m3; activations are e4m3 too, and the GEMMs are torch._scaled_mm with unit scales
-    and BF16 output (cuBLASLt FP8)."""
+                 sequence (ep_decompress_many) into their own buffers, then the block's GEMMs run.
+    value = serial / gemm - 1 (the overhead); the overlap and block figures are reported beside it.
+    fp8: the layers hold FP8 e4m3 codes of W / s_w (one scale per tensor) compressed at 5 bpp and decoded
+    into e4m3; the activations are cast to e4m3 once, before timing (CompressedLinear.quantize_input), and
+    each forward runs torch._scaled_mm (cuBLASLt FP8) with BF16 output."""
     import decode_ep_b200 as ep
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     layers = layer_list(args.layers)
     target = 5.0 if fp8 else args.target_bpp
-    wdt = torch.float8_e4m3fn if fp8 else torch.bfloat16
-    ws = [synth.dit_layer(i, shape=(M, N)).to(device) for i, _, M, N in layers]
-    if fp8:
-        ws = [to_e4m3_rows(w) for w in ws]
     streams_enc = [torch.cuda.Stream(device) for _ in range(4)]
 
     def enc(k):
+        _, _, M, N = layers[k]
         with torch.cuda.stream(streams_enc[k % 4]):
-            return ep.compress(ws[k], ep.EntroPackLossyConfig(target, encoder="cuda"))
+            w = synth.dit_layer(k, shape=(M, N)).to(device)
+            bias = torch.zeros(M, dtype=torch.bfloat16, device=device)
+            cfg = ep.EntroPackLossyConfig(target, encoder="cuda")
+            if fp8:
+                wf = w.float()
+                scale = float(wf.abs().max()) / 448.0
+                codes = (wf / scale).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+                return ep.CompressedLinear.from_fp8(codes, scale, bias, cfg)
+            return ep.CompressedLinear(ep.compress(w, cfg), bias).to(device)
 
     with cf.ThreadPoolExecutor(max_workers=4) as ex:
-        blobs = list(ex.map(enc, range(len(layers))))
+        cl = list(ex.map(enc, range(len(layers))))
     torch.cuda.synchronize(device)
-    resident = [ep.decompress(c, device=device) for c in blobs]  # what the GEMM-only pass reads
-    del ws
+    resident = [l.decode_weight() for l in cl]  # what the GEMM-only pass reads
     g = torch.Generator(device=device).manual_seed(7)
     xs = {N: torch.randn(tokens, N, generator=g, device=device, dtype=torch.bfloat16) for _, _, _, N in layers}
-    if fp8:
-        xs = {N: x.clamp(-448.0, 448.0).to(torch.float8_e4m3fn) for N, x in xs.items()}
-        one = torch.ones((), device=device, dtype=torch.float32)
-    max_numel = max(M * N for _, _, M, N in layers)
-    y = torch.empty(tokens * max(M for _, _, M, _ in layers), dtype=torch.bfloat16, device=device)
-    wbuf = [torch.empty(max_numel, dtype=wdt, device=device) for _ in range(2)]
+    sxs = {N: None for N in xs}
+    if fp8:  # activations cast to e4m3 once, outside the timed passes, as an FP8 pipeline would pass them
+        for N in list(xs):
+            xs[N], sxs[N] = ep.CompressedLinear.quantize_input(xs[N])
+    wdt = cl[0].weight_dtype
     main = torch.cuda.current_stream(device)
-    side = torch.cuda.Stream(device)
-
-    def gemm(k, w):
-        _, _, M, N = layers[k]
-        wk = w.reshape(-1)[: M * N].view(M, N).t()
-        if fp8:
-            torch._scaled_mm(xs[N], wk, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
-        else:
-            torch.matmul(xs[N], wk, out=y[: tokens * M].view(tokens, M))
 
     def step_gemm():
-        for k in range(len(layers)):
-            gemm(k, resident[k])
+        for k, l in enumerate(cl):
+            N = layers[k][3]
+            l.forward_with(xs[N], resident[k], sxs[N])
+
+    def step_layers():
+        for k, l in enumerate(cl):
+            N = layers[k][3]
+            l(xs[N], sxs[N])
 
     # Blocks of consecutive layers decoded as one sequence each, into per-layer views of one buffer.
     block_of_layer = [min(i // 8, 34) for i in range(len(layers))]
@@ -703,6 +697,7 @@ def run_gemm_overhead(args, tokens=4096, fp8=False):
         blocks.setdefault(bi, []).append(k)
     block_elems = max(sum(layers[k][2] * layers[k][3] for k in ks) for ks in blocks.values())
     bbuf = torch.empty(block_elems, dtype=wdt, device=device)
+    comps = [ep.CompressedTensor.from_blob(bytes(l.blob.cpu().numpy().tobytes())) for l in cl]
     block_runs = []
     for ks in blocks.values():
         views, off = [], 0
@@ -710,44 +705,14 @@ def run_gemm_overhead(args, tokens=4096, fp8=False):
             _, _, M, N = layers[k]
             views.append(bbuf[off: off + M * N].view(M, N))
             off += M * N
-        block_runs.append((ks, views, ep.LayerBatch([(blobs[k], v) for k, v in zip(ks, views)], main)))
+        block_runs.append((ks, views, ep.LayerBatch([(comps[k], v) for k, v in zip(ks, views)], main)))
 
     def step_blocks():
         for ks, views, batch in block_runs:
             batch.run()
             for k, v in zip(ks, views):
-                gemm(k, v)
-
-    def step_serial():
-        for k, c in enumerate(blobs):
-            out = wbuf[0][: c.shape[0] * c.shape[1]].view(c.shape)
-            ep.decompress_into(c, out, main)
-            gemm(k, out)
-
-    def step_overlap():
-        done = [torch.cuda.Event(), torch.cuda.Event()]   # GEMM that last read wbuf[b] is done
-        ready = [torch.cuda.Event(), torch.cuda.Event()]  # decode into wbuf[b] is done
-        first = [True, True]
-
-        def decode(k):
-            b = k & 1
-            c = blobs[k]
-            with torch.cuda.stream(side):
-                if not first[b]:
-                    side.wait_event(done[b])
-                first[b] = False
-                ep.decompress_into(c, wbuf[b][: c.shape[0] * c.shape[1]].view(c.shape), side)
-                ready[b].record(side)
-
-        decode(0)
-        for k in range(len(layers)):
-            if k + 1 < len(layers):
-                decode(k + 1)
-            b = k & 1
-            main.wait_event(ready[b])
-            gemm(k, wbuf[b])
-            done[b].record(main)
-        main.wait_stream(side)
+                N = layers[k][3]
+                cl[k].forward_with(xs[N], v, sxs[N])
 
     def timed(fn):
         for _ in range(args.warmup):
@@ -763,28 +728,33 @@ def run_gemm_overhead(args, tokens=4096, fp8=False):
 
     with ClockSampler(local) as clk:
         ms_gemm = timed(step_gemm)
-        ms_serial = timed(step_serial)
-        ms_overlap = timed(step_overlap)
+        ep.link_prefetch([])
+        for l in cl:
+            l.next_layer = None
+        ms_serial = timed(step_layers)
+        ep.link_prefetch(cl)
+        ms_overlap = timed(step_layers)
         ms_blocks = timed(step_blocks)
     if ep.device_status(main):
         raise RuntimeError("device status set")
     flops = 2.0 * tokens * sum(M * N for _, _, M, N in layers)
     kind = "FP8 e4m3 at 5 bpp, FP8 GEMMs" if fp8 else "BF16 at 4 bpp, BF16 GEMMs"
     return {
-        "metric": f"decode overhead on the 276 layer GEMMs of a 4096-token prefill ({kind}; serial decode+GEMM / GEMM - 1)",
+        "metric": f"decode overhead on the 276 layer GEMMs of a 4096-token prefill ({kind}; CompressedLinear "
+                  f"decode+GEMM / GEMM - 1)",
         "value": round(100.0 * (ms_serial / ms_gemm - 1.0), 2), "unit": "%", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_serial, 3), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": ("fp8" if fp8 else "bf16") + " GEMM; u32+f32 decode", "data": "synthetic",
         "config": {"workload": "dit276_fp8_gemm_overhead" if fp8 else "dit276_gemm_overhead", "tokens": tokens,
                    "layers": len(layers), "target_bpp": target, "gemm_tflops": round(flops / (ms_gemm * 1e-3) / 1e12, 1),
-                   "ms_gemm_only": round(ms_gemm, 3), "ms_decode_then_gemm": round(ms_serial, 3),
-                   "ms_decode_overlapped": round(ms_overlap, 3),
-                   "overlap_overhead_pct": round(100.0 * (ms_overlap / ms_gemm - 1.0), 2),
+                   "module": "decode_ep_b200.CompressedLinear", "ms_gemm_only": round(ms_gemm, 3),
+                   "ms_decode_then_gemm": round(ms_serial, 3), "ms_decode_prefetched": round(ms_overlap, 3),
+                   "prefetched_overhead_pct": round(100.0 * (ms_overlap / ms_gemm - 1.0), 2),
                    "ms_block_sequences": round(ms_blocks, 3),
                    "block_sequences_overhead_pct": round(100.0 * (ms_blocks / ms_gemm - 1.0), 2),
-                   "gemm": ("torch._scaled_mm (cuBLASLt), FP8 e4m3 x e4m3 -> BF16, unit scales" if fp8 else
-                            "torch.matmul (cuBLAS), BF16") + ", weights (out, in) used transposed",
-                   "actual_bpp": round(8 * sum(len(c.blob) for c in blobs) / sum(M * N for _, _, M, N in layers), 4)},
+                   "gemm": ("torch._scaled_mm (cuBLASLt), e4m3 x e4m3 -> BF16, per-tensor scales, activations cast "
+                            "to e4m3 before timing" if fp8 else "torch.nn.functional.linear (cuBLAS), BF16") + ", with bias",
+                   "actual_bpp": round(sum(l.compressed_bits for l in cl) / sum(M * N for _, _, M, N in layers), 4)},
         "clocks": clk.summary(), "gpu_launches": args.steps * len(layers),  # the serial pass's decodes
     }
 

@@ -11,6 +11,7 @@ API, after the EntroPack README (quick-start and Config sections):
     c = compress(tensor, cfg)                  # CompressedTensor; c.actual_bpp counts metadata
     w = decompress(c)                          # CUDA tensor, same shape and dtype
     decompress_into(c, out, stream=None)       # hot path: preallocated output, async on a stream
+    layer = CompressedLinear.from_linear(linear, cfg)   # README, section 使用 Compressed Linear
 """
 from __future__ import annotations
 
@@ -24,7 +25,8 @@ import torch
 from . import build as _build
 
 __all__ = ["EntroPackLossyConfig", "CompressedTensor", "EntroPackError", "LayerBatch", "compress", "decompress",
-           "decompress_into", "decompress_many", "decode_coords", "device_status", "blob_info", "plan_bitrates", "lib"]
+           "decompress_into", "decompress_many", "decode_coords", "device_status", "blob_info", "plan_bitrates", "lib",
+           "CompressedLinear", "DecodeWorkspace", "link_prefetch"]
 
 EP_BF16, EP_FP16, EP_FP32, EP_FP8_E4M3, EP_INT8 = 1, 2, 3, 4, 5
 _TORCH_TO_EP = {torch.bfloat16: EP_BF16, torch.float16: EP_FP16, torch.float32: EP_FP32,
@@ -324,3 +326,6 @@ def device_status(stream=None) -> int:
     flags = ctypes.c_int32()
     _check(lib().ep_get_device_status(_stream_ptr(stream), ctypes.byref(flags)), "device_status")
     return flags.value
+
+
+from .linear import CompressedLinear, DecodeWorkspace, link_prefetch  # noqa: E402  (uses the names above)
