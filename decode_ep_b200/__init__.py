@@ -18,6 +18,7 @@ from __future__ import annotations
 import ctypes
 import math
 import os
+import threading
 from dataclasses import dataclass, field
 
 import torch
@@ -48,48 +49,56 @@ class _Options(ctypes.Structure):
 
 
 _lib = None
+_lib_lock = threading.Lock()
 
 
 def lib() -> ctypes.CDLL:
-    """The loaded libentropack.so. The library is built in-tree if it is missing or out of date."""
-    global _lib
+    """The loaded libentropack.so. The library is built in-tree if it is missing or out of date. Threads that
+    ask for it at once wait for one build and load."""
     if _lib is None:
-        path = _build.LIB
-        if not os.path.exists(path) or _build.stale():
-            path = _build.build()
-        L = ctypes.CDLL(path)
-        c = ctypes
-        L.ep_options_default.argtypes = [c.POINTER(_Options)]
-        L.ep_compress.argtypes = [c.c_void_p, c.c_int, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_double,
-                                  c.POINTER(_Options), c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
-                                  c.POINTER(c.c_double)]
-        L.ep_compress_cuda.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_double,
-                                       c.POINTER(_Options), c.c_void_p, c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
-                                       c.POINTER(c.c_double)]
-        L.ep_compress_cuda_noalloc.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_double,
-                                               c.POINTER(_Options), c.c_void_p, c.c_void_p, c.c_size_t,
-                                               c.POINTER(c.c_size_t), c.POINTER(c.c_double)]
-        L.ep_compress_cuda_noalloc.restype = c.c_int
-        L.ep_blob_free.argtypes = [c.c_void_p]
-        L.ep_blob_info.argtypes = [c.c_void_p, c.c_size_t, c.POINTER(c.c_int), c.POINTER(c.c_int64),
-                                   c.POINTER(c.c_int64), c.POINTER(c.c_double)]
-        for name in ("ep_decompress_into", "ep_decode_coords_into"):
-            getattr(L, name).argtypes = [c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p, c.c_size_t, c.c_void_p]
-        L.ep_decompress.argtypes = [c.c_void_p, c.c_void_p, c.c_size_t, c.POINTER(c.c_void_p), c.c_void_p]
-        L.ep_decompress_many.argtypes = [c.c_int, c.POINTER(c.c_char_p), c.POINTER(c.c_void_p),
-                                         c.POINTER(c.c_size_t), c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
-                                         c.c_void_p]
-        L.ep_get_device_status.argtypes = [c.c_void_p, c.POINTER(c.c_int32)]
-        L.ep_plan_bitrates.argtypes = [c.c_int64, c.POINTER(c.c_int64), c.POINTER(c.c_int64), c.POINTER(c.c_double),
-                                       c.c_double, c.c_double, c.c_double, c.POINTER(_Options), c.POINTER(c.c_double)]
-        L.ep_status_string.restype = c.c_char_p
-        L.ep_status_string.argtypes = [c.c_int]
-        L.ep_last_error.restype = c.c_char_p
-        for name in ("ep_compress", "ep_compress_cuda", "ep_blob_info", "ep_decompress_into", "ep_decode_coords_into", "ep_decompress",
-                     "ep_get_device_status", "ep_decompress_many", "ep_plan_bitrates"):
-            getattr(L, name).restype = c.c_int
-        _lib = L
+        with _lib_lock:
+            if _lib is None:
+                _load()
     return _lib
+
+
+def _load() -> None:
+    global _lib
+    path = _build.LIB
+    if not os.path.exists(path) or _build.stale():
+        path = _build.build()
+    L = ctypes.CDLL(path)
+    c = ctypes
+    L.ep_options_default.argtypes = [c.POINTER(_Options)]
+    L.ep_compress.argtypes = [c.c_void_p, c.c_int, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_double,
+                              c.POINTER(_Options), c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
+                              c.POINTER(c.c_double)]
+    L.ep_compress_cuda.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_double,
+                                   c.POINTER(_Options), c.c_void_p, c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
+                                   c.POINTER(c.c_double)]
+    L.ep_compress_cuda_noalloc.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_double,
+                                           c.POINTER(_Options), c.c_void_p, c.c_void_p, c.c_size_t,
+                                           c.POINTER(c.c_size_t), c.POINTER(c.c_double)]
+    L.ep_compress_cuda_noalloc.restype = c.c_int
+    L.ep_blob_free.argtypes = [c.c_void_p]
+    L.ep_blob_info.argtypes = [c.c_void_p, c.c_size_t, c.POINTER(c.c_int), c.POINTER(c.c_int64),
+                               c.POINTER(c.c_int64), c.POINTER(c.c_double)]
+    for name in ("ep_decompress_into", "ep_decode_coords_into"):
+        getattr(L, name).argtypes = [c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p, c.c_size_t, c.c_void_p]
+    L.ep_decompress.argtypes = [c.c_void_p, c.c_void_p, c.c_size_t, c.POINTER(c.c_void_p), c.c_void_p]
+    L.ep_decompress_many.argtypes = [c.c_int, c.POINTER(c.c_char_p), c.POINTER(c.c_void_p),
+                                     c.POINTER(c.c_size_t), c.POINTER(c.c_void_p), c.POINTER(c.c_size_t),
+                                     c.c_void_p]
+    L.ep_get_device_status.argtypes = [c.c_void_p, c.POINTER(c.c_int32)]
+    L.ep_plan_bitrates.argtypes = [c.c_int64, c.POINTER(c.c_int64), c.POINTER(c.c_int64), c.POINTER(c.c_double),
+                                   c.c_double, c.c_double, c.c_double, c.POINTER(_Options), c.POINTER(c.c_double)]
+    L.ep_status_string.restype = c.c_char_p
+    L.ep_status_string.argtypes = [c.c_int]
+    L.ep_last_error.restype = c.c_char_p
+    for name in ("ep_compress", "ep_compress_cuda", "ep_blob_info", "ep_decompress_into", "ep_decode_coords_into", "ep_decompress",
+                 "ep_get_device_status", "ep_decompress_many", "ep_plan_bitrates"):
+        getattr(L, name).restype = c.c_int
+    _lib = L
 
 
 def _check(st: int, what: str) -> None:

@@ -32,7 +32,10 @@
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdlib>
+#include <cstring>
+#include <memory>
 #include <mutex>
 #include <vector>
 
@@ -113,6 +116,13 @@ struct Params {
 
 __device__ int g_status;
 
+// Acquire load at GPU scope: the memory operations that follow it in this thread are ordered after it.
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // ------------------------------------------------------------------------- PTX helpers
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -137,6 +147,7 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+__device__ __forceinline__ void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 // (a0 - k0, a1 - k1), then times c: two binary32 values per instruction (packed f32x2, sm_100).
 __device__ __forceinline__ void sub_mul_f32x2(float a0, float a1, float k0, float k1, float c, float& y0, float& y1) {
     uint64_t a, kk, cc, r;
@@ -395,24 +406,28 @@ struct RowCursor {
     // s - alpha * q0 (Markstein). This matches IEEE division for every bf16 s >= 2^-96 with a quotient
     // in [2^-96, 2^96] (checked exhaustively over all such s for thousands of alphas). Anything else,
     // zero rows included, takes the IEEE division.
-    static __device__ __forceinline__ float scale_of(const Params& p, const uint16_t* scales, uint32_t r) {
+    template <class P>
+    static __device__ __forceinline__ float scale_of(const P& p, const uint16_t* scales, uint32_t r) {
         const float s = __uint_as_float(uint32_t(__ldg(scales + r)) << 16);
         const float q0 = __fmul_rn(s, p.inv_alpha);
         const float q = __fmaf_rn(__fmaf_rn(-p.alpha, q0, s), p.inv_alpha, q0);
         return (s >= 0x1p-96f && q >= 0x1p-96f && q <= 0x1p96f) ? q : __fdiv_rn(s, p.alpha);
     }
-    __device__ __forceinline__ void load_scale(const Params& p, const uint16_t* scales) {
+    template <class P>
+    __device__ __forceinline__ void load_scale(const P& p, const uint16_t* scales) {
         if (row >= p.M) return;  // lanes past the last group
         c_row = scale_of(p, scales, row);
     }
-    __device__ __forceinline__ void start(const Params& p, const uint16_t* scales, uint32_t g) {
+    template <class P>
+    __device__ __forceinline__ void start(const P& p, const uint16_t* scales, uint32_t g) {
         row = g / p.gpr;
         col = g - row * p.gpr;
         c_row = 0.f;
         load_scale(p, scales);
     }
     // Next round: 32 groups further. The scale is reloaded only when the row changes.
-    __device__ __forceinline__ void advance(const Params& p, const uint16_t* scales) {
+    template <class P>
+    __device__ __forceinline__ void advance(const P& p, const uint16_t* scales) {
         col += 32;
         if (col >= p.gpr) {
             col -= p.gpr;
@@ -1058,12 +1073,14 @@ __device__ __forceinline__ uint32_t entry_template_v2(int c, int sym, uint32_t f
 // context sums to 256. Pass 2: each thread fills slots, finding the symbol that owns each by binary search.
 // Byte `threadIdx.x` of the serialised tables (zero past their end): loaded first thing in the kernel, so
 // that it does not queue behind the tiles' copies.
-__device__ __forceinline__ uint32_t table_byte(const Params& p) {
+template <class P>
+__device__ __forceinline__ uint32_t table_byte(const P& p) {
     const uint32_t tlen = p.tables_len < kScratchTableCap ? p.tables_len : kScratchTableCap;
     return threadIdx.x < tlen ? uint32_t(__ldg(p.blob + p.off_tables + threadIdx.x)) : 0u;
 }
 
-__device__ void build_tables_v2(const Params& p, uint8_t* tables, uint8_t* scratch, uint32_t tbyte) {
+template <class P>
+__device__ void build_tables_v2(const P& p, uint8_t* tables, uint8_t* scratch, uint32_t tbyte, bool report) {
     uint16_t* F = reinterpret_cast<uint16_t*>(scratch + kScratchF);
     uint16_t* cum = reinterpret_cast<uint16_t*>(scratch + kScratchCum);
     uint8_t* tb = scratch + kScratchBytesOff;
@@ -1103,7 +1120,7 @@ __device__ void build_tables_v2(const Params& p, uint8_t* tables, uint8_t* scrat
         if (lane == 0) {
             cum[c * 129 + 128] = uint16_t(total);
             const bool ok = cnt == 0 ? total == 0 : (total == kProbScaleV2 && cnt >= 2);
-            if (!ok && blockIdx.x == 0) atomicOr(&g_status, int(EP_DEV_BAD_TABLES));
+            if (!ok && report) atomicOr(&g_status, int(EP_DEV_BAD_TABLES));
         }
     }
     __syncthreads();
@@ -1125,9 +1142,10 @@ __device__ void build_tables_v2(const Params& p, uint8_t* tables, uint8_t* scrat
 }
 
 // One symbol step: the fused entry of the context block B at slot x & 255, then x <- f (x >> 8) + slot - cum.
-__device__ __forceinline__ uint32_t symbol(const Params& p, uint32_t B, uint32_t& x) {
+template <class K>
+__device__ __forceinline__ uint32_t symbol(const K& k, uint32_t B, uint32_t& x) {
     const uint32_t q = x >> 8;
-    const uint32_t e = ld_shared_u32((x + q * p.kneg256) * p.k4 + B);  // B + 4 (x mod 256)
+    const uint32_t e = ld_shared_u32((x + q * k.kneg256) * k.k4 + B);  // B + 4 (x mod 256)
     x = __byte_perm(e, 0u, 0x4442u) * q + (e >> 24);
     return e;
 }
@@ -1158,8 +1176,8 @@ __device__ __forceinline__ void refill(uint32_t& x, uint32_t& pa, uint32_t lt_ma
 // Values of one group from the value bits mb[i]: 1.5 * 2^22 + F/2 with F = 2 idx + b at positions 0..6 and
 // 4 idx + b at position 7 (before pi is added), built by ORing the entries' value fields into the mantissa
 // (see round_fast of version 1). two_pi = 2 pi comes from the XOR of the idx parities.
-template <int MODE, bool WAIT>
-__device__ __forceinline__ void store_fast(const Params& p, const uint32_t* mb, uint32_t two_pi, uint32_t g, float c) {
+template <int MODE, bool WAIT, class P>
+__device__ __forceinline__ void store_fast(const P& p, const uint32_t* mb, uint32_t two_pi, uint32_t g, float c) {
     float m[8], y[8];
     int32_t z[8];
 #pragma unroll
@@ -1179,8 +1197,8 @@ __device__ __forceinline__ void store_fast(const Params& p, const uint32_t* mb, 
 
 // Values of one group in general: hi from the entries or the escape words, lo from the raw section, then
 // t = hi 2^r + lo, u_7 = 2 t_7 + pi, z = 2u + b and y = RN(z/2 * c).
-template <int MODE>
-__device__ __forceinline__ void store_general(const Params& p, const uint32_t* e, const int32_t* hesc, uint32_t escm,
+template <int MODE, class P>
+__device__ __forceinline__ void store_general(const P& p, const uint32_t* e, const int32_t* hesc, uint32_t escm,
                                               const uint32_t* win, uint32_t g, float c) {
     const int r = p.r;
     int32_t t[8];
@@ -1249,31 +1267,31 @@ __device__ __forceinline__ uint32_t or3(uint32_t a, uint32_t b, uint32_t c) {
 // escape (its offset entry says so). Then, when some lane of the warp met one in this round, its words are
 // read after the fourth pair, and each escaped position's value bits and parity are rebuilt from the word's
 // hi (an escape's field, 2 * 63 + b or 4 * 63 + b, marks it).
-template <int MODE, bool WAIT, bool ESC>
-__device__ __forceinline__ void round_fast_v2(const Params& p, uint32_t t0, uint32_t& x, uint32_t& pa, uint32_t g,
+template <int MODE, bool WAIT, bool ESC, class P, class K>
+__device__ __forceinline__ void round_fast_v2(const P& p, const K& kc, uint32_t t0, uint32_t ts, uint32_t& x, uint32_t& pa, uint32_t g,
                                               uint32_t lt_mask, float c, uint32_t k2) {
     uint32_t mb[8], e, e2, par, escs;
-    e = symbol(p, t0 | kStartOffset, x);
+    e = symbol(kc, ts, x);
     mb[0] = and_or(e, 0x7Fu, kHalfMagic);
     const uint32_t gbase = and_or(e, kCosetBit, t0);
-    e2 = symbol(p, and_or(e, kClassBit, gbase), x);
+    e2 = symbol(kc, and_or(e, kClassBit, gbase), x);
     mb[1] = and_or(e2, 0x7Fu, kHalfMagic);
     par = e ^ e2;
     escs = e | e2;
     refill(x, pa, lt_mask, k2);
 #pragma unroll
     for (int i = 2; i < 6; i += 2) {
-        e = symbol(p, and_or(e2, kClassBit, gbase), x);
+        e = symbol(kc, and_or(e2, kClassBit, gbase), x);
         mb[i] = and_or(e, 0x7Fu, kHalfMagic);
-        e2 = symbol(p, and_or(e, kClassBit, gbase), x);
+        e2 = symbol(kc, and_or(e, kClassBit, gbase), x);
         mb[i + 1] = and_or(e2, 0x7Fu, kHalfMagic);
         par = xor3(par, e, e2);
         escs = or3(escs, e, e2);
         refill(x, pa, lt_mask, k2);
     }
-    e = symbol(p, and_or(e2, kClassBit, gbase), x);
+    e = symbol(kc, and_or(e2, kClassBit, gbase), x);
     mb[6] = and_or(e, 0x7Fu, kHalfMagic);
-    e2 = symbol(p, and_or(e, kClassBit, gbase | kPos7Bit), x);
+    e2 = symbol(kc, and_or(e, kClassBit, gbase | kPos7Bit), x);
     mb[7] = and_or(e2, 0xFFu, kHalfMagic);
     par ^= e;
     escs = or3(escs, e, e2);
@@ -1304,8 +1322,8 @@ __device__ __forceinline__ void round_fast_v2(const Params& p, uint32_t t0, uint
 
 // General round: ragged rounds (PARTIAL: some lanes hold no group), raw low bits, and streams read from
 // global memory with bounds checks (Words = GlobalWords) or from the ring (RingWords).
-template <int MODE, bool PARTIAL, class Words>
-__device__ __forceinline__ void round_general_v2(const Params& p, uint32_t t0, const Words& words, const uint8_t* rawsec,
+template <int MODE, bool PARTIAL, class Words, class P>
+__device__ __forceinline__ void round_general_v2(const P& p, uint32_t t0, uint32_t ts, const Words& words, const uint8_t* rawsec,
                                               uint32_t raw_avail, TileState& st, uint32_t q, bool active, uint32_t g,
                                               uint32_t lt_mask, float c) {
     const bool on = !PARTIAL || active;
@@ -1313,7 +1331,7 @@ __device__ __forceinline__ void round_general_v2(const Params& p, uint32_t t0, c
     raw_window(rawsec, raw_avail, q, on ? p.r : 0, win);
     uint32_t x = st.x, pb = st.pb;
     uint32_t e[8];
-    uint32_t gbase = t0, B = t0 | kStartOffset;
+    uint32_t gbase = t0, B = ts;
 #pragma unroll
     for (int pr = 0; pr < 4; ++pr) {
 #pragma unroll
@@ -1364,8 +1382,8 @@ static_assert(kTablesBytes + kScratchSize + kSlackBytes >= kOverrunBytes, "a cor
 // lane i computes the factor of row row0 + i once, and each round takes its row's factor by a shuffle, with
 // no load on the round's path. kr: the first round's column in its row, in rounds. Otherwise the lanes'
 // rows move on their own (RowCursor).
-template <int MODE, bool ESC, bool UNIFORM>
-__device__ __forceinline__ uint32_t fast_rounds_v2(const Params& p, uint32_t t0, TileState& st, uint32_t ring_base,
+template <int MODE, bool ESC, bool UNIFORM, class P, class K>
+__device__ __forceinline__ uint32_t fast_rounds_v2(const P& p, const K& kc, uint32_t t0, uint32_t ts, TileState& st, uint32_t ring_base,
                                                    uint32_t g, uint32_t lt_mask, uint32_t Rf, uint32_t row0, uint32_t kr,
                                                    const uint16_t* scales, RowCursor& rc, bool& waited) {
     uint32_t k = 0, x = st.x, pa = ring_base + st.pb;
@@ -1374,7 +1392,7 @@ __device__ __forceinline__ uint32_t fast_rounds_v2(const Params& p, uint32_t t0,
         const float cvec = row0 + lane < p.M ? RowCursor::scale_of(p, scales, row0 + lane) : 0.f;
         uint32_t ri = 0;
         if (!waited && Rf > 0) {
-            round_fast_v2<MODE, true, ESC>(p, t0, x, pa, g, lt_mask, __shfl_sync(kFullMask, cvec, 0), p.k2);
+            round_fast_v2<MODE, true, ESC>(p, kc, t0, ts, x, pa, g, lt_mask, __shfl_sync(kFullMask, cvec, 0), kc.k2);
             waited = true;
             k = 1;
             g += 32;
@@ -1384,7 +1402,7 @@ __device__ __forceinline__ uint32_t fast_rounds_v2(const Params& p, uint32_t t0,
             }
         }
         for (; k < Rf; ++k, g += 32) {
-            round_fast_v2<MODE, false, ESC>(p, t0, x, pa, g, lt_mask, __shfl_sync(kFullMask, cvec, ri), p.k2);
+            round_fast_v2<MODE, false, ESC>(p, kc, t0, ts, x, pa, g, lt_mask, __shfl_sync(kFullMask, cvec, ri), kc.k2);
             if (++kr == rpr) {
                 kr = 0;
                 ++ri;
@@ -1392,14 +1410,14 @@ __device__ __forceinline__ uint32_t fast_rounds_v2(const Params& p, uint32_t t0,
         }
     } else {
         if (!waited && Rf > 0) {
-            round_fast_v2<MODE, true, ESC>(p, t0, x, pa, g, lt_mask, rc.scale(), p.k2);
+            round_fast_v2<MODE, true, ESC>(p, kc, t0, ts, x, pa, g, lt_mask, rc.scale(), kc.k2);
             rc.advance(p, scales);
             waited = true;
             k = 1;
             g += 32;
         }
         for (; k < Rf; ++k, g += 32) {
-            round_fast_v2<MODE, false, ESC>(p, t0, x, pa, g, lt_mask, rc.scale(), p.k2);
+            round_fast_v2<MODE, false, ESC>(p, kc, t0, ts, x, pa, g, lt_mask, rc.scale(), kc.k2);
             rc.advance(p, scales);
         }
     }
@@ -1412,7 +1430,8 @@ __device__ __forceinline__ uint32_t fast_rounds_v2(const Params& p, uint32_t t0,
 struct TileOffs {
     uint32_t e0, e1;
 };
-__device__ __forceinline__ TileOffs load_offs(const Params& p, const uint32_t* toff, uint32_t tile) {
+template <class P>
+__device__ __forceinline__ TileOffs load_offs(const P& p, const uint32_t* toff, uint32_t tile) {
     TileOffs o{0u, 0u};
     if (tile < p.T) {
         o.e0 = __ldg(toff + tile);
@@ -1421,7 +1440,8 @@ __device__ __forceinline__ TileOffs load_offs(const Params& p, const uint32_t* t
     return o;
 }
 // Byte size of a tile whose offsets are sane (start <= end <= payload, at least its 128 bytes of states), else 0.
-__device__ __forceinline__ uint32_t tile_size(const Params& p, const TileOffs& o) {
+template <class P>
+__device__ __forceinline__ uint32_t tile_size(const P& p, const TileOffs& o) {
     const uint64_t start = uint64_t(o.e0 & 0x7FFFFFFFu) * 16, end = uint64_t(o.e1 & 0x7FFFFFFFu) * 16;
     return (end >= start + 128 && end <= p.payload_bytes && end - start <= 0x7FFFFFF0ull) ? uint32_t(end - start) : 0u;
 }
@@ -1473,7 +1493,7 @@ __global__ void __launch_bounds__(kThreadsV2, 1) decode_kernel(const Params p) {
             pending = 1;
         }
     }
-    build_tables_v2(p, tables, scratch, tbyte);
+    build_tables_v2(p, tables, scratch, tbyte, blockIdx.x == 0);
     bool waited = false;
 
     // Every decision below is taken for the whole warp (a vote, or values of the tile index and the kernel
@@ -1524,12 +1544,12 @@ __global__ void __launch_bounds__(kThreadsV2, 1) decode_kernel(const Params p) {
                 const uint32_t row0 = gt0 / p.gpr, kr0 = (gt0 - row0 * p.gpr) / 32;
                 const bool esc = __any_sync(kFullMask, cur.e0 >> 31);
                 if (p.gpr % 32 == 0) {
-                    k = esc ? fast_rounds_v2<MODE, true, true>(p, t0, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited)
-                            : fast_rounds_v2<MODE, false, true>(p, t0, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited);
+                    k = esc ? fast_rounds_v2<MODE, true, true>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited)
+                            : fast_rounds_v2<MODE, false, true>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited);
                 } else {
                     rc.start(p, scales, gt0 + lane);
-                    k = esc ? fast_rounds_v2<MODE, true, false>(p, t0, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited)
-                            : fast_rounds_v2<MODE, false, false>(p, t0, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited);
+                    k = esc ? fast_rounds_v2<MODE, true, false>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited)
+                            : fast_rounds_v2<MODE, false, false>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited);
                 }
             }
             if (k < R) {
@@ -1544,9 +1564,9 @@ __global__ void __launch_bounds__(kThreadsV2, 1) decode_kernel(const Params p) {
                     const bool full = 32 * k + 32 <= ng;
                     // Ring reads of a round stay within the tile's own bytes (a round takes at most 768).
                     if (in_ring && full && __all_sync(kFullMask, st.pb + 2 * kRoundWords <= sz)) {
-                        round_general_v2<MODE, false>(p, t0, ring, rawsec, raw_avail, st, q, true, g, lt_mask, rc.scale());
+                        round_general_v2<MODE, false>(p, t0, t0 | kStartOffset, ring, rawsec, raw_avail, st, q, true, g, lt_mask, rc.scale());
                     } else {
-                        round_general_v2<MODE, true>(p, t0, gwords, rawsec, raw_avail, st, q, q < ng, g, lt_mask,
+                        round_general_v2<MODE, true>(p, t0, t0 | kStartOffset, gwords, rawsec, raw_avail, st, q, q < ng, g, lt_mask,
                                                       rc.scale());
                     }
                     rc.advance(p, scales);
@@ -1572,6 +1592,361 @@ __global__ void __launch_bounds__(kThreadsV2, 1) decode_kernel(const Params p) {
     if (!waited) grid_dependency_wait();
 }
 
+
+// ------------------------------------------------------------------------- one launch for a sequence
+//
+// ep_decompress_many of version-2 blobs that share one output type runs as two launches: prep_tables_kernel
+// builds every layer's fused entries once into global scratch, and seq_kernel, one CTA per SM for all the
+// layers, decodes them. The tiles of all the layers are dealt round-robin as one list: the sequence's k-th
+// tile goes to CTA k mod grid, and a CTA's own tiles go to its warps in turn, so a layer with few tiles shares
+// the SMs with the next one, and no launch boundary, table build or wait for a whole previous layer sits
+// between layers. Each CTA holds the tables of kWindows consecutive layers in shared windows: the window of
+// layer L is refilled with layer L + kWindows by bulk copies once all of the CTA's warps are done with L. A tile
+// writes only after the tiles of earlier layers that wrote the same bytes are done (per-layer tile-done
+// bitmasks in global memory, bounded waits), so the buffer ends as a sequence of separate launches leaves it.
+
+constexpr uint32_t kMaxSeqLayers = 280;
+constexpr uint16_t kNoDep = 0xFFFFu;
+
+struct LayerDesc {
+    const uint8_t* blob;
+    void* dst;
+    uint64_t payload_bytes;
+    uint32_t gpr, T, G, NG, M;
+    int r;
+    float alpha, inv_alpha;
+    uint32_t off_scales, off_offsets, off_payload, off_tables, tables_len;
+    uint32_t tile0;        // the layer's first tile in the sequence's deal order
+    uint32_t bits;         // word offset of the layer's tile-done bitmask in the order scratch
+    uint32_t need_prefix;  // layers [0, need_prefix) are complete before any store of this layer
+    // Groups [seg_lo[d], seg_hi[d]) of this layer were last written, before it, by layer seg_layer[d]
+    // (kNoDep: no such segment). Older writers, if any, are covered by need_prefix.
+    uint32_t seg_lo[2], seg_hi[2];
+    uint16_t seg_layer[2];
+};
+
+struct SeqParams {
+    uint32_t count;
+    uint32_t k2, k4, kneg256;  // multipliers kept out of the compiler's sight (see Params)
+    uint32_t ordered;          // some layer overwrites an earlier one's output: tiles wait and publish
+    uint32_t use_prefix;       // some layer has need_prefix > 0: tiles are counted per layer
+    uint32_t counts_off;       // word offset of the per-layer done counters in the order scratch
+    uint32_t prefix_off;       // word offset of the number of leading complete layers
+    const uint32_t* tables;    // prepared fused entries, kTablesBytes per layer, in shared-window layout
+    uint32_t* order;           // tile-done bitmasks, done counters, prefix (zeroed before the launch)
+    LayerDesc L[kMaxSeqLayers];
+};
+static_assert(sizeof(SeqParams) <= 32764, "kernel parameters are limited to 32764 bytes");
+
+// One CTA per layer: builds the layer's fused entries into global memory.
+__global__ void __launch_bounds__(kThreadsV2, 1) prep_tables_kernel(const __grid_constant__ SeqParams sp) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    const LayerDesc& p = sp.L[blockIdx.x];
+    const uint32_t tbyte = table_byte(p);
+    uint32_t* out = const_cast<uint32_t*>(sp.tables) + size_t(blockIdx.x) * (kTablesBytes / 4);
+    build_tables_v2(p, reinterpret_cast<uint8_t*>(out), smem_raw, tbyte, true);
+}
+
+// Table windows: a CTA holds the tables of kWindows consecutive layers. A window is the 8 KB of context
+// blocks, on an 8 KB boundary so that the (b, class, position 7) bits combine by OR, plus a 1 KB START block
+// of its own. Layout: rings, then the context blocks of every window, their START blocks, then the window
+// barriers and done counters. More than kOverrunBytes follow the last ring.
+constexpr uint32_t kWindows = 4;  // a power of two
+constexpr uint32_t kCtxRegion = kStartOffset;  // contexts 1..8
+constexpr uint32_t kSeqSmemBytes = 16 + kRingsBytes + kCtxRegion + kWindows * kTablesBytes + kWindows * 16 +
+                                   kMaxSeqLayers * 4;
+static_assert(kSeqSmemBytes <= 227 * 1024, "exceeds the per-block shared memory of sm_100");
+static_assert(kWindows * kTablesBytes >= kOverrunBytes, "a corrupt stream could read past the allocation");
+
+// Starts the bulk copies of layer L's entries into window (ctx, start); thread 0 only.
+__device__ __noinline__ void load_window(const SeqParams& sp, uint32_t L, uint32_t ctx, uint32_t start,
+                                            uint32_t bar) {
+    mbar_expect_tx(bar, kTablesBytes);
+    const uint32_t* src = sp.tables + size_t(L) * (kTablesBytes / 4);
+    for (uint32_t c = 0; c < kCtxRegion / kCtxBytes; ++c)
+        bulk_copy_g2s(ctx + c * kCtxBytes, src + c * (kCtxBytes / 4), kCtxBytes, bar);
+    bulk_copy_g2s(start, src + kStartOffset / 4, kCtxBytes, bar);
+}
+
+// The CTA's tiles of layer L: t0, t0 + grid, ... (the return value counts them).
+__device__ __forceinline__ uint32_t cta_tiles(const SeqParams& sp, uint32_t L, uint32_t& t0) {
+    const uint32_t T = sp.L[L].T, grid = gridDim.x;
+    t0 = (blockIdx.x + grid - sp.L[L].tile0 % grid) % grid;
+    return t0 < T ? (T - t0 + grid - 1) / grid : 0u;
+}
+// This warp's first tile of layer L, or T when it has none there. nb: the CTA's tiles in the layers before L,
+// which sets where the warps' turns stand.
+__device__ __forceinline__ uint32_t first_tile(const SeqParams& sp, uint32_t L, uint32_t nb, uint32_t warp) {
+    uint32_t t0;
+    const uint32_t cnt = cta_tiles(sp, L, t0);
+    const uint32_t j0 = (warp + 32u - nb % 32u) % 32u;
+    return j0 < cnt ? t0 + j0 * gridDim.x : sp.L[L].T;
+}
+
+// A position in this warp's walk over the sequence; L == count at the end.
+struct Pos {
+    uint32_t L, tile;
+};
+// The warp's next tile after q. nbs[L]: the CTA's tiles in the layers before L (shared memory).
+__device__ __forceinline__ Pos next_pos(const SeqParams& sp, const uint32_t* nbs, Pos q, uint32_t warp) {
+    q.tile += 32u * gridDim.x;
+    while (q.L < sp.count && q.tile >= sp.L[q.L].T) {
+        ++q.L;
+        if (q.L < sp.count) q.tile = first_tile(sp, q.L, nbs[q.L], warp);
+    }
+    return q;
+}
+__device__ __forceinline__ const uint32_t* pos_toff(const SeqParams& sp, const Pos& q) {
+    const LayerDesc& p = sp.L[q.L];
+    return reinterpret_cast<const uint32_t*>(p.blob + p.off_offsets) + q.tile;
+}
+__device__ __forceinline__ TileOffs pos_offs(const SeqParams& sp, const Pos& q) {
+    if (q.L >= sp.count) return TileOffs{0u, 0u};
+    const uint32_t* t = pos_toff(sp, q);
+    return TileOffs{__ldg(t), __ldg(t + 1)};
+}
+
+constexpr uint32_t kDepSpins = 1u << 20;  // bounded waits: about a quarter second, then a status bit
+
+// Before the first store of a tile of layer p (groups [g0, g0 + ng), es bytes an element): the layers before
+// need_prefix complete, and, for each segment the tile meets, the tiles of the segment's writer that cover the
+// common bytes done. The flags are read in parallel, one word a lane: lane 0 the prefix, lanes 1-15 segment
+// 0's bitmask words, lanes 16-31 segment 1's. A lane's acquire orders the warp's stores after it through the
+// closing warp barrier.
+__device__ __forceinline__ void seq_wait(const SeqParams& sp, const LayerDesc& p, uint32_t g0, uint32_t ng,
+                                         uint32_t es) {
+    const uint32_t lane = threadIdx.x & 31;
+    const uint32_t d = lane >> 4, first = d ? lane - 16 : lane - 1, step = d ? 16u : 15u;
+    const uint32_t* bits = nullptr;
+    uint32_t k0 = 1, k1 = 0;  // tiles [k0, k1] of the writer (empty unless set below)
+    if (lane != 0 && p.seg_layer[d] != kNoDep) {
+        const uint32_t a = max(g0, p.seg_lo[d]), b = min(g0 + ng, p.seg_hi[d]);
+        if (a < b) {
+            const LayerDesc& q = sp.L[p.seg_layer[d]];
+            const uint64_t qlo = reinterpret_cast<uint64_t>(q.dst), qhi = qlo + uint64_t(q.NG) * 8 * es;
+            const uint64_t base = reinterpret_cast<uint64_t>(p.dst);
+            const uint64_t lo = max(base + uint64_t(a) * 8 * es, qlo), hi = min(base + uint64_t(b) * 8 * es, qhi);
+            if (lo < hi) {
+                const uint64_t tb = uint64_t(32) * q.G * 8 * es;  // output bytes of one full tile of q
+                k0 = uint32_t((lo - qlo) / tb);
+                k1 = min(uint32_t((hi - qlo - 1) / tb), q.T - 1);
+                bits = sp.order + q.bits;
+            }
+        }
+    }
+    for (uint32_t n = 0;; ++n) {
+        bool ok = true;
+        if (lane == 0 && p.need_prefix) ok = ld_acquire(sp.order + sp.prefix_off) >= p.need_prefix;
+        if (bits) {
+            for (uint32_t w = k0 / 32 + first; w <= k1 / 32; w += step) {
+                const uint32_t lo = w * 32 > k0 ? 0u : k0 % 32, hi = w * 32 + 31 < k1 ? 31u : k1 % 32;
+                const uint32_t m = (hi == 31 ? ~0u : (2u << hi) - 1u) & ~((1u << lo) - 1u);
+                ok = ok && (ld_acquire(bits + w) & m) == m;
+            }
+        }
+        if (__all_sync(kFullMask, ok)) break;
+        if (n >= kDepSpins) {
+            if (lane == 0) atomicOr(&g_status, int(EP_DEV_DEP_WAIT));
+            break;
+        }
+        __nanosleep(256);
+    }
+    __syncwarp();
+}
+
+// Moves the prefix of complete layers on from j while layer j is complete (an empty layer always is). The
+// prefix only moves by compare-and-swap from j to j + 1, so a caller that finds it elsewhere stops. Two
+// callers racing over neighbouring layers cannot both stop short: each makes its update, fences, then reads
+// the other's, so at least one sees both and moves on.
+__device__ __forceinline__ void advance_prefix(const SeqParams& sp, uint32_t j) {
+    for (; j < sp.count; ++j) {
+        if (ld_acquire(sp.order + sp.counts_off + j) != sp.L[j].T) break;
+        if (atomicCAS(sp.order + sp.prefix_off, j, j + 1) != j) break;
+        __threadfence();
+    }
+}
+
+// After the last store of tile `tile` of layer L: publish it, count it, and when it completes its layer,
+// advance the prefix of complete layers (a layer that completes while an earlier one is open leaves the
+// advance to that layer's last tile).
+__device__ __forceinline__ void seq_done(const SeqParams& sp, uint32_t L, uint32_t tile) {
+    __syncwarp();
+    if ((threadIdx.x & 31) != 0) return;
+    __threadfence();
+    atomicOr(sp.order + sp.L[L].bits + tile / 32, 1u << (tile % 32));
+    if (!sp.use_prefix) return;
+    const uint32_t c = atomicAdd(sp.order + sp.counts_off + L, 1u) + 1u;
+    if (c != sp.L[L].T) return;
+    __threadfence();
+    advance_prefix(sp, L);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreadsV2, 1) seq_kernel(const __grid_constant__ SeqParams sp) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    constexpr uint32_t es = MODE == kFP32 ? 4u : (MODE == kBF16 || MODE == kFP16) ? 2u : 1u;
+    const uint32_t raw_base = smem_addr(smem_raw);
+    const uint32_t rings0 = (raw_base + 15u) & ~15u;
+    const uint32_t win0 = (rings0 + kRingsBytes + kCtxRegion - 1) & ~(kCtxRegion - 1);
+    const uint32_t starts = win0 + kWindows * kCtxRegion;
+    const uint32_t bars = starts + kWindows * kCtxBytes;  // kWindows mbarriers, then kWindows done counters
+    uint32_t* done_cnt = reinterpret_cast<uint32_t*>(smem_raw + (bars + 8u * kWindows - raw_base));
+    uint32_t* nbs = done_cnt + kWindows;  // per layer: the CTA's tiles in the layers before it
+    const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const uint32_t ring_base = rings0 + warp * kRingBytes;
+    const uint32_t n = sp.count;
+
+    if (threadIdx.x < kWindows) {
+        mbar_init(bars + 8 * threadIdx.x, 1);
+        done_cnt[threadIdx.x] = 0;
+    }
+    if (warp == 0) {  // nbs: an exclusive scan of the CTA's tile counts over the layers
+        uint32_t carry = 0;
+        for (uint32_t base = 0; base < n; base += 32) {
+            uint32_t t0c, c = base + lane < n ? cta_tiles(sp, base + lane, t0c) : 0u, incl = c;
+#pragma unroll
+            for (int dd = 1; dd < 32; dd <<= 1) {
+                const uint32_t v = __shfl_up_sync(kFullMask, incl, dd);
+                if (lane >= uint32_t(dd)) incl += v;
+            }
+            if (base + lane < n) nbs[base + lane] = carry + incl - c;
+            carry += __shfl_sync(kFullMask, incl, 31);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        for (uint32_t s = 0; s < kWindows && s < n; ++s)
+            load_window(sp, s, win0 + s * kCtxRegion, starts + s * kCtxBytes, bars + 8 * s);
+    // Leading empty layers never complete a tile: move the prefix over them.
+    if (sp.use_prefix && blockIdx.x == 0 && threadIdx.x == 0) advance_prefix(sp, 0);
+
+    Pos cur{0u, n ? first_tile(sp, 0, 0, warp) : 0u};
+    if (n && cur.tile >= sp.L[0].T) cur = next_pos(sp, nbs, cur, warp);
+    Pos nxt = next_pos(sp, nbs, cur, warp);
+    TileOffs co = pos_offs(sp, cur), no = pos_offs(sp, nxt);
+    uint32_t place = 0, pending = 0;
+    if (cur.L < n) {
+        const LayerDesc& p = sp.L[cur.L];
+        const uint32_t sz = tile_size(p, co);
+        if (sz && sz <= kRingBytes) {
+            copy_tile(ring_base, p.blob + p.off_payload + uint64_t(co.e0 & 0x7FFFFFFFu) * 16, sz, lane);
+            cp_async_commit();
+            pending = 1;
+        }
+    }
+    bool waited = true;  // no launch-level wait: stores wait tile by tile (seq_wait)
+
+    for (uint32_t L = 0; L < n; ++L) {
+        const uint32_t s = L % kWindows, t0 = win0 + s * kCtxRegion, ts = starts + s * kCtxBytes;
+        if (!mbar_wait(bars + 8 * s, (L / kWindows) & 1u, kTableWaitTries) && lane == 0)
+            atomicOr(&g_status, int(EP_DEV_TABLE_COPY));
+        const LayerDesc& p = sp.L[L];
+        const uint16_t* scales = reinterpret_cast<const uint16_t*>(p.blob + p.off_scales);
+        const uint8_t* payload = p.blob + p.off_payload;
+        const uint32_t per_tile = 32 * p.G;
+        while (cur.L == L) {
+            const uint32_t tile = cur.tile;
+            const uint32_t ng = min(per_tile, p.NG - tile * per_tile);
+            const uint32_t raw = (ng * uint32_t(p.r) + 3u) & ~3u, s0 = 128 + raw;
+            const uint32_t sz = __shfl_sync(kFullMask, tile_size(p, co), 0);
+            const bool ok = sz >= s0;
+            const bool in_ring = ok && sz <= kRingBytes;
+            const Pos aft = next_pos(sp, nbs, nxt, warp);
+            const LayerDesc& pn = sp.L[nxt.L < n ? nxt.L : L];
+            const uint32_t nsz = nxt.L < n ? __shfl_sync(kFullMask, tile_size(pn, no), 0) : 0u;
+            const bool early = nsz && (in_ring ? sz + nsz <= kRingBytes : nsz <= kRingBytes);
+            const uint32_t nplace = early && in_ring && place == 0 ? kRingBytes - nsz : 0u;
+            if (aft.L < n) prefetch_l1(pos_toff(sp, aft));  // read at the end of the tile
+            cp_async_wait<0>();
+            __syncwarp();
+            pending = 0;
+            const uint8_t* nsrc = pn.blob + pn.off_payload + uint64_t(no.e0 & 0x7FFFFFFFu) * 16;
+            if (early) {
+                copy_tile(ring_base + nplace, nsrc, nsz, lane);
+                cp_async_commit();
+                pending = 1;
+            }
+            if (!ok) {
+                if (lane == 0) atomicOr(&g_status, int(EP_DEV_BAD_OFFSETS));
+            } else {
+                const uint32_t rb = ring_base + place;
+                const uint8_t* tp = payload + uint64_t(co.e0 & 0x7FFFFFFFu) * 16;
+                TileState st;
+                st.x = in_ring ? ld_shared_u32(rb + 4 * lane) : __ldg(reinterpret_cast<const uint32_t*>(tp) + lane);
+                st.pb = s0;
+                const GlobalWords gwords{tp, s0, sz};
+                RowCursor rc;
+                const uint8_t* rawsec = tp + 128;
+                const uint32_t raw_avail = sz - 128;
+                const uint32_t R = (ng + 31) / 32;
+                const uint32_t gt0 = tile * per_tile;
+                if (sp.ordered) seq_wait(sp, p, gt0, ng, es);
+                uint32_t k = 0;
+                if (in_ring && p.r == 0) {
+                    const uint32_t Rf = min(ng / 32, kMaxFastRounds);
+                    const uint32_t row0 = gt0 / p.gpr, kr0 = (gt0 - row0 * p.gpr) / 32;
+                    const bool esc = __any_sync(kFullMask, co.e0 >> 31);
+                    if (p.gpr % 32 == 0) {
+                        k = esc ? fast_rounds_v2<MODE, true, true>(p, sp, t0, ts, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited)
+                                : fast_rounds_v2<MODE, false, true>(p, sp, t0, ts, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited);
+                    } else {
+                        rc.start(p, scales, gt0 + lane);
+                        k = esc ? fast_rounds_v2<MODE, true, false>(p, sp, t0, ts, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited)
+                                : fast_rounds_v2<MODE, false, false>(p, sp, t0, ts, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited);
+                    }
+                }
+                if (k < R) {
+                    rc.start(p, scales, gt0 + 32 * k + lane);
+                    const RingWords ring{rb};
+                    for (; k < R; ++k) {
+                        const uint32_t q = 32 * k + lane, g = gt0 + q;
+                        const bool full = 32 * k + 32 <= ng;
+                        if (in_ring && full && __all_sync(kFullMask, st.pb + 2 * kRoundWords <= sz)) {
+                            round_general_v2<MODE, false>(p, t0, ts, ring, rawsec, raw_avail, st, q, true, g, lt_mask, rc.scale());
+                        } else {
+                            round_general_v2<MODE, true>(p, t0, ts, gwords, rawsec, raw_avail, st, q, q < ng, g, lt_mask,
+                                                          rc.scale());
+                        }
+                        rc.advance(p, scales);
+                    }
+                }
+                __syncwarp();
+                const uint32_t used = st.pb - s0, cap = sz - s0;
+                const bool good = __all_sync(kFullMask, st.x == kRansL) && used <= cap && cap - used <= 14;
+                if (!good && lane == 0) atomicOr(&g_status, int(EP_DEV_CORRUPT_TILE));
+            }
+            if (sp.ordered) seq_done(sp, L, tile);  // bad tiles too: nothing may wait for them in vain
+            if (!early && nsz && nsz <= kRingBytes) {
+                __syncwarp();
+                copy_tile(ring_base, nsrc, nsz, lane);
+                cp_async_commit();
+                pending = 1;
+            }
+            place = early ? nplace : 0u;
+            cur = nxt;
+            co = no;
+            nxt = aft;
+            no = pos_offs(sp, aft);
+        }
+        // Done with layer L. The last of the CTA's warps to get here refills the window with layer
+        // L + kWindows, once every warp's reads of it are ordered before the copy.
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence_block();
+            if (atomicAdd(done_cnt + s, 1u) == 31u) {
+                __threadfence_block();
+                done_cnt[s] = 0;
+                if (L + kWindows < n) {
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    load_window(sp, L + kWindows, t0, ts, bars + 8 * s);
+                }
+            }
+        }
+    }
+    if (pending) cp_async_wait<0>();
+}
+
 }  // namespace v2
 
 
@@ -1585,6 +1960,7 @@ struct DeviceInfo {
     int sms = 0;
     bool configured[8] = {false};     // version 1 kernels, by mode
     bool configured_v2[8] = {false};  // version 2 kernels, by mode
+    bool configured_seq[8] = {false}; // version 2 sequence kernels, by mode
 };
 std::mutex g_dev_mu;
 DeviceInfo g_dev[64];
@@ -1709,6 +2085,137 @@ extern "C" ep_status ep_decompress_into(const uint8_t* host_hdr, const void* dev
     return launch_decode(host_hdr, dev_blob, blob_bytes, dst, dst_bytes, h.dtype, cuda_stream, false);
 }
 
+// ep_decompress_many of version-2 blobs with one output type: prep_tables_kernel, then seq_kernel (see there),
+// for up to kMaxSeqLayers blobs a launch pair; longer sequences take several pairs, in stream order. Returns
+// EP_ERR_NOMEM, having launched nothing, when the stream-ordered scratch cannot be had.
+template <int MODE>
+ep_status decompress_seq(int count, const uint8_t* const* host_hdrs, const void* const* dev_blobs, void* const* dsts,
+                         cudaStream_t stream, int device) {
+    using dev::v2::LayerDesc;
+    using dev::v2::SeqParams;
+    {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        bool& configured = g_dev[device].configured_seq[MODE];
+        if (!configured) {
+            cudaError_t e = cudaFuncSetAttribute(dev::v2::seq_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 int(dev::v2::kSeqSmemBytes));
+            if (e != cudaSuccess) return fail(EP_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+            configured = true;
+        }
+    }
+    auto sp = std::make_unique<SeqParams>();
+    for (int c0 = 0; c0 < count; c0 += int(dev::v2::kMaxSeqLayers)) {
+        const int n = std::min(count - c0, int(dev::v2::kMaxSeqLayers));
+        std::memset(sp.get(), 0, sizeof(SeqParams));
+        sp->count = uint32_t(n);
+        sp->k2 = 2;
+        sp->k4 = 4;
+        sp->kneg256 = 0xFFFFFF00u;
+        std::vector<uint64_t> lo(static_cast<size_t>(n)), hi(static_cast<size_t>(n));
+        uint32_t tiles = 0, words = 0;
+        for (int i = 0; i < n; ++i) {
+            Header h;
+            parse_header(host_hdrs[c0 + i], h);
+            LayerDesc& d = sp->L[i];
+            d.blob = static_cast<const uint8_t*>(dev_blobs[c0 + i]);
+            d.dst = dsts[c0 + i];
+            d.payload_bytes = h.total - h.off_payload;
+            d.gpr = h.N / 8;
+            d.T = h.T;
+            d.G = uint32_t(h.G);
+            d.NG = uint32_t(h.groups());
+            d.M = h.M;
+            d.r = h.r;
+            d.alpha = h.alpha;
+            d.inv_alpha = 1.0f / h.alpha;  // IEEE binary32 division: RN(1 / alpha)
+            d.off_scales = h.off_scales;
+            d.off_offsets = h.off_offsets;
+            d.off_payload = h.off_payload;
+            d.off_tables = h.off_tables;
+            d.tables_len = h.off_offsets - h.off_tables;
+            d.tile0 = tiles;
+            d.bits = words;
+            tiles += h.T;
+            words += (h.T + 31) / 32;
+            lo[size_t(i)] = reinterpret_cast<uint64_t>(d.dst);
+            hi[size_t(i)] = lo[size_t(i)] + uint64_t(h.M) * h.N * uint64_t(elem_bytes(h.dtype));
+            // The latest earlier writer of each byte of this layer's output: split the range by going back
+            // through the layers; a writer's pieces merge into their hull (waiting for a few more of its tiles
+            // is harmless). The two latest writers are waited for tile by tile, older ones as whole layers.
+            d.seg_layer[0] = d.seg_layer[1] = dev::v2::kNoDep;
+            const uint64_t gb = 8 * uint64_t(elem_bytes(h.dtype));
+            std::vector<std::pair<uint64_t, uint64_t>> open{{lo[size_t(i)], hi[size_t(i)]}};
+            int nd = 0;
+            for (int j = i - 1; j >= 0 && hi[size_t(i)] > lo[size_t(i)] && !open.empty(); --j) {
+                if (hi[size_t(j)] <= lo[size_t(j)]) continue;
+                std::vector<std::pair<uint64_t, uint64_t>> rest;
+                uint64_t a0 = ~0ull, b0 = 0;
+                for (const auto& u : open) {
+                    const uint64_t a = std::max(u.first, lo[size_t(j)]), b = std::min(u.second, hi[size_t(j)]);
+                    if (a >= b) {
+                        rest.push_back(u);
+                        continue;
+                    }
+                    a0 = std::min(a0, a);
+                    b0 = std::max(b0, b);
+                    if (u.first < a) rest.emplace_back(u.first, a);
+                    if (b < u.second) rest.emplace_back(b, u.second);
+                }
+                open.swap(rest);
+                if (b0 == 0) continue;
+                if (nd < 2) {
+                    d.seg_layer[nd] = uint16_t(j);
+                    d.seg_lo[nd] = uint32_t((a0 - lo[size_t(i)]) / gb);
+                    d.seg_hi[nd] = uint32_t((b0 - lo[size_t(i)] + gb - 1) / gb);
+                    ++nd;
+                } else {
+                    d.need_prefix = uint32_t(j + 1);  // the latest of the older writers
+                    break;
+                }
+            }
+            if (d.need_prefix) sp->use_prefix = 1;
+            if (nd) sp->ordered = 1;
+        }
+        sp->counts_off = words;
+        sp->prefix_off = words + uint32_t(n);
+        const size_t order_words = size_t(sp->prefix_off) + 1;
+        const size_t table_bytes = size_t(n) * dev::v2::kTablesBytes;
+        cudaMemPool_t pool;
+        uint8_t* scratch = nullptr;
+        if (scratch_pool(&pool) != cudaSuccess ||
+            cudaMallocFromPoolAsync(reinterpret_cast<void**>(&scratch), table_bytes + order_words * 4, pool, stream) !=
+                cudaSuccess) {
+            cudaGetLastError();
+            return fail(EP_ERR_NOMEM, "ep_decompress_many: no stream-ordered scratch for the sequence tables");
+        }
+        sp->tables = reinterpret_cast<const uint32_t*>(scratch);
+        sp->order = reinterpret_cast<uint32_t*>(scratch + table_bytes);
+        cudaError_t e = sp->ordered ? cudaMemsetAsync(sp->order, 0, order_words * 4, stream) : cudaSuccess;
+        if (e == cudaSuccess) {
+            dev::v2::prep_tables_kernel<<<unsigned(n), dev::v2::kThreadsV2, dev::v2::kScratchSize, stream>>>(*sp);
+            e = cudaGetLastError();
+        }
+        if (e == cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(unsigned(g_dev[device].sms));
+            cfg.blockDim = dim3(dev::v2::kThreadsV2);
+            cfg.dynamicSmemBytes = dev::v2::kSeqSmemBytes;
+            cfg.stream = stream;
+            // Every CTA is resident at once: a tile may wait for a tile of another CTA.
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeCooperative;
+            attr[0].val.cooperative = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            e = cudaLaunchKernelEx(&cfg, dev::v2::seq_kernel<MODE>, *sp);
+            if (e == cudaSuccess) e = cudaGetLastError();
+        }
+        cudaFreeAsync(scratch, stream);
+        if (e != cudaSuccess) return fail(EP_ERR_CUDA, "sequence decode launch: %s", cudaGetErrorString(e));
+    }
+    return EP_OK;
+}
+
 extern "C" ep_status ep_decompress_many(int count, const uint8_t* const* host_hdrs, const void* const* dev_blobs,
                                         const size_t* blob_bytes, void* const* dsts, const size_t* dst_bytes,
                                         void* cuda_stream) {
@@ -1739,6 +2246,42 @@ extern "C" ep_status ep_decompress_many(int count, const uint8_t* const* host_hd
         }
     }
     const int n1 = int(v1.size());
+    // Version-2 blobs that share one output type: the sequence kernel, after the checks every launch makes.
+    bool one_type = count >= 2 && n1 == 0;
+    int dtype = -1;
+    for (int i = 0; one_type && i < count; ++i) {
+        Header h;
+        parse_header(host_hdrs[i], h);
+        if (dtype < 0) dtype = h.dtype;
+        one_type = h.dtype == dtype;
+        if (!dev_blobs[i] || !dsts[i]) return fail(EP_ERR_ARG, "ep_decompress_many: NULL blob or dst %d", i);
+        if ((reinterpret_cast<uintptr_t>(dev_blobs[i]) & 15) || (reinterpret_cast<uintptr_t>(dsts[i]) & 15))
+            return fail(EP_ERR_BUFFER, "ep_decompress_many: blob and dst %d must be 16-byte aligned", i);
+        const uint64_t need = uint64_t(h.M) * h.N * uint64_t(elem_bytes(h.dtype));
+        if (dst_bytes[i] < need)
+            return fail(EP_ERR_BUFFER, "ep_decompress_many: dst %d holds %zu bytes, need %llu", i, dst_bytes[i],
+                        (unsigned long long)need);
+    }
+    if (one_type) {
+        int device = 0;
+        cudaError_t e = cudaGetDevice(&device);
+        if (e != cudaSuccess || device < 0 || device >= 64) return fail(EP_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+        {
+            std::lock_guard<std::mutex> lk(g_dev_mu);
+            if (!g_dev[device].sms) {
+                e = cudaDeviceGetAttribute(&g_dev[device].sms, cudaDevAttrMultiProcessorCount, device);
+                if (e != cudaSuccess) return fail(EP_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+            }
+        }
+        switch (dtype) {
+            case dev::kBF16: return decompress_seq<dev::kBF16>(count, host_hdrs, dev_blobs, dsts, stream, device);
+            case dev::kFP16: return decompress_seq<dev::kFP16>(count, host_hdrs, dev_blobs, dsts, stream, device);
+            case dev::kFP32: return decompress_seq<dev::kFP32>(count, host_hdrs, dev_blobs, dsts, stream, device);
+            case dev::kFP8: return decompress_seq<dev::kFP8>(count, host_hdrs, dev_blobs, dsts, stream, device);
+            case dev::kINT8: return decompress_seq<dev::kINT8>(count, host_hdrs, dev_blobs, dsts, stream, device);
+        }
+        return fail(EP_ERR_DTYPE, "ep_decompress_many: unknown dtype %d", dtype);
+    }
     uint32_t* pre = nullptr;
     if (count >= 2 && n1 >= 1) {
         cudaMemPool_t pool;

@@ -62,8 +62,11 @@ typedef enum {
 /* Bits of the device status word: set by the decode kernel, read by ep_get_device_status. */
 #define EP_DEV_CORRUPT_TILE 1u  /* a tile's final rANS states or its word count did not check out */
 #define EP_DEV_BAD_OFFSETS 2u   /* a tile offset points outside the payload */
-#define EP_DEV_BAD_TABLES 4u    /* a frequency table does not sum to 4096 */
-#define EP_DEV_TABLE_COPY 8u    /* a sequence's prepared tables did not reach a CTA in time; it decoded nothing */
+#define EP_DEV_BAD_TABLES 4u    /* a frequency table does not sum to its scale (4096 in version 1, 256 in 2) */
+#define EP_DEV_TABLE_COPY 8u    /* a sequence's prepared tables did not reach a CTA in time; in version 1 it
+                                   decoded nothing, in version 2 it decoded with whatever the window held */
+#define EP_DEV_DEP_WAIT 16u     /* in a version-2 sequence, a tile waited too long for an earlier layer's tile
+                                   that writes the same bytes, and stored without it */
 
 /* Encoder options. Start from ep_options_default(). */
 typedef struct {
@@ -224,26 +227,36 @@ ep_status ep_decompress_into(const uint8_t* host_hdr, const void* dev_blob, size
 /*
  * ep_decompress_many: decodes `count` blobs in order on one stream: blob i into dsts[i], with the
  * argument rules of ep_decompress_into for each one. This is the layer-sequence form of the hot
- * path, for example all linear layers of a model before a forward pass.
+ * path, for example all linear layers of a model before a forward pass. Overlapping dsts end as if
+ * the blobs were decoded one after another in list order. One requirement follows from reads made
+ * while earlier decodes run: no blob in the list may be written by the decodes listed before it.
+ * Every header, size and alignment is checked before anything launches, so an error launches nothing.
  *
- * With two or more blobs, one expand kernel first builds every blob's fused decode tables (144 KB per
- * blob) into device scratch, taken stream-ordered from a memory pool that the library keeps per
- * device and released stream-ordered after the last decode. Each decode CTA then takes its tables
- * by bulk copies (TMA, completed on a shared-memory barrier) instead of rebuilding them. Its wait for
- * them is bounded; a copy that has not landed in time sets EP_DEV_TABLE_COPY, and that CTA decodes
- * nothing. If the scratch cannot be had, each CTA builds its own tables, as ep_decompress_into does.
+ * Two or more format-version-2 blobs of one container dtype (the usual case) take the sequence path:
+ * per group of up to 280 blobs, a table kernel builds every blob's fused tables (9 KB each) into
+ * device scratch, then one persistent kernel (one CTA per SM, launched cooperatively, so all of them
+ * are resident at once) decodes the whole group. The tiles of all the blobs are dealt round-robin as
+ * one list, so a small layer shares the GPU with the next one, and each CTA keeps four blobs' tables in
+ * shared memory, refilled by bulk copies (TMA, no multicast). When some dst overlaps an earlier one,
+ * each tile waits, before its first store, for the tiles of earlier blobs that last wrote the same
+ * bytes (per-tile done flags in the scratch, with release and acquire ordering); the waits are bounded
+ * and set EP_DEV_DEP_WAIT if they run out, and a window copy that does not land in time sets
+ * EP_DEV_TABLE_COPY. The scratch (9 KB per blob plus a bit per tile) comes stream-ordered from a pool
+ * the library keeps per device and is released stream-ordered after the group; if it cannot be had,
+ * the call returns EP_ERR_NOMEM with nothing of that group launched (earlier groups stay queued).
  *
- * The first decode is ordered after earlier work on the stream, the expand kernel included, as
- * usual. Each later decode is a programmatic dependent launch of the one before it: it may load
- * its tables, prefetch its first tiles, pull the next blob's metadata into L2 and decode each
- * warp's first round while the previous decode drains, and it stores nothing until that decode has
- * finished. Overlapping dsts are therefore written in order. One requirement follows from the early
- * reads: no blob in the list may be written by the decodes listed before it.
- * Every header is validated before anything launches, so an error launches nothing.
- * Errors: as ep_decompress_into, for the first failing blob.
+ * Other lists (any version-1 blob, or mixed dtypes) launch one decode per blob. With two or more blobs,
+ * an expand kernel first builds every version-1 blob's tables (144 KB each) into the same kind of
+ * scratch, and those decodes take them by bulk copies; a copy that has not landed in time sets
+ * EP_DEV_TABLE_COPY and that CTA decodes nothing. If the scratch cannot be had, each CTA builds its own
+ * tables. The first decode is ordered after earlier work on the stream as usual; each later one is a
+ * programmatic dependent launch of the one before it that stores nothing until that decode has
+ * finished.
+ *
+ * Errors: as ep_decompress_into, for the first failing blob; EP_ERR_NOMEM as above.
  * Test hook: with the environment variable EPK_TEST_TABLE_COPY_TIMEOUT set to 1 when the call is made,
- * the table copies are not issued, so every CTA's bounded wait runs out (each poll suspends about
- * 1 us, 2^14 polls twice) and EP_DEV_TABLE_COPY is set. The test suite uses it to check that path.
+ * the version-1 table copies are not issued, so every CTA's bounded wait runs out (each poll suspends
+ * about 1 us, 2^14 polls twice) and EP_DEV_TABLE_COPY is set. The test suite uses it to check that path.
  */
 ep_status ep_decompress_many(int count, const uint8_t* const* host_hdrs, const void* const* dev_blobs,
                              const size_t* blob_bytes, void* const* dsts, const size_t* dst_bytes,

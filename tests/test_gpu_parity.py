@@ -280,8 +280,9 @@ def test_streams_and_allocating_entry(orc):
 
 
 def test_decompress_many_matches_single_decodes(orc):
-    """The layer-sequence entry (programmatic dependent launches) gives the same bytes as one-by-one
-    decodes. The last output is one buffer shared by several layers, written in list order."""
+    """The layer-sequence entry in its launch-per-blob form (the list mixes format versions and dtypes)
+    gives the same bytes as one-by-one decodes. The last output is one buffer shared by several layers,
+    written in list order."""
     comps = [ep.compress(synth.dit_layer(i, shape=shp), 4.0)
              for i, shp in enumerate([(384, 256), (1024, 512), (64, 3840), (3840, 64), (1536, 256)])]
     comps.append(ep.compress(synth.fp8_codes(256, 512, seed=5), 5.0))
@@ -390,8 +391,8 @@ def test_decompress_many_edge_counts(orc):
 @pytest.mark.slow
 def test_full_276_layer_sequence_sampled(orc):
     """The benchmark's launch configuration at full size: all 276 DiT-like layers (6.17 G parameters at
-    4 bpp, CUDA encoder) decoded by one ep_decompress_many (tables prepared once, chained launches), each
-    layer into its own buffer. The first, a middle and the last (ragged) tile of every layer are compared
+    4 bpp, CUDA encoder) decoded by one ep_decompress_many (the sequence kernel: one launch for all the
+    layers), each layer into its own buffer. The first, a middle and the last (ragged) tile of every layer are compared
     with the oracle's decode of the same tiles."""
     import concurrent.futures as cf
     shapes = synth.dit_layer_shapes()
@@ -426,3 +427,109 @@ def test_full_276_layer_sequence_sampled(orc):
         for i, want, mask in ex.map(one, range(len(shapes))):
             got = gpu_bits(outs[i])
             assert np.array_equal(got[mask], want[mask]), f"layer {i}"
+
+
+def test_version2_sequence_into_one_buffer_keeps_write_order(orc):
+    """The sequence kernel orders its layers tile by tile: each tile waits only for the tiles of earlier layers
+    that last wrote its bytes. Layers of mixed sizes decoded into one shared buffer (a small one between two large ones, so
+    that a later layer overwrites a region the layer before it left alone) must leave, at every byte, the value
+    of the last layer that wrote it. The expected buffer is assembled on the host from the oracle's decodes."""
+    shapes = [(1024, 768), (96, 256), (768, 512), (64, 3840), (1536, 256), (256, 256), (1024, 640)]
+    comps = [ep.compress(synth.dit_layer(60 + i, shape=s), ep.EntroPackLossyConfig(3.0 + 0.5 * (i % 3)))
+             for i, s in enumerate(shapes)]
+    assert all(int.from_bytes(c.blob[4:6], "little") == 2 for c in comps)
+    total = max(M * N for M, N in shapes)
+    shared = torch.zeros(total, dtype=torch.bfloat16, device="cuda")
+    views = [shared[: M * N].view(M, N) for M, N in shapes]
+    want = np.zeros(total, np.uint16)
+    for c in comps:
+        d = orc.decompress(c.blob).reshape(-1)
+        want[: d.size] = d
+    for _ in range(3):
+        shared.zero_()
+        ep.decompress_many(list(zip(comps, views)))
+        torch.cuda.synchronize()
+        status_clean()
+        assert np.array_equal(gpu_bits(shared), want)
+
+
+def _bits_any(t):
+    b = gpu_bits(t)
+    return b.view(np.uint32) if b.dtype == np.float32 else b
+
+
+def _want_any(orc, c):
+    w = orc.decompress(c.blob)
+    return w.view(np.uint32) if w.dtype == np.float32 else w
+
+
+@pytest.mark.parametrize("kind", ["bf16", "fp16", "fp32", "fp8", "int8"])
+def test_sequence_kernel_every_dtype(orc, kind):
+    """A list of version-2 blobs of one container dtype runs as the sequence kernel; layers of assorted
+    shapes (one tile up to several per CTA, ragged last tiles, r = 0 and r > 0) all match the oracle."""
+    if kind == "fp8":
+        comps = [ep.compress(synth.fp8_codes(64 + 16 * i, 512, seed=i), 5.0) for i in range(6)]
+    elif kind == "int8":
+        comps = [ep.compress(synth.int8_codes(64 + 8 * i, 256, seed=i), 3.0) for i in range(6)]
+    else:
+        comps = [ep.compress(synth.gaussian(8 + 37 * i % 300, 8 * (1 + i % 40), seed=i, container=kind), 2.0 + i % 6)
+                 for i in range(12)]
+        comps.append(ep.compress(synth.gaussian(200, 96, seed=99, container=kind), 9.0))  # raw low bits (r > 0)
+    outs = [torch.empty(c.shape, dtype=c.dtype, device="cuda") for c in comps]
+    for _ in range(2):
+        ep.decompress_many(list(zip(comps, outs)))
+    torch.cuda.synchronize()
+    status_clean()
+    for c, o in zip(comps, outs):
+        assert np.array_equal(_bits_any(o), _want_any(orc, c))
+
+
+def test_sequence_kernel_two_launch_groups(orc):
+    """330 small layers: more than one sequence launch takes (280), so two groups run in stream order. Into
+    separate outputs, then all into one buffer, where every element holds the last layer that wrote it."""
+    comps = [ep.compress(synth.gaussian(1 + (i * 7) % 23, 8 * (1 + (i * 5) % 9), seed=2000 + i, container="bf16"),
+                         1.0 + i % 9) for i in range(330)]
+    outs = [torch.empty(c.shape, dtype=c.dtype, device="cuda") for c in comps]
+    ep.decompress_many(list(zip(comps, outs)))
+    torch.cuda.synchronize()
+    status_clean()
+    dec = [_want_any(orc, c) for c in comps]
+    for d, o in zip(dec, outs):
+        assert np.array_equal(gpu_bits(o), d)
+    mx = max(c.shape[0] * c.shape[1] for c in comps)
+    buf = torch.zeros(mx, dtype=torch.bfloat16, device="cuda")
+    want = np.zeros(mx, np.uint16)
+    for d in dec:
+        want[: d.size] = d.reshape(-1)
+    ep.decompress_many([(c, buf[: c.shape[0] * c.shape[1]].view(c.shape)) for c in comps])
+    torch.cuda.synchronize()
+    status_clean()
+    assert np.array_equal(gpu_bits(buf), want)
+
+
+@pytest.mark.parametrize("layout", ["one", "ping_pong", "offset"])
+def test_sequence_kernel_overlapping_outputs(orc, layout):
+    """Layers of mixed sizes (up to 14.7 M parameters) written into shared buffers: all into one, alternating
+    between two, or into one at staggered offsets, so that a layer overwrites parts of several earlier ones.
+    Each buffer must end as list-order decoding leaves it; run three times."""
+    shapes = [(1024, 768), (96, 256), (768, 512), (64, 3840), (1536, 256), (256, 256), (1024, 640), (15360, 256),
+              (3840, 3840), (2048, 512)]
+    comps = [ep.compress(synth.dit_layer(60 + i, shape=s), 3.0 + 0.5 * (i % 3)) for i, s in enumerate(shapes)]
+    dec = [_want_any(orc, c).reshape(-1) for c in comps]
+    mx = max(M * N for M, N in shapes)
+    bufs = [torch.zeros(mx + 4096, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    wants = [np.zeros(mx + 4096, np.uint16) for _ in range(2)]
+    pairs = []
+    for i, (c, (M, N)) in enumerate(zip(comps, shapes)):
+        b = i % 2 if layout == "ping_pong" else 0
+        off = (i * 1032) % 4096 // 8 * 8 if layout == "offset" else 0
+        pairs.append((c, bufs[b][off: off + M * N].view(M, N)))
+        wants[b][off: off + M * N] = dec[i]
+    for _ in range(3):
+        for b in bufs:
+            b.zero_()
+        ep.decompress_many(pairs)
+        torch.cuda.synchronize()
+        status_clean()
+        for b, w in zip(bufs, wants):
+            assert np.array_equal(gpu_bits(b), w)
