@@ -1401,12 +1401,15 @@ __device__ __forceinline__ uint32_t fast_rounds_v2(const P& p, const K& kc, uint
                 ++ri;
             }
         }
-        for (; k < Rf; ++k, g += 32) {
-            round_fast_v2<MODE, false, ESC>(p, kc, t0, ts, x, pa, g, lt_mask, __shfl_sync(kFullMask, cvec, ri), kc.k2);
-            if (++kr == rpr) {
-                kr = 0;
-                ++ri;
-            }
+        // Row by row: the factor is taken once per row, and the inner loop only counts rounds.
+        while (k < Rf) {
+            const uint32_t run = min(rpr - kr, Rf - k);
+            const float c = __shfl_sync(kFullMask, cvec, ri);
+            const uint32_t gend = g + 32 * run;
+            for (; g != gend; g += 32) round_fast_v2<MODE, false, ESC>(p, kc, t0, ts, x, pa, g, lt_mask, c, kc.k2);
+            k += run;
+            kr = 0;
+            ++ri;
         }
     } else {
         if (!waited && Rf > 0) {
