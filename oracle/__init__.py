@@ -21,6 +21,7 @@ import numpy as np
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "liboracle.so")
 SRC_PATH = os.path.join(HERE, "entropack_oracle.c")
+SOURCES = [SRC_PATH, os.path.join(HERE, "tileans_oracle.c")]
 
 DTYPES = {"bf16": 1, "fp16": 2, "fp32": 3, "fp8_e4m3": 4, "int8": 5}
 ELEM = {1: 2, 2: 2, 3: 4, 4: 1, 5: 1}
@@ -29,9 +30,10 @@ NP_CONTAINER = {1: np.uint16, 2: np.uint16, 3: np.float32, 4: np.uint8, 5: np.in
 
 def build(force: bool = False) -> str:
     """Compile the oracle with gcc (-O2, no FMA contraction)."""
-    if force or not os.path.exists(LIB_PATH) or os.path.getmtime(LIB_PATH) < os.path.getmtime(SRC_PATH):
+    newest = max(os.path.getmtime(f) for f in SOURCES + [os.path.join(HERE, "entropack_oracle.h")])
+    if force or not os.path.exists(LIB_PATH) or os.path.getmtime(LIB_PATH) < newest:
         cmd = ["gcc", "-O2", "-std=c11", "-Wall", "-ffp-contract=off", "-fPIC", "-shared",
-               SRC_PATH, "-o", LIB_PATH, "-lm"]
+               *SOURCES, "-o", LIB_PATH, "-lm"]
         subprocess.run(cmd, check=True)
     return LIB_PATH
 
@@ -65,6 +67,12 @@ def lib():
         L.orc_decompress.argtypes = [c.c_void_p, c.c_size_t, c.c_void_p, c.c_void_p]
         L.orc_quantize.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_float, c.c_void_p,
                                    c.c_void_p]
+        L.orc_tans_compress.argtypes = [c.c_void_p, c.c_int, c.c_int, c.c_void_p, c.c_int, c.POINTER(c.c_void_p),
+                                        c.POINTER(c.c_size_t)]
+        L.orc_tans_info.argtypes = [c.c_void_p, c.c_size_t, c.POINTER(c.c_int), c.POINTER(c.c_int), c.c_void_p,
+                                    c.POINTER(c.c_int), c.POINTER(c.c_uint32), c.POINTER(c.c_int)]
+        L.orc_tans_decode_tiles.argtypes = [c.c_void_p, c.c_size_t, c.c_uint32, c.c_uint32, c.c_void_p]
+        L.orc_tans_decompress.argtypes = [c.c_void_p, c.c_size_t, c.c_void_p]
         _lib = L
     return _lib
 
@@ -182,3 +190,49 @@ def quantize(data: np.ndarray, dtype: int, alpha: float) -> tuple[np.ndarray, np
     s = np.zeros(M, np.uint16)
     _check(lib().orc_quantize(_ptr(a), dtype, M, N, float(alpha), _ptr(z), _ptr(s)), "quantize")
     return z, s
+
+
+# ------------------------------------------------------------------ lossless tile-ANS (EPL1)
+
+TANS_NP = {1: np.uint16, 2: np.uint16, 3: np.uint32, 4: np.uint8, 5: np.uint8}
+
+
+def tans_compress(bits: np.ndarray, dtype: int, K: int = 0) -> bytes:
+    """Lossless tile-ANS blob of an array of raw bit patterns (``TANS_NP[dtype]``; any shape, ndim <= 8)."""
+    a = np.asarray(bits)
+    if not a.flags.c_contiguous:
+        a = a.copy(order="C")  # (np.ascontiguousarray would turn a 0-d array into a 1-d one)
+    if a.dtype != TANS_NP[dtype]:
+        raise ValueError("tans_compress: bits must hold the dtype's raw patterns")
+    dims = (ctypes.c_int64 * max(1, a.ndim))(*a.shape)
+    p, n = ctypes.c_void_p(), ctypes.c_size_t()
+    _check(lib().orc_tans_compress(a.ctypes.data if a.size else None, dtype, a.ndim, dims, K, ctypes.byref(p),
+                                   ctypes.byref(n)), "tans_compress")
+    try:
+        return ctypes.string_at(p.value, n.value)
+    finally:
+        lib().orc_free(p)
+
+
+def tans_info(blob: bytes) -> dict:
+    c = ctypes
+    dt, nd, K, T, mask = c.c_int(), c.c_int(), c.c_int(), c.c_uint32(), c.c_int()
+    dims = (c.c_int64 * 8)()
+    _check(lib().orc_tans_info(blob, len(blob), c.byref(dt), c.byref(nd), dims, c.byref(K), c.byref(T),
+                               c.byref(mask)), "tans_info")
+    return {"dtype": dt.value, "shape": tuple(dims[i] for i in range(nd.value)), "K": K.value,
+            "num_tiles": T.value, "coded_mask": mask.value}
+
+
+def tans_decompress(blob: bytes) -> np.ndarray:
+    """The raw bit patterns, in the blob's shape."""
+    info = tans_info(blob)
+    out = np.zeros(info["shape"], TANS_NP[info["dtype"]])
+    _check(lib().orc_tans_decompress(blob, len(blob), out.ctypes.data if out.size else None), "tans_decompress")
+    return out
+
+
+def tans_decode_tiles(blob: bytes, t0: int, t1: int, out: np.ndarray) -> None:
+    """Decode tiles [t0, t1) into ``out`` (the whole tensor's array of raw bit patterns)."""
+    _check(lib().orc_tans_decode_tiles(blob, len(blob), t0, t1, out.ctypes.data if out.size else None),
+           "tans_decode_tiles")

@@ -1,5 +1,6 @@
 /*
- * EntroPack oracle — plain, slow CPU encoder and decoder of the EPK1 blob.
+ * EntroPack oracle — plain, slow CPU encoders and decoders of the EPK1 (lossy) and EPL1 (lossless
+ * tile-ANS) blobs.
  *
  * TEST INFRASTRUCTURE, NOT PRODUCT CODE. The test suite, the smoke check and
  * the benchmark's CPU-baseline leg are its only users; the product library
@@ -64,6 +65,19 @@ int orc_decompress(const uint8_t* blob, size_t bytes, void* dst, int32_t* zout);
  * point per coordinate, scales_out[M] = bf16 bits of s_row. */
 int orc_quantize(const void* data, int dtype, int64_t M, int64_t N, float alpha, int32_t* zout,
                  uint16_t* scales_out);
+
+/* Lossless tile-ANS (EPL1 blob, tileans_oracle.c). data: numel = prod(dims) elements of the dtype's
+ * size, read as raw bit patterns; ndim 0..8 (ndim 0 is one element). K: elements per lane per tile,
+ * 1..1024, or 0 for 128. The blob is malloc'd; release it with orc_free. */
+int orc_tans_compress(const void* data, int dtype, int ndim, const int64_t* dims, int K, uint8_t** blob,
+                      size_t* bytes);
+/* Full validation (header, tables, offsets, CRC) and the header fields; dims receives ndim values. */
+int orc_tans_info(const uint8_t* blob, size_t bytes, int* dtype, int* ndim, int64_t* dims, int* K, uint32_t* T,
+                  int* coded_mask);
+/* Decode tiles [t0, t1) into dst (the whole tensor's buffer; only those tiles' elements are written). */
+int orc_tans_decode_tiles(const uint8_t* blob, size_t bytes, uint32_t t0, uint32_t t1, void* dst);
+/* Decode every tile. */
+int orc_tans_decompress(const uint8_t* blob, size_t bytes, void* dst);
 
 #ifdef __cplusplus
 }
