@@ -66,7 +66,8 @@ def parse_args():
     ap.add_argument("--workload", default="dit276_bf16_4bpp",
                     choices=["dit276_bf16_4bpp", "quickstart256_bf16_3.5bpp", "lognormal3072_bf16_4bpp", "sweep4096",
                              "fp8_8192x28672_5bpp", "int8_8192x28672_3bpp", "dit276_gemm_overhead",
-                             "dit276_fp8_gemm_overhead", "dit276_mixed_2.3bpp", "cuda_encode_gate_10240x3840"],
+                             "dit276_fp8_gemm_overhead", "dit276_mixed_2.3bpp", "cuda_encode_gate_10240x3840",
+                             "tileans_lossless"],
                     help="the default is the headline line; the others print one line per tensor")
     return ap.parse_args()
 
@@ -646,6 +647,104 @@ def oracle_rate(blob, shape, seconds, workers):
     return done / (time.perf_counter() - t0)
 
 
+def tans_items():
+    """(label, tensor factory) for the lossless tile-ANS workload: weights of the lossy workloads' recipes,
+    in shapes that are not 2-D where the recipe allows it."""
+    return [
+        ("tans_bf16_4x4096x4096", lambda: synth.gaussian(4 * 4096, 4096, seed=31, container="bf16").view(4, 4096, 4096)),
+        ("tans_fp16_64x1024x1024", lambda: synth.gaussian(64 * 1024, 1024, seed=32, container="fp16").view(64, 1024, 1024)),
+        ("tans_fp32_8192x8192", lambda: synth.gaussian(8192, 8192, seed=33, container="fp32")),
+        ("tans_fp8_8192x28672", lambda: synth.fp8_codes(8192, 28672, seed=3)),
+        ("tans_int8_8192x28672", lambda: synth.int8_codes(8192, 28672, seed=4)),
+    ]
+
+
+def run_tans(args):
+    """One JSON line per tensor of the lossless tile-ANS workload. A step is one ep_tans_decompress_into of the
+    tensor, with a 256 MB write between steps that flushes the 126 MB L2; value = elements / median step
+    time. The line also carries the compression ratio, the host encoder's time and the oracle's decode rate
+    on a sample of tiles."""
+    import decode_ep_b200 as ep
+    import oracle
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    L = ep.lib()
+    stream = torch.cuda.current_stream(device)
+    sptr = stream.cuda_stream
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    peak, peak_kind = measured_hbm_peak()
+    lines = []
+    for label, make in tans_items():
+        w = make()
+        t_enc = time.perf_counter()
+        c = ep.compress(w, ep.TileANSConfig())
+        t_enc = time.perf_counter() - t_enc
+        n = w.numel()
+        d = c.device_blob(device)
+        out = torch.empty(w.shape, dtype=w.dtype, device=device)
+        out_bytes = n * out.element_size()
+
+        def launch():
+            st = L.ep_tans_decompress_into(c.header, d.data_ptr(), len(c.blob), out.data_ptr(), out_bytes, sptr)
+            if st:
+                raise RuntimeError(L.ep_last_error().decode())
+
+        for _ in range(args.warmup):
+            launch()
+        torch.cuda.synchronize(device)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        with ClockSampler(local) as clk:
+            for a, b in evs:
+                flush.fill_(1)
+                a.record(stream)
+                launch()
+                b.record(stream)
+            torch.cuda.synchronize(device)
+        times = sorted(a.elapsed_time(b) for a, b in evs)
+        med, best = statistics.median(times), times[0]
+        if ep.device_status(stream):
+            raise RuntimeError(f"{label}: device status set")
+        exact = bool(torch.equal(out.cpu().view(torch.uint8), w.contiguous().view(torch.uint8)))
+        alg = len(c.blob) + out_bytes
+        achieved = alg / (med * 1e-3) / 1e9
+        cpu = None
+        if rank == 0 and not args.no_cpu_baseline:
+            oracle.build()
+            info = oracle.tans_info(c.blob)
+            T = info["num_tiles"]
+            host = np.zeros(tuple(w.shape), oracle.TANS_NP[info["dtype"]])
+            runs = [(t, min(T, t + 16)) for t in range(0, T, 16)]
+            cores = os.cpu_count() or 1
+            done, k, t0 = 0, 0, time.perf_counter()
+            with cf.ThreadPoolExecutor(max_workers=cores) as ex:
+                while time.perf_counter() - t0 < args.cpu_seconds / 4:
+                    batch = [runs[(k + j) % len(runs)] for j in range(2 * cores)]
+                    k += len(batch)
+                    list(ex.map(lambda r: oracle.tans_decode_tiles(c.blob, r[0], r[1], host), batch))
+                    done += sum(min(r[1] * 4096, n) - r[0] * 4096 for r in batch)
+            cpu = {"value": round(done / (time.perf_counter() - t0) / 1e9, 5), "unit": "Gelements/s", "cores": cores,
+                   "kind": "oracle", "sample": f"runs of 16 tiles of this blob, cycled, C oracle for "
+                                               f"{args.cpu_seconds / 4:.1f} s on {cores} threads"}
+        lines.append({
+            "metric": "lossless tile-ANS decode Gelements/s on 1 B200", "value": round(n / (med * 1e-3) / 1e9, 3),
+            "unit": "Gelements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(med, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "u8 planes", "data": "synthetic",
+            "config": {"workload": label, "shape": list(w.shape), "container": str(w.dtype).replace("torch.", ""),
+                       "elements": n, "blob_bytes": len(c.blob), "bits_per_element": round(8 * len(c.blob) / n, 4),
+                       "ratio": round(out_bytes / len(c.blob), 4), "coded_planes_mask": ep.blob_info(c.blob)["coded_mask"],
+                       "bit_exact": exact, "best_ms": round(best, 5), "host_encode_s": round(t_enc, 3),
+                       "l2": "flushed between steps (256 MB write)"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": None, "peak_source": f"{peak_kind} copy bandwidth",
+                         "per_launch_algorithmic_bytes": alg, "duration_source": "median of the timed launches"},
+            "cpu_baseline": cpu, "e2e": None, "clocks": clk.summary(), "gpu_launches": args.steps,
+        })
+        del w, out, d
+    return lines
+
+
 def run_gemm_overhead(args, tokens=4096, fp8=False):
     """Decode overhead against the layer GEMMs of a prefill-sized forward pass, through the library's
     CompressedLinear layers (the pages measure it as the denoising-step time with compressed vs BF16 weights;
@@ -1035,6 +1134,8 @@ def main():
         lines = [run_ours(args)]
     elif args.workload == "cuda_encode_gate_10240x3840":
         lines = [run_cuda_encode_gate(args)]
+    elif args.workload == "tileans_lossless":
+        lines = run_tans(args)
     else:
         lines = run_workload(args)
     for line in lines or []:

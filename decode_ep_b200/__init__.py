@@ -25,7 +25,7 @@ import torch
 
 from . import build as _build
 
-__all__ = ["EntroPackLossyConfig", "CompressedTensor", "EntroPackError", "LayerBatch", "compress", "decompress",
+__all__ = ["EntroPackLossyConfig", "TileANSConfig", "CompressedTensor", "EntroPackError", "LayerBatch", "compress", "decompress",
            "decompress_into", "decompress_many", "decode_coords", "device_status", "blob_info", "plan_bitrates", "lib",
            "CompressedLinear", "DecodeWorkspace", "link_prefetch"]
 
@@ -34,6 +34,7 @@ _TORCH_TO_EP = {torch.bfloat16: EP_BF16, torch.float16: EP_FP16, torch.float32: 
                 torch.float8_e4m3fn: EP_FP8_E4M3, torch.int8: EP_INT8}
 _EP_TO_TORCH = {v: k for k, v in _TORCH_TO_EP.items()}
 HEADER_BYTES = 64
+TANS_HEADER_BYTES = 96  # lossless tile-ANS (EPL1) blobs
 
 
 class EntroPackError(RuntimeError):
@@ -95,8 +96,14 @@ def _load() -> None:
     L.ep_status_string.restype = c.c_char_p
     L.ep_status_string.argtypes = [c.c_int]
     L.ep_last_error.restype = c.c_char_p
+    L.ep_tans_compress.argtypes = [c.c_void_p, c.c_int, c.c_int, c.c_void_p, c.c_uint32, c.c_int,
+                                   c.POINTER(c.c_void_p), c.POINTER(c.c_size_t)]
+    L.ep_tans_info.argtypes = [c.c_void_p, c.c_size_t, c.POINTER(c.c_int), c.POINTER(c.c_int), c.c_void_p,
+                               c.POINTER(c.c_uint32), c.POINTER(c.c_uint32)]
+    L.ep_tans_decompress_into.argtypes = [c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p, c.c_size_t, c.c_void_p]
     for name in ("ep_compress", "ep_compress_cuda", "ep_blob_info", "ep_decompress_into", "ep_decode_coords_into", "ep_decompress",
-                 "ep_get_device_status", "ep_decompress_many", "ep_plan_bitrates"):
+                 "ep_get_device_status", "ep_decompress_many", "ep_plan_bitrates", "ep_tans_compress", "ep_tans_info",
+                 "ep_tans_decompress_into"):
         getattr(L, name).restype = c.c_int
     _lib = L
 
@@ -136,6 +143,17 @@ class EntroPackLossyConfig:
 
 
 @dataclass
+class TileANSConfig:
+    """Lossless tile-ANS (README, Config table: TileANSConfig): exact restoration of BF16, FP16, FP32, FP8 and
+    INT8 tensors of any shape (up to 8 dimensions); the ratio depends on the data. The elements' bytes are
+    split into planes; clustered planes (sign and exponent bytes) are rANS-coded, the others stored as they
+    are. elems_per_lane: K, a tile holds 32 x K elements (0 means 128). threads: host encoder threads (0: all
+    cores)."""
+    elems_per_lane: int = 0
+    threads: int = 0
+
+
+@dataclass
 class CompressedTensor:
     """A compressed 2-D tensor: the blob bytes plus a cached device copy per CUDA device."""
     blob: bytes
@@ -145,8 +163,12 @@ class CompressedTensor:
     _device_blobs: dict = field(default_factory=dict, repr=False)
 
     @property
+    def lossless(self) -> bool:
+        return self.blob[:4] == b"EPL1"
+
+    @property
     def header(self) -> bytes:
-        return self.blob[:HEADER_BYTES]
+        return self.blob[:TANS_HEADER_BYTES if self.lossless else HEADER_BYTES]
 
     @property
     def compressed_bits(self) -> int:
@@ -168,20 +190,54 @@ class CompressedTensor:
     @staticmethod
     def from_blob(blob: bytes) -> "CompressedTensor":
         info = blob_info(blob)
-        return CompressedTensor(bytes(blob), (info["rows"], info["cols"]), _EP_TO_TORCH[info["dtype"]],
-                                info["actual_bpp"])
+        return CompressedTensor(bytes(blob), info["shape"], _EP_TO_TORCH[info["dtype"]], info["actual_bpp"])
 
 
 def blob_info(blob: bytes) -> dict:
-    """Full host validation of a blob (header, tables, offsets, CRC) and its description."""
+    """Full host validation of a blob (header, tables, offsets, CRC) and its description. Lossy (EPK1) and
+    lossless (EPL1) blobs both give dtype, shape and actual_bpp; lossy ones also rows and cols, lossless
+    ones coded_mask (bit j: byte plane j is rANS-coded) and elems_per_lane."""
     c = ctypes
+    if bytes(blob[:4]) == b"EPL1":
+        dt, nd, mask, K = c.c_int(), c.c_int(), c.c_uint32(), c.c_uint32()
+        dims = (c.c_int64 * 8)()
+        _check(lib().ep_tans_info(blob, len(blob), c.byref(dt), c.byref(nd), dims, c.byref(mask), c.byref(K)),
+               "blob_info")
+        shape = tuple(dims[i] for i in range(nd.value))
+        numel = math.prod(shape)
+        return {"dtype": dt.value, "shape": shape, "coded_mask": mask.value, "elems_per_lane": K.value,
+                "actual_bpp": 8 * len(blob) / numel if numel else 0.0}
     dt, M, N, bpp = c.c_int(), c.c_int64(), c.c_int64(), c.c_double()
     _check(lib().ep_blob_info(blob, len(blob), c.byref(dt), c.byref(M), c.byref(N), c.byref(bpp)), "blob_info")
-    return {"dtype": dt.value, "rows": M.value, "cols": N.value, "actual_bpp": bpp.value}
+    return {"dtype": dt.value, "rows": M.value, "cols": N.value, "shape": (M.value, N.value),
+            "actual_bpp": bpp.value}
 
 
-def compress(tensor: torch.Tensor, config: EntroPackLossyConfig | float) -> CompressedTensor:
-    """Lossy compression of a 2-D tensor (CPU or CUDA). The library runs rate control and encoding."""
+def _compress_lossless(tensor: torch.Tensor, config: TileANSConfig) -> CompressedTensor:
+    if tensor.dtype not in _TORCH_TO_EP:
+        raise EntroPackError(-2, f"compress: unsupported dtype {tensor.dtype}")
+    if tensor.dim() > 8:
+        raise EntroPackError(-3, "compress: tile-ANS takes tensors of at most 8 dimensions")
+    host = tensor.detach().contiguous().cpu()
+    dims = (ctypes.c_int64 * max(1, host.dim()))(*host.shape)
+    blob_p, nbytes = ctypes.c_void_p(), ctypes.c_size_t()
+    _check(lib().ep_tans_compress(host.data_ptr() if host.numel() else None, _TORCH_TO_EP[host.dtype], host.dim(),
+                                  dims, int(config.elems_per_lane), int(config.threads), ctypes.byref(blob_p),
+                                  ctypes.byref(nbytes)), "compress")
+    try:
+        blob = ctypes.string_at(blob_p.value, nbytes.value)
+    finally:
+        lib().ep_blob_free(blob_p)
+    numel = host.numel()
+    return CompressedTensor(blob, tuple(host.shape), tensor.dtype, 8 * len(blob) / numel if numel else 0.0)
+
+
+def compress(tensor: torch.Tensor, config: EntroPackLossyConfig | TileANSConfig | float) -> CompressedTensor:
+    """Compression of a tensor (CPU or CUDA). EntroPackLossyConfig (or a bare target in bits per parameter):
+    lossy, 2-D tensors; the library runs rate control and encoding. TileANSConfig: lossless, any shape, on
+    the host encoder."""
+    if isinstance(config, TileANSConfig):
+        return _compress_lossless(tensor, config)
     if not isinstance(config, EntroPackLossyConfig):
         config = EntroPackLossyConfig(float(config))
     if tensor.dim() != 2:
@@ -276,8 +332,9 @@ def decompress_into(compressed: CompressedTensor, out: torch.Tensor, stream=None
     if not out.is_cuda or not out.is_contiguous() or out.dtype != compressed.dtype:
         raise EntroPackError(-9, "decompress_into: out must be a contiguous CUDA tensor of the blob's dtype")
     dblob = compressed.device_blob(out.device)
-    _check(lib().ep_decompress_into(compressed.header, dblob.data_ptr(), len(compressed.blob), out.data_ptr(),
-                                    out.numel() * out.element_size(), _stream_ptr(stream)), "decompress_into")
+    fn = lib().ep_tans_decompress_into if compressed.lossless else lib().ep_decompress_into
+    _check(fn(compressed.header, dblob.data_ptr(), len(compressed.blob), out.data_ptr(),
+              out.numel() * out.element_size(), _stream_ptr(stream)), "decompress_into")
     return out
 
 

@@ -17,10 +17,10 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libentropack.so")
-SOURCES = ["decode.cu", "host_encoder.cpp", "capi.cpp", "plan.cpp"]
+SOURCES = ["decode.cu", "host_encoder.cpp", "capi.cpp", "plan.cpp", "tans_host.cpp"]
 # Compiled on their own with --fmad=false: the CUDA encoder must round every double operation alone.
 NOFMA_SOURCES = ["gpu_encoder.cu"]
-HEADERS = ["epk_format.h", "capi_internal.h", "encoder_common.h", "lattice_code.h"]
+HEADERS = ["epk_format.h", "capi_internal.h", "encoder_common.h", "lattice_code.h", "tans_format.h", "tans_decode.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

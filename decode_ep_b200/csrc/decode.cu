@@ -36,6 +36,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <memory>
+#include <type_traits>
 #include <mutex>
 #include <vector>
 
@@ -2372,3 +2373,7 @@ extern "C" ep_status ep_get_device_status(void* cuda_stream, int32_t* flags) {
     *flags = v;
     return EP_OK;
 }
+
+// Lossless tile-ANS decode (shares the status word and the device table above).
+#include "tans_format.h"
+#include "tans_decode.cuh"

@@ -292,6 +292,49 @@ const char* ep_status_string(ep_status st);
 /* Message for the calling thread's last failed call ("" if none). Valid until that thread's next call. */
 const char* ep_last_error(void);
 
+/*
+ * Lossless tile-ANS ("EPL1" blobs; the EntroPack README's Config table, TileANSConfig: exact restoration of
+ * BF16, FP16, FP32, FP8 and INT8 tensors of any shape, with a ratio that depends on the data). The raw bit
+ * patterns of the elements are cut into byte planes (byte j of every element, little-endian); a plane whose
+ * values cluster is rANS-coded under its own 12-bit table in tiles of 32 interleaved lanes, the others are
+ * stored verbatim. No value is interpreted: NaN payloads, signed zeros and subnormals come back as they were.
+ */
+#define EP_TANS_HEADER_BYTES 96
+
+/*
+ * ep_tans_compress: host encoder. data: numel = dims[0] x ... x dims[ndim-1] elements of `dtype`, host
+ * memory, row-major, read only (ndim 0..8; ndim 0 is one element; a zero dim gives an empty tensor).
+ * elems_per_lane: K, a tile holds 32 x K elements (1..1024, or 0 for 128). threads: host threads (0 = all
+ * cores); the blob does not depend on it. The blob is malloc'd; release it with ep_blob_free.
+ * Errors: EP_ERR_ARG (NULL pointer, K out of range), EP_ERR_DTYPE, EP_ERR_SHAPE (a dim above 2^32 - 1, or a
+ * blob above 64 GB), EP_ERR_NOMEM.
+ */
+ep_status ep_tans_compress(const void* data, ep_dtype dtype, int ndim, const int64_t* dims, uint32_t elems_per_lane,
+                           int threads, uint8_t** blob_out, size_t* bytes_out);
+
+/*
+ * ep_tans_info: full host validation of an EPL1 blob (header, tables, tile offsets, metadata CRC) and its
+ * description. dims receives ndim values (at most 8). Every out-pointer may be NULL.
+ * Errors: EP_ERR_ARG, EP_ERR_CORRUPT.
+ */
+ep_status ep_tans_info(const uint8_t* blob, size_t blob_bytes, ep_dtype* dt, int* ndim, int64_t* dims,
+                       uint32_t* coded_mask, uint32_t* elems_per_lane);
+
+/*
+ * ep_tans_decompress_into: decode of an EPL1 blob into a caller-owned device buffer, on the GPU.
+ * host_hdr    host copy of at least the first 96 bytes of the blob (the header).
+ * dev_blob    device copy of the whole blob, 16-byte aligned, blob_bytes long; read only.
+ * dst         device buffer of numel elements of the blob's dtype, 16-byte aligned; dst_bytes its size.
+ *             It may be NULL for an empty tensor, which launches nothing.
+ * cuda_stream cudaStream_t to launch on; NULL means the legacy default stream.
+ * One kernel, no allocation, no synchronisation. Host-detectable errors: EP_ERR_ARG, EP_ERR_CORRUPT (bad
+ * header), EP_ERR_BUFFER (size or alignment), EP_ERR_CUDA. The kernel checks every tile's final states and
+ * word count and bounds its reads; corruption sets EP_DEV_* bits of the device status word
+ * (ep_get_device_status) instead of faulting, and a corrupt tile's elements are unspecified.
+ */
+ep_status ep_tans_decompress_into(const uint8_t* host_hdr, const void* dev_blob, size_t blob_bytes, void* dst,
+                                  size_t dst_bytes, void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif
