@@ -1,7 +1,8 @@
 // Lossless tile-ANS (EPL1) decode for sm_100a, and its ABI entry ep_tans_decompress_into. Included by
 // decode.cu, so that it shares the device status word.
 //
-// One warp per tile, tiles dealt round-robin over the CTAs first. A round gives each lane one element:
+// One warp per tile, tiles dealt round-robin over the CTAs first; the warp first copies its tile into its
+// shared buffer. A round gives each lane one element:
 // for each byte plane in order, a coded plane decodes one symbol from the lane's rANS state (the fused
 // entry of slot x mod 4096 in the plane's shared table, then the lanes with x < 2^16 take the next words
 // of the tile's stream in lane order), a raw plane reads its byte from the tile's raw section; the bytes
@@ -17,6 +18,7 @@ constexpr int kThreadsT = kWarpsT * 32;
 constexpr uint32_t kEntries = 4096;                   // slots of a 12-bit table
 constexpr uint32_t kTableBytesT = kEntries * 4;       // fused entries of one coded plane: 16 KB
 constexpr uint32_t kScratchT = 4 * (256 + 257) * 4;   // f and cum of up to four planes
+constexpr uint32_t kMaxSmemT = 227 * 1024;             // per-CTA limit of sm_100
 
 struct TParams {
     const uint8_t* blob;
@@ -25,6 +27,7 @@ struct TParams {
     uint64_t payload_bytes;
     uint32_t K, T, mask;   // elements per lane per tile, tiles, coded planes
     uint32_t off_tables, off_offsets, off_payload;
+    uint32_t buf_bytes;    // per-warp tile buffer (a multiple of 16)
 };
 
 // Fused entry: symbol (bits 24-31) | slot - cum (bits 12-23) | f (bits 0-11).
@@ -80,7 +83,7 @@ __device__ void build_tans_tables(const TParams& p, uint32_t* tables, uint32_t* 
     }
     __syncthreads();
     const int nc = __popc(p.mask);
-    for (uint32_t k = threadIdx.x; k < uint32_t(nc) * kEntries; k += kThreadsT) {
+    for (uint32_t k = threadIdx.x; k < uint32_t(nc) * kEntries; k += blockDim.x) {
         const uint32_t cc = k >> 12, t = k & (kEntries - 1);
         const uint32_t* cu = cum + cc * 257;
         uint32_t s = 0;
@@ -94,6 +97,104 @@ __device__ void build_tans_tables(const TParams& p, uint32_t* tables, uint32_t* 
     __syncthreads();
 }
 
+__device__ __forceinline__ uint32_t ld_shared_u8(uint32_t addr) {
+    uint16_t v;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+
+// The bytes of one tile, in the warp's shared buffer (SMEM) or read from global memory in place.
+template <bool SMEM>
+struct TileBytes {
+    const uint8_t* g;  // the tile in global memory
+    uint32_t s;        // its shared-memory copy
+    __device__ __forceinline__ uint32_t u32(uint32_t o) const {
+        if constexpr (SMEM) return ld_shared_u32(s + o);
+        else return __ldg(reinterpret_cast<const uint32_t*>(g + o));
+    }
+    __device__ __forceinline__ uint32_t u16(uint32_t o) const {
+        if constexpr (SMEM) return ld_shared_u16(s + o);
+        else return __ldg(reinterpret_cast<const uint16_t*>(g + o));
+    }
+    __device__ __forceinline__ uint32_t u8(uint32_t o) const {
+        if constexpr (SMEM) return ld_shared_u8(s + o);
+        else return __ldg(g + o);
+    }
+};
+
+// One round of a tile: each lane's element i (act: it exists; PARTIAL: some lane's may not). MASK, the coded
+// planes, is a compile-time constant, so the planes unroll with no test. A word index past the tile's stream
+// reads the last word (shared copy, whose buffer has slack past the tile) or zero (in place): the values then
+// come out wrong, and the tile check flags the tile.
+template <int E, uint32_t MASK, bool SMEM, bool PARTIAL, class Elem>
+__device__ __forceinline__ void tans_round(const TileBytes<SMEM>& tb, uint32_t t_base, uint32_t raw_run,
+                                           uint32_t words_off, uint32_t cap, uint32_t capm1, uint32_t& x, uint32_t& pw,
+                                           uint32_t i,
+                                           bool act, Elem* o, uint32_t lt_mask) {
+    constexpr uint32_t raw0 = MASK ? 128u : 0u;
+    uint32_t val = 0;
+    int c = 0, r = 0;
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+        uint32_t byte = 0;
+        if ((MASK >> j) & 1u) {
+            if (!PARTIAL || act) {
+                const uint32_t e = ld_shared_u32(t_base + 4 * (uint32_t(c) * kEntries + (x & (kEntries - 1))));
+                x = (e & 0xFFFu) * (x >> 12) + ((e >> 12) & 0xFFFu);
+                byte = e >> 24;
+            }
+            const bool need = (!PARTIAL || act) && x < 65536u;
+            const uint32_t m = __ballot_sync(kFullMask, need);
+            if (need) {
+                const uint32_t idx = pw + __popc(m & lt_mask);
+                if constexpr (SMEM) x = (x << 16) | tb.u16(words_off + 2 * min(idx, capm1));
+                else x = (x << 16) | (idx < cap ? tb.u16(words_off + 2 * idx) : 0u);
+            }
+            pw += __popc(m);
+            ++c;
+        } else {
+            if (!PARTIAL || act) byte = tb.u8(raw0 + uint32_t(r) * raw_run + i);
+            ++r;
+        }
+        val |= byte << (8 * j);
+    }
+    if (!PARTIAL || act) o[i] = Elem(val);
+}
+
+// Decodes one tile of ne elements (output o, the tile's first element) whose bytes tb holds; returns whether
+// its checks pass.
+template <int E, uint32_t MASK, bool SMEM, class Elem>
+__device__ __forceinline__ bool tans_tile(const TileBytes<SMEM>& tb, uint32_t t_base, uint32_t size, uint32_t ne,
+                                          Elem* o, uint32_t lane, uint32_t lt_mask) {
+    constexpr int NC = __builtin_popcount(MASK);
+    const uint32_t raw_run = (ne + 3) & ~3u;
+    const uint32_t words_off = (NC ? 128u : 0u) + uint32_t(E - NC) * raw_run;
+    const uint32_t cap = (size - words_off) / 2;
+    const uint32_t capm1 = cap ? cap - 1 : 0u;  // with cap = 0 the clamped read stays inside the tile's slack
+    uint32_t x = NC ? tb.u32(4 * lane) : 0u;
+    uint32_t pw = 0;
+    const uint32_t full = ne / 32;
+    for (uint32_t k = 0; k < full; ++k)
+        tans_round<E, MASK, SMEM, false>(tb, t_base, raw_run, words_off, cap, capm1, x, pw, 32 * k + lane, true, o,
+                                         lt_mask);
+    if (ne % 32) {
+        const uint32_t i = 32 * full + lane;
+        tans_round<E, MASK, SMEM, true>(tb, t_base, raw_run, words_off, cap, capm1, x, pw, i, i < ne, o, lt_mask);
+    }
+    return NC == 0 || (__all_sync(kFullMask, x == 65536u) && pw <= cap && cap - pw <= 7);
+}
+
+// tans_tile for the runtime mask: one instantiation per possible set of coded planes.
+template <int E, uint32_t M, bool SMEM, class Elem>
+__device__ __forceinline__ bool tans_tile_any(uint32_t mask, const TileBytes<SMEM>& tb, uint32_t t_base, uint32_t size,
+                                              uint32_t ne, Elem* o, uint32_t lane, uint32_t lt_mask) {
+    if (mask == M) return tans_tile<E, M, SMEM>(tb, t_base, size, ne, o, lane, lt_mask);
+    if constexpr (M + 1 < (1u << E)) return tans_tile_any<E, M + 1, SMEM>(mask, tb, t_base, size, ne, o, lane, lt_mask);
+    return false;
+}
+
+// The whole kernel. Each warp copies its tile into its shared buffer (buf_bytes, cp.async, 16 bytes a lane)
+// when it fits, and reads it in place from global memory otherwise.
 template <int E>
 __global__ void __launch_bounds__(kThreadsT, 1) tans_decode_kernel(const TParams p) {
     extern __shared__ __align__(16) uint8_t smem_t[];
@@ -105,57 +206,35 @@ __global__ void __launch_bounds__(kThreadsT, 1) tans_decode_kernel(const TParams
     const uint32_t* toff = reinterpret_cast<const uint32_t*>(p.blob + p.off_offsets);
     const uint8_t* payload = p.blob + p.off_payload;
     const uint32_t t_base = smem_addr(tables);
+    const uint32_t buf = t_base + uint32_t(__popc(p.mask)) * kTableBytesT + warp * p.buf_bytes;
     const int nc = __popc(p.mask);
     const uint64_t per_tile = 32ull * p.K;
     using Elem = typename std::conditional<E == 4, uint32_t, typename std::conditional<E == 2, uint16_t, uint8_t>::type>::type;
     Elem* out = static_cast<Elem*>(p.dst);
-    for (uint32_t tile = warp * gridDim.x + blockIdx.x; tile < p.T; tile += kWarpsT * gridDim.x) {
+    const uint32_t warps = blockDim.x / 32;
+    for (uint32_t tile = warp * gridDim.x + blockIdx.x; tile < p.T; tile += warps * gridDim.x) {
         const uint64_t start = 16ull * __ldg(toff + tile), end = 16ull * __ldg(toff + tile + 1);
         const uint64_t i0 = uint64_t(tile) * per_tile;
         const uint32_t ne = uint32_t(per_tile < p.n - i0 ? per_tile : p.n - i0);
-        const uint32_t raw_run = (ne + 3) & ~3u;
-        const uint32_t words_off = (nc ? 128u : 0u) + uint32_t(E - nc) * raw_run;
+        const uint32_t words_off = (nc ? 128u : 0u) + uint32_t(E - nc) * ((ne + 3) & ~3u);
         if (end < start || end > p.payload_bytes || end - start < words_off) {
             if (lane == 0) atomicOr(&g_status, int(EP_DEV_BAD_OFFSETS));
             continue;
         }
-        const uint8_t* tp = payload + start;
-        const uint16_t* words = reinterpret_cast<const uint16_t*>(tp + words_off);
-        const uint32_t cap = uint32_t((end - start - words_off) / 2);
-        uint32_t x = nc ? __ldg(reinterpret_cast<const uint32_t*>(tp) + lane) : 0u;
-        uint32_t pw = 0;
-        const uint32_t R = (ne + 31) / 32;
-        for (uint32_t k = 0; k < R; ++k) {
-            const uint32_t i = 32 * k + lane;
-            const bool act = i < ne;
-            uint32_t val = 0;
-            int c = 0, r = 0;
-#pragma unroll
-            for (int j = 0; j < E; ++j) {
-                uint32_t byte = 0;
-                if ((p.mask >> j) & 1u) {
-                    if (act) {
-                        const uint32_t e = ld_shared_u32(t_base + 4 * (uint32_t(c) * kEntries + (x & (kEntries - 1))));
-                        x = (e & 0xFFFu) * (x >> 12) + ((e >> 12) & 0xFFFu);
-                        byte = e >> 24;
-                    }
-                    const bool need = act && x < 65536u;
-                    const uint32_t m = __ballot_sync(kFullMask, need);
-                    if (need) {
-                        const uint32_t idx = pw + __popc(m & lt_mask);
-                        x = (x << 16) | (idx < cap ? uint32_t(__ldg(words + idx)) : 0u);
-                    }
-                    pw += __popc(m);
-                    ++c;
-                } else {
-                    if (act) byte = __ldg(tp + (nc ? 128u : 0u) + uint32_t(r) * raw_run + i);
-                    ++r;
-                }
-                val |= byte << (8 * j);
-            }
-            if (act) out[i0 + i] = Elem(val);
+        const uint32_t size = uint32_t(end - start);
+        Elem* o = out + i0;
+        bool good;
+        // The buffer keeps 16 bytes past the tile, so that a clamped word read of an empty stream stays inside.
+        if (size + 16 <= p.buf_bytes) {
+            v2::copy_tile(buf, payload + start, size, lane);
+            cp_async_commit();
+            cp_async_wait<0>();
+            __syncwarp();
+            good = tans_tile_any<E, 0>(p.mask, TileBytes<true>{payload + start, buf}, t_base, size, ne, o, lane, lt_mask);
+            __syncwarp();  // the buffer's reads are done before the next tile's copy
+        } else {
+            good = tans_tile_any<E, 0>(p.mask, TileBytes<false>{payload + start, 0u}, t_base, size, ne, o, lane, lt_mask);
         }
-        const bool good = nc == 0 || (__all_sync(kFullMask, x == 65536u) && pw <= cap && cap - pw <= 7);
         if (!good && lane == 0) atomicOr(&g_status, int(EP_DEV_CORRUPT_TILE));
     }
 }
@@ -200,7 +279,21 @@ extern "C" ep_status ep_tans_decompress_into(const uint8_t* host_hdr, const void
     p.off_tables = h.off_tables;
     p.off_offsets = h.off_offsets;
     p.off_payload = h.off_payload;
-    const uint32_t smem = kScratchT + uint32_t(h.coded_planes()) * kTableBytesT;
+    // Per-warp tile buffers fill what the tables leave of the CTA's shared memory. The CTA takes as many warps
+    // (32 down to 8) as can each hold an average tile with 15 % to spare (a 4096-element tile of 2-byte values
+    // takes 6-7 KB, of 4-byte values about 14 KB); tiles that do not fit are read in place.
+    const uint32_t fixed = kScratchT + uint32_t(h.coded_planes()) * kTableBytesT;
+    const uint64_t avg = (h.total - h.off_payload) / h.T;
+    const uint64_t need = ((avg + avg / 7 + 15) & ~uint64_t(15)) + 64;
+    uint32_t warps = 8;
+    for (uint32_t w = uint32_t(kWarpsT); w >= 8; w -= 4)
+        if ((kMaxSmemT - fixed) / w >= need) {
+            warps = w;
+            break;
+        }
+    const uint32_t buf = ((kMaxSmemT - fixed) / warps) & ~15u;
+    p.buf_bytes = buf;
+    const uint32_t smem = fixed + warps * buf;
     const void* fn = h.e == 4   ? reinterpret_cast<const void*>(tans_decode_kernel<4>)
                      : h.e == 2 ? reinterpret_cast<const void*>(tans_decode_kernel<2>)
                                 : reinterpret_cast<const void*>(tans_decode_kernel<1>);
@@ -214,16 +307,17 @@ extern "C" ep_status ep_tans_decompress_into(const uint8_t* host_hdr, const void
         sms = g_dev[device].sms;
         bool& conf = g_tans_configured[device][h.e];
         if (!conf) {
-            e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kScratchT + 4 * kTableBytesT));
+            e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kMaxSmemT));
             if (e != cudaSuccess) return fail(EP_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
             conf = true;
         }
     }
     const uint32_t grid = h.T < uint32_t(sms) ? h.T : uint32_t(sms);
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-    if (h.e == 4) tans_decode_kernel<4><<<grid, kThreadsT, smem, stream>>>(p);
-    else if (h.e == 2) tans_decode_kernel<2><<<grid, kThreadsT, smem, stream>>>(p);
-    else tans_decode_kernel<1><<<grid, kThreadsT, smem, stream>>>(p);
+    const uint32_t threads = warps * 32;
+    if (h.e == 4) tans_decode_kernel<4><<<grid, threads, smem, stream>>>(p);
+    else if (h.e == 2) tans_decode_kernel<2><<<grid, threads, smem, stream>>>(p);
+    else tans_decode_kernel<1><<<grid, threads, smem, stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(EP_ERR_CUDA, "tile-ANS decode launch: %s", cudaGetErrorString(e));
     return EP_OK;
