@@ -1178,13 +1178,13 @@ __device__ __forceinline__ void refill(uint32_t& x, uint32_t& pa, uint32_t lt_ma
 // 4 idx + b at position 7 (before pi is added), built by ORing the entries' value fields into the mantissa
 // (see round_fast of version 1). two_pi = 2 pi comes from the XOR of the idx parities.
 template <int MODE, bool WAIT, class P>
-__device__ __forceinline__ void store_fast(const P& p, const uint32_t* mb, uint32_t two_pi, uint32_t g, float c) {
+__device__ __forceinline__ void store_fast(const P& p, const uint32_t* mb, uint32_t two_pi, uint32_t g, float c,
+                                           float K = kHalfMagicF + 31.0f, float K7 = kHalfMagicF + 62.0f) {
     float m[8], y[8];
     int32_t z[8];
 #pragma unroll
     for (int i = 0; i < 7; ++i) m[i] = __uint_as_float(mb[i]);
     m[7] = __uint_as_float(mb[7] + two_pi);
-    const float K = kHalfMagicF + 31.0f, K7 = kHalfMagicF + 62.0f;
 #pragma unroll
     for (int i = 0; i < 6; i += 2) sub_mul_f32x2(m[i], m[i + 1], K, K, c, y[i], y[i + 1]);
     sub_mul_f32x2(m[6], m[7], K, K7, c, y[6], y[7]);
@@ -1268,9 +1268,9 @@ __device__ __forceinline__ uint32_t or3(uint32_t a, uint32_t b, uint32_t c) {
 // escape (its offset entry says so). Then, when some lane of the warp met one in this round, its words are
 // read after the fourth pair, and each escaped position's value bits and parity are rebuilt from the word's
 // hi (an escape's field, 2 * 63 + b or 4 * 63 + b, marks it).
-template <int MODE, bool WAIT, bool ESC, class P, class K>
+template <int MODE, bool WAIT, bool ESC, class P, class K, bool RAW = false>
 __device__ __forceinline__ void round_fast_v2(const P& p, const K& kc, uint32_t t0, uint32_t ts, uint32_t& x, uint32_t& pa, uint32_t g,
-                                              uint32_t lt_mask, float c, uint32_t k2) {
+                                              uint32_t lt_mask, float c, uint32_t k2, uint32_t rawb = 0, uint32_t q = 0) {
     uint32_t mb[8], e, e2, par, escs;
     e = symbol(kc, ts, x);
     mb[0] = and_or(e, 0x7Fu, kHalfMagic);
@@ -1318,7 +1318,35 @@ __device__ __forceinline__ void round_fast_v2(const P& p, const K& kc, uint32_t 
             }
         }
     }
-    store_fast<MODE, WAIT>(p, mb, ~par & 2u, g, c);
+    if constexpr (RAW) {
+        // r >= 1 raw low bits a coordinate, in a tile with no escape (so |hi| <= 31 and every field below stays
+        // under 2^22): t = hi 2^r + lo, so m_i = 1.5*2^22 + 2 idx 2^r + 2 lo + b (i < 7) and
+        // m_7 = 1.5*2^22 + 4 idx 2^r + 4 lo_7 + 2 pi + b, pi the parity of the seven lo's; the group's 8r
+        // bits sit at bit 8 r q of the tile's raw section, in shared memory (rawb).
+        const uint32_t r = uint32_t(p.r), o = q * r, a = o & ~3u, sh = (o & 3u) * 8, lmask = (1u << r) - 1u;
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] = ld_shared_u32(rawb + a + 4 * j);
+        uint32_t lpar = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t bp = uint32_t(i) * r + sh, sel = bp >> 5, s5 = bp & 31;
+            const uint32_t wa = sel == 0 ? w[0] : (sel == 1 ? w[1] : (sel == 2 ? w[2] : w[3]));
+            const uint32_t wb = sel == 0 ? w[1] : (sel == 1 ? w[2] : w[3]);
+            const uint32_t lo = __funnelshift_r(wa, wb, s5) & lmask;
+            const uint32_t f = mb[i] & 0xFFu;
+            if (i < 7) {
+                lpar ^= lo;
+                mb[i] = kHalfMagic + ((f & 0x7Eu) << r) + (lo << 1) + (f & 1u);
+            } else {
+                mb[7] = kHalfMagic + ((f & 0xFCu) << r) + (lo << 2) + ((lpar & 1u) << 1) + (f & 1u);
+            }
+        }
+        const float sc = float(1u << r);
+        store_fast<MODE, WAIT>(p, mb, 0u, g, c, kHalfMagicF + 31.0f * sc, kHalfMagicF + 62.0f * sc);
+    } else {
+        store_fast<MODE, WAIT>(p, mb, ~par & 2u, g, c);
+    }
 }
 
 // General round: ragged rounds (PARTIAL: some lanes hold no group), raw low bits, and streams read from
@@ -1383,17 +1411,18 @@ static_assert(kTablesBytes + kScratchSize + kSlackBytes >= kOverrunBytes, "a cor
 // lane i computes the factor of row row0 + i once, and each round takes its row's factor by a shuffle, with
 // no load on the round's path. kr: the first round's column in its row, in rounds. Otherwise the lanes'
 // rows move on their own (RowCursor).
-template <int MODE, bool ESC, bool UNIFORM, class P, class K>
+template <int MODE, bool ESC, bool UNIFORM, class P, class K, bool RAW = false>
 __device__ __forceinline__ uint32_t fast_rounds_v2(const P& p, const K& kc, uint32_t t0, uint32_t ts, TileState& st, uint32_t ring_base,
                                                    uint32_t g, uint32_t lt_mask, uint32_t Rf, uint32_t row0, uint32_t kr,
-                                                   const uint16_t* scales, RowCursor& rc, bool& waited) {
+                                                   const uint16_t* scales, RowCursor& rc, bool& waited, uint32_t rawb = 0) {
     uint32_t k = 0, x = st.x, pa = ring_base + st.pb;
+    const uint32_t g0 = g - (threadIdx.x & 31);  // the tile's first group: q = g - g0
     if constexpr (UNIFORM) {
         const uint32_t rpr = p.gpr / 32, lane = threadIdx.x & 31;
         const float cvec = row0 + lane < p.M ? RowCursor::scale_of(p, scales, row0 + lane) : 0.f;
         uint32_t ri = 0;
         if (!waited && Rf > 0) {
-            round_fast_v2<MODE, true, ESC>(p, kc, t0, ts, x, pa, g, lt_mask, __shfl_sync(kFullMask, cvec, 0), kc.k2);
+            round_fast_v2<MODE, true, ESC, P, K, RAW>(p, kc, t0, ts, x, pa, g, lt_mask, __shfl_sync(kFullMask, cvec, 0), kc.k2, rawb, g - g0);
             waited = true;
             k = 1;
             g += 32;
@@ -1407,21 +1436,21 @@ __device__ __forceinline__ uint32_t fast_rounds_v2(const P& p, const K& kc, uint
             const uint32_t run = min(rpr - kr, Rf - k);
             const float c = __shfl_sync(kFullMask, cvec, ri);
             const uint32_t gend = g + 32 * run;
-            for (; g != gend; g += 32) round_fast_v2<MODE, false, ESC>(p, kc, t0, ts, x, pa, g, lt_mask, c, kc.k2);
+            for (; g != gend; g += 32) round_fast_v2<MODE, false, ESC, P, K, RAW>(p, kc, t0, ts, x, pa, g, lt_mask, c, kc.k2, rawb, g - g0);
             k += run;
             kr = 0;
             ++ri;
         }
     } else {
         if (!waited && Rf > 0) {
-            round_fast_v2<MODE, true, ESC>(p, kc, t0, ts, x, pa, g, lt_mask, rc.scale(), kc.k2);
+            round_fast_v2<MODE, true, ESC, P, K, RAW>(p, kc, t0, ts, x, pa, g, lt_mask, rc.scale(), kc.k2, rawb, g - g0);
             rc.advance(p, scales);
             waited = true;
             k = 1;
             g += 32;
         }
         for (; k < Rf; ++k, g += 32) {
-            round_fast_v2<MODE, false, ESC>(p, kc, t0, ts, x, pa, g, lt_mask, rc.scale(), kc.k2);
+            round_fast_v2<MODE, false, ESC, P, K, RAW>(p, kc, t0, ts, x, pa, g, lt_mask, rc.scale(), kc.k2, rawb, g - g0);
             rc.advance(p, scales);
         }
     }
@@ -1543,11 +1572,18 @@ __global__ void __launch_bounds__(kThreadsV2, 1) decode_kernel(const Params p) {
             const uint32_t gt0 = tile * per_tile;
 
             uint32_t k = 0;
-            if (in_ring && p.r == 0) {
+            const bool esc = __any_sync(kFullMask, cur.e0 >> 31);
+            if (in_ring && (p.r == 0 || !esc)) {
                 const uint32_t Rf = min(ng / 32, kMaxFastRounds);
                 const uint32_t row0 = gt0 / p.gpr, kr0 = (gt0 - row0 * p.gpr) / 32;
-                const bool esc = __any_sync(kFullMask, cur.e0 >> 31);
-                if (p.gpr % 32 == 0) {
+                if (p.r != 0) {  // raw low bits, no escape in the tile
+                    if (p.gpr % 32 == 0) {
+                        k = fast_rounds_v2<MODE, false, true, Params, Params, true>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited, rb + 128);
+                    } else {
+                        rc.start(p, scales, gt0 + lane);
+                        k = fast_rounds_v2<MODE, false, false, Params, Params, true>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited, rb + 128);
+                    }
+                } else if (p.gpr % 32 == 0) {
                     k = esc ? fast_rounds_v2<MODE, true, true>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited)
                             : fast_rounds_v2<MODE, false, true>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited);
                 } else {
@@ -1887,7 +1923,7 @@ __global__ void __launch_bounds__(kThreadsV2, 1) seq_kernel(const __grid_constan
                 const uint32_t gt0 = tile * per_tile;
                 if (sp.ordered) seq_wait(sp, p, gt0, ng, es);
                 uint32_t k = 0;
-                if (in_ring && p.r == 0) {
+                if (in_ring && p.r == 0) {  // (tiles with raw low bits take the general rounds here)
                     const uint32_t Rf = min(ng / 32, kMaxFastRounds);
                     const uint32_t row0 = gt0 / p.gpr, kr0 = (gt0 - row0 * p.gpr) / 32;
                     const bool esc = __any_sync(kFullMask, co.e0 >> 31);
