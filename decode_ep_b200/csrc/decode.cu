@@ -1,32 +1,26 @@
 // Fused EntroPack decode for sm_100a (B200): rANS symbols -> E8 coordinates -> s_row * v / alpha ->
-// container. One kernel does all of it. No symbol tensor and no codebook sit in between; the
-// arithmetic inverse of the lattice map and the per-row rescale are fused with the symbol decode
-// (modelscope paper page, summary; paper page abstract).
+// container, in one pass. No symbol tensor and no codebook sit in between; the arithmetic inverse of the
+// lattice map and the per-row rescale are fused with the symbol decode (modelscope paper page, summary;
+// paper page abstract). This file holds four kernels and their C-ABI launchers:
 //
-// Kernel shape: a persistent grid with one 1024-thread CTA per SM (32 warps).
-//   - Tables. Each CTA first expands the blob's 9 twelve-bit frequency tables into fused 32-bit
-//     decode entries in shared memory: 9 contexts x 4096 slots, 144 KB. One entry holds
-//       a value field (bits 0-6; 0-7 at position 7), the magnitude class of the decoded coordinate
-//       (bit 7, which picks the next context), f (bits 8-19) and slot - cum (bits 20-31).
-//     A symbol step is therefore one random 4-byte shared load and a handful of integer operations.
-//     There are no symbol, record or codebook tables. The field sits at the bottom of the entry, so
-//     one AND-OR gives the value's float bits.
-//   - Tiles. Each warp decodes whole tiles. Lane L owns the groups 32k + L of the tile. After every
-//     symbol step, the lanes that must refill take the next 16-bit words of the shared stream in
-//     lane order, found with a warp ballot and a popcount prefix.
-//   - Stream staging. The words come from a 2 KB per-warp ring in shared memory, filled by
-//     asynchronous 16-byte copies (cp.async) in 512-byte chunks, so no refill waits on DRAM. The first
-//     2 KB of a tile's stream (all of it, for most tiles at 4 bpp) land in one batch. A longer stream
-//     gets its next chunk copied into the slot that the rounds have left behind.
-//   - Values. v = hi + b/2 is rebuilt with no conversion instruction. The value field is ORed into
-//     the mantissa of 1.5 * 2^22, a float whose last-place unit is 1/2, and the bias is subtracted.
-//     Each lane then writes its 8 values with one 16-byte store (BF16/FP16), so a warp writes 512
-//     contiguous bytes.
-//   - Layer sequences. Successive launches are chained with programmatic dependent launch. A
-//     kernel builds its tables and fills its first rings while the previous kernel drains, and it
-//     waits on the grid dependency only before its first store.
-// The loop is bound by integer issue and shared-memory bandwidth, not by tensor cores: decode has
-// no dense contraction.
+//   - v2::decode_kernel, one layer of format version 2 (the default; ep_decompress_into). A persistent grid
+//     of 1024-thread CTAs, one per SM. Each CTA builds the blob's 9 x 256 fused 32-bit entries in shared
+//     memory (value field, escape and class bits, coset bit, f, slot - cum): a symbol step is one random
+//     4-byte shared load and a handful of integer operations, and one refill (ballot, popcount prefix, one
+//     16-bit word in lane order) serves each pair of coordinates. Each warp copies its whole tile into a 5 KB
+//     shared buffer with cp.async, the next tile landing in the other end while it decodes the current one.
+//     v = u + b/2 is rebuilt with no conversion instruction (the value field ORed into the mantissa of
+//     1.5 * 2^22), rescaled in packed f32x2, and each lane stores its 8 values at once.
+//   - v2::prep_tables_kernel and v2::seq_kernel, a list of version-2 layers of one dtype (ep_decompress_many):
+//     the tables of every layer built once into global scratch, then one cooperative persistent launch
+//     deals all the layers' tiles round-robin over CTAs and warps, keeps four layers' tables per CTA in
+//     shared windows refilled by bulk copies, and orders the stores of overlapping outputs tile by tile.
+//   - decode_kernel, one layer of format version 1 (12-bit tables, 144 KB of fused entries, a refill per
+//     symbol); with expand_tables_kernel for version-1 sequences, chained with programmatic dependent launch.
+//   - tans_decode_kernel (tans_decode.cuh, included at the end): the lossless tile-ANS blobs.
+//
+// The decode is bound by integer issue and shared-memory latency, not by tensor cores: it has no dense
+// contraction.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -2272,7 +2266,8 @@ extern "C" ep_status ep_decompress_many(int count, const uint8_t* const* host_hd
     // The fused entries of every version-1 blob, built once for the sequence into stream-ordered scratch
     // (144 KB per blob). The first decode launches in plain stream order behind the expand kernel, and every
     // later one starts after it, so all of them read finished tables. Without the scratch, each CTA builds
-    // its own tables. Version-2 tables (9 KB) are always built by each CTA: that takes about a microsecond.
+    // its own tables. (A list of version-2 blobs of one dtype has returned through decompress_seq above; in a
+    // mixed list, each version-2 decode builds its 9 KB of tables in each CTA.)
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     constexpr size_t kWords = dev::kTablesBytes / 4;
     std::vector<int> v1;  // indices of the version-1 blobs, in order; blob v1[j] takes prepared slot j
