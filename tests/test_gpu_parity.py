@@ -518,3 +518,46 @@ def test_sequence_kernel_overlapping_outputs(orc, layout):
         status_clean()
         for b, w in zip(bufs, wants):
             assert np.array_equal(gpu_bits(b), w)
+
+
+@pytest.mark.parametrize("layout", ["separate", "one"])
+def test_sequence_kernel_corrupt_blob_is_flagged_and_the_rest_decodes(orc, layout):
+    """A corrupted word stream in one layer of a sequence: the sequence kernel flags it (EP_DEV_CORRUPT_TILE),
+    every tile still publishes itself, so no wait runs out (no EP_DEV_DEP_WAIT) and the call completes; the
+    other layers come out exact. With one shared buffer, the bytes the corrupt layer wrote last are the only
+    ones left unspecified."""
+    shapes = [(512, 512), (256, 768), (1024, 256), (384, 512)]
+    comps = [ep.compress(synth.dit_layer(80 + i, shape=s), 4.0) for i, s in enumerate(shapes)]
+    bad = bytearray(comps[1].blob)
+    off_payload = int.from_bytes(bad[40:44], "little")
+    for k in range(off_payload + 300, len(bad) - 64, 97):
+        bad[k] ^= 0x5A
+    comps[1] = ep.CompressedTensor(bytes(bad), comps[1].shape, comps[1].dtype, comps[1].actual_bpp)
+    dec = {i: orc.decompress(c.blob).reshape(-1) for i, c in enumerate(comps) if i != 1}
+    status_clean()
+    if layout == "separate":
+        outs = [torch.zeros(c.shape, dtype=c.dtype, device="cuda") for c in comps]
+        ep.decompress_many(list(zip(comps, outs)))
+        st = ep.device_status()
+        assert st & 1 and not st & 16, st
+        for i, o in enumerate(outs):
+            if i != 1:
+                assert np.array_equal(gpu_bits(o).reshape(-1), dec[i]), f"layer {i}"
+    else:
+        mx = max(M * N for M, N in shapes)
+        buf = torch.zeros(mx, dtype=torch.bfloat16, device="cuda")
+        ep.decompress_many([(c, buf[: c.shape[0] * c.shape[1]].view(c.shape)) for c in comps])
+        st = ep.device_status()
+        assert st & 1 and not st & 16, st
+        got = gpu_bits(buf)
+        last = np.full(mx, -1)
+        for i, (M, N) in enumerate(shapes):
+            last[: M * N] = i
+        for i in dec:
+            n = shapes[i][0] * shapes[i][1]
+            sel = np.flatnonzero(last[:n] == i)
+            assert np.array_equal(got[sel], dec[i][sel]), f"layer {i}"
+    # the context stays usable
+    good = ep.compress(synth.dit_layer(90, shape=(256, 256)), 4.0)
+    assert np.array_equal(gpu_bits(ep.decompress(good)), orc.decompress(good.blob))
+    status_clean()
