@@ -161,6 +161,64 @@ __device__ __forceinline__ void tans_round(const TileBytes<SMEM>& tb, uint32_t t
     if (!PARTIAL || act) o[i] = Elem(val);
 }
 
+// One full round of a tile held in shared memory: lane's raw bytes at rp[r] + off, its word stream at words
+// (shared addresses). Every lane reads a word, at its clamped index, and only the lanes that refill keep it:
+// the refill takes no branch.
+template <int E, uint32_t MASK>
+__device__ __forceinline__ uint32_t tans_round_smem(uint32_t t_base, const uint32_t* rp, uint32_t off, uint32_t words,
+                                                    uint32_t capm1, uint32_t& x, uint32_t& pw, uint32_t lt_mask) {
+    uint32_t val = 0;
+    int c = 0, r = 0;
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+        uint32_t byte;
+        if ((MASK >> j) & 1u) {
+            const uint32_t e = ld_shared_u32(t_base + uint32_t(c) * kTableBytesT + 4u * (x & (kEntries - 1)));
+            x = (e & 0xFFFu) * (x >> 12) + ((e >> 12) & 0xFFFu);
+            byte = e >> 24;
+            const bool need = x < 65536u;
+            const uint32_t m = __ballot_sync(kFullMask, need);
+            const uint32_t w = ld_shared_u16(words + 2u * min(pw + __popc(m & lt_mask), capm1));
+            if (need) x = __byte_perm(w, x, 0x5410);  // (x << 16) | w
+            pw += __popc(m);
+            ++c;
+        } else {
+            byte = ld_shared_u8(rp[r] + off);
+            ++r;
+        }
+        val |= byte << (8 * j);
+    }
+    return val;
+}
+
+// The full rounds of a tile held in shared memory, four to a step: the raw planes' shared addresses and the
+// output pointer advance once a step, and the rounds inside it use constant offsets from them.
+template <int E, uint32_t MASK, class Elem>
+__device__ __forceinline__ void tans_rounds_smem(uint32_t t_base, uint32_t raw_lane, uint32_t raw_run, uint32_t words,
+                                                 uint32_t capm1, uint32_t& x, uint32_t& pw, uint32_t rounds, Elem* o,
+                                                 uint32_t lt_mask) {
+    constexpr int NR = E - __builtin_popcount(MASK);
+    constexpr uint32_t U = 4;
+    uint32_t rp[NR > 0 ? NR : 1];
+#pragma unroll
+    for (int r = 0; r < (NR > 0 ? NR : 1); ++r) rp[r] = raw_lane + uint32_t(r) * raw_run;
+    uint32_t k = 0;
+    for (; k + U <= rounds; k += U) {
+#pragma unroll
+        for (uint32_t u = 0; u < U; ++u)
+            o[32 * u] = Elem(tans_round_smem<E, MASK>(t_base, rp, 32 * u, words, capm1, x, pw, lt_mask));
+#pragma unroll
+        for (int r = 0; r < NR; ++r) rp[r] += 32 * U;
+        o += 32 * U;
+    }
+    for (; k < rounds; ++k) {
+        *o = Elem(tans_round_smem<E, MASK>(t_base, rp, 0, words, capm1, x, pw, lt_mask));
+#pragma unroll
+        for (int r = 0; r < NR; ++r) rp[r] += 32;
+        o += 32;
+    }
+}
+
 // Decodes one tile of ne elements (output o, the tile's first element) whose bytes tb holds; returns whether
 // its checks pass.
 template <int E, uint32_t MASK, bool SMEM, class Elem>
@@ -174,9 +232,14 @@ __device__ __forceinline__ bool tans_tile(const TileBytes<SMEM>& tb, uint32_t t_
     uint32_t x = NC ? tb.u32(4 * lane) : 0u;
     uint32_t pw = 0;
     const uint32_t full = ne / 32;
-    for (uint32_t k = 0; k < full; ++k)
-        tans_round<E, MASK, SMEM, false>(tb, t_base, raw_run, words_off, cap, capm1, x, pw, 32 * k + lane, true, o,
-                                         lt_mask);
+    if constexpr (SMEM) {
+        tans_rounds_smem<E, MASK>(t_base, tb.s + (NC ? 128u : 0u) + lane, raw_run, tb.s + words_off, capm1, x, pw,
+                                  full, o + lane, lt_mask);
+    } else {
+        for (uint32_t k = 0; k < full; ++k)
+            tans_round<E, MASK, SMEM, false>(tb, t_base, raw_run, words_off, cap, capm1, x, pw, 32 * k + lane, true,
+                                             o, lt_mask);
+    }
     if (ne % 32) {
         const uint32_t i = 32 * full + lane;
         tans_round<E, MASK, SMEM, true>(tb, t_base, raw_run, words_off, cap, capm1, x, pw, i, i < ne, o, lt_mask);
