@@ -69,6 +69,7 @@ def parse_args():
                              "dit276_fp8_gemm_overhead", "dit276_mixed_2.3bpp", "cuda_encode_gate_10240x3840",
                              "tileans_lossless"],
                     help="the default is the headline line; the others print one line per tensor")
+    ap.add_argument("--only", default="", help="single-tensor workloads: run only the tensors whose label contains this")
     return ap.parse_args()
 
 
@@ -1002,6 +1003,8 @@ def run_workload(args):
     peak, peak_kind = measured_hbm_peak()
     lines = []
     for label, make, target, G in workload_items(args.workload):
+        if args.only and args.only not in label:
+            continue
         w = make()
         t_enc = time.perf_counter()
         c = ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G))

@@ -1291,7 +1291,52 @@ __device__ __forceinline__ void round_fast_v2(const P& p, const K& kc, uint32_t 
     par ^= e;
     escs = or3(escs, e, e2);
     refill(x, pa, lt_mask, k2);
-    if (ESC && __any_sync(kFullMask, escs & kEscBit)) {
+    if constexpr (RAW && ESC) {
+        // A round in which some lane met an escape: its words follow the fourth pair, position by position and
+        // lane by lane, as in the general round. Each position's t = hi 2^r + lo (hi from the entry, or any
+        // int16 from the escape word; lo from the group's raw bits in shared memory) replaces its value bits,
+        // and the values come from the integer formula.
+        if (__any_sync(kFullMask, escs & kEscBit)) {
+            const uint32_t r = uint32_t(p.r), o = q * r, a = o & ~3u, sh = (o & 3u) * 8, lmask = (1u << r) - 1u;
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w[j] = ld_shared_u32(rawb + a + 4 * j);
+            uint32_t A = __funnelshift_r(w[0], w[1], sh), B = __funnelshift_r(w[1], w[2], sh), C = __funnelshift_r(w[2], w[3], sh);
+            const int32_t b = int32_t(mb[0] & 1u);
+            int32_t s7 = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const bool esc = i < 7 ? (mb[i] & 0x7Eu) == 0x7Eu : (mb[7] & 0xFCu) == 0xFCu;
+                const uint32_t me = __ballot_sync(kFullMask, esc);
+                int32_t hi = int32_t(i < 7 ? (mb[i] >> 1) & 63u : (mb[7] >> 2) & 63u) - 31;
+                if (me) {
+                    const uint32_t wd = ld_shared_u16(pa + __popc(me & lt_mask) * k2);
+                    pa += __popc(me) * k2;
+                    if (esc) hi = int32_t(int16_t(wd));
+                }
+                const int32_t t = hi * (1 << r) + int32_t(A & lmask);
+                if (i < 7) {
+                    A = __funnelshift_r(A, B, r);
+                    B = __funnelshift_r(B, C, r);
+                    C >>= r;
+                }
+                if (i < 7) s7 += t;
+                mb[i] = uint32_t(t);
+            }
+            float y[8];
+            int32_t z[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int32_t u = i < 7 ? int32_t(mb[i]) : 2 * int32_t(mb[7]) + (s7 & 1);
+                z[i] = 2 * u + b;
+                y[i] = __fmul_rn(__int2float_rn(z[i]) * 0.5f, c);
+            }
+            if constexpr (WAIT) grid_dependency_wait();
+            store_group<MODE>(p.dst, g, y, z);
+            return;
+        }
+    }
+    if (!RAW && ESC && __any_sync(kFullMask, escs & kEscBit)) {
         const uint32_t b = mb[0] & 1u;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -1318,22 +1363,28 @@ __device__ __forceinline__ void round_fast_v2(const P& p, const K& kc, uint32_t 
         // m_7 = 1.5*2^22 + 4 idx 2^r + 4 lo_7 + 2 pi + b, pi the parity of the seven lo's; the group's 8r
         // bits sit at bit 8 r q of the tile's raw section, in shared memory (rawb).
         const uint32_t r = uint32_t(p.r), o = q * r, a = o & ~3u, sh = (o & 3u) * 8, lmask = (1u << r) - 1u;
+        const uint32_t pow2r = 1u << r;
         uint32_t w[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) w[j] = ld_shared_u32(rawb + a + 4 * j);
+        // The group's 8r bits from bit 0 of (A, B, C): each position takes the low r bits of A, then the three
+        // words shift right by r together.
+        uint32_t A = __funnelshift_r(w[0], w[1], sh), B = __funnelshift_r(w[1], w[2], sh), C = __funnelshift_r(w[2], w[3], sh);
         uint32_t lpar = 0;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const uint32_t bp = uint32_t(i) * r + sh, sel = bp >> 5, s5 = bp & 31;
-            const uint32_t wa = sel == 0 ? w[0] : (sel == 1 ? w[1] : (sel == 2 ? w[2] : w[3]));
-            const uint32_t wb = sel == 0 ? w[1] : (sel == 1 ? w[2] : w[3]);
-            const uint32_t lo = __funnelshift_r(wa, wb, s5) & lmask;
-            const uint32_t f = mb[i] & 0xFFu;
+            const uint32_t lo = A & lmask;
+            if (i < 7) {
+                A = __funnelshift_r(A, B, r);
+                B = __funnelshift_r(B, C, r);
+                C >>= r;
+            }
+            // mb & ~0xFE is 1.5*2^22 + b: the entry's value field sits in the low 8 bits.
             if (i < 7) {
                 lpar ^= lo;
-                mb[i] = kHalfMagic + ((f & 0x7Eu) << r) + (lo << 1) + (f & 1u);
+                mb[i] = (mb[i] & ~0xFEu) + (mb[i] & 0x7Eu) * pow2r + (lo << 1);
             } else {
-                mb[7] = kHalfMagic + ((f & 0xFCu) << r) + (lo << 2) + ((lpar & 1u) << 1) + (f & 1u);
+                mb[7] = (mb[7] & ~0xFEu) + (mb[7] & 0xFCu) * pow2r + (lo << 2) + ((lpar & 1u) << 1);
             }
         }
         const float sc = float(1u << r);
@@ -1567,15 +1618,17 @@ __global__ void __launch_bounds__(kThreadsV2, 1) decode_kernel(const Params p) {
 
             uint32_t k = 0;
             const bool esc = __any_sync(kFullMask, cur.e0 >> 31);
-            if (in_ring && (p.r == 0 || !esc)) {
+            if (in_ring) {
                 const uint32_t Rf = min(ng / 32, kMaxFastRounds);
                 const uint32_t row0 = gt0 / p.gpr, kr0 = (gt0 - row0 * p.gpr) / 32;
-                if (p.r != 0) {  // raw low bits, no escape in the tile
+                if (p.r != 0) {  // raw low bits
                     if (p.gpr % 32 == 0) {
-                        k = fast_rounds_v2<MODE, false, true, Params, Params, true>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited, rb + 128);
+                        k = esc ? fast_rounds_v2<MODE, true, true, Params, Params, true>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited, rb + 128)
+                                : fast_rounds_v2<MODE, false, true, Params, Params, true>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited, rb + 128);
                     } else {
                         rc.start(p, scales, gt0 + lane);
-                        k = fast_rounds_v2<MODE, false, false, Params, Params, true>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited, rb + 128);
+                        k = esc ? fast_rounds_v2<MODE, true, false, Params, Params, true>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited, rb + 128)
+                                : fast_rounds_v2<MODE, false, false, Params, Params, true>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited, rb + 128);
                     }
                 } else if (p.gpr % 32 == 0) {
                     k = esc ? fast_rounds_v2<MODE, true, true>(p, p, t0, t0 | kStartOffset, st, rb, gt0 + lane, lt_mask, Rf, row0, kr0, scales, rc, waited)
