@@ -328,6 +328,16 @@ def run_ours(args):
         b.record(stream)
     torch.cuda.synchronize(device)
     kernel_ms = sum(a.elapsed_time(b) for a, b in evs)
+    by_shape = {}
+    for (a, b), (_, _, M, N) in zip(evs, layers):
+        e = by_shape.setdefault(f"{M}x{N}", {"layers": 0, "ms": 0.0})
+        e["layers"] += 1
+        e["ms"] += a.elapsed_time(b)
+    for k, e in by_shape.items():
+        M, N = map(int, k.split("x"))
+        e["us_per_layer"] = round(1e3 * e["ms"] / e["layers"], 2)
+        e["gparams_s"] = round(e["layers"] * M * N / (e["ms"] * 1e-3) / 1e9, 1)
+        e["ms"] = round(e["ms"], 4)
     shared = outs[int(max(range(len(layers)), key=lambda i: layers[i][2] * layers[i][3]))].view(-1)
     one_buf = ep.LayerBatch([(c, shared[: M * N].view(M, N)) for c, (_, _, M, N) in zip(blobs, layers)], stream)
     one_buf.run()
@@ -382,6 +392,7 @@ def run_ours(args):
                      "duration_source": "timed region: ms_per_step (sequence kernel + table kernel)",
                      "isolated_launches_ms_per_pass": round(kernel_ms, 4),
                      "isolated_launches_frac": round(alg_bytes / (kernel_ms * 1e-3) / 1e9 / peak, 4),
+                     "isolated_launches_by_shape": by_shape,
                      "frac_of_nominal_8TBs": round(achieved / 8000.0, 4)},
         "cpu_baseline": cpu,
         "e2e": e2e,
