@@ -137,6 +137,48 @@ def test_parity_r12_extremes(orc, version):
     check_full(orc, ep.CompressedTensor.from_blob(blob))
 
 
+def tile_mix(blob: bytes):
+    """(r, tiles that hold an escape and fit the one-layer kernel's 5 KB tile buffer, tiles that fit
+    without one, tiles too large for it): r is header byte 7, T the u32 at 24, the tile offsets (u32, in
+    16-byte units, bit 31 set when the tile holds an escape) start at the u32 offset at 36."""
+    import struct
+    r = blob[7]
+    T, = struct.unpack_from("<I", blob, 24)
+    off, = struct.unpack_from("<I", blob, 36)
+    offs = np.frombuffer(blob, np.uint32, T + 1, off).astype(np.int64)
+    esc = (offs[:T] >> 31).astype(bool)
+    start = offs & 0x7FFFFFFF
+    fit = (start[1:] - start[:T]) * 16 <= 5 * 1024
+    return r, int((esc & fit).sum()), int((~esc & fit).sum()), int((~fit).sum())
+
+
+@pytest.mark.parametrize("kind", ["bf16_6bpp", "fp32_8bpp", "fp16_11bpp", "int16_escapes_r4", "int16_escapes_r7"])
+def test_parity_raw_bit_tiles_with_escapes(orc, kind):
+    """Tiles with raw low bits (r >= 1) decoded by the one-layer kernel's raw-bit fast rounds, with and
+    without escapes, the escape rounds building integer values (escape words far outside the entries' +-31:
+    |z| up to 128001 at r = 7). The blobs are checked to hold the kinds of tile asked for, whole in the tile
+    buffer; every value and lattice coordinate is compared with the oracle."""
+    if kind.startswith("int16"):
+        g = torch.Generator().manual_seed(6)
+        w = torch.randn(64, 4096, generator=g) * 1e-3
+        w[:, 7] = 1.0
+        w[::2, 9] = -1.0
+        w[5::7, 100] = 0.5
+        blob, _ = orc.compress(w.numpy(), 3, 6.0, 16, 100.0 if kind.endswith("r4") else 1000.0)
+        c = ep.CompressedTensor.from_blob(blob)
+        r, esc_fit, plain_fit, too_big = tile_mix(blob)
+        assert r == (4 if kind.endswith("r4") else 7) and esc_fit == 64 and too_big == 0
+    else:
+        cont, rate = kind.split("_")
+        target = float(rate[:-3])
+        G = 12 if target > 10 else 0
+        w = synth.gaussian(1024, 2048, 41, container=cont)
+        c = ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G))
+        r, esc_fit, plain_fit, too_big = tile_mix(c.blob)
+        assert r >= 1 and esc_fit >= 100 and plain_fit >= 100 and too_big == 0
+    check_full(orc, c)
+
+
 @pytest.mark.parametrize("version", VERSIONS)
 def test_parity_random_fuzz(orc, version):
     rng = np.random.default_rng(2024)
