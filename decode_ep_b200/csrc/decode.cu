@@ -1358,8 +1358,8 @@ __device__ __forceinline__ void round_fast_v2(const P& p, const K& kc, uint32_t 
         }
     }
     if constexpr (RAW) {
-        // r >= 1 raw low bits a coordinate, in a tile with no escape (so |hi| <= 31 and every field below stays
-        // under 2^22): t = hi 2^r + lo, so m_i = 1.5*2^22 + 2 idx 2^r + 2 lo + b (i < 7) and
+        // r >= 1 raw low bits a coordinate, in a round where no lane met an escape (so |hi| <= 31 and every field
+        // below stays under 2^22): t = hi 2^r + lo, so m_i = 1.5*2^22 + 2 idx 2^r + 2 lo + b (i < 7) and
         // m_7 = 1.5*2^22 + 4 idx 2^r + 4 lo_7 + 2 pi + b, pi the parity of the seven lo's; the group's 8r
         // bits sit at bit 8 r q of the tile's raw section, in shared memory (rawb).
         const uint32_t r = uint32_t(p.r), o = q * r, a = o & ~3u, sh = (o & 3u) * 8, lmask = (1u << r) - 1u;
