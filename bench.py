@@ -638,6 +638,11 @@ def workload_items(name):
     raise SystemExit(f"unknown workload {name}")
 
 
+def selected_items(name, only=""):
+    """workload_items(name), keeping the tensors whose label contains `only` (all when it is empty)."""
+    return [it for it in workload_items(name) if not only or only in it[0]]
+
+
 def oracle_rate(blob, shape, seconds, workers):
     """Oracle decode rate (params/s) on `workers` threads over runs of 16 tiles, bounded by `seconds`."""
     import oracle
@@ -1013,9 +1018,7 @@ def run_workload(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     peak, peak_kind = measured_hbm_peak()
     lines = []
-    for label, make, target, G in workload_items(args.workload):
-        if args.only and args.only not in label:
-            continue
+    for label, make, target, G in selected_items(args.workload, args.only):
         w = make()
         t_enc = time.perf_counter()
         c = ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G))

@@ -64,3 +64,24 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
         warmup, steps, target_bpp = 3, 2, 4.0
 
     assert bench.run_reference(Args()) is None
+
+
+def test_single_tensor_selection_by_label():
+    assert len(bench.selected_items("sweep4096")) == 24
+    assert [it[0] for it in bench.selected_items("sweep4096", "bf16_6bpp")] == ["gauss4096_bf16_6bpp"]
+    fp32 = bench.selected_items("sweep4096", "fp32")
+    assert len(fp32) == 8 and all(it[0].startswith("gauss4096_fp32_") for it in fp32)
+    assert [it[2] for it in fp32] == [0.5, 1.0, 2.3, 3.0, 5.0, 6.0, 8.0, 11.0]
+    assert bench.selected_items("fp8_8192x28672_5bpp", "nothing") == []
+
+
+def test_committed_traffic_figure_is_consistent():
+    """The DRAM traffic per algorithmic byte that the bench line reports: its ratio is the capture's read +
+    write bytes over the algorithmic bytes, and it is used only while the kernel source hash matches."""
+    import json
+    d = json.load(open(bench.os.path.join(bench.ROOT, "profiles", "decode_traffic.json")))
+    ratio = (d["dram_bytes_read"] + d["dram_bytes_write"]) / d["algorithmic_bytes"]
+    assert abs(ratio - d["dram_bytes_per_algorithmic_byte"]) < 1e-12
+    assert 0.5 < ratio < 1.5
+    got = bench.committed_traffic()
+    assert (got is not None) == (d["kernel_source_sha256_16"] == bench.kernel_source_hash())
