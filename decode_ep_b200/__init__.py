@@ -155,7 +155,8 @@ class TileANSConfig:
 
 @dataclass
 class CompressedTensor:
-    """A compressed 2-D tensor: the blob bytes plus a cached device copy per CUDA device."""
+    """A compressed tensor: the blob bytes (EPK1 lossy, 2-D; or EPL1 lossless, any shape) plus a cached device
+    copy per CUDA device."""
     blob: bytes
     shape: tuple
     dtype: torch.dtype
@@ -176,7 +177,8 @@ class CompressedTensor:
 
     def device_blob(self, device=None) -> torch.Tensor:
         """The blob as a uint8 CUDA tensor (cached). cudaMalloc alignment (256 B) meets the 16 B rule."""
-        dev = torch.device("cuda", torch.cuda.current_device() if device is None else torch.device(device).index)
+        idx = None if device is None else torch.device(device).index
+        dev = torch.device("cuda", torch.cuda.current_device() if idx is None else idx)
         t = self._device_blobs.get(dev.index)
         if t is None:
             host = torch.frombuffer(bytearray(self.blob), dtype=torch.uint8)
@@ -232,6 +234,12 @@ def _compress_lossless(tensor: torch.Tensor, config: TileANSConfig) -> Compresse
     return CompressedTensor(blob, tuple(host.shape), tensor.dtype, 8 * len(blob) / numel if numel else 0.0)
 
 
+def _rows_dense(t: torch.Tensor) -> torch.Tensor:
+    """t itself when its rows are dense and do not overlap (the encoders take a row stride of at least cols),
+    else a contiguous copy: transposed, expanded and other strided views."""
+    return t if t.stride(1) == 1 and t.stride(0) >= t.shape[1] else t.contiguous()
+
+
 def compress(tensor: torch.Tensor, config: EntroPackLossyConfig | TileANSConfig | float) -> CompressedTensor:
     """Compression of a tensor (CPU or CUDA). EntroPackLossyConfig (or a bare target in bits per parameter):
     lossy, 2-D tensors; the library runs rate control and encoding. TileANSConfig: lossless, any shape, on
@@ -244,7 +252,7 @@ def compress(tensor: torch.Tensor, config: EntroPackLossyConfig | TileANSConfig 
         raise EntroPackError(-3, "compress: EntroPack lossy mode takes 2-D tensors only")
     if tensor.dtype not in _TORCH_TO_EP:
         raise EntroPackError(-2, f"compress: unsupported dtype {tensor.dtype}")
-    t = tensor if tensor.stride(1) == 1 else tensor.contiguous()
+    t = _rows_dense(tensor)
     rows, cols = t.shape
     blob_p, nbytes, actual = ctypes.c_void_p(), ctypes.c_size_t(), ctypes.c_double()
     opt = config._options()
@@ -284,7 +292,7 @@ def compress_cuda_noalloc(tensor: torch.Tensor, config: EntroPackLossyConfig | f
         raise EntroPackError(-1, "compress_cuda_noalloc: takes a 2-D CUDA tensor")
     if tensor.dtype not in _TORCH_TO_EP:
         raise EntroPackError(-2, f"compress_cuda_noalloc: unsupported dtype {tensor.dtype}")
-    t = tensor if tensor.stride(1) == 1 else tensor.contiguous()
+    t = _rows_dense(tensor)
     rows, cols = t.shape
     cap = 8 * rows * cols + 2 * rows + 4096
     buf = (ctypes.c_uint8 * cap)()
@@ -326,9 +334,9 @@ def _stream_ptr(stream) -> int | None:
 
 
 def decompress_into(compressed: CompressedTensor, out: torch.Tensor, stream=None) -> torch.Tensor:
-    """Fused decode into a preallocated CUDA tensor (contiguous, the blob's dtype and shape).
-    Asynchronous on ``stream`` (default: the current stream). It allocates nothing and does not
-    synchronise."""
+    """Decode into a preallocated CUDA tensor (contiguous, the blob's dtype and element count): the fused
+    lossy decode (ep_decompress_into) or the lossless one (ep_tans_decompress_into). Asynchronous on
+    ``stream`` (default: the current stream). It allocates nothing and does not synchronise."""
     if not out.is_cuda or not out.is_contiguous() or out.dtype != compressed.dtype:
         raise EntroPackError(-9, "decompress_into: out must be a contiguous CUDA tensor of the blob's dtype")
     dblob = compressed.device_blob(out.device)
@@ -339,9 +347,10 @@ def decompress_into(compressed: CompressedTensor, out: torch.Tensor, stream=None
 
 
 class LayerBatch:
-    """A fixed list of (compressed tensor, output tensor) pairs, marshalled once. Each call to
-    ``run()`` is one ``ep_decompress_many`` call: the whole sequence of fused decodes, chained with
-    programmatic dependent launch, on one stream."""
+    """A fixed list of (compressed lossy tensor, output tensor) pairs, marshalled once. Each call to
+    ``run()`` is one ``ep_decompress_many`` call on one stream: for version-2 blobs of one dtype, a table
+    kernel and one persistent kernel over all the layers' tiles; otherwise one decode per blob, chained
+    with programmatic dependent launch. Overlapping outputs end as if decoded in list order."""
 
     def __init__(self, pairs, stream=None):
         c = ctypes

@@ -93,6 +93,13 @@ def test_strided_input(ep):
     a = ep.compress(view, 3.0).blob
     b = ep.compress(view.contiguous(), 3.0).blob
     assert a == b
+    # Views whose rows are not dense (row stride below cols) are copied before encoding.
+    row = synth.gaussian(1, 64, seed=13, container="bf16")
+    expanded = row.expand(8, 64)
+    assert expanded.stride(0) == 0
+    assert ep.compress(expanded, 4.0).blob == ep.compress(expanded.contiguous(), 4.0).blob
+    transposed = synth.gaussian(64, 32, seed=14, container="bf16").t()
+    assert ep.compress(transposed, 4.0).blob == ep.compress(transposed.contiguous(), 4.0).blob
 
 
 def test_status_codes(ep):
