@@ -40,7 +40,10 @@ class DecodeWorkspace:
 
     A slot is a flat byte buffer, grown to the largest weight decoded into it. A layer's GEMM reads the
     slot its weight was decoded into; an event recorded after that GEMM marks the slot free again, and the
-    next decode into the slot waits for it on the GPU (never on the host)."""
+    next decode into the slot waits for it on the GPU (never on the host). Each stream that writes or reads
+    a slot is recorded on its buffer, so a buffer given up when its slot grows is not reused by the
+    allocator before that work is done. The slots' bookkeeping is host state: the layers of one device run
+    their forwards one at a time (one thread), as a model's layers do."""
 
     _lock = threading.Lock()
     _by_device: dict = {}
@@ -75,6 +78,8 @@ class DecodeWorkspace:
         if self.free[slot] is not None:
             stream.wait_event(self.free[slot])
         layer.decode_weight(out=w, stream=stream)
+        if self.buffers[slot].numel():
+            self.buffers[slot].record_stream(stream)
         ev = torch.cuda.Event()
         ev.record(stream)
         self.ready[slot] = ev
@@ -95,6 +100,8 @@ class DecodeWorkspace:
 
     def release(self, slot: int, stream) -> None:
         """Marks the slot free once the work queued so far on `stream` (the GEMM) is done."""
+        if self.buffers[slot].numel():
+            self.buffers[slot].record_stream(stream)
         ev = torch.cuda.Event()
         ev.record(stream)
         self.free[slot] = ev
