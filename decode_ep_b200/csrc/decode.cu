@@ -2309,12 +2309,20 @@ extern "C" ep_status ep_decompress_many(int count, const uint8_t* const* host_hd
     clear_error();
     if (count < 0 || (count > 0 && (!host_hdrs || !dev_blobs || !blob_bytes || !dsts || !dst_bytes)))
         return fail(EP_ERR_ARG, "ep_decompress_many: bad arguments");
-    // Validate every header before launching anything, so a failure launches nothing.
+    // Validate every header, size, pointer and alignment before launching anything, so a failure launches
+    // nothing, whichever path the list then takes.
     for (int i = 0; i < count; ++i) {
         Header h;
         if (!host_hdrs[i] || !parse_header(host_hdrs[i], h))
             return fail(EP_ERR_CORRUPT, "ep_decompress_many: blob %d has a malformed header", i);
         if (h.total != blob_bytes[i]) return fail(EP_ERR_BUFFER, "ep_decompress_many: blob %d size mismatch", i);
+        if (!dev_blobs[i] || !dsts[i]) return fail(EP_ERR_ARG, "ep_decompress_many: NULL blob or dst %d", i);
+        if ((reinterpret_cast<uintptr_t>(dev_blobs[i]) & 15) || (reinterpret_cast<uintptr_t>(dsts[i]) & 15))
+            return fail(EP_ERR_BUFFER, "ep_decompress_many: blob and dst %d must be 16-byte aligned", i);
+        const uint64_t need = uint64_t(h.M) * h.N * uint64_t(elem_bytes(h.dtype));
+        if (dst_bytes[i] < need)
+            return fail(EP_ERR_BUFFER, "ep_decompress_many: dst %d holds %zu bytes, need %llu", i, dst_bytes[i],
+                        (unsigned long long)need);
     }
     // The fused entries of every version-1 blob, built once for the sequence into stream-ordered scratch
     // (144 KB per blob). The first decode launches in plain stream order behind the expand kernel, and every
@@ -2334,7 +2342,7 @@ extern "C" ep_status ep_decompress_many(int count, const uint8_t* const* host_hd
         }
     }
     const int n1 = int(v1.size());
-    // Version-2 blobs that share one output type: the sequence kernel, after the checks every launch makes.
+    // Version-2 blobs that share one output type: the sequence kernel.
     bool one_type = count >= 2 && n1 == 0;
     int dtype = -1;
     for (int i = 0; one_type && i < count; ++i) {
@@ -2342,13 +2350,6 @@ extern "C" ep_status ep_decompress_many(int count, const uint8_t* const* host_hd
         parse_header(host_hdrs[i], h);
         if (dtype < 0) dtype = h.dtype;
         one_type = h.dtype == dtype;
-        if (!dev_blobs[i] || !dsts[i]) return fail(EP_ERR_ARG, "ep_decompress_many: NULL blob or dst %d", i);
-        if ((reinterpret_cast<uintptr_t>(dev_blobs[i]) & 15) || (reinterpret_cast<uintptr_t>(dsts[i]) & 15))
-            return fail(EP_ERR_BUFFER, "ep_decompress_many: blob and dst %d must be 16-byte aligned", i);
-        const uint64_t need = uint64_t(h.M) * h.N * uint64_t(elem_bytes(h.dtype));
-        if (dst_bytes[i] < need)
-            return fail(EP_ERR_BUFFER, "ep_decompress_many: dst %d holds %zu bytes, need %llu", i, dst_bytes[i],
-                        (unsigned long long)need);
     }
     if (one_type) {
         int device = 0;

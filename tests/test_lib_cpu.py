@@ -149,6 +149,41 @@ def test_decode_rejects_bad_arguments_without_launching(ep):
     assert L.ep_decompress_into(None, fake_dev, len(c.blob), fake_dev, 1 << 20, None) == -1
 
 
+def test_decompress_many_checks_every_entry_before_launching(ep):
+    """ep_decompress_many checks every header, size, pointer and alignment before its first CUDA call, whichever
+    path the list takes (one sequence kernel, or one decode per blob for version-1 or mixed-dtype lists): a bad
+    last entry is refused with nothing launched."""
+    import ctypes as c
+    L = ep.lib()
+    w = synth.gaussian(64, 128, seed=21, container="bf16")
+    v2 = ep.compress(w, 3.0)
+    v1 = ep.compress(w, ep.EntroPackLossyConfig(3.0, format_version=1))
+    f16 = ep.compress(synth.gaussian(64, 128, seed=22, container="fp16"), 3.0)
+    comps = [v2, v1, f16]
+    fake = 0x100000  # aligned and never dereferenced: every case fails on the host first
+
+    def call(hdrs=None, blobs=None, sizes=None, dsts=None, dst_sizes=None, count=3):
+        n = len(comps)
+        H = (c.c_char_p * n)(*(hdrs or [x.header for x in comps]))
+        B = (c.c_void_p * n)(*(blobs or [fake] * n))
+        S = (c.c_size_t * n)(*(sizes or [len(x.blob) for x in comps]))
+        D = (c.c_void_p * n)(*(dsts or [fake + 0x100000 * (k + 1) for k in range(n)]))
+        Z = (c.c_size_t * n)(*(dst_sizes or [2 * 64 * 128] * n))
+        return L.ep_decompress_many(count, H, B, S, D, Z, None)
+
+    assert L.ep_decompress_many(-1, None, None, None, None, None, None) == -1
+    assert L.ep_decompress_many(2, None, None, None, None, None, None) == -1
+    assert L.ep_decompress_many(0, None, None, None, None, None, None) == 0
+    good_dsts = [fake + 0x100000 * (k + 1) for k in range(3)]
+    assert call(dsts=good_dsts[:2] + [good_dsts[2] + 8]) == -9            # last dst misaligned
+    assert call(dst_sizes=[2 * 64 * 128, 2 * 64 * 128, 1000]) == -9        # last dst too small
+    assert call(dsts=good_dsts[:2] + [None]) == -1                         # last dst NULL
+    assert call(blobs=[fake, fake, fake + 4]) == -9                        # last blob misaligned
+    assert call(sizes=[len(v2.blob), len(v1.blob) - 16, len(f16.blob)]) == -9  # a blob size mismatch
+    assert call(hdrs=[v2.header, v1.header, b"EPKX" + f16.header[4:]]) == -6   # last header malformed
+    assert L.ep_last_error().decode().startswith("ep_decompress_many")
+
+
 def _fuzz_case(seed):
     """A seeded random tensor, target and tile size: shapes from one row to a few hundred, every container."""
     import random
