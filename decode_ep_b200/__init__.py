@@ -397,7 +397,8 @@ def decode_coords(compressed: CompressedTensor, device=None, stream=None) -> tor
 
 
 def device_status(stream=None) -> int:
-    """Synchronises the stream, then reads and clears the device status word (EP_DEV_* bits)."""
+    """Synchronises the stream, then reads and clears the device status word (EP_DEV_* bits). Decodes still
+    running on other streams may set bits between the read and the clear: synchronise them first."""
     flags = ctypes.c_int32()
     _check(lib().ep_get_device_status(_stream_ptr(stream), ctypes.byref(flags)), "device_status")
     return flags.value

@@ -282,7 +282,9 @@ ep_status ep_decode_coords_into(const uint8_t* host_hdr, const void* dev_blob, s
 /*
  * ep_get_device_status: synchronises cuda_stream, then reads and clears the device status word of the
  * current device. That word is the OR of the EP_DEV_* bits that the decode kernels set since the last
- * read. Errors: EP_ERR_ARG, EP_ERR_CUDA.
+ * read. The read and the clear are two copies: a bit that a decode still running on another stream sets
+ * between them is lost, so synchronise the streams whose decodes should be reported before the call.
+ * Errors: EP_ERR_ARG, EP_ERR_CUDA.
  */
 ep_status ep_get_device_status(void* cuda_stream, int32_t* flags);
 
