@@ -152,28 +152,38 @@ def tile_mix(blob: bytes):
     return r, int((esc & fit).sum()), int((~esc & fit).sum()), int((~fit).sum())
 
 
-@pytest.mark.parametrize("kind", ["bf16_6bpp", "fp32_8bpp", "fp16_11bpp", "int16_escapes_r4", "int16_escapes_r7"])
-def test_parity_raw_bit_tiles_with_escapes(orc, kind):
+RAW_ESC = [
+    # (id, container or None for an oracle-encoded int16-escape blob, rows, cols, target bpp, G or forced alpha)
+    ("bf16_6bpp", "bf16", 1024, 2048, 6.0, 0),
+    ("fp32_8bpp", "fp32", 1024, 2048, 8.0, 0),
+    ("fp16_11bpp", "fp16", 1024, 2048, 11.0, 12),
+    ("bf16_6bpp_rows_of_255_groups", "bf16", 1024, 2040, 6.0, 0),
+    ("int16_escapes_r4", None, 64, 4096, 6.0, 100.0),
+    ("int16_escapes_r7", None, 64, 4096, 6.0, 1000.0),
+    ("int16_escapes_r4_rows_of_511_groups", None, 64, 4088, 6.0, 100.0),
+]
+
+
+@pytest.mark.parametrize("kind,cont,M,N,target,arg", RAW_ESC, ids=[e[0] for e in RAW_ESC])
+def test_parity_raw_bit_tiles_with_escapes(orc, kind, cont, M, N, target, arg):
     """Tiles with raw low bits (r >= 1) decoded by the one-layer kernel's raw-bit fast rounds, with and
     without escapes, the escape rounds building integer values (escape words far outside the entries' +-31:
-    |z| up to 128001 at r = 7). The blobs are checked to hold the kinds of tile asked for, whole in the tile
-    buffer; every value and lattice coordinate is compared with the oracle."""
-    if kind.startswith("int16"):
+    |z| up to 128001 at r = 7), in rows of whole rounds and in rows that are not (255 and 511 groups). The
+    blobs are checked to hold the kinds of tile asked for, whole in the tile buffer; every value and lattice
+    coordinate is compared with the oracle."""
+    if cont is None:
         g = torch.Generator().manual_seed(6)
-        w = torch.randn(64, 4096, generator=g) * 1e-3
+        w = torch.randn(M, N, generator=g) * 1e-3
         w[:, 7] = 1.0
         w[::2, 9] = -1.0
         w[5::7, 100] = 0.5
-        blob, _ = orc.compress(w.numpy(), 3, 6.0, 16, 100.0 if kind.endswith("r4") else 1000.0)
+        blob, _ = orc.compress(w.numpy(), 3, target, 16, arg)
         c = ep.CompressedTensor.from_blob(blob)
         r, esc_fit, plain_fit, too_big = tile_mix(blob)
-        assert r == (4 if kind.endswith("r4") else 7) and esc_fit == 64 and too_big == 0
+        assert r == (4 if arg == 100.0 else 7) and esc_fit >= 60 and too_big == 0
     else:
-        cont, rate = kind.split("_")
-        target = float(rate[:-3])
-        G = 12 if target > 10 else 0
-        w = synth.gaussian(1024, 2048, 41, container=cont)
-        c = ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=G))
+        w = synth.gaussian(M, N, 41, container=cont)
+        c = ep.compress(w, ep.EntroPackLossyConfig(target, rounds_per_tile=int(arg)))
         r, esc_fit, plain_fit, too_big = tile_mix(c.blob)
         assert r >= 1 and esc_fit >= 100 and plain_fit >= 100 and too_big == 0
     check_full(orc, c)
