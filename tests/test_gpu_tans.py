@@ -16,7 +16,7 @@ if not torch.cuda.is_available():
 import decode_ep_b200 as ep  # noqa: E402
 
 from test_oracle_tileans import DTYPES, SHAPES, bits_of  # noqa: E402
-from test_tans_cpu import VIEW, tensor_of  # noqa: E402
+from test_tans_cpu import VIEW, several_coded_planes, tensor_of  # noqa: E402
 
 
 def raw_bits(t: torch.Tensor, kind: str) -> np.ndarray:
@@ -61,6 +61,19 @@ def test_decode_tile_sizes(orc, K):
         got = ep.decompress(c)
         status_clean()
         assert np.array_equal(raw_bits(got, kind), orc.tans_decompress(c.blob))
+
+
+def test_decode_several_coded_planes(orc):
+    """Tiles with two to four rANS-coded byte planes, each decoded from the lane's one state in plane order
+    (coded masks 3, 15 and 11, a raw plane between coded ones included, and ragged tiles of 7 elements a
+    lane): every element against the oracle and the input."""
+    for kind, b, K, mask in several_coded_planes():
+        c = ep.compress(tensor_of(kind, b), ep.TileANSConfig(elems_per_lane=K))
+        assert ep.blob_info(c.blob)["coded_mask"] == mask
+        got = ep.decompress(c)
+        status_clean()
+        assert np.array_equal(raw_bits(got, kind), orc.tans_decompress(c.blob))
+        assert np.array_equal(raw_bits(got, kind), b)
 
 
 def test_decode_special_patterns_and_all_raw(orc):

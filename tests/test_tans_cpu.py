@@ -21,6 +21,32 @@ def tensor_of(kind: str, bits: np.ndarray) -> torch.Tensor:
     return t.view(TORCH[kind]).reshape(bits.shape)
 
 
+def several_coded_planes():
+    """(kind, raw bits, K, coded planes mask) of tensors with two or more coded byte planes: values from a set of
+    33 levels (every byte plane clusters), and FP32 copies of BF16 weights (zero low bytes and a clustered top
+    byte coded around a raw one); one of them in ragged tiles of 7 elements a lane."""
+    rng = np.random.default_rng(5)
+    levels = torch.tensor(np.arange(-16, 17) / 8.0, dtype=torch.float32)
+    idx = torch.from_numpy(rng.integers(0, 33, size=(3, 1000, 37)))
+    cases = []
+    for kind, mask in (("bf16", 3), ("fp16", 3), ("fp32", 15)):
+        x = levels[idx].to(TORCH[kind])
+        cases.append((kind, x.view(VIEW[kind]).numpy().view(np.uint32 if kind == "fp32" else np.uint16), 0, mask))
+    y = (torch.from_numpy(rng.standard_normal((2000, 64))).float() * 0.02).to(torch.bfloat16).to(torch.float32)
+    cases.append(("fp32", y.view(torch.int32).numpy().view(np.uint32), 0, 11))
+    x = levels[torch.from_numpy(rng.integers(0, 33, size=(7, 3001)))].to(torch.bfloat16)
+    cases.append(("bf16", x.view(torch.int16).numpy().view(np.uint16), 7, 3))
+    return cases
+
+
+def test_host_encoder_several_coded_planes():
+    for kind, b, K, mask in several_coded_planes():
+        c = ep.compress(tensor_of(kind, b), ep.TileANSConfig(elems_per_lane=K))
+        assert ep.blob_info(c.blob)["coded_mask"] == mask, kind
+        assert c.blob == orc.tans_compress(b, DTYPES[kind], K=K or 128), kind
+        assert np.array_equal(orc.tans_decompress(c.blob), b), kind
+
+
 @pytest.mark.parametrize("kind", list(DTYPES))
 @pytest.mark.parametrize("shape", SHAPES)
 def test_host_encoder_matches_oracle(kind, shape):
